@@ -1,0 +1,242 @@
+// Host side of libmosaic: argument validation, TMA descriptors and kernel dispatch
+// behind the C ABI declared in mosaic.h.
+#include <atomic>
+#include <cstdio>
+#include <cstring>
+
+#include "common.cuh"
+#include "gemm.cuh"
+
+namespace mq {
+
+// launchers (quant.cu, select.cu, gemm.cu)
+int amax_grid(int64_t n8);
+cudaError_t launch_quant_weight(const uint16_t* W, int N, int K, uint8_t* codes, uint8_t* sf, uint8_t* sf_swz,
+                                float* g, uint8_t* rcodes, uint8_t* rsf, float* partial, cudaStream_t s);
+cudaError_t launch_quant_act(const uint16_t* X, int M, int K, uint8_t* codes, uint8_t* sf, uint8_t* sf_swz,
+                             float* g, cudaStream_t s);
+cudaError_t launch_hessian(const uint16_t* X, int T, int K, float* H, cudaStream_t s);
+cudaError_t launch_delta(const uint16_t* W, int N, int K, const float* H, const float* g, double* delta,
+                         cudaStream_t s);
+cudaError_t launch_topk(const double* delta, int B, int budget, int32_t* rank, int32_t* sel, cudaStream_t s);
+cudaError_t launch_pack(const uint8_t* rcodes, const uint8_t* rsf, int N, int K, const int32_t* sel, int budget,
+                        uint8_t* blk_codes, uint8_t* blk_sf, int32_t* blk_kt, int32_t* tile_ptr, uint32_t* bitmap,
+                        cudaStream_t s);
+
+}  // namespace mq
+
+using namespace mq;
+
+static std::atomic<uint64_t> g_launches{0};
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    }
+    return fn;
+}
+
+// 2-D byte tensor [rows][row_bytes] (row-major), 128-byte swizzled boxes of
+// box_bytes x box_rows; rows outside the tensor read as zero.
+static bool make_tmap_bytes(CUtensorMap* map, const void* base, uint64_t row_bytes, uint64_t rows,
+                            uint32_t box_bytes, uint32_t box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {row_bytes, rows};
+    cuuint64_t strides[1] = {row_bytes};
+    cuuint32_t box[2] = {box_bytes, box_rows};
+    cuuint32_t es[2] = {1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, es,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+static inline cudaStream_t as_stream(mq_stream s) { return reinterpret_cast<cudaStream_t>(s); }
+
+static inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+static mq_status launched(cudaError_t e, int kernels) {
+    if (e != cudaSuccess) return MQ_ERR_CUDA;
+    g_launches.fetch_add((uint64_t)kernels, std::memory_order_relaxed);
+    return MQ_OK;
+}
+
+static bool nvfp4_shape_ok(int rows, int cols) { return rows > 0 && cols > 0 && cols % 64 == 0; }
+
+extern "C" {
+
+size_t mq_sf_swz_bytes(int rows, int cols) {
+    if (rows <= 0 || cols <= 0 || cols % 64) return 0;
+    return (size_t)((rows + 127) / 128) * 128 * (size_t)(cols / 16);
+}
+
+int mq_budget_blocks(int N, int K, double frac) {
+    if (N <= 0 || K <= 0 || N % 64 || K % 64 || !(frac >= 0.0 && frac <= 1.0)) return -1;
+    const double nb = (double)(N / 64) * (double)(K / 64);
+    return (int)(frac * nb + 1e-9);
+}
+
+size_t mq_quantize_weight_workspace_bytes(int N, int K) {
+    (void)N;
+    (void)K;
+    return (size_t)148 * 8 * sizeof(float);
+}
+
+size_t mq_delta_topk_workspace_bytes(int N, int K, int budget) {
+    (void)N;
+    (void)K;
+    (void)budget;
+    return 0;
+}
+
+size_t mq_gemm_workspace_bytes(int M, int N, int K, unsigned flags) {
+    (void)flags;
+    if (M <= 0 || N <= 0 || K <= 0 || N % 128 || K % 256) return 0;
+    return decode_workspace_bytes(M, N, K);
+}
+
+mq_status mq_quantize_weight(const mq_bf16* W, int N, int K, mq_nvfp4_mat* base, mq_nvfp4_mat* resid_full,
+                             void* ws, size_t ws_bytes, mq_stream stream) {
+    if (!W || !base || !resid_full || !nvfp4_shape_ok(N, K) || N % 64) return MQ_ERR_INVALID_ARG;
+    if (!base->codes || !base->sf_swz || !base->gscale || !resid_full->codes || !resid_full->sf)
+        return MQ_ERR_INVALID_ARG;
+    if (base->rows != N || base->cols != K || resid_full->rows != N || resid_full->cols != K)
+        return MQ_ERR_INVALID_ARG;
+    if (!aligned(W, 16) || !aligned(base->codes, 8) || !aligned(resid_full->codes, 8) || !aligned(base->sf_swz, 4))
+        return MQ_ERR_INVALID_ARG;
+    if (!ws || ws_bytes < mq_quantize_weight_workspace_bytes(N, K)) return MQ_ERR_WORKSPACE;
+    cudaError_t e = launch_quant_weight(W, N, K, base->codes, base->sf, base->sf_swz, base->gscale,
+                                        resid_full->codes, resid_full->sf, static_cast<float*>(ws),
+                                        as_stream(stream));
+    return launched(e, 2);
+}
+
+mq_status mq_hessian_diag(const mq_bf16* Xcal, int T, int K, float* H, mq_stream stream) {
+    if (!Xcal || !H || T <= 0 || K <= 0 || K % 64) return MQ_ERR_INVALID_ARG;
+    return launched(launch_hessian(Xcal, T, K, H, as_stream(stream)), 1);
+}
+
+mq_status mq_delta_score_topk(const mq_bf16* W, const float* H, const mq_nvfp4_mat* base,
+                              const mq_nvfp4_mat* resid_full, int budget, double* delta, int32_t* rank,
+                              int32_t* sel, void* ws, size_t ws_bytes, mq_stream stream) {
+    (void)resid_full;
+    (void)ws;
+    (void)ws_bytes;
+    if (!W || !H || !base || !base->gscale || !delta) return MQ_ERR_INVALID_ARG;
+    const int N = base->rows, K = base->cols;
+    if (!nvfp4_shape_ok(N, K) || N % 64 || !aligned(W, 16)) return MQ_ERR_INVALID_ARG;
+    const int B = (N / 64) * (K / 64);
+    if (budget < 0 || budget > B) return MQ_ERR_INVALID_ARG;
+    if (budget > 0 && (!rank || !sel)) return MQ_ERR_INVALID_ARG;
+    cudaStream_t s = as_stream(stream);
+    cudaError_t e = launch_delta(W, N, K, H, base->gscale, delta, s);
+    if (e != cudaSuccess) return MQ_ERR_CUDA;
+    g_launches.fetch_add(1);
+    return launched(launch_topk(delta, B, budget, rank, sel, s), budget > 0 ? 2 : 0);
+}
+
+mq_status mq_pack_residual(const mq_nvfp4_mat* resid_full, const int32_t* sel, int budget, mq_residual_packed* out,
+                           mq_stream stream) {
+    if (!resid_full || !out || !resid_full->codes || !resid_full->sf) return MQ_ERR_INVALID_ARG;
+    const int N = resid_full->rows, K = resid_full->cols;
+    if (!nvfp4_shape_ok(N, K) || N % 64) return MQ_ERR_INVALID_ARG;
+    if (out->N != N || out->K != K || out->nblk != budget || budget < 0 || budget > (N / 64) * (K / 64))
+        return MQ_ERR_INVALID_ARG;
+    if (!out->tile_ptr || !out->bitmap) return MQ_ERR_INVALID_ARG;
+    if (budget > 0 && (!sel || !out->blk_codes || !out->blk_sf || !out->blk_kt)) return MQ_ERR_INVALID_ARG;
+    if (budget > 0 && (!aligned(out->blk_codes, 16) || !aligned(out->blk_sf, 16))) return MQ_ERR_INVALID_ARG;
+    return launched(launch_pack(resid_full->codes, resid_full->sf, N, K, sel, budget, out->blk_codes, out->blk_sf,
+                                out->blk_kt, out->tile_ptr, out->bitmap, as_stream(stream)),
+                    1);
+}
+
+mq_status mq_quantize_act(const mq_bf16* X, int M, int K, mq_nvfp4_mat* xq, mq_stream stream) {
+    if (!X || !xq || !xq->codes || !xq->sf_swz || !xq->gscale || !nvfp4_shape_ok(M, K)) return MQ_ERR_INVALID_ARG;
+    if (xq->rows != M || xq->cols != K || !aligned(X, 16) || !aligned(xq->codes, 8) || !aligned(xq->sf_swz, 4))
+        return MQ_ERR_INVALID_ARG;
+    return launched(launch_quant_act(X, M, K, xq->codes, xq->sf, xq->sf_swz, xq->gscale, as_stream(stream)), 1);
+}
+
+mq_status mq_gemm(const mq_nvfp4_mat* xq, const mq_nvfp4_mat* wq, const mq_residual_packed* r, mq_bf16* Y, int M,
+                  int N, int K, unsigned flags, void* ws, size_t ws_bytes, mq_stream stream) {
+    if (!xq || !wq || !Y || M <= 0 || N <= 0 || K <= 0 || N % 64 || K % 64) return MQ_ERR_INVALID_ARG;
+    if (N % 128 || K % 256) return MQ_ERR_UNSUPPORTED_SHAPE;
+    if (!xq->codes || !xq->sf_swz || !xq->gscale || !wq->codes || !wq->sf_swz || !wq->gscale)
+        return MQ_ERR_INVALID_ARG;
+    if (xq->rows != M || xq->cols != K || wq->rows != N || wq->cols != K) return MQ_ERR_INVALID_ARG;
+    if ((flags & MQ_GEMM_BASE_ONLY) && (flags & MQ_GEMM_RESIDUAL_ONLY)) return MQ_ERR_INVALID_ARG;
+    if (!aligned(xq->codes, 16) || !aligned(wq->codes, 16) || !aligned(xq->sf_swz, 16) || !aligned(wq->sf_swz, 16))
+        return MQ_ERR_INVALID_ARG;
+    const bool has_r = r && r->nblk > 0 && !(flags & MQ_GEMM_BASE_ONLY);
+    if (r && r->nblk > 0) {
+        if (r->N != N || r->K != K || !r->blk_codes || !r->blk_sf || !r->tile_ptr || !r->bitmap)
+            return MQ_ERR_INVALID_ARG;
+        if (!aligned(r->blk_codes, 16) || !aligned(r->blk_sf, 16)) return MQ_ERR_INVALID_ARG;
+    }
+    DecodePlan d = plan_decode(M, N, K);
+    const size_t need = decode_workspace_bytes(M, N, K);
+    if (need > 0 && (!ws || ws_bytes < need || !aligned(ws, 16))) return MQ_ERR_WORKSPACE;
+
+    CUtensorMap tw, tx;
+    if (!make_tmap_bytes(&tw, wq->codes, (uint64_t)K / 2, (uint64_t)N, 128, 128)) return MQ_ERR_CUDA;
+    if (!make_tmap_bytes(&tx, xq->codes, (uint64_t)K / 2, (uint64_t)M, 128, (uint32_t)d.BN)) return MQ_ERR_CUDA;
+
+    GemmParams p;
+    memset(&p, 0, sizeof p);
+    p.w_sf = wq->sf_swz;
+    p.x_sf = xq->sf_swz;
+    p.g_w = wq->gscale;
+    p.g_x = xq->gscale;
+    if (has_r) {
+        p.blk_codes = r->blk_codes;
+        p.blk_sf = r->blk_sf;
+        p.tile_ptr = r->tile_ptr;
+        p.bitmap = r->bitmap;
+    }
+    p.has_resid = has_r ? 1 : 0;
+    p.Y = Y;
+    p.M = M;
+    p.N = N;
+    p.K = K;
+    p.mode = (flags & MQ_GEMM_BASE_ONLY) ? 1 : (flags & MQ_GEMM_RESIDUAL_ONLY) ? 2 : 0;
+    if (need > 0) {
+        size_t part = (size_t)d.splits * d.tiles_m * d.BN * N * sizeof(float);
+        part = (part + 255) & ~size_t(255);
+        p.partial = static_cast<float*>(ws);
+        p.counters = reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + part);
+    }
+    return launched(launch_gemm_decode(tw, tx, p, d, as_stream(stream)), 1);
+}
+
+mq_status mq_get_error(mq_stream stream) {
+    if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return MQ_ERR_CUDA;
+    int v = 0;
+    if (read_clear_error(&v) != cudaSuccess) return MQ_ERR_CUDA;
+    return v ? (mq_status)v : MQ_OK;
+}
+
+const char* mq_status_string(mq_status s) {
+    switch (s) {
+        case MQ_OK: return "ok";
+        case MQ_ERR_INVALID_ARG: return "invalid argument";
+        case MQ_ERR_UNSUPPORTED_SHAPE: return "shape not supported by the GEMM kernels";
+        case MQ_ERR_WORKSPACE: return "workspace missing or too small";
+        case MQ_ERR_CUDA: return "CUDA error";
+        case MQ_ERR_TIMEOUT: return "device pipeline wait timed out";
+    }
+    return "unknown status";
+}
+
+uint64_t mq_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+}  // extern "C"

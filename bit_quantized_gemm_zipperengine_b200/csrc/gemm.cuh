@@ -1,0 +1,41 @@
+// Types and entry points of the fused GEMM shared by the kernels and the host API.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace mq {
+
+struct GemmParams {
+    const uint8_t* w_sf;     // tiled scales of W
+    const uint8_t* x_sf;     // tiled scales of X
+    const float* g_w;        // [1]
+    const float* g_x;        // [M]
+    const uint8_t* blk_codes;
+    const uint8_t* blk_sf;
+    const int32_t* tile_ptr;
+    const uint32_t* bitmap;
+    uint16_t* Y;
+    float* partial;          // split-K partials [splits][tiles_m * BN][N]
+    int* counters;           // [tiles_m * tiles_n], zero between calls
+    int M, N, K;
+    int splits, iters_per_split;
+    int mode;                // 0 fused, 1 base only, 2 residual only
+    int has_resid;
+};
+
+// Decode kernel tiling: token tile BN, grid tiles_n x splits x tiles_m, `iters`
+// K stages (256 elements each) per split.
+struct DecodePlan {
+    int BN, tiles_m, tiles_n, splits, iters;
+};
+
+DecodePlan plan_decode(int M, int N, int K);
+size_t decode_workspace_bytes(int M, int N, int K);
+cudaError_t launch_gemm_decode(const CUtensorMap& tw, const CUtensorMap& tx, GemmParams p, const DecodePlan& d,
+                               cudaStream_t s);
+cudaError_t read_clear_error(int* value);
+
+}  // namespace mq

@@ -1,0 +1,236 @@
+"""ctypes binding of libmosaic (include/mosaic.h).
+
+Argument marshalling only: every step of the path runs in the CUDA library. PyTorch
+provides device memory and the current stream. There is no CPU fallback: a missing
+library or a non-CUDA tensor raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libmosaic.so")
+_lib = None
+
+MQ_OK = 0
+MQ_GEMM_AUTO = 0
+MQ_GEMM_DECODE = 1
+MQ_GEMM_PREFILL = 2
+MQ_GEMM_BASE_ONLY = 4
+MQ_GEMM_RESIDUAL_ONLY = 8
+
+EXPORTED = (
+    "mq_sf_swz_bytes", "mq_budget_blocks", "mq_quantize_weight_workspace_bytes", "mq_delta_topk_workspace_bytes",
+    "mq_gemm_workspace_bytes", "mq_quantize_weight", "mq_hessian_diag", "mq_delta_score_topk", "mq_pack_residual",
+    "mq_quantize_act", "mq_gemm", "mq_get_error", "mq_status_string", "mq_launch_count",
+)
+
+
+class MosaicError(RuntimeError):
+    pass
+
+
+class NVFP4Mat(ctypes.Structure):
+    _fields_ = [("rows", ctypes.c_int), ("cols", ctypes.c_int), ("codes", ctypes.c_void_p), ("sf", ctypes.c_void_p),
+                ("sf_swz", ctypes.c_void_p), ("gscale", ctypes.c_void_p)]
+
+
+class ResidualPacked(ctypes.Structure):
+    _fields_ = [("N", ctypes.c_int), ("K", ctypes.c_int), ("nblk", ctypes.c_int), ("blk_codes", ctypes.c_void_p),
+                ("blk_sf", ctypes.c_void_p), ("blk_kt", ctypes.c_void_p), ("tile_ptr", ctypes.c_void_p),
+                ("bitmap", ctypes.c_void_p)]
+
+
+def lib():
+    """Load libmosaic.so (built by ``__graft_entry__.build()`` or ``build.py``)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise MosaicError(f"libmosaic.so is not built ({LIB_PATH}); run __graft_entry__.build()")
+    L = ctypes.CDLL(LIB_PATH)
+    vp, i32, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    P = ctypes.POINTER
+    L.mq_sf_swz_bytes.argtypes = [i32, i32]
+    L.mq_sf_swz_bytes.restype = sz
+    L.mq_budget_blocks.argtypes = [i32, i32, ctypes.c_double]
+    L.mq_budget_blocks.restype = i32
+    L.mq_quantize_weight_workspace_bytes.argtypes = [i32, i32]
+    L.mq_quantize_weight_workspace_bytes.restype = sz
+    L.mq_delta_topk_workspace_bytes.argtypes = [i32, i32, i32]
+    L.mq_delta_topk_workspace_bytes.restype = sz
+    L.mq_gemm_workspace_bytes.argtypes = [i32, i32, i32, ctypes.c_uint]
+    L.mq_gemm_workspace_bytes.restype = sz
+    L.mq_quantize_weight.argtypes = [vp, i32, i32, P(NVFP4Mat), P(NVFP4Mat), vp, sz, vp]
+    L.mq_hessian_diag.argtypes = [vp, i32, i32, vp, vp]
+    L.mq_delta_score_topk.argtypes = [vp, vp, P(NVFP4Mat), P(NVFP4Mat), i32, vp, vp, vp, vp, sz, vp]
+    L.mq_pack_residual.argtypes = [P(NVFP4Mat), vp, i32, P(ResidualPacked), vp]
+    L.mq_quantize_act.argtypes = [vp, i32, i32, P(NVFP4Mat), vp]
+    L.mq_gemm.argtypes = [P(NVFP4Mat), P(NVFP4Mat), P(ResidualPacked), vp, i32, i32, i32, ctypes.c_uint, vp, sz, vp]
+    for f in ("mq_quantize_weight", "mq_hessian_diag", "mq_delta_score_topk", "mq_pack_residual", "mq_quantize_act",
+              "mq_gemm", "mq_get_error"):
+        getattr(L, f).restype = i32
+    L.mq_get_error.argtypes = [vp]
+    L.mq_status_string.argtypes = [i32]
+    L.mq_status_string.restype = ctypes.c_char_p
+    L.mq_launch_count.argtypes = []
+    L.mq_launch_count.restype = ctypes.c_uint64
+    _lib = L
+    return L
+
+
+def _check(status: int, what: str):
+    if status != MQ_OK:
+        raise MosaicError(f"{what}: {lib().mq_status_string(status).decode()} (status {status})")
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise MosaicError("libmosaic takes CUDA tensors only")
+    return t.data_ptr()
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _u8(*shape, device):
+    return torch.empty(shape, dtype=torch.uint8, device=device)
+
+
+def mat(d: dict) -> NVFP4Mat:
+    return NVFP4Mat(d["rows"], d["cols"], _ptr(d.get("codes")), _ptr(d.get("sf")), _ptr(d.get("sf_swz")),
+                    _ptr(d.get("gscale")))
+
+
+def packed_struct(p: dict | None) -> ResidualPacked | None:
+    if p is None:
+        return None
+    return ResidualPacked(p["N"], p["K"], p["nblk"], _ptr(p.get("blk_codes")), _ptr(p.get("blk_sf")),
+                          _ptr(p.get("blk_kt")), _ptr(p.get("tile_ptr")), _ptr(p.get("bitmap")))
+
+
+# ------------------------------------------------------------------ allocation helpers
+def alloc_weight(N: int, K: int, device, with_sf: bool = True) -> tuple[dict, dict]:
+    L = lib()
+    base = {"rows": N, "cols": K, "codes": _u8(N, K // 2, device=device),
+            "sf": _u8(N, K // 16, device=device) if with_sf else None,
+            "sf_swz": _u8(L.mq_sf_swz_bytes(N, K), device=device),
+            "gscale": torch.empty(1, dtype=torch.float32, device=device)}
+    resid = {"rows": N, "cols": K, "codes": _u8(N, K // 2, device=device), "sf": _u8(N, K // 16, device=device),
+             "sf_swz": None, "gscale": None}
+    return base, resid
+
+
+def alloc_act(M: int, K: int, device, with_sf: bool = False) -> dict:
+    L = lib()
+    return {"rows": M, "cols": K, "codes": _u8(M, K // 2, device=device),
+            "sf": _u8(M, K // 16, device=device) if with_sf else None,
+            "sf_swz": _u8(L.mq_sf_swz_bytes(M, K), device=device),
+            "gscale": torch.empty(M, dtype=torch.float32, device=device)}
+
+
+def alloc_packed(N: int, K: int, budget: int, device) -> dict:
+    KB = K // 64
+    KW = (KB + 31) // 32
+    nb = max(budget, 1)
+    return {"N": N, "K": K, "nblk": budget, "blk_codes": _u8(nb, 2048, device=device),
+            "blk_sf": _u8(nb, 512, device=device), "blk_kt": torch.empty(nb, dtype=torch.int32, device=device),
+            "tile_ptr": torch.empty(N // 64 + 1, dtype=torch.int32, device=device),
+            "bitmap": torch.empty((N // 64, KW), dtype=torch.int32, device=device)}
+
+
+# ------------------------------------------------------------------ the path (C names)
+def mq_quantize_weight(W: torch.Tensor, base: dict, resid: dict, ws: torch.Tensor, stream=None):
+    N, K = W.shape
+    _check(lib().mq_quantize_weight(_ptr(W), N, K, ctypes.byref(mat(base)), ctypes.byref(mat(resid)), _ptr(ws),
+                                    ws.numel() * ws.element_size(), _stream(stream)), "mq_quantize_weight")
+
+
+def mq_hessian_diag(Xcal: torch.Tensor, H: torch.Tensor, stream=None):
+    T, K = Xcal.shape
+    _check(lib().mq_hessian_diag(_ptr(Xcal), T, K, _ptr(H), _stream(stream)), "mq_hessian_diag")
+
+
+def mq_delta_score_topk(W, H, base: dict, resid: dict | None, budget: int, delta, rank, sel, ws=None, stream=None):
+    wsb = 0 if ws is None else ws.numel() * ws.element_size()
+    rs = None if resid is None else ctypes.byref(mat(resid))
+    _check(lib().mq_delta_score_topk(_ptr(W), _ptr(H), ctypes.byref(mat(base)), rs, budget, _ptr(delta), _ptr(rank),
+                                     _ptr(sel), _ptr(ws), wsb, _stream(stream)), "mq_delta_score_topk")
+
+
+def mq_pack_residual(resid: dict, sel, budget: int, packed: dict, stream=None):
+    _check(lib().mq_pack_residual(ctypes.byref(mat(resid)), _ptr(sel), budget, ctypes.byref(packed_struct(packed)),
+                                  _stream(stream)), "mq_pack_residual")
+
+
+def mq_quantize_act(X: torch.Tensor, xq: dict, stream=None):
+    M, K = X.shape
+    _check(lib().mq_quantize_act(_ptr(X), M, K, ctypes.byref(mat(xq)), _stream(stream)), "mq_quantize_act")
+
+
+def mq_gemm(xq: dict, wq: dict, packed: dict | None, Y: torch.Tensor, M: int, N: int, K: int, flags: int = 0,
+            ws: torch.Tensor | None = None, stream=None):
+    ps = packed_struct(packed)
+    wsb = 0 if ws is None else ws.numel() * ws.element_size()
+    _check(lib().mq_gemm(ctypes.byref(mat(xq)), ctypes.byref(mat(wq)), None if ps is None else ctypes.byref(ps),
+                         _ptr(Y), M, N, K, flags, _ptr(ws), wsb, _stream(stream)), "mq_gemm")
+
+
+def mq_get_error(stream=None) -> int:
+    return lib().mq_get_error(_stream(stream))
+
+
+def mq_launch_count() -> int:
+    return int(lib().mq_launch_count())
+
+
+def gemm_workspace(M: int, N: int, K: int, flags: int, device) -> torch.Tensor | None:
+    """Zero-initialised workspace for mq_gemm (the tile counters must start at zero)."""
+    n = lib().mq_gemm_workspace_bytes(M, N, K, flags)
+    return torch.zeros(max(n, 16), dtype=torch.uint8, device=device) if n else None
+
+
+# ------------------------------------------------------------------ convenience
+class Layer:
+    """One linear layer through the whole path: quantize W, H from calibration tokens,
+    Delta + top-K, pack, then per call quantize X and run the fused GEMM. Buffers are
+    allocated once (torch) and reused."""
+
+    def __init__(self, N: int, K: int, budget: int, device="cuda", with_sf: bool = True):
+        self.N, self.K, self.budget, self.device = N, K, budget, device
+        self.base, self.resid = alloc_weight(N, K, device, with_sf)
+        self.qws = torch.empty(lib().mq_quantize_weight_workspace_bytes(N, K), dtype=torch.uint8, device=device)
+        self.H = torch.empty(K, dtype=torch.float32, device=device)
+        self.delta = torch.empty((N // 64) * (K // 64), dtype=torch.float64, device=device)
+        self.rank = torch.empty(max(budget, 1), dtype=torch.int32, device=device)
+        self.sel = torch.empty(max(budget, 1), dtype=torch.int32, device=device)
+        self.packed = alloc_packed(N, K, budget, device)
+        self._act = {}
+
+    def prepare(self, W: torch.Tensor, Xcal: torch.Tensor, stream=None):
+        mq_quantize_weight(W, self.base, self.resid, self.qws, stream)
+        mq_hessian_diag(Xcal, self.H, stream)
+        mq_delta_score_topk(W, self.H, self.base, None, self.budget, self.delta, self.rank, self.sel, None, stream)
+        mq_pack_residual(self.resid, self.sel, self.budget, self.packed, stream)
+
+    def act_buffers(self, M: int, flags: int = 0):
+        key = (M, flags)
+        if key not in self._act:
+            self._act[key] = (alloc_act(M, self.K, self.device),
+                              torch.empty((M, self.N), dtype=torch.bfloat16, device=self.device),
+                              gemm_workspace(M, self.N, self.K, flags, self.device))
+        return self._act[key]
+
+    def forward(self, X: torch.Tensor, flags: int = 0, stream=None) -> torch.Tensor:
+        M = X.shape[0]
+        xq, Y, ws = self.act_buffers(M, flags)
+        mq_quantize_act(X, xq, stream)
+        mq_gemm(xq, self.base, self.packed, Y, M, self.N, self.K, flags, ws, stream)
+        return Y

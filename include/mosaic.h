@@ -1,0 +1,213 @@
+/*
+ * mosaic.h -- C ABI of libmosaic, the B200 (sm_100a) MosaicQuant / ZipperEngine path.
+ *
+ * The method (MosaicQuant technical summary, "Methodology"; arXiv 2606.15652 abstract):
+ * the weight matrix W is split into a dense 4-bit base Q(W) plus a 4-bit residual R,
+ * W ~ Q(W) + R (section 1, "Inlier-outlier disaggregation"); R is kept only on the
+ * top-K 64x64 blocks ranked by a Hessian-guided Delta-score (section 2, "Block-wise
+ * residual allocation"); ZipperEngine runs base and sparse residual in one fused GEMM,
+ * with activation quantization and the reduce-sum in the same pipeline (section 3).
+ *
+ * Number format (NVFP4): E2M1 values {0, 0.5, 1, 1.5, 2, 3, 4, 6} with a sign bit, one
+ * E4M3 scale per 16 consecutive K elements, and an fp32 tensor scale g (one per weight
+ * matrix, one per token for activations). g = amax / 2688 (1 if amax = 0). Per group:
+ * s = amax_group / (6 g); sf = E4M3_rne_satfinite(s); d = dec(sf) * g;
+ * code_i = E2M1_rne_satfinite(a_i / d) (a signed zero when d = 0). All fp32 IEEE
+ * operations, no fused multiply-add; codes and scales are bit-exact with the CPU oracle.
+ *
+ * Conventions for every call:
+ *  - All pointers are DEVICE pointers unless stated otherwise; the caller allocates and
+ *    frees every buffer. The library allocates no device memory.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default stream).
+ *    The returned status covers argument validation and launch errors only; a device
+ *    side timeout (a pipeline wait that gave up) is reported by mq_get_error().
+ *  - Shapes: N and K must be multiples of 64 (MQ_ERR_INVALID_ARG otherwise); the GEMM
+ *    additionally needs N % 128 == 0 and K % 256 == 0 (MQ_ERR_UNSUPPORTED_SHAPE).
+ *    M >= 1. Inputs must be finite (NaN/Inf is a precondition violation).
+ *  - bf16 buffers are passed as raw 16-bit patterns (mq_bf16).
+ */
+#ifndef MOSAIC_H_
+#define MOSAIC_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t mq_bf16;
+typedef void* mq_stream; /* cudaStream_t */
+
+typedef enum {
+    MQ_OK = 0,
+    MQ_ERR_INVALID_ARG = 1,       /* null pointer, bad shape, budget out of range */
+    MQ_ERR_UNSUPPORTED_SHAPE = 2, /* valid NVFP4 shape the GEMM kernels do not tile */
+    MQ_ERR_WORKSPACE = 3,         /* workspace missing or smaller than required */
+    MQ_ERR_CUDA = 4,              /* a CUDA runtime/driver call or launch failed */
+    MQ_ERR_TIMEOUT = 5            /* a device pipeline wait gave up (see mq_get_error) */
+} mq_status;
+
+/* GEMM flags. */
+enum {
+    MQ_GEMM_AUTO = 0,          /* pick the decode or prefill kernel from M */
+    MQ_GEMM_DECODE = 1,        /* small-M kernel: W as the MMA's M side, split-K */
+    MQ_GEMM_PREFILL = 2,       /* large-M kernel: X as the MMA's M side */
+    MQ_GEMM_BASE_ONLY = 4,     /* skip the residual blocks (dense-only reference) */
+    MQ_GEMM_RESIDUAL_ONLY = 8  /* only the residual blocks (linearity check) */
+};
+
+/*
+ * An NVFP4 matrix, rows x cols (weights: N x K; activations: M x K).
+ *  codes : [rows][cols/2] bytes; element 2j of a row in the low nibble of byte j,
+ *          element 2j+1 in the high nibble. Nibble = sign (bit 3) | E2M1 magnitude.
+ *  sf    : [rows][cols/16] E4M3 bytes, row-major (group q of row r at r*cols/16 + q).
+ *          May be NULL where a call says so.
+ *  sf_swz: the GEMM's tiled scale layout, mq_sf_swz_bytes(rows, cols) bytes: rows in
+ *          tiles of 128 and groups in steps of 4 (64 K elements); each (row tile,
+ *          K step) is a 512-byte chunk at ((r/128)*(cols/64) + q/4)*512, and inside it
+ *          row t = r%128, group q%4 sit at (t%32)*16 + (t/32)*4 + q%4. Rows past `rows`
+ *          up to the next multiple of 128 hold zero.
+ *  gscale: fp32 tensor scale(s): [1] for weights, [rows] for activations.
+ */
+typedef struct {
+    int rows;
+    int cols;
+    uint8_t* codes;
+    uint8_t* sf;
+    uint8_t* sf_swz;
+    float* gscale;
+} mq_nvfp4_mat;
+
+/*
+ * Packed sparse residual of an N x K weight, nblk selected blocks in ascending block
+ * index b = nt*(K/64) + kt (nt = block row, kt = block column).
+ *  blk_codes: [nblk][2048]; block row r (0..63), packed byte j (0..31) of that row at
+ *             (r/8)*256 + (j/16)*128 + (r%8)*16 + (j%16) (8-row x 16-byte core
+ *             matrices, the MMA's no-swizzle K-major operand layout).
+ *  blk_sf   : [nblk][512]; the block's 64x4 scales written into the 128-row scale chunk
+ *             of its 128-row band (tile row t = 64*(nt%2) + r, group q at
+ *             (t%32)*16 + (t/32)*4 + q), every other byte zero.
+ *  blk_kt   : [nblk] block column of each entry.
+ *  tile_ptr : [N/64 + 1] CSR over block rows: entries of block row nt are
+ *             [tile_ptr[nt], tile_ptr[nt+1]).
+ *  bitmap   : [N/64][ceil((K/64)/32)] u32; bit kt%32 of word kt/32 set iff (nt, kt)
+ *             is selected.
+ */
+typedef struct {
+    int N;
+    int K;
+    int nblk;
+    uint8_t* blk_codes;
+    uint8_t* blk_sf;
+    int32_t* blk_kt;
+    int32_t* tile_ptr;
+    uint32_t* bitmap;
+} mq_residual_packed;
+
+/* ---- sizes (host only, no device work) ---------------------------------------- */
+
+/* Bytes of an sf_swz buffer for a rows x cols matrix: ceil(rows/128)*128*(cols/16). */
+size_t mq_sf_swz_bytes(int rows, int cols);
+
+/* floor(frac * (N/64) * (K/64)); -1 on a bad shape or frac outside [0, 1]. */
+int mq_budget_blocks(int N, int K, double frac);
+
+/* Workspace of mq_quantize_weight (per-CTA partial maxima). */
+size_t mq_quantize_weight_workspace_bytes(int N, int K);
+
+/* Workspace of mq_delta_score_topk for `budget` selected blocks. */
+size_t mq_delta_topk_workspace_bytes(int N, int K, int budget);
+
+/* Workspace of mq_gemm: split-K fp32 partials plus per-tile counters. The counter
+ * region must be zero before the first call on a workspace; every call leaves it zero
+ * again when it completes. Calls sharing a workspace must not overlap on the GPU. */
+size_t mq_gemm_workspace_bytes(int M, int N, int K, unsigned flags);
+
+/* ---- the path ----------------------------------------------------------------- */
+
+/*
+ * A1. Weight quantization (MosaicQuant summary, "Methodology", section 1).
+ * W: bf16 [N][K]. Writes base = NVFP4(W, g_w) and resid_full = NVFP4(W - deq Q(W), g_w)
+ * for EVERY element (the residual uses the base's tensor scale g_w; selection happens
+ * later). base: codes, sf_swz and gscale[1] required, sf optional (NULL skips it).
+ * resid_full: codes and sf required; its sf_swz is not written; its gscale may be NULL
+ * (the residual shares base->gscale). ws: mq_quantize_weight_workspace_bytes.
+ */
+mq_status mq_quantize_weight(const mq_bf16* W, int N, int K, mq_nvfp4_mat* base, mq_nvfp4_mat* resid_full,
+                             void* ws, size_t ws_bytes, mq_stream stream);
+
+/*
+ * A2. Diagonal Hessian estimate of the input channels (summary, "Methodology",
+ * section 2): H_k = fp32( sum_t fp64(x_tk)^2 / T ), sum in t order. Xcal: bf16 [T][K],
+ * H: fp32 [K]. T >= 1, K % 64 == 0.
+ */
+mq_status mq_hessian_diag(const mq_bf16* Xcal, int T, int K, float* H, mq_stream stream);
+
+/*
+ * A3 + A4. Delta-score and top-K block selection (summary, "Methodology", section 2:
+ * marginal reduction of the output distortion per block, residual error weighted by
+ * the diagonal Hessian). For block b = (nt, kt):
+ *   Delta_b = T64_k( fp64(H_k) * T64_r( fp64(e)^2 - fp64(e')^2 ) ),
+ *   e = fp32(W - deq Q(W)), e' = fp32(e - deq R),
+ * where T64 is the pairwise tree v[i] += v[i+32], +16, +8, +4, +2, +1 over the block's
+ * 64 rows (inner) and 64 columns (outer). The kernel recomputes e and e' from W and the
+ * tensor scale base->gscale, bit-identical to mq_quantize_weight's codes; base->codes and
+ * resid_full are not read (they may be NULL).
+ * Then blocks are ordered by (Delta descending, b ascending): rank[0..budget) = the
+ * first `budget` indices in that order, sel[0..budget) = the same set ascending.
+ * delta: fp64 [(N/64)*(K/64)]. 0 <= budget <= number of blocks.
+ * ws: mq_delta_topk_workspace_bytes.
+ */
+mq_status mq_delta_score_topk(const mq_bf16* W, const float* H, const mq_nvfp4_mat* base,
+                              const mq_nvfp4_mat* resid_full, int budget, double* delta, int32_t* rank,
+                              int32_t* sel, void* ws, size_t ws_bytes, mq_stream stream);
+
+/*
+ * A5. Pack the selected residual blocks (the sparse residual of section 1, stored per
+ * block for the fused GEMM's "sparse block computation", arXiv abstract).
+ * resid_full: codes and sf of mq_quantize_weight. sel: ascending block indices [budget].
+ * out: N, K, nblk = budget, and buffers sized as in mq_residual_packed.
+ */
+mq_status mq_pack_residual(const mq_nvfp4_mat* resid_full, const int32_t* sel, int budget,
+                           mq_residual_packed* out, mq_stream stream);
+
+/*
+ * A6. Activation quantization (summary, "Methodology", section 3: quantization inside
+ * the pipeline). X: bf16 [M][K]. Per token m: g_x[m] = amax(X[m,:]) / 2688 (1 if 0),
+ * then NVFP4 with that scale. xq: codes, sf_swz and gscale[M] required, sf optional.
+ */
+mq_status mq_quantize_act(const mq_bf16* X, int M, int K, mq_nvfp4_mat* xq, mq_stream stream);
+
+/*
+ * A7 + A8. ZipperEngine fused GEMM (summary, "Methodology", section 3; arXiv abstract):
+ *   Y[m,n] = bf16_rn( acc[m,n] * fp32(g_x[m] * g_w) ),
+ *   acc[m,n] = sum_k xh[m,k] * ( wh[n,k] + [block (n/64, k/64) selected] rh[n,k] ),
+ * with xh, wh, rh the scaled E2M1 values (val * dec(sf)). Base and residual blocks
+ * accumulate into one fp32 tensor-memory accumulator (tcgen05 kind::mxf4nvf4 MMAs, one
+ * extra MMA per selected block); the decode kernel then adds its split-K partials in a
+ * fixed order. r == NULL (or r->nblk == 0) is the dense base alone.
+ * xq: codes, sf_swz, gscale [M]. wq: codes, sf_swz, gscale [1]. Y: bf16 [M][N].
+ * flags: MQ_GEMM_* (one of AUTO/DECODE/PREFILL, optionally BASE_ONLY or RESIDUAL_ONLY).
+ * ws: mq_gemm_workspace_bytes(M, N, K, flags) bytes (see there); may be NULL if that
+ * size is 0.
+ */
+mq_status mq_gemm(const mq_nvfp4_mat* xq, const mq_nvfp4_mat* wq, const mq_residual_packed* r, mq_bf16* Y,
+                  int M, int N, int K, unsigned flags, void* ws, size_t ws_bytes, mq_stream stream);
+
+/* Synchronizes `stream`, then returns (and clears) the device error word: MQ_OK, or
+ * MQ_ERR_TIMEOUT if a kernel gave up on a pipeline wait, or MQ_ERR_CUDA if the
+ * synchronization itself failed. */
+mq_status mq_get_error(mq_stream stream);
+
+/* Static description of a status code. */
+const char* mq_status_string(mq_status status);
+
+/* Number of kernel launches the library has issued in this process (for accounting). */
+uint64_t mq_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOSAIC_H_ */

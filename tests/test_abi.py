@@ -1,0 +1,65 @@
+"""The C ABI library loads on a machine without a GPU, exports every call that
+include/mosaic.h declares, and validates arguments on the host before any launch."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    from bit_quantized_gemm_zipperengine_b200 import build, mosaic
+    build.build()
+    return mosaic.lib()
+
+
+def declared():
+    with open(os.path.join(ROOT, "include", "mosaic.h")) as f:
+        text = f.read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(mq_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = declared()
+    assert len(names) >= 14
+    for n in names:
+        assert hasattr(L, n), n
+    from bit_quantized_gemm_zipperengine_b200 import mosaic
+    assert set(mosaic.EXPORTED) == set(names)
+
+
+def test_size_helpers(L):
+    assert L.mq_sf_swz_bytes(16, 4096) == 128 * 256
+    assert L.mq_sf_swz_bytes(300, 512) == 384 * 32
+    assert L.mq_sf_swz_bytes(16, 100) == 0
+    assert L.mq_budget_blocks(256, 512, 0.10) == 3
+    assert L.mq_budget_blocks(4096, 4096, 0.10) == 409
+    assert L.mq_budget_blocks(28672, 8192, 0.05) == 2867
+    assert L.mq_budget_blocks(256, 512, 1.5) == -1
+    assert L.mq_quantize_weight_workspace_bytes(4096, 4096) >= 4 * 148 * 8
+    # decode GEMM at M=16, N=K=4096: 32 weight tiles x 4 K splits -> fp32 partials + counters
+    ws = L.mq_gemm_workspace_bytes(16, 4096, 4096, 0)
+    assert ws == 4 * 16 * 4096 * 4 + 32 * 4
+
+
+def test_host_validation_rejects_bad_arguments(L):
+    from bit_quantized_gemm_zipperengine_b200 import mosaic
+    m = mosaic.NVFP4Mat(16, 4096, None, None, None, None)
+    # null pointers and bad shapes are rejected before any CUDA call
+    assert L.mq_quantize_act(None, 16, 4096, ctypes.byref(m), None) == 1
+    assert L.mq_hessian_diag(None, 8, 64, None, None) == 1
+    assert L.mq_gemm(ctypes.byref(m), ctypes.byref(m), None, None, 16, 4096, 4096, 0, None, 0, None) == 1
+    fake = ctypes.c_void_p(0x10000)
+    xm = mosaic.NVFP4Mat(16, 4096, fake, None, fake, fake)
+    wm = mosaic.NVFP4Mat(4096 + 64, 4096, fake, None, fake, fake)
+    assert L.mq_gemm(ctypes.byref(xm), ctypes.byref(wm), None, fake, 16, 4096 + 64, 4096, 0, None, 0, None) == 2
+    wm2 = mosaic.NVFP4Mat(4096, 4096, fake, None, fake, fake)
+    assert L.mq_gemm(ctypes.byref(xm), ctypes.byref(wm2), None, fake, 16, 4096, 4096,
+                     mosaic.MQ_GEMM_BASE_ONLY | mosaic.MQ_GEMM_RESIDUAL_ONLY, None, 0, None) == 1
+    # decode split-K needs its workspace
+    assert L.mq_gemm(ctypes.byref(xm), ctypes.byref(wm2), None, fake, 16, 4096, 4096, 0, None, 0, None) == 3
+    assert L.mq_status_string(3) == b"workspace missing or too small"

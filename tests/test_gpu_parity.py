@@ -1,0 +1,144 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle on the same seeded
+inputs. Codes, scales, H, Delta (fp64 bits), ranking, selection and the packed store are
+compared bit for bit; the GEMM within the stated tolerance."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from gpu_path import check_gemm, gpu_run, oracle_ref, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def dev():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    return torch.device("cuda:0")
+
+
+_cache = {}
+
+
+def _pair(name, dev, M=None):
+    key = (name, M)
+    if key not in _cache:
+        L = synth.layer(name, M=M)
+        budget = synth.budget_blocks(L["N"], L["K"], 0.10)
+        _cache[key] = (L, budget, gpu_run(L, budget, dev), oracle_ref(L, budget))
+    return _cache[key]
+
+
+WORKLOADS = ["tiny", "llama3_8b_qproj_decode"]
+
+
+@pytest.mark.parametrize("name", WORKLOADS)
+def test_quantize_weight_bit_exact(name, dev):
+    L, budget, g, o = _pair(name, dev)
+    wq = o["wq"]
+    assert g["g"] == wq["g"]
+    assert np.array_equal(g["codes"], wq["codes"])
+    assert np.array_equal(g["sf"], wq["sf"])
+    assert np.array_equal(g["sf_swz"], oracle.sf_tile(wq["sf"], L["N"], L["K"]))
+    assert np.array_equal(g["r_codes"], wq["r_codes"])
+    assert np.array_equal(g["r_sf"], wq["r_sf"])
+
+
+@pytest.mark.parametrize("name", WORKLOADS)
+def test_hessian_bit_exact(name, dev):
+    L, budget, g, o = _pair(name, dev)
+    assert np.array_equal(g["H"].view(np.uint32), o["H"].view(np.uint32))
+
+
+@pytest.mark.parametrize("name", WORKLOADS)
+def test_delta_and_selection_bit_exact(name, dev):
+    L, budget, g, o = _pair(name, dev)
+    assert np.array_equal(g["delta"].view(np.uint64), o["delta"].view(np.uint64))
+    assert np.array_equal(g["rank"], o["rank"])
+    assert np.array_equal(g["sel"], o["sel"])
+
+
+@pytest.mark.parametrize("name", WORKLOADS)
+def test_pack_bit_exact(name, dev):
+    L, budget, g, o = _pair(name, dev)
+    for k in ("blk_codes", "blk_sf", "blk_kt", "tile_ptr"):
+        assert np.array_equal(g["packed"][k], o["packed"][k]), k
+    assert np.array_equal(g["packed"]["bitmap"].view(np.uint32), o["packed"]["bitmap"])
+
+
+@pytest.mark.parametrize("name", WORKLOADS)
+def test_quantize_act_bit_exact(name, dev):
+    L, budget, g, o = _pair(name, dev)
+    xq = o["xq"]
+    assert np.array_equal(g["xq_codes"], xq["codes"])
+    assert np.array_equal(g["xq_g"], xq["g"])
+    assert np.array_equal(g["xq_swz"], oracle.sf_tile(xq["sf"], L["M"], L["K"]))
+
+
+@pytest.mark.parametrize("name", WORKLOADS)
+def test_gemm_fused_within_tolerance(name, dev):
+    L, budget, g, o = _pair(name, dev)
+    check_gemm(g["Y"], o["y"], o["yabs"], name)
+
+
+@pytest.mark.parametrize("M", [1, 5, 16, 37, 64, 100, 128, 130, 300])
+def test_gemm_ragged_token_counts(M, dev):
+    """Token counts that are not a multiple of the token tile (ragged tail), across the
+    16/32/64/128 token tiles and several token tiles."""
+    L = synth.layer("tiny", M=M)
+    budget = synth.budget_blocks(L["N"], L["K"], 0.10)
+    g = gpu_run(L, budget, dev)
+    o = oracle_ref(L, budget)
+    assert np.array_equal(g["xq_codes"], o["xq"]["codes"])
+    check_gemm(g["Y"], o["y"], o["yabs"], f"M={M}")
+
+
+def test_gemm_base_only_paths_identical(dev):
+    """r = NULL, a zero budget and the BASE_ONLY flag all give the dense base, bit for bit,
+    and match the oracle's base-only GEMM."""
+    from bit_quantized_gemm_zipperengine_b200 import mosaic
+    L, budget, g, o = _pair("llama3_8b_qproj_decode", dev)
+    layer = g["layer"]
+    M, N, K = L["M"], L["N"], L["K"]
+    xq, _, ws = layer.act_buffers(M)
+    outs = []
+    for packed, flags in ((None, 0), (layer.packed, mosaic.MQ_GEMM_BASE_ONLY)):
+        Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        mosaic.mq_gemm(xq, layer.base, packed, Y, M, N, K, flags, ws)
+        outs.append(Y)
+    zero = mosaic.alloc_packed(N, K, 0, dev)
+    mosaic.mq_pack_residual(layer.resid, layer.sel, 0, zero)
+    Y0 = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    mosaic.mq_gemm(xq, layer.base, zero, Y0, M, N, K, 0, ws)
+    torch.cuda.synchronize()
+    assert torch.equal(outs[0], outs[1]) and torch.equal(outs[0], Y0)
+    yb, yba = oracle.gemm_rows(o["xq"], o["wq"], o["sel"], M, N, K, 1)
+    check_gemm(outs[0].float().cpu().numpy().astype(np.float64), yb, yba, "base only")
+
+
+def test_gemm_linearity(dev):
+    """Fused = base-only + residual-only (one accumulator, summed by linearity)."""
+    from bit_quantized_gemm_zipperengine_b200 import mosaic
+    L, budget, g, o = _pair("llama3_8b_qproj_decode", dev)
+    layer = g["layer"]
+    M, N, K = L["M"], L["N"], L["K"]
+    xq, _, ws = layer.act_buffers(M)
+    Yr = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    mosaic.mq_gemm(xq, layer.base, layer.packed, Yr, M, N, K, mosaic.MQ_GEMM_RESIDUAL_ONLY, ws)
+    torch.cuda.synchronize()
+    yr, yra = oracle.gemm_rows(o["xq"], o["wq"], o["sel"], M, N, K, 2)
+    check_gemm(Yr.float().cpu().numpy().astype(np.float64), yr, yra, "residual only")
+    assert np.abs(yr).max() > 0
+
+
+def test_repeat_calls_deterministic(dev):
+    """Same inputs twice: quantization, Delta, selection and the GEMM output repeat bit for
+    bit (the split-K partials are added in a fixed order)."""
+    L, budget, g, o = _pair("llama3_8b_qproj_decode", dev)
+    g2 = gpu_run(L, budget, dev)
+    for k in ("codes", "sf", "r_codes", "r_sf", "H", "rank", "sel"):
+        assert np.array_equal(g[k], g2[k]), k
+    assert np.array_equal(g["delta"].view(np.uint64), g2["delta"].view(np.uint64))
+    assert np.array_equal(g["Y"], g2["Y"])
