@@ -218,6 +218,41 @@ mq_status mq_gemm(const mq_nvfp4_mat* xq, const mq_nvfp4_mat* wq, const mq_resid
     return launched(launch_gemm_decode(tw, tx, p, d, as_stream(stream)), 1);
 }
 
+mq_status mq_run_layer(const mq_bf16* W, const mq_bf16* X, const mq_bf16* Xcal, mq_bf16* Y, int M, int N, int K,
+                       int T, int budget, unsigned flags, int host, mq_layer_buffers* buf, mq_stream stream) {
+    if (!W || !X || !Xcal || !Y || !buf || M <= 0 || N <= 0 || K <= 0 || T <= 0) return MQ_ERR_INVALID_ARG;
+    cudaStream_t s = as_stream(stream);
+    const mq_bf16 *w = W, *x = X, *xc = Xcal;
+    mq_bf16* y = Y;
+    if (host) {
+        if (!buf->W_dev || !buf->X_dev || !buf->Xcal_dev || !buf->Y_dev) return MQ_ERR_INVALID_ARG;
+        if (cudaMemcpyAsync(buf->W_dev, W, (size_t)N * K * 2, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+            cudaMemcpyAsync(buf->Xcal_dev, Xcal, (size_t)T * K * 2, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+            cudaMemcpyAsync(buf->X_dev, X, (size_t)M * K * 2, cudaMemcpyHostToDevice, s) != cudaSuccess)
+            return MQ_ERR_CUDA;
+        w = buf->W_dev;
+        x = buf->X_dev;
+        xc = buf->Xcal_dev;
+        y = buf->Y_dev;
+    }
+    mq_status st;
+    if ((st = mq_quantize_weight(w, N, K, &buf->base, &buf->resid_full, buf->ws_quant, buf->ws_quant_bytes,
+                                 stream)) != MQ_OK)
+        return st;
+    if ((st = mq_hessian_diag(xc, T, K, buf->H, stream)) != MQ_OK) return st;
+    if ((st = mq_delta_score_topk(w, buf->H, &buf->base, &buf->resid_full, budget, buf->delta, buf->rank, buf->sel,
+                                  NULL, 0, stream)) != MQ_OK)
+        return st;
+    if ((st = mq_pack_residual(&buf->resid_full, buf->sel, budget, &buf->packed, stream)) != MQ_OK) return st;
+    if ((st = mq_quantize_act(x, M, K, &buf->xq, stream)) != MQ_OK) return st;
+    if ((st = mq_gemm(&buf->xq, &buf->base, &buf->packed, y, M, N, K, flags, buf->ws_gemm, buf->ws_gemm_bytes,
+                      stream)) != MQ_OK)
+        return st;
+    if (host && cudaMemcpyAsync(Y, buf->Y_dev, (size_t)M * N * 2, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return MQ_ERR_CUDA;
+    return MQ_OK;
+}
+
 mq_status mq_get_error(mq_stream stream) {
     if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return MQ_ERR_CUDA;
     int v = 0;

@@ -25,7 +25,7 @@ MQ_GEMM_RESIDUAL_ONLY = 8
 EXPORTED = (
     "mq_sf_swz_bytes", "mq_budget_blocks", "mq_quantize_weight_workspace_bytes", "mq_delta_topk_workspace_bytes",
     "mq_gemm_workspace_bytes", "mq_quantize_weight", "mq_hessian_diag", "mq_delta_score_topk", "mq_pack_residual",
-    "mq_quantize_act", "mq_gemm", "mq_get_error", "mq_status_string", "mq_launch_count",
+    "mq_quantize_act", "mq_gemm", "mq_run_layer", "mq_get_error", "mq_status_string", "mq_launch_count",
 )
 
 
@@ -42,6 +42,14 @@ class ResidualPacked(ctypes.Structure):
     _fields_ = [("N", ctypes.c_int), ("K", ctypes.c_int), ("nblk", ctypes.c_int), ("blk_codes", ctypes.c_void_p),
                 ("blk_sf", ctypes.c_void_p), ("blk_kt", ctypes.c_void_p), ("tile_ptr", ctypes.c_void_p),
                 ("bitmap", ctypes.c_void_p)]
+
+
+class LayerBuffers(ctypes.Structure):
+    _fields_ = [("base", NVFP4Mat), ("resid_full", NVFP4Mat), ("xq", NVFP4Mat), ("H", ctypes.c_void_p),
+                ("delta", ctypes.c_void_p), ("rank", ctypes.c_void_p), ("sel", ctypes.c_void_p),
+                ("packed", ResidualPacked), ("ws_quant", ctypes.c_void_p), ("ws_quant_bytes", ctypes.c_size_t),
+                ("ws_gemm", ctypes.c_void_p), ("ws_gemm_bytes", ctypes.c_size_t), ("W_dev", ctypes.c_void_p),
+                ("X_dev", ctypes.c_void_p), ("Xcal_dev", ctypes.c_void_p), ("Y_dev", ctypes.c_void_p)]
 
 
 def lib():
@@ -73,6 +81,8 @@ def lib():
     for f in ("mq_quantize_weight", "mq_hessian_diag", "mq_delta_score_topk", "mq_pack_residual", "mq_quantize_act",
               "mq_gemm", "mq_get_error"):
         getattr(L, f).restype = i32
+    L.mq_run_layer.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, ctypes.c_uint, i32, P(LayerBuffers), vp]
+    L.mq_run_layer.restype = i32
     L.mq_get_error.argtypes = [vp]
     L.mq_status_string.argtypes = [i32]
     L.mq_status_string.restype = ctypes.c_char_p
@@ -183,6 +193,19 @@ def mq_gemm(xq: dict, wq: dict, packed: dict | None, Y: torch.Tensor, M: int, N:
                          _ptr(Y), M, N, K, flags, _ptr(ws), wsb, _stream(stream)), "mq_gemm")
 
 
+def mq_run_layer(W, X, Xcal, Y, M: int, N: int, K: int, T: int, budget: int, flags: int, host: bool,
+                 buf: LayerBuffers, stream=None):
+    """Whole path in one call. With host=True, W/X/Xcal/Y are pinned CPU tensors."""
+    def p(t):
+        if host:
+            if t.is_cuda:
+                raise MosaicError("host=True expects CPU tensors")
+            return t.data_ptr()
+        return _ptr(t)
+    _check(lib().mq_run_layer(p(W), p(X), p(Xcal), p(Y), M, N, K, T, budget, flags, 1 if host else 0,
+                              ctypes.byref(buf), _stream(stream)), "mq_run_layer")
+
+
 def mq_get_error(stream=None) -> int:
     return lib().mq_get_error(_stream(stream))
 
@@ -227,6 +250,26 @@ class Layer:
                               torch.empty((M, self.N), dtype=torch.bfloat16, device=self.device),
                               gemm_workspace(M, self.N, self.K, flags, self.device))
         return self._act[key]
+
+    def buffers(self, M: int, T: int, flags: int = 0, staging: bool = False) -> LayerBuffers:
+        """The ctypes struct mq_run_layer takes (staging buffers for host inputs)."""
+        xq, Y, ws = self.act_buffers(M, flags)
+        b = LayerBuffers()
+        b.base, b.resid_full, b.xq = mat(self.base), mat(self.resid), mat(xq)
+        b.H, b.delta, b.rank, b.sel = _ptr(self.H), _ptr(self.delta), _ptr(self.rank), _ptr(self.sel)
+        b.packed = packed_struct(self.packed)
+        b.ws_quant, b.ws_quant_bytes = _ptr(self.qws), self.qws.numel()
+        b.ws_gemm, b.ws_gemm_bytes = (_ptr(ws), ws.numel()) if ws is not None else (None, 0)
+        if staging:
+            key = ("staging", M, T)
+            if key not in self._act:
+                bf = torch.bfloat16
+                self._act[key] = (torch.empty((self.N, self.K), dtype=bf, device=self.device),
+                                  torch.empty((M, self.K), dtype=bf, device=self.device),
+                                  torch.empty((T, self.K), dtype=bf, device=self.device))
+            w, x, xc = self._act[key]
+            b.W_dev, b.X_dev, b.Xcal_dev, b.Y_dev = _ptr(w), _ptr(x), _ptr(xc), _ptr(Y)
+        return b
 
     def forward(self, X: torch.Tensor, flags: int = 0, stream=None) -> torch.Tensor:
         M = X.shape[0]

@@ -195,6 +195,41 @@ mq_status mq_quantize_act(const mq_bf16* X, int M, int K, mq_nvfp4_mat* xq, mq_s
 mq_status mq_gemm(const mq_nvfp4_mat* xq, const mq_nvfp4_mat* wq, const mq_residual_packed* r, mq_bf16* Y,
                   int M, int N, int K, unsigned flags, void* ws, size_t ws_bytes, mq_stream stream);
 
+/*
+ * Device buffers of one layer for mq_run_layer (all caller-owned; sizes as in the
+ * individual calls above). W_dev, X_dev, Xcal_dev and Y_dev are staging buffers used
+ * only when mq_run_layer is given host pointers.
+ */
+typedef struct {
+    mq_nvfp4_mat base;        /* sf may be NULL */
+    mq_nvfp4_mat resid_full;  /* codes and sf */
+    mq_nvfp4_mat xq;          /* codes, sf_swz, gscale [M] */
+    float* H;                 /* [K] */
+    double* delta;            /* [(N/64)*(K/64)] */
+    int32_t* rank;            /* [budget] */
+    int32_t* sel;             /* [budget] */
+    mq_residual_packed packed;
+    void* ws_quant;           /* mq_quantize_weight_workspace_bytes */
+    size_t ws_quant_bytes;
+    void* ws_gemm;            /* mq_gemm_workspace_bytes (counters zeroed once) */
+    size_t ws_gemm_bytes;
+    mq_bf16* W_dev;           /* [N][K]  staging when host != 0 */
+    mq_bf16* X_dev;           /* [M][K]  staging when host != 0 */
+    mq_bf16* Xcal_dev;        /* [T][K]  staging when host != 0 */
+    mq_bf16* Y_dev;           /* [M][N]  staging when host != 0 */
+} mq_layer_buffers;
+
+/*
+ * The whole path for one layer in the method's order: A1 quantize W, A2 H from the T
+ * calibration tokens, A3+A4 Delta and top-`budget` selection, A5 pack, A6 quantize X,
+ * A7+A8 fused GEMM into Y. With host == 0, W, X, Xcal and Y are device pointers. With
+ * host != 0 they are HOST pointers (page-locked for the copies to be asynchronous):
+ * the inputs are copied into buf->W_dev, X_dev, Xcal_dev and the result from buf->Y_dev
+ * back to Y, all on `stream`. Errors as the individual calls.
+ */
+mq_status mq_run_layer(const mq_bf16* W, const mq_bf16* X, const mq_bf16* Xcal, mq_bf16* Y, int M, int N, int K,
+                       int T, int budget, unsigned flags, int host, mq_layer_buffers* buf, mq_stream stream);
+
 /* Synchronizes `stream`, then returns (and clears) the device error word: MQ_OK, or
  * MQ_ERR_TIMEOUT if a kernel gave up on a pipeline wait, or MQ_ERR_CUDA if the
  * synchronization itself failed. */
