@@ -26,6 +26,7 @@ EXPORTED = (
     "mq_sf_swz_bytes", "mq_budget_blocks", "mq_quantize_weight_workspace_bytes", "mq_delta_topk_workspace_bytes",
     "mq_gemm_workspace_bytes", "mq_quantize_weight", "mq_hessian_diag", "mq_delta_score_topk", "mq_pack_residual",
     "mq_quantize_act", "mq_gemm", "mq_run_layer", "mq_get_error", "mq_status_string", "mq_launch_count",
+    "mq_gemm_noalloc", "mq_gemm_noalloc_scratch_limit",
 )
 
 
@@ -83,6 +84,10 @@ def lib():
         getattr(L, f).restype = i32
     L.mq_run_layer.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, ctypes.c_uint, i32, P(LayerBuffers), vp]
     L.mq_run_layer.restype = i32
+    L.mq_gemm_noalloc.argtypes = [P(NVFP4Mat), P(NVFP4Mat), P(ResidualPacked), vp, i32, i32, i32, ctypes.c_uint, vp]
+    L.mq_gemm_noalloc.restype = i32
+    L.mq_gemm_noalloc_scratch_limit.argtypes = []
+    L.mq_gemm_noalloc_scratch_limit.restype = sz
     L.mq_get_error.argtypes = [vp]
     L.mq_status_string.argtypes = [i32]
     L.mq_status_string.restype = ctypes.c_char_p
@@ -204,6 +209,15 @@ def mq_run_layer(W, X, Xcal, Y, M: int, N: int, K: int, T: int, budget: int, fla
         return _ptr(t)
     _check(lib().mq_run_layer(p(W), p(X), p(Xcal), p(Y), M, N, K, T, budget, flags, 1 if host else 0,
                               ctypes.byref(buf), _stream(stream)), "mq_run_layer")
+
+
+def mq_gemm_noalloc(xq: dict, wq: dict, packed: dict | None, Y: torch.Tensor, M: int, N: int, K: int,
+                    flags: int = 0, stream=None):
+    """mq_gemm for callers that cannot allocate device memory: no workspace argument,
+    the split-K scratch is a static buffer inside the library (see include/mosaic.h)."""
+    ps = packed_struct(packed)
+    _check(lib().mq_gemm_noalloc(ctypes.byref(mat(xq)), ctypes.byref(mat(wq)), None if ps is None else ctypes.byref(ps),
+                                 _ptr(Y), M, N, K, flags, _stream(stream)), "mq_gemm_noalloc")
 
 
 def mq_get_error(stream=None) -> int:

@@ -230,6 +230,28 @@ typedef struct {
 mq_status mq_run_layer(const mq_bf16* W, const mq_bf16* X, const mq_bf16* Xcal, mq_bf16* Y, int M, int N, int K,
                        int T, int budget, unsigned flags, int host, mq_layer_buffers* buf, mq_stream stream);
 
+/*
+ * mq_gemm without a workspace argument, for callers that cannot allocate device memory
+ * (for example code embedded in a framework that owns all device memory and offers no
+ * workspace hook, or paths where an allocation is not allowed). The paper has no
+ * counterpart to this call; it exists for such integrations.
+ * Same arguments, checks and results as mq_gemm, minus ws/ws_bytes. The split-K scratch
+ * is a static array inside the library, mq_gemm_noalloc_scratch_limit() bytes (8 MiB)
+ * on every GPU that loads the library, held until the process exits. A problem whose
+ * mq_gemm_workspace_bytes() exceeds that limit is rejected with MQ_ERR_WORKSPACE (use
+ * mq_gemm with a workspace instead). The first call on each device looks up the
+ * array's device address (set-up, once per device, with that device current); make
+ * that first call before any stream capture. Each call clears the scratch's tile
+ * counters on `stream` before its kernel. All calls share the one array, which keeps
+ * the last call's contents: calls that overlap on the GPU race and must be serialized
+ * by the caller. Allocates nothing (no cudaMalloc/cudaFree).
+ */
+mq_status mq_gemm_noalloc(const mq_nvfp4_mat* xq, const mq_nvfp4_mat* wq, const mq_residual_packed* r, mq_bf16* Y,
+                          int M, int N, int K, unsigned flags, mq_stream stream);
+
+/* Size in bytes of mq_gemm_noalloc's static scratch array. */
+size_t mq_gemm_noalloc_scratch_limit(void);
+
 /* Synchronizes `stream`, then returns (and clears) the device error word: MQ_OK, or
  * MQ_ERR_TIMEOUT if a kernel gave up on a pipeline wait, or MQ_ERR_CUDA if the
  * synchronization itself failed. */
