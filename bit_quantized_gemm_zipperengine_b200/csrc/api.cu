@@ -18,6 +18,9 @@ cudaError_t launch_quant_act(const uint16_t* X, int M, int K, uint8_t* codes, ui
 cudaError_t launch_hessian(const uint16_t* X, int T, int K, float* H, cudaStream_t s);
 cudaError_t launch_delta(const uint16_t* W, int N, int K, const float* H, const float* g, double* delta,
                          cudaStream_t s);
+cudaError_t launch_quant_delta(const uint16_t* W, int N, int K, const float* H, uint8_t* codes, uint8_t* sf,
+                               uint8_t* sf_swz, float* g, uint8_t* rcodes, uint8_t* rsf, double* delta,
+                               float* partial, cudaStream_t s);
 cudaError_t launch_topk(const double* delta, int B, int budget, int32_t* rank, int32_t* sel, cudaStream_t s);
 cudaError_t launch_pack(const uint8_t* rcodes, const uint8_t* rsf, int N, int K, const int32_t* sel, int budget,
                         uint8_t* blk_codes, uint8_t* blk_sf, int32_t* blk_kt, int32_t* tile_ptr, uint32_t* bitmap,
@@ -142,7 +145,31 @@ mq_status mq_delta_score_topk(const mq_bf16* W, const float* H, const mq_nvfp4_m
     cudaError_t e = launch_delta(W, N, K, H, base->gscale, delta, s);
     if (e != cudaSuccess) return MQ_ERR_CUDA;
     g_launches.fetch_add(1);
-    return launched(launch_topk(delta, B, budget, rank, sel, s), budget > 0 ? 2 : 0);
+    return launched(launch_topk(delta, B, budget, rank, sel, s), budget <= 0 ? 0 : budget <= 1024 ? 1 : 2);
+}
+
+mq_status mq_quantize_weight_delta(const mq_bf16* W, int N, int K, const float* H, mq_nvfp4_mat* base,
+                                   mq_nvfp4_mat* resid_full, double* delta, void* ws, size_t ws_bytes,
+                                   mq_stream stream) {
+    if (!W || !H || !delta || !base || !resid_full || !nvfp4_shape_ok(N, K) || N % 64) return MQ_ERR_INVALID_ARG;
+    if (!base->codes || !base->sf_swz || !base->gscale || !resid_full->codes || !resid_full->sf)
+        return MQ_ERR_INVALID_ARG;
+    if (base->rows != N || base->cols != K || resid_full->rows != N || resid_full->cols != K)
+        return MQ_ERR_INVALID_ARG;
+    if (!aligned(W, 16) || !aligned(base->codes, 8) || !aligned(resid_full->codes, 8) || !aligned(base->sf_swz, 4) ||
+        !aligned(resid_full->sf, 4) || (base->sf && !aligned(base->sf, 4)))
+        return MQ_ERR_INVALID_ARG;
+    if (!ws || ws_bytes < mq_quantize_weight_workspace_bytes(N, K)) return MQ_ERR_WORKSPACE;
+    cudaError_t e = launch_quant_delta(W, N, K, H, base->codes, base->sf, base->sf_swz, base->gscale, resid_full->codes,
+                                       resid_full->sf, delta, static_cast<float*>(ws), as_stream(stream));
+    return launched(e, 2);
+}
+
+mq_status mq_topk_blocks(const double* delta, int nblk, int budget, int32_t* rank, int32_t* sel, mq_stream stream) {
+    if (!delta || nblk <= 0 || budget < 0 || budget > nblk) return MQ_ERR_INVALID_ARG;
+    if (budget > 0 && (!rank || !sel)) return MQ_ERR_INVALID_ARG;
+    const int kernels = budget <= 0 ? 0 : budget <= 1024 ? 1 : 2;
+    return launched(launch_topk(delta, nblk, budget, rank, sel, as_stream(stream)), kernels);
 }
 
 mq_status mq_pack_residual(const mq_nvfp4_mat* resid_full, const int32_t* sel, int budget, mq_residual_packed* out,
@@ -210,7 +237,7 @@ mq_status mq_gemm(const mq_nvfp4_mat* xq, const mq_nvfp4_mat* wq, const mq_resid
     p.K = K;
     p.mode = (flags & MQ_GEMM_BASE_ONLY) ? 1 : (flags & MQ_GEMM_RESIDUAL_ONLY) ? 2 : 0;
     if (need > 0) {
-        size_t part = (size_t)d.splits * d.tiles_m * d.BN * N * sizeof(float);
+        size_t part = (size_t)d.splits * d.tiles_m * d.BN * N * sizeof(float);  // workspace path only
         part = (part + 255) & ~size_t(255);
         p.partial = static_cast<float*>(ws);
         p.counters = reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + part);
@@ -236,12 +263,11 @@ mq_status mq_run_layer(const mq_bf16* W, const mq_bf16* X, const mq_bf16* Xcal, 
         y = buf->Y_dev;
     }
     mq_status st;
-    if ((st = mq_quantize_weight(w, N, K, &buf->base, &buf->resid_full, buf->ws_quant, buf->ws_quant_bytes,
-                                 stream)) != MQ_OK)
-        return st;
     if ((st = mq_hessian_diag(xc, T, K, buf->H, stream)) != MQ_OK) return st;
-    if ((st = mq_delta_score_topk(w, buf->H, &buf->base, &buf->resid_full, budget, buf->delta, buf->rank, buf->sel,
-                                  NULL, 0, stream)) != MQ_OK)
+    if ((st = mq_quantize_weight_delta(w, N, K, buf->H, &buf->base, &buf->resid_full, buf->delta, buf->ws_quant,
+                                       buf->ws_quant_bytes, stream)) != MQ_OK)
+        return st;
+    if ((st = mq_topk_blocks(buf->delta, (N / 64) * (K / 64), budget, buf->rank, buf->sel, stream)) != MQ_OK)
         return st;
     if ((st = mq_pack_residual(&buf->resid_full, buf->sel, budget, &buf->packed, stream)) != MQ_OK) return st;
     if ((st = mq_quantize_act(x, M, K, &buf->xq, stream)) != MQ_OK) return st;

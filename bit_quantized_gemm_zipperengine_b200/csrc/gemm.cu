@@ -10,9 +10,16 @@
 // chunks, and every selected residual block of the tile's two 64-row block rows.
 // The MMA thread issues 4 base MMAs (K = 64 each) and one more MMA per selected
 // residual block into the SAME fp32 accumulator: the residual block's rows fill one
-// half of a 128-row operand whose other half carries zero scales. Split-K partials
-// are added in a fixed order by the last CTA of each tile (a tile counter in the
-// workspace), then scaled by g_x[m] * g_w and stored as bf16.
+// half of a 128-row operand whose other half carries zero scales.
+// Split-K: the K splits of a tile run as one thread-block cluster; each CTA leaves its
+// fp32 partial in its own shared memory and, after a cluster barrier, reduces a slice of
+// the tile's rows by reading its peers' partials (distributed shared memory) in split
+// order, then scales by g_x[m] * g_w and stores bf16. Above 8 splits (narrow layers) the
+// partials go through a global workspace instead, added in the same order by the last
+// CTA of the tile (a tile counter).
+// The kernel is launched with programmatic dependent launch: its prologue and the W,
+// W-scale and residual loads (written by earlier kernels) overlap the preceding kernel;
+// it waits for that kernel before loading X and its scales.
 #include <cuda_bf16.h>
 
 #include "common.cuh"
@@ -47,6 +54,9 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
     }
 }
 
+constexpr int kMaxSplits = 16;        // split-K factor bound of the decode plan
+constexpr int kMaxClusterSplits = 8;  // splits reduced through a thread-block cluster
+
 template <int BN>
 struct DecodeCfg {
     static constexpr int kStages = BN >= 128 ? 3 : 4;
@@ -57,7 +67,7 @@ struct DecodeCfg {
     static constexpr int kOffRC = kOffSFX + 2048;        // 4 x (128 rows x 32 B), no swizzle
     static constexpr int kOffRSF = kOffRC + 16384;       // 8 x 512 B
     static constexpr int kStageBytes = kOffRSF + 4096;
-    static constexpr int kCtrlBytes = 256;
+    static constexpr int kCtrlBytes = 256;  // 3 barriers per stage, accumulator barrier, TMEM address, masks
     static constexpr int kSmemBytes = kStages * kStageBytes + kCtrlBytes + 1024;
     static constexpr int kThreads = 192;
     static constexpr uint32_t kTmemCols = 512;
@@ -66,23 +76,41 @@ struct DecodeCfg {
     static_assert(kSmemBytes <= 232448, "shared memory budget");
 };
 
-// Residual blocks of block row nt among block columns [kt0, kt0 + 4): returns a 4-bit
-// presence mask and fills idx[kk] with the packed index of block (nt, kt0 + kk).
-__device__ __forceinline__ uint32_t resid_lookup(const GemmParams& p, int nt, int kt0, int (&idx)[4]) {
-    const int KB = p.K / 64, KW = (KB + 31) / 32;
-    const uint32_t* row = p.bitmap + (int64_t)nt * KW;
-    const int w = kt0 >> 5, sh = kt0 & 31;  // kt0 % 4 == 0, so the 4 bits share a word
-    const uint32_t word = __ldg(row + w);
-    const uint32_t m = (word >> sh) & 15u;
-    if (m) {
-        int base = __ldg(p.tile_ptr + nt);
-        for (int j = 0; j < w; ++j) base += __popc(__ldg(row + j));
-        base += __popc(sh ? (word & ((1u << sh) - 1u)) : 0u);
+// Walks the selected blocks of one block row in increasing block-column order: the
+// packed index of the next selected block and the bitmap word being read.
+struct RowCursor {
+    const uint32_t* words;
+    int idx;   // packed index of the first selected block at or after the cursor
+    int w;     // index of the bitmap word held in `word`
+    uint32_t word;
+};
+
+// Cursor at block column kt_begin (a multiple of 4) of block row nt.
+__device__ __forceinline__ RowCursor row_cursor(const GemmParams& p, int nt, int kt_begin) {
+    const int KW = (p.K / 64 + 31) / 32;
+    RowCursor c;
+    c.words = p.bitmap + (int64_t)nt * KW;
+    c.w = kt_begin >> 5;
+    c.word = __ldg(c.words + c.w);
+    int idx = __ldg(p.tile_ptr + nt);
+    for (int j = 0; j < c.w; ++j) idx += __popc(__ldg(c.words + j));
+    const int sh = kt_begin & 31;
+    c.idx = idx + __popc(sh ? (c.word & ((1u << sh) - 1u)) : 0u);
+    return c;
+}
+
+// Presence bits of block columns kt0..kt0+3 (kt0 % 4 == 0, increasing from call to
+// call) and the packed index of each present block.
+__device__ __forceinline__ uint32_t row_step(RowCursor& c, int kt0, int (&idx)[4]) {
+    if ((kt0 >> 5) != c.w) {
+        c.w = kt0 >> 5;
+        c.word = __ldg(c.words + c.w);
+    }
+    const uint32_t m = (c.word >> (kt0 & 31)) & 15u;
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-            idx[kk] = base;
-            base += (m >> kk) & 1u;
-        }
+    for (int kk = 0; kk < 4; ++kk) {
+        idx[kk] = c.idx;
+        c.idx += (m >> kk) & 1u;
     }
     return m;
 }
@@ -91,11 +119,12 @@ __device__ __forceinline__ bool tile_has_mma(const GemmParams& p, int n_tile, in
     if (ks_end <= ks_begin) return false;
     if (p.mode != 2) return true;
     if (!p.has_resid) return false;
-    for (int ks = ks_begin; ks < ks_end; ++ks)
-        for (int h = 0; h < 2; ++h) {
-            int idx[4];
-            if (resid_lookup(p, n_tile * 2 + h, ks * 4, idx)) return true;
-        }
+    const int KB = p.K / 64, KW = (KB + 31) / 32;
+    for (int h = 0; h < 2; ++h) {
+        const uint32_t* row = p.bitmap + (int64_t)(n_tile * 2 + h) * KW;
+        for (int kt = ks_begin * 4; kt < ks_end * 4; kt += 4)
+            if ((__ldg(row + (kt >> 5)) >> (kt & 31)) & 15u) return true;
+    }
     return false;
 }
 
@@ -106,9 +135,10 @@ __global__ void __launch_bounds__(192, 1)
     using C = DecodeCfg<BN>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kStages * C::kStageBytes);
-    uint64_t* empty = full + C::kStages;
-    uint64_t* accf = empty + C::kStages;
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kStages * C::kStageBytes);  // W, X and scales landed
+    uint64_t* rfull = full + C::kStages;                                                // residual blocks landed
+    uint64_t* empty = rfull + C::kStages;                                               // stage consumed
+    uint64_t* accf = empty + C::kStages;                                                // accumulator complete
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(accf + 1);
     uint32_t* rmask = tmem_holder + 1;  // [kStages]
 
@@ -123,6 +153,7 @@ __global__ void __launch_bounds__(192, 1)
     if (warp == 0 && lane == 0) {
         for (int s = 0; s < C::kStages; ++s) {
             mbar_init(&full[s], 1);
+            mbar_init(&rfull[s], 1);
             mbar_init(&empty[s], 1);
         }
         mbar_init(accf, 1);
@@ -144,41 +175,69 @@ __global__ void __launch_bounds__(192, 1)
             // ------------------------------------------------ producer
             const uint8_t* xsf_tile = p.x_sf + (int64_t)(m0 / 128) * KS64 * 512;
             const uint8_t* wsf_tile = p.w_sf + (int64_t)n_tile * KS64 * 512;
-            int issued = 0;
-            for (int it = 0; it < n_iters; ++it) {
-                const int s = it % C::kStages;
-                const uint32_t use = it / C::kStages;
-                if (it >= C::kStages && !mbar_wait(&empty[s], (use - 1) & 1)) break;
-                const int ks = ks_begin + it;
+            // W tile and W scales: written by earlier kernels, loaded before the wait
+            auto issue_w = [&](int it) {
+                const int st_i = it % C::kStages, ks = ks_begin + it;
+                uint8_t* st = smem + st_i * C::kStageBytes;
+                mbar_arrive_expect_tx(&full[st_i], 16384 + BN * 128 + 2048 + 2048);
+                tma_load_2d(st + C::kOffW, &tmap_w, &full[st_i], ks * 128, n0);
+                bulk_load(st + C::kOffSFW, wsf_tile + (int64_t)ks * 4 * 512, 2048, &full[st_i]);
+            };
+            // X tile and X scales: written by the previous kernel
+            auto issue_x = [&](int it) {
+                const int st_i = it % C::kStages, ks = ks_begin + it;
+                uint8_t* st = smem + st_i * C::kStageBytes;
+                tma_load_2d(st + C::kOffX, &tmap_x, &full[st_i], ks * 128, m0);
+                bulk_load(st + C::kOffSFX, xsf_tile + (int64_t)ks * 4 * 512, 2048, &full[st_i]);
+            };
+            RowCursor cur0, cur1;
+            auto issue_resid = [&](int it) {
+                const int s = it % C::kStages, ks = ks_begin + it;
+                uint8_t* st = smem + s * C::kStageBytes;
                 uint32_t m = 0;
                 int idx0[4] = {0, 0, 0, 0}, idx1[4] = {0, 0, 0, 0};
                 if (p.has_resid) {
-                    const uint32_t m0b = resid_lookup(p, n_tile * 2 + 0, ks * 4, idx0);
-                    const uint32_t m1b = resid_lookup(p, n_tile * 2 + 1, ks * 4, idx1);
+                    const uint32_t m0b = row_step(cur0, ks * 4, idx0);
+                    const uint32_t m1b = row_step(cur1, ks * 4, idx1);
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk) m |= (((m0b >> kk) & 1u) << (2 * kk)) | (((m1b >> kk) & 1u) << (2 * kk + 1));
+                    for (int kk = 0; kk < 4; ++kk)
+                        m |= (((m0b >> kk) & 1u) << (2 * kk)) | (((m1b >> kk) & 1u) << (2 * kk + 1));
                 }
                 rmask[s] = m;
-                uint8_t* st = smem + s * C::kStageBytes;
-                const uint32_t bytes = 16384 + BN * 128 + 2048 + 2048 + __popc(m) * (2048 + 512);
-                mbar_arrive_expect_tx(&full[s], bytes);
-                tma_load_2d(st + C::kOffW, &tmap_w, &full[s], ks * 128, n0);
-                tma_load_2d(st + C::kOffX, &tmap_x, &full[s], ks * 128, m0);
-                bulk_load(st + C::kOffSFW, wsf_tile + (int64_t)ks * 4 * 512, 2048, &full[s]);
-                bulk_load(st + C::kOffSFX, xsf_tile + (int64_t)ks * 4 * 512, 2048, &full[s]);
+                mbar_arrive_expect_tx(&rfull[s], __popc(m) * (2048 + 512));
 #pragma unroll 1
                 for (int j = 0; j < 8; ++j) {
                     if (!((m >> j) & 1u)) continue;
                     const int kk = j >> 1, h = j & 1;
                     const int idx = h ? idx1[kk] : idx0[kk];
-                    bulk_load(st + C::kOffRC + kk * 4096 + h * 2048, p.blk_codes + (int64_t)idx * 2048, 2048, &full[s]);
-                    bulk_load(st + C::kOffRSF + j * 512, p.blk_sf + (int64_t)idx * 512, 512, &full[s]);
+                    bulk_load(st + C::kOffRC + kk * 4096 + h * 2048, p.blk_codes + (int64_t)idx * 2048, 2048,
+                              &rfull[s]);
+                    bulk_load(st + C::kOffRSF + j * 512, p.blk_sf + (int64_t)idx * 512, 512, &rfull[s]);
                 }
+            };
+            const int first = min(C::kStages, n_iters);
+            for (int it = 0; it < first; ++it) issue_w(it);  // nothing to wait for yet
+            if (p.has_resid && n_iters > 0) {
+                cur0 = row_cursor(p, n_tile * 2 + 0, ks_begin * 4);
+                cur1 = row_cursor(p, n_tile * 2 + 1, ks_begin * 4);
+            }
+            for (int it = 0; it < first; ++it) issue_resid(it);
+            griddep_wait();
+            for (int it = 0; it < first; ++it) issue_x(it);
+            int issued = first;
+            for (int it = first; it < n_iters; ++it) {
+                const int st_i = it % C::kStages;
+                if (!mbar_wait(&empty[st_i], ((it / C::kStages) - 1) & 1)) break;
+                issue_w(it);
+                issue_x(it);
+                issue_resid(it);
                 ++issued;
             }
             // Do not leave while copies into this CTA's shared memory are in flight.
-            for (int it = max(0, issued - C::kStages); it < issued; ++it)
+            for (int it = max(0, issued - C::kStages); it < issued; ++it) {
                 mbar_wait(&full[it % C::kStages], (it / C::kStages) & 1);
+                mbar_wait(&rfull[it % C::kStages], (it / C::kStages) & 1);
+            }
         }
     } else if (warp == 1) {
         if (lane == 0) {
@@ -187,40 +246,37 @@ __global__ void __launch_bounds__(192, 1)
             uint32_t acc = 0;
             for (int it = 0; it < n_iters; ++it) {
                 const int s = it % C::kStages;
-                const uint32_t use = it / C::kStages;
-                if (!mbar_wait(&full[s], use & 1)) break;
+                const uint32_t par = (it / C::kStages) & 1;
+                if (!mbar_wait(&full[s], par)) break;
                 tc_fence_after();
                 uint8_t* st = smem + s * C::kStageBytes;
                 const uint32_t sfc = tmem + C::kSfCol0 + s * 64;
-                const uint32_t m = rmask[s];
+                const uint32_t aw = smem_u32(st + C::kOffW), bx = smem_u32(st + C::kOffX);
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) {
                     tc_cp_sf_chunk(sfc + 4 * kk, smem_desc(smem_u32(st + C::kOffSFW + kk * 512), 0, 128, 0));
                     tc_cp_sf_chunk(sfc + 16 + 4 * kk, smem_desc(smem_u32(st + C::kOffSFX + kk * 512), 0, 128, 0));
                 }
-#pragma unroll 1
-                for (int j = 0; j < 8; ++j)
-                    if ((m >> j) & 1u)
-                        tc_cp_sf_chunk(sfc + 32 + 4 * j, smem_desc(smem_u32(st + C::kOffRSF + j * 512), 0, 128, 0));
-                const uint32_t aw = smem_u32(st + C::kOffW), bx = smem_u32(st + C::kOffX);
+                if (p.mode != 2) {
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-                    const uint64_t bdesc = smem_desc(bx + 32 * kk, 16, 1024, 2);
-                    if (p.mode != 2) {
-                        mma_mxf4nvf4(tmem, smem_desc(aw + 32 * kk, 16, 1024, 2), bdesc, idesc, sfc + 4 * kk,
-                                     sfc + 16 + 4 * kk, acc);
+                    for (int kk = 0; kk < 4; ++kk) {
+                        mma_mxf4nvf4(tmem, smem_desc(aw + 32 * kk, 16, 1024, 2), smem_desc(bx + 32 * kk, 16, 1024, 2),
+                                     idesc, sfc + 4 * kk, sfc + 16 + 4 * kk, acc);
                         acc = 1;
                     }
-                    if (p.mode != 1) {
-#pragma unroll
-                        for (int h = 0; h < 2; ++h) {
-                            const int j = 2 * kk + h;
-                            if (!((m >> j) & 1u)) continue;
-                            const uint64_t adesc = smem_desc(smem_u32(st + C::kOffRC + kk * 4096), 128, 256, 0);
-                            mma_mxf4nvf4(tmem, adesc, bdesc, idesc, sfc + 32 + 4 * j, sfc + 16 + 4 * kk, acc);
-                            acc = 1;
-                        }
-                    }
+                }
+                if (!mbar_wait(&rfull[s], par)) break;
+                tc_fence_after();
+                const uint32_t m = p.mode != 1 ? rmask[s] : 0u;
+#pragma unroll 1
+                for (int j = 0; j < 8; ++j) {
+                    if (!((m >> j) & 1u)) continue;
+                    const int kk = j >> 1;
+                    tc_cp_sf_chunk(sfc + 32 + 4 * j, smem_desc(smem_u32(st + C::kOffRSF + j * 512), 0, 128, 0));
+                    mma_mxf4nvf4(tmem, smem_desc(smem_u32(st + C::kOffRC + kk * 4096), 128, 256, 0),
+                                 smem_desc(bx + 32 * kk, 16, 1024, 2), idesc, sfc + 32 + 4 * j, sfc + 16 + 4 * kk,
+                                 acc);
+                    acc = 1;
                 }
                 tc_commit(&empty[s]);
             }
@@ -229,34 +285,44 @@ __global__ void __launch_bounds__(192, 1)
     } else {
         // ---------------------------------------------------- epilogue (warps 2..5)
         const int q = warp & 3;
-        const int n = n0 + 32 * q + lane;
-        float acc[BN];
+        const int nl = 32 * q + lane, n = n0 + nl;
+        griddep_wait();  // g_x, Y and the workspace follow the previous kernel
         const bool waited = mbar_wait(accf, 0);
         tc_fence_after();
-        if (waited && tile_has_mma(p, n_tile, ks_begin, ks_end)) {
+        const bool have = waited && tile_has_mma(p, n_tile, ks_begin, ks_end);
+        const float gw = __ldg(p.g_w);
+        const int Mp = gridDim.z * BN;
+        float* red = reinterpret_cast<float*>(smem);  // [BN][128] partial (stages are free now)
+#pragma unroll 1
+        for (int c0 = 0; c0 < BN; c0 += 16) {
+            float acc[16];
+            if (have) {
+                tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + c0, acc);
+            } else {
 #pragma unroll
-            for (int c = 0; c < BN / 16; ++c) tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + 16 * c, acc + 16 * c);
-        } else {
+                for (int j = 0; j < 16; ++j) acc[j] = 0.0f;
+            }
+            if (p.splits == 1) {
 #pragma unroll
-            for (int j = 0; j < BN; ++j) acc[j] = 0.0f;
+                for (int j = 0; j < 16; ++j) {
+                    const int mm = m0 + c0 + j;
+                    if (mm < p.M) {
+                        const float sc = __fmul_rn(__ldg(p.g_x + mm), gw);
+                        const __nv_bfloat16 y = __float2bfloat16_rn(__fmul_rn(acc[j], sc));
+                        p.Y[(int64_t)mm * p.N + n] = *reinterpret_cast<const uint16_t*>(&y);
+                    }
+                }
+            } else if (p.cluster) {
+#pragma unroll
+                for (int j = 0; j < 16; ++j) red[(c0 + j) * 128 + nl] = acc[j];
+            } else {
+                float* part = p.partial + ((int64_t)split * Mp + m0) * p.N + n;
+#pragma unroll
+                for (int j = 0; j < 16; ++j) __stcg(part + (int64_t)(c0 + j) * p.N, acc[j]);
+            }
         }
         tc_fence_before();
-        const float gw = __ldg(p.g_w);
-        if (p.splits == 1) {
-#pragma unroll
-            for (int j = 0; j < BN; ++j) {
-                const int mm = m0 + j;
-                if (mm < p.M) {
-                    const float sc = __fmul_rn(__ldg(p.g_x + mm), gw);
-                    const __nv_bfloat16 y = __float2bfloat16_rn(__fmul_rn(acc[j], sc));
-                    p.Y[(int64_t)mm * p.N + n] = *reinterpret_cast<const uint16_t*>(&y);
-                }
-            }
-        } else {
-            const int Mp = gridDim.z * BN;
-            float* part = p.partial + ((int64_t)split * Mp + m0) * p.N + n;
-#pragma unroll
-            for (int j = 0; j < BN; ++j) __stcg(part + (int64_t)j * p.N, acc[j]);
+        if (p.splits > 1 && !p.cluster) {
             __threadfence();
             asm volatile("bar.sync 1, 128;" ::: "memory");
             __shared__ int s_last;
@@ -265,21 +331,61 @@ __global__ void __launch_bounds__(192, 1)
             asm volatile("bar.sync 1, 128;" ::: "memory");
             if (s_last) {
                 __threadfence();
+                // the last CTA of the tile adds all splits' partials in split order
                 const float* base = p.partial + (int64_t)m0 * p.N + n;
+                const int64_t sstride = (int64_t)Mp * p.N;
 #pragma unroll 1
-                for (int j = 0; j < BN; ++j) {
-                    const int mm = m0 + j;
-                    if (mm >= p.M) break;
-                    float sum = __ldcg(base + (int64_t)j * p.N);
-                    for (int s2 = 1; s2 < p.splits; ++s2)
-                        sum = __fadd_rn(sum, __ldcg(base + ((int64_t)s2 * Mp + j) * p.N));
-                    const float sc = __fmul_rn(__ldg(p.g_x + mm), gw);
-                    const __nv_bfloat16 y = __float2bfloat16_rn(__fmul_rn(sum, sc));
-                    p.Y[(int64_t)mm * p.N + n] = *reinterpret_cast<const uint16_t*>(&y);
+                for (int c0 = 0; c0 < BN && m0 + c0 < p.M; c0 += 8) {
+                    float sum[8];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) sum[j] = __ldcg(base + (int64_t)(c0 + j) * p.N);
+#pragma unroll 4
+                    for (int s2 = 1; s2 < p.splits; ++s2) {
+                        float v[8];
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) v[j] = __ldcg(base + s2 * sstride + (int64_t)(c0 + j) * p.N);
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) sum[j] = __fadd_rn(sum[j], v[j]);
+                    }
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const int mm = m0 + c0 + j;
+                        if (mm < p.M) {
+                            const float sc = __fmul_rn(__ldg(p.g_x + mm), gw);
+                            const __nv_bfloat16 y = __float2bfloat16_rn(__fmul_rn(sum[j], sc));
+                            p.Y[(int64_t)mm * p.N + n] = *reinterpret_cast<const uint16_t*>(&y);
+                        }
+                    }
                 }
                 if (threadIdx.x == 64) *ctr = 0;
             }
         }
+    }
+    griddep_launch();
+    if (p.splits > 1 && p.cluster) {
+        // every CTA of the cluster holds its partial in shared memory; CTA r adds rows
+        // [r*128/S, (r+1)*128/S) of all splits in split order
+        __syncwarp();
+        cluster_sync();
+        if (warp >= 2) {
+            const uint32_t S = (uint32_t)p.splits, r = cluster_ctarank();
+            const int r0 = (int)(r * 128 / S), r1 = (int)((r + 1) * 128 / S), rows = r1 - r0;
+            const float* red = reinterpret_cast<const float*>(smem);
+            const float gw = __ldg(p.g_w);
+            for (int e = threadIdx.x - 64; e < rows * BN; e += 128) {
+                const int j = e / rows, nl = r0 + e % rows;
+                const int mm = m0 + j;
+                float sum = ld_dsmem_f32(red + j * 128 + nl, 0);
+                for (uint32_t s2 = 1; s2 < S; ++s2) sum = __fadd_rn(sum, ld_dsmem_f32(red + j * 128 + nl, s2));
+                if (mm < p.M) {
+                    const float sc = __fmul_rn(__ldg(p.g_x + mm), gw);
+                    const __nv_bfloat16 y = __float2bfloat16_rn(__fmul_rn(sum, sc));
+                    p.Y[(int64_t)mm * p.N + n0 + nl] = *reinterpret_cast<const uint16_t*>(&y);
+                }
+            }
+        }
+        __syncwarp();
+        cluster_sync();  // peers may still be reading this CTA's partial until here
     }
     __syncthreads();
     if (warp == 1) {
@@ -298,15 +404,17 @@ DecodePlan plan_decode(int M, int N, int K) {
     const int tiles = d.tiles_m * d.tiles_n;
     int s = 148 / tiles;
     if (s < 1) s = 1;
+    if (s > kMaxSplits) s = kMaxSplits;
     if (s > KS) s = KS;
     d.iters = (KS + s - 1) / s;
     d.splits = (KS + d.iters - 1) / d.iters;
+    d.cluster = d.splits > 1 && d.splits <= kMaxClusterSplits;
     return d;
 }
 
 size_t decode_workspace_bytes(int M, int N, int K) {
     DecodePlan d = plan_decode(M, N, K);
-    if (d.splits <= 1) return 0;
+    if (d.splits <= 1 || d.cluster) return 0;
     size_t part = (size_t)d.splits * d.tiles_m * d.BN * N * sizeof(float);
     part = (part + 255) & ~size_t(255);
     return part + (size_t)d.tiles_m * d.tiles_n * sizeof(int);
@@ -324,14 +432,15 @@ static cudaError_t launch_decode_bn(const CUtensorMap& tw, const CUtensorMap& tx
         attr_set = true;
     }
     dim3 grid(d.tiles_n, d.splits, d.tiles_m);
-    k_gemm_decode<BN><<<grid, C::kThreads, C::kSmemBytes, s>>>(tw, tx, p);
-    return cudaGetLastError();
+    return launch_pdl(k_gemm_decode<BN>, grid, dim3(C::kThreads), C::kSmemBytes, s, d.cluster ? d.splits : 1, tw, tx,
+                      p);
 }
 
 cudaError_t launch_gemm_decode(const CUtensorMap& tw, const CUtensorMap& tx, GemmParams p, const DecodePlan& d,
                                cudaStream_t s) {
     p.splits = d.splits;
     p.iters_per_split = d.iters;
+    p.cluster = d.cluster ? 1 : 0;
     switch (d.BN) {
         case 16: return launch_decode_bn<16>(tw, tx, p, d, s);
         case 32: return launch_decode_bn<32>(tw, tx, p, d, s);

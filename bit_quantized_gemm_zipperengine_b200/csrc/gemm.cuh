@@ -24,12 +24,14 @@ struct GemmParams {
     int splits, iters_per_split;
     int mode;                // 0 fused, 1 base only, 2 residual only
     int has_resid;
+    int cluster;             // split-K reduced through the cluster's shared memory
 };
 
 // Decode kernel tiling: token tile BN, grid tiles_n x splits x tiles_m, `iters`
 // K stages (256 elements each) per split.
 struct DecodePlan {
     int BN, tiles_m, tiles_n, splits, iters;
+    bool cluster;  // splits reduced in a (1, splits, 1) cluster, no workspace
 };
 
 DecodePlan plan_decode(int M, int N, int K);

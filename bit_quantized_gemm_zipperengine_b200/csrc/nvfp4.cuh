@@ -1,30 +1,15 @@
-// NVFP4 arithmetic on the GPU: E2M1 / E4M3 encoders written from the bit layouts and
-// the per-group quantization rule, in fp32 IEEE operations with explicit rounding
-// intrinsics so that no multiply-add is contracted (codes and scales must match the
-// CPU oracle bit for bit).
+// NVFP4 arithmetic on the GPU: the per-group quantization rule in fp32 IEEE operations
+// with explicit rounding intrinsics (no multiply-add is contracted; codes and scales
+// must match the CPU oracle bit for bit), an E4M3 encoder written from the bit layout,
+// and the hardware E2M1 conversions.
 #pragma once
 
 #include <cstdint>
+#include <cuda_fp16.h>
 
 namespace mq {
 
 __device__ __forceinline__ float bf16_bits_to_f32(uint32_t h) { return __uint_as_float(h << 16); }
-
-// E2M1 code of v: round to nearest, ties to the even code, saturate at 6, keep the sign.
-// The magnitude code counts the grid midpoints below |v|; a midpoint itself goes to
-// the even neighbour, hence the alternating strict / non-strict comparisons.
-__device__ __forceinline__ uint32_t e2m1_encode(float v) {
-    const float a = fabsf(v);
-    uint32_t m = (a > 0.25f) + (a >= 0.75f) + (a > 1.25f) + (a >= 1.75f) + (a > 2.5f) + (a >= 3.5f) + (a > 5.0f);
-    return m | ((__float_as_uint(v) >> 28) & 8u);
-}
-
-// |value| of an E2M1 magnitude code (0..7): {0, 0.5, 1, 1.5, 2, 3, 4, 6}.
-__device__ __forceinline__ float e2m1_mag(uint32_t m) {
-    // exponent field e = m >> 1 (bias 1), mantissa bit m & 1; e = 0 is subnormal (m * 0.5)
-    const uint32_t e = m >> 1, f = m & 1u;
-    return e == 0 ? 0.5f * (float)f : __uint_as_float(((e + 126u) << 23) | (f << 22));
-}
 
 // E4M3 (fn) encode of a non-negative finite fp32: round to nearest even, saturate to 448.
 __device__ __forceinline__ uint32_t e4m3_encode_nonneg(float s) {
@@ -48,10 +33,70 @@ __device__ __forceinline__ float e4m3_value(uint32_t c) {
     return e == 0 ? __fmul_rn((float)m, 0.001953125f) : __uint_as_float(((e + 120u) << 23) | (m << 20));
 }
 
+// Packed fp32 multiply (sm_100 mul.rn.f32x2): each lane is one IEEE fp32 multiply with
+// round-to-nearest-even, bit-identical to __fmul_rn (a product's sign, zeros included,
+// is the xor of the operands' signs). Packed add/sub/fma are not used: on B200,
+// sub.rn.f32x2 returned -0 for (-x) - (-x), where IEEE round-to-nearest gives +0, and
+// the sign of a zero residual is part of its code.
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
+    float2 d;
+    asm("{\n\t.reg .b64 a, b, d;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
+        "mul.rn.f32x2 d, a, b;\n\tmov.b64 {%0, %1}, d;\n\t}"
+        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+
+// Eight scaled values -> eight E2M1 codes packed in a word (element 0 in the low nibble
+// of byte 0). The E2M1 rule: round to nearest with ties to the even code, saturate at 6,
+// keep the sign (-0.1 -> 0x8). cvt.rn.satfinite.e2m1x2 implements exactly this rule:
+// it was compared on B200 with an encoder written from the format's bit layout over
+// every finite fp32 value, with no difference.
+__device__ __forceinline__ uint32_t e2m1x8(float q0, float q1, float q2, float q3, float q4, float q5, float q6,
+                                           float q7) {
+    uint32_t w;
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+        "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+        : "=r"(w)
+        : "f"(q0), "f"(q1), "f"(q2), "f"(q3), "f"(q4), "f"(q5), "f"(q6), "f"(q7));
+    return w;
+}
+
+// Signed E2M1 values of the eight codes of a word (exact in f16, widened to fp32).
+__device__ __forceinline__ void e2m1x8_values(uint32_t w, float* v) {
+    uint32_t h[4];
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+        : "=r"(h[0]), "=r"(h[1]), "=r"(h[2]), "=r"(h[3])
+        : "r"(w));
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const __half2 x = *reinterpret_cast<const __half2*>(&h[j]);
+        const float2 f = __half22float2(x);
+        v[2 * j] = f.x;
+        v[2 * j + 1] = f.y;
+    }
+}
+
+// Codes of 16 values that all round to a signed zero (the group scale is zero).
+__device__ __forceinline__ uint32_t sign_nibbles8(const float* a) {
+    uint32_t w = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) w |= ((__float_as_uint(a[i]) >> 28) & 8u) << (4 * i);
+    return w;
+}
+
 // One 16-element group with tensor scale g (g6 = fp32(6 g)):
-//   s = amax / g6; sf = E4M3(s); d = dec(sf) * g; code_i = E2M1(a_i / d) (signed zero if
-//   d == 0); deq_i = val(code_i) * d.
-// Returns the scale byte; packs codes (element 2j low nibble of byte j) into lo/hi words.
+//   s = amax / g6; sf = E4M3(s); d = dec(sf) * g; r = 1 / d;
+//   code_i = E2M1(a_i * r) (a signed zero if d == 0); deq_i = val(code_i) * d.
+// Returns the scale byte; codes (element 2j in the low nibble of byte j) in lo/hi.
 __device__ __forceinline__ uint32_t nvfp4_group(const float (&a)[16], float g, float g6, uint32_t& lo, uint32_t& hi,
                                                 float (&deq)[16]) {
     float amax = 0.0f;
@@ -60,18 +105,28 @@ __device__ __forceinline__ uint32_t nvfp4_group(const float (&a)[16], float g, f
     const float s = __fdiv_rn(amax, g6);
     const uint32_t sf = e4m3_encode_nonneg(s);
     const float d = __fmul_rn(e4m3_value(sf), g);
-    uint32_t w[2] = {0u, 0u};
+    if (d > 0.0f) {
+        const float r = __frcp_rn(d);
+        const float2 rr = make_float2(r, r);
+        float2 q[8];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-        uint32_t c;
-        if (d > 0.0f) c = e2m1_encode(__fdiv_rn(a[i], d));
-        else c = (__float_as_uint(a[i]) >> 28) & 8u;
-        const float mag = __fmul_rn(e2m1_mag(c & 7u), d);
-        deq[i] = (c & 8u) ? -mag : mag;
-        w[i >> 3] |= c << (4 * (i & 7));
+        for (int j = 0; j < 8; ++j) q[j] = mul2(make_float2(a[2 * j], a[2 * j + 1]), rr);
+        lo = e2m1x8(q[0].x, q[0].y, q[1].x, q[1].y, q[2].x, q[2].y, q[3].x, q[3].y);
+        hi = e2m1x8(q[4].x, q[4].y, q[5].x, q[5].y, q[6].x, q[6].y, q[7].x, q[7].y);
+    } else {
+        lo = sign_nibbles8(a);
+        hi = sign_nibbles8(a + 8);
     }
-    lo = w[0];
-    hi = w[1];
+    float v[16];
+    e2m1x8_values(lo, v);
+    e2m1x8_values(hi, v + 8);
+    const float2 dd = make_float2(d, d);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const float2 t = mul2(make_float2(v[2 * j], v[2 * j + 1]), dd);
+        deq[2 * j] = t.x;
+        deq[2 * j + 1] = t.y;
+    }
     return sf;
 }
 

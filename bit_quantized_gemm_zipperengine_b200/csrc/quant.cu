@@ -1,9 +1,10 @@
 // Weight and activation quantization to NVFP4 (the dense 4-bit base and the 4-bit
 // residual of MosaicQuant, summary "Methodology" section 1) and the diagonal Hessian
 // estimate (section 2). HBM-bound elementwise kernels: 16-byte vector loads, one
-// thread per 16-element group, warp-shuffle maxima.
+// thread per 16-element group, warp-shuffle maxima, hardware E2M1 conversions.
 #include "common.cuh"
 #include "nvfp4.cuh"
+#include "quant.cuh"
 
 namespace mq {
 
@@ -13,32 +14,36 @@ __device__ __forceinline__ float warp_max(float v) {
     return v;
 }
 
-__device__ __forceinline__ void load16_bf16(const uint16_t* p, float (&a)[16]) {
-    const uint4* q = reinterpret_cast<const uint4*>(p);
-    uint4 v0 = __ldg(q), v1 = __ldg(q + 1);
-    const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        a[2 * i] = bf16_bits_to_f32(w[i] & 0xFFFFu);
-        a[2 * i + 1] = bf16_bits_to_f32(w[i] >> 16);
-    }
-}
-
-// Per-CTA maxima of |W| over a grid-stride range of 8-element vectors.
-__global__ void __launch_bounds__(256) k_amax_partial(const uint16_t* __restrict__ W, int64_t n8,
+// Per-CTA maxima of |W| over a grid-stride range of 8-element vectors (kAmaxBlocks
+// CTAs, 4 independent 16-byte loads in flight per thread).
+__global__ void __launch_bounds__(512) k_amax_partial(const uint16_t* __restrict__ W, int64_t n8,
                                                       float* __restrict__ partial) {
+    griddep_wait();
+    griddep_launch();
     float m = 0.0f;
     const uint4* v = reinterpret_cast<const uint4*>(W);
-    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n8; i += (int64_t)gridDim.x * blockDim.x) {
-        uint4 x = __ldg(v + i);
-        const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+    for (; i + 3 * stride < n8; i += 4 * stride) {
+        uint4 x[4];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            m = fmaxf(m, fabsf(bf16_bits_to_f32(w[j] & 0xFFFFu)));
-            m = fmaxf(m, fabsf(bf16_bits_to_f32(w[j] >> 16)));
+        for (int u = 0; u < 4; ++u) x[u] = __ldg(v + i + u * stride);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const uint32_t w[4] = {x[u].x, x[u].y, x[u].z, x[u].w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) m = fmaxf(m, fmaxf(fabsf(bf16_bits_to_f32(w[j] & 0xFFFFu)),
+                                                           fabsf(bf16_bits_to_f32(w[j] >> 16))));
         }
     }
-    __shared__ float red[8];
+    for (; i < n8; i += stride) {
+        const uint4 x = __ldg(v + i);
+        const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            m = fmaxf(m, fmaxf(fabsf(bf16_bits_to_f32(w[j] & 0xFFFFu)), fabsf(bf16_bits_to_f32(w[j] >> 16))));
+    }
+    __shared__ float red[16];
     m = warp_max(m);
     if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
     __syncthreads();
@@ -47,19 +52,6 @@ __global__ void __launch_bounds__(256) k_amax_partial(const uint16_t* __restrict
         t = warp_max(t);
         if (threadIdx.x == 0) partial[blockIdx.x] = t;
     }
-}
-
-// Tensor scale from the partial maxima: g = amax / 2688, or 1 for an all-zero tensor.
-__device__ __forceinline__ float reduce_scale(const float* partial, int P) {
-    __shared__ float s_g;
-    if (threadIdx.x < 32) {
-        float m = 0.0f;
-        for (int i = threadIdx.x; i < P; i += 32) m = fmaxf(m, partial[i]);
-        m = warp_max(m);
-        if (threadIdx.x == 0) s_g = (m == 0.0f) ? 1.0f : __fdiv_rn(m, 2688.0f);
-    }
-    __syncthreads();
-    return s_g;
 }
 
 // Gathers the scale bytes of 4 consecutive groups (lanes l..l+3, l % 4 == 0) into one
@@ -72,14 +64,16 @@ __device__ __forceinline__ uint32_t gather4(uint32_t b) {
 }
 
 // A1: base NVFP4(W, g) and residual NVFP4(W - deq Q(W), g) for every group.
-// One thread per group; the group count is a multiple of 32 (K % 64 == 0 gives
-// K/16 % 4 == 0 and N*K/16 % 32 == 0 needs N % 8 == 0, true for N % 64 == 0).
+// One thread per group; the group count is a multiple of 32 (K % 64 == 0 and
+// N % 64 == 0), so whole warps stay together for the 4-group scale gather.
 __global__ void __launch_bounds__(256) k_quant_weight(const uint16_t* __restrict__ W, int N, int K,
-                                                      const float* __restrict__ partial, int P,
+                                                      const float* __restrict__ partial,
                                                       uint8_t* __restrict__ codes, uint8_t* __restrict__ sf,
                                                       uint8_t* __restrict__ sf_swz, float* __restrict__ g_out,
                                                       uint8_t* __restrict__ rcodes, uint8_t* __restrict__ rsf) {
-    const float g = reduce_scale(partial, P);
+    griddep_wait();
+    griddep_launch();
+    const float g = tensor_scale(partial);
     if (blockIdx.x == 0 && threadIdx.x == 0) *g_out = g;
     const float g6 = __fmul_rn(6.0f, g);
     const int G = K / 16;
@@ -113,48 +107,59 @@ __global__ void __launch_bounds__(256) k_quant_weight(const uint16_t* __restrict
     }
 }
 
-// A6: one CTA per (padded) token row. Rows >= M only clear their tiled scales.
-__global__ void __launch_bounds__(128) k_quant_act(const uint16_t* __restrict__ X, int M, int K,
-                                                   uint8_t* __restrict__ codes, uint8_t* __restrict__ sf,
-                                                   uint8_t* __restrict__ sf_swz, float* __restrict__ g_x) {
+// A6: one CTA per (padded) token row, every group held in registers (kGPT groups per
+// thread, groups tid + j * blockDim), so the row is read once. Rows >= M only clear
+// their tiled scales.
+template <int kGPT>
+__global__ void __launch_bounds__(1024) k_quant_act(const uint16_t* __restrict__ X, int M, int K,
+                                                    uint8_t* __restrict__ codes, uint8_t* __restrict__ sf,
+                                                    uint8_t* __restrict__ sf_swz, float* __restrict__ g_x) {
+    griddep_wait();
+    griddep_launch();
     const int m = blockIdx.x;
     const int G = K / 16;
-    const int lane = threadIdx.x & 31;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     if (m >= M) {
         for (int q = threadIdx.x * 4; q < G; q += blockDim.x * 4)
             *reinterpret_cast<uint32_t*>(sf_swz + sf_swz_offset(m, q, K)) = 0u;
         return;
     }
     const uint16_t* row = X + (int64_t)m * K;
+    float a[kGPT][16];
     float amax = 0.0f;
-    for (int q = threadIdx.x; q < G; q += blockDim.x) {
-        float a[16];
-        load16_bf16(row + q * 16, a);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(a[i]));
+    for (int j = 0; j < kGPT; ++j) {
+        const int q = threadIdx.x + j * blockDim.x;
+        if (q < G) {
+            load16_bf16(row + q * 16, a[j]);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(a[j][i]));
+        }
     }
-    __shared__ float red[4];
+    __shared__ float red[32];
     __shared__ float s_g;
     amax = warp_max(amax);
-    if (lane == 0) red[threadIdx.x >> 5] = amax;
+    if (lane == 0) red[warp] = amax;
     __syncthreads();
-    if (threadIdx.x == 0) {
-        float t = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
-        s_g = (t == 0.0f) ? 1.0f : __fdiv_rn(t, 2688.0f);
-        g_x[m] = s_g;
+    if (warp == 0) {
+        float t = lane < (int)(blockDim.x >> 5) ? red[lane] : 0.0f;
+        t = warp_max(t);
+        if (lane == 0) {
+            s_g = (t == 0.0f) ? 1.0f : __fdiv_rn(t, 2688.0f);
+            g_x[m] = s_g;
+        }
     }
     __syncthreads();
     const float g = s_g, g6 = __fmul_rn(6.0f, g);
-    // G is a multiple of 4; iterate whole warps so the 4-group gather stays aligned.
-    for (int q0 = (threadIdx.x & ~31); q0 < G; q0 += blockDim.x) {
-        const int q = q0 + lane;
+#pragma unroll
+    for (int j = 0; j < kGPT; ++j) {
+        const int q = threadIdx.x + j * blockDim.x;
         const bool live = q < G;
         uint32_t sfb = 0;
         if (live) {
-            float a[16], deq[16];
+            float deq[16];
             uint32_t lo, hi;
-            load16_bf16(row + q * 16, a);
-            sfb = nvfp4_group(a, g, g6, lo, hi, deq);
+            sfb = nvfp4_group(a[j], g, g6, lo, hi, deq);
             reinterpret_cast<uint2*>(codes + (int64_t)m * (K / 2))[q] = make_uint2(lo, hi);
             if (sf) sf[(int64_t)m * G + q] = (uint8_t)sfb;
         }
@@ -163,58 +168,98 @@ __global__ void __launch_bounds__(128) k_quant_act(const uint16_t* __restrict__ 
     }
 }
 
-// A2: H_k = fp32( sum_t x_tk^2 / T ) with the fp64 sum taken in t order (one thread per
-// column; the squares of bf16 values are exact in fp64, so a fused add is harmless).
-__global__ void __launch_bounds__(128) k_hessian(const uint16_t* __restrict__ X, int T, int K, float* __restrict__ H) {
-    const int k = blockIdx.x * blockDim.x + threadIdx.x;
-    if (k >= K) return;
-    double s = 0.0;
-    int t = 0;
-    for (; t + 8 <= T; t += 8) {
-        uint16_t v[8];
+// A2: H_k = fp32( sum_t x_tk^2 / T ), the fp64 sum taken in t order. A CTA owns 32
+// columns; all threads stage 128-row chunks of those columns in shared memory (a ring
+// of kHChunks chunks in flight with cp.async), one warp runs the 32 sequential sums.
+constexpr int kHCols = 32, kHRows = 128, kHChunks = 4, kHThreads = 256;
+
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, bool pred) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(pred ? 16 : 0)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+__global__ void __launch_bounds__(kHThreads) k_hessian(const uint16_t* __restrict__ X, int T, int K,
+                                                       float* __restrict__ H) {
+    griddep_wait();
+    griddep_launch();
+    __shared__ __align__(16) uint16_t buf[kHChunks][kHRows][kHCols];
+    const int k0 = blockIdx.x * kHCols;
+    const int nchunks = (T + kHRows - 1) / kHRows;
+    auto issue = [&](int c) {
+        if (c < nchunks) {
+            // 128 rows x 64 bytes = 512 16-byte pieces, two per thread
 #pragma unroll
-        for (int j = 0; j < 8; ++j) v[j] = __ldg(X + (int64_t)(t + j) * K + k);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const double x = (double)bf16_bits_to_f32(v[j]);
-            s = __dadd_rn(s, __dmul_rn(x, x));
+            for (int u = 0; u < 2; ++u) {
+                const int piece = threadIdx.x + u * kHThreads;
+                const int r = piece >> 2, part = piece & 3;
+                const int t = c * kHRows + r;
+                const bool ok = t < T;
+                cp_async16(&buf[c % kHChunks][r][part * 8], X + (int64_t)(ok ? t : 0) * K + k0 + part * 8, ok);
+            }
         }
+        cp_async_commit();
+    };
+#pragma unroll
+    for (int c = 0; c < kHChunks - 1; ++c) issue(c);
+    double s = 0.0;
+    for (int c = 0; c < nchunks; ++c) {
+        issue(c + kHChunks - 1);
+        cp_async_wait<kHChunks - 1>();
+        __syncthreads();
+        if (threadIdx.x < kHCols) {
+            const int rows = min(kHRows, T - c * kHRows);
+            const uint16_t(*b)[kHCols] = buf[c % kHChunks];
+            int r = 0;
+            for (; r + 8 <= rows; r += 8) {
+                double x[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) x[j] = (double)bf16_bits_to_f32(b[r + j][threadIdx.x]);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) s = __dadd_rn(s, __dmul_rn(x[j], x[j]));
+            }
+            for (; r < rows; ++r) {
+                const double x = (double)bf16_bits_to_f32(b[r][threadIdx.x]);
+                s = __dadd_rn(s, __dmul_rn(x, x));
+            }
+        }
+        __syncthreads();
     }
-    for (; t < T; ++t) {
-        const double x = (double)bf16_bits_to_f32(__ldg(X + (int64_t)t * K + k));
-        s = __dadd_rn(s, __dmul_rn(x, x));
-    }
-    H[k] = __double2float_rn(__ddiv_rn(s, (double)T));
+    if (threadIdx.x < kHCols) H[k0 + threadIdx.x] = __double2float_rn(__ddiv_rn(s, (double)T));
 }
 
 // ------------------------------------------------------------------ launchers
-int amax_grid(int64_t n8) {
-    int64_t blocks = (n8 + 255) / 256;
-    return (int)(blocks < 148 * 8 ? (blocks < 1 ? 1 : blocks) : 148 * 8);
+cudaError_t launch_amax(const uint16_t* W, int64_t n, float* partial, cudaStream_t s) {
+    return launch_pdl(k_amax_partial, dim3(kAmaxBlocks), dim3(512), 0, s, 1, W, n / 8, partial);
 }
 
 cudaError_t launch_quant_weight(const uint16_t* W, int N, int K, uint8_t* codes, uint8_t* sf, uint8_t* sf_swz,
                                 float* g, uint8_t* rcodes, uint8_t* rsf, float* partial, cudaStream_t s) {
-    const int64_t n8 = (int64_t)N * K / 8;
-    const int P = amax_grid(n8);
-    k_amax_partial<<<P, 256, 0, s>>>(W, n8, partial);
+    cudaError_t e = launch_amax(W, (int64_t)N * K, partial, s);
+    if (e != cudaSuccess) return e;
     const int64_t ngrp = (int64_t)N * (K / 16);
     int64_t blocks = (ngrp + 255) / 256;
     if (blocks > 148 * 16) blocks = 148 * 16;
-    k_quant_weight<<<(int)blocks, 256, 0, s>>>(W, N, K, partial, P, codes, sf, sf_swz, g, rcodes, rsf);
-    return cudaGetLastError();
+    return launch_pdl(k_quant_weight, dim3((unsigned)blocks), dim3(256), 0, s, 1, W, N, K, (const float*)partial,
+                      codes, sf, sf_swz, g, rcodes, rsf);
 }
 
 cudaError_t launch_quant_act(const uint16_t* X, int M, int K, uint8_t* codes, uint8_t* sf, uint8_t* sf_swz,
                              float* g, cudaStream_t s) {
     const int Mp = (M + 127) / 128 * 128;
-    k_quant_act<<<Mp, 128, 0, s>>>(X, M, K, codes, sf, sf_swz, g);
-    return cudaGetLastError();
+    const int G = K / 16;
+    const int gpt = G <= 1024 ? 1 : G <= 2048 ? 2 : 4;
+    int threads = (G + gpt - 1) / gpt;
+    threads = (threads + 31) / 32 * 32;
+    if (gpt == 1) return launch_pdl(k_quant_act<1>, dim3(Mp), dim3(threads), 0, s, 1, X, M, K, codes, sf, sf_swz, g);
+    if (gpt == 2) return launch_pdl(k_quant_act<2>, dim3(Mp), dim3(threads), 0, s, 1, X, M, K, codes, sf, sf_swz, g);
+    return launch_pdl(k_quant_act<4>, dim3(Mp), dim3(threads), 0, s, 1, X, M, K, codes, sf, sf_swz, g);
 }
 
 cudaError_t launch_hessian(const uint16_t* X, int T, int K, float* H, cudaStream_t s) {
-    k_hessian<<<(K + 127) / 128, 128, 0, s>>>(X, T, K, H);
-    return cudaGetLastError();
+    return launch_pdl(k_hessian, dim3(K / kHCols), dim3(kHThreads), 0, s, 1, X, T, K, H);
 }
 
 }  // namespace mq

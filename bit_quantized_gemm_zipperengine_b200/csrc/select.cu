@@ -3,65 +3,119 @@
 // block budget, and packing of the selected residual blocks for the fused GEMM.
 #include "common.cuh"
 #include "nvfp4.cuh"
+#include "quant.cuh"
 
 namespace mq {
 
 // ------------------------------------------------------------------ Delta-score
-// One CTA per block (nt, kt), thread (r = tid/4, q = tid%4) owns one 16-group of the
-// block. e and e' are recomputed from W and the tensor scale exactly as the weight
-// quantizer computes them, so no codes are re-read. The reductions follow the fixed
-// pairwise tree v[i] += v[i+32], +16, +8, +4, +2, +1 (rows first, then columns).
-constexpr int kTauStride = 65;  // fp64 words per smem row (pad: conflict-free columns)
+// One CTA (4 warps) per 64x64 block (nt, kt). Warp q owns group column q (16 K
+// elements); lane r owns block rows r and r+32, so the first level of the fixed
+// pairwise row tree (v[i] += v[i+32]) happens in registers. The remaining levels
+// (+16, +8, +4, +2, +1) run as a butterfly over the lanes that at each level also
+// halves the set of columns a lane keeps: the adds are exactly the tree's pairs, and
+// at the end lanes 2c and 2c+1 hold column c of the group. e and e' are recomputed
+// from W and the tensor scale with the weight quantizer's arithmetic, so they are
+// bit-identical to the stored codes. tau = fma(e, e, -fp32(e'^2)) (fp32); the column
+// sums are widened to fp64 for p_k = H_k c_k and the 64-column tree.
+template <bool kWriteCodes>
+__device__ __forceinline__ void quant_delta_block(const uint16_t* __restrict__ W, int K, const float* __restrict__ H,
+                                                  float g, int nt, int kt, uint8_t* __restrict__ codes,
+                                                  uint8_t* __restrict__ sf, uint8_t* __restrict__ sf_swz,
+                                                  uint8_t* __restrict__ rcodes, uint8_t* __restrict__ rsf,
+                                                  double* __restrict__ delta_out) {
+    __shared__ double pcol[64];
+    __shared__ uint32_t sf_s[64], rsf_s[64];  // the 4 group scales of each block row
+    const int q = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const float g6 = __fmul_rn(6.0f, g);
+    // both rows' loads first, so 64 bytes per thread are in flight before any arithmetic
+    float a2[2][16];
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+        load16_bf16(W + ((int64_t)nt * 64 + lane + 32 * h) * K + kt * 64 + q * 16, a2[h]);
+    float v[16];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const int rl = lane + 32 * h;
+        const int64_t row = (int64_t)nt * 64 + rl;
+        float deq[16], R[16], rdeq[16];
+        uint32_t lo, hi, rlo, rhi;
+        const uint32_t sfb = nvfp4_group(a2[h], g, g6, lo, hi, deq);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) R[i] = __fsub_rn(a2[h][i], deq[i]);
+        const uint32_t rsb = nvfp4_group(R, g, g6, rlo, rhi, rdeq);
+        if (kWriteCodes) {
+            *reinterpret_cast<uint2*>(codes + row * (K / 2) + kt * 32 + q * 8) = make_uint2(lo, hi);
+            *reinterpret_cast<uint2*>(rcodes + row * (K / 2) + kt * 32 + q * 8) = make_uint2(rlo, rhi);
+            reinterpret_cast<uint8_t*>(sf_s)[rl * 4 + q] = (uint8_t)sfb;
+            reinterpret_cast<uint8_t*>(rsf_s)[rl * 4 + q] = (uint8_t)rsb;
+        }
+        // tau = fma(e, e, -fp32(e'^2)) with e = R, e' = R - deqR; the squares of e' are
+        // taken in pairs
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const float e0 = R[2 * j], e1 = R[2 * j + 1];
+            const float f0 = __fsub_rn(e0, rdeq[2 * j]), f1 = __fsub_rn(e1, rdeq[2 * j + 1]);
+            const float2 sq = mul2(make_float2(f0, f1), make_float2(f0, f1));
+            const float t0 = __fmaf_rn(e0, e0, -sq.x), t1 = __fmaf_rn(e1, e1, -sq.y);
+            v[2 * j] = h ? __fadd_rn(v[2 * j], t0) : t0;
+            v[2 * j + 1] = h ? __fadd_rn(v[2 * j + 1], t1) : t1;
+        }
+    }
+    // butterfly: masks 16, 8, 4, 2 keep n = 8, 4, 2, 1 columns; then mask 1 adds pairs
+#pragma unroll
+    for (int m = 16, n = 8; m >= 2; m >>= 1, n >>= 1) {
+        const bool upper = (lane & m) != 0;
+#pragma unroll
+        for (int j = 0; j < n; ++j) {
+            const float send = upper ? v[j] : v[j + n];
+            const float keep = upper ? v[j + n] : v[j];
+            v[j] = __fadd_rn(keep, __shfl_xor_sync(0xffffffffu, send, m));
+        }
+    }
+    const float colsum = __fadd_rn(v[0], __shfl_xor_sync(0xffffffffu, v[0], 1));
+    const int c = (lane >> 1) & 15;
+    if ((lane & 1) == 0) pcol[q * 16 + c] = __dmul_rn((double)__ldg(H + kt * 64 + q * 16 + c), (double)colsum);
+    __syncthreads();
+    if (q == 0) {
+        double d = __dadd_rn(pcol[lane], pcol[lane + 32]);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) d = __dadd_rn(d, __shfl_down_sync(0xffffffffu, d, o));
+        if (lane == 0) *delta_out = d;
+    }
+    if (kWriteCodes && threadIdx.x < 64) {
+        const int64_t row = (int64_t)nt * 64 + threadIdx.x;
+        const uint32_t wsf = sf_s[threadIdx.x], wr = rsf_s[threadIdx.x];
+        if (sf) *reinterpret_cast<uint32_t*>(sf + row * (K / 16) + kt * 4) = wsf;
+        *reinterpret_cast<uint32_t*>(rsf + row * (K / 16) + kt * 4) = wr;
+        *reinterpret_cast<uint32_t*>(sf_swz + sf_swz_offset(row, (int64_t)kt * 4, K)) = wsf;
+    }
+}
 
-__global__ void __launch_bounds__(256) k_delta(const uint16_t* __restrict__ W, int N, int K,
+// A3: Delta-score from W, H and the tensor scale (no codes written).
+__global__ void __launch_bounds__(128) k_delta(const uint16_t* __restrict__ W, int N, int K,
                                                const float* __restrict__ H, const float* __restrict__ gptr,
                                                double* __restrict__ delta) {
-    __shared__ double tau[64 * kTauStride];
-    __shared__ double p[64];
-    const int KB = K / 64;
-    const int b = blockIdx.x;
-    const int nt = b / KB, kt = b % KB;
-    const int r = threadIdx.x >> 2, q = threadIdx.x & 3;
-    const float g = __ldg(gptr);
-    const float g6 = __fmul_rn(6.0f, g);
-    {
-        float a[16], deq[16], R[16], rdeq[16];
-        const uint4* src = reinterpret_cast<const uint4*>(W + (int64_t)(nt * 64 + r) * K + kt * 64 + q * 16);
-        const uint4 v0 = __ldg(src), v1 = __ldg(src + 1);
-        const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            a[2 * i] = bf16_bits_to_f32(w[i] & 0xFFFFu);
-            a[2 * i + 1] = bf16_bits_to_f32(w[i] >> 16);
-        }
-        uint32_t lo, hi;
-        nvfp4_group(a, g, g6, lo, hi, deq);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) R[i] = __fsub_rn(a[i], deq[i]);
-        nvfp4_group(R, g, g6, lo, hi, rdeq);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const double e = (double)R[i];
-            const double e2 = (double)__fsub_rn(R[i], rdeq[i]);
-            tau[r * kTauStride + q * 16 + i] = __dsub_rn(__dmul_rn(e, e), __dmul_rn(e2, e2));
-        }
-    }
-    __syncthreads();
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-#pragma unroll 1
-    for (int c = warp * 8; c < warp * 8 + 8; ++c) {
-        double v = __dadd_rn(tau[lane * kTauStride + c], tau[(lane + 32) * kTauStride + c]);
-#pragma unroll
-        for (int h = 16; h > 0; h >>= 1) v = __dadd_rn(v, __shfl_down_sync(0xffffffffu, v, h));
-        if (lane == 0) p[c] = __dmul_rn((double)__ldg(H + kt * 64 + c), v);
-    }
-    __syncthreads();
-    if (warp == 0) {
-        double v = __dadd_rn(p[lane], p[lane + 32]);
-#pragma unroll
-        for (int h = 16; h > 0; h >>= 1) v = __dadd_rn(v, __shfl_down_sync(0xffffffffu, v, h));
-        if (lane == 0) delta[b] = v;
-    }
+    griddep_wait();
+    griddep_launch();
+    const int KB = K / 64, b = blockIdx.x;
+    quant_delta_block<false>(W, K, H, __ldg(gptr), b / KB, b % KB, nullptr, nullptr, nullptr, nullptr, nullptr,
+                             delta + b);
+}
+
+// A1 + A3 in one pass over W: base and residual codes/scales and the Delta-score of
+// every block, with the tensor scale from the |W| maximum pass.
+__global__ void __launch_bounds__(128) k_quant_delta(const uint16_t* __restrict__ W, int N, int K,
+                                                     const float* __restrict__ H, const float* __restrict__ partial,
+                                                     uint8_t* __restrict__ codes, uint8_t* __restrict__ sf,
+                                                     uint8_t* __restrict__ sf_swz, float* __restrict__ g_out,
+                                                     uint8_t* __restrict__ rcodes, uint8_t* __restrict__ rsf,
+                                                     double* __restrict__ delta) {
+    griddep_wait();
+    griddep_launch();
+    const float g = tensor_scale(partial);
+    if (blockIdx.x == 0 && threadIdx.x == 0) *g_out = g;
+    const int KB = K / 64, b = blockIdx.x;
+    quant_delta_block<true>(W, K, H, g, b / KB, b % KB, codes, sf, sf_swz, rcodes, rsf, delta + b);
 }
 
 // ------------------------------------------------------------------ top-K
@@ -103,49 +157,88 @@ __device__ __forceinline__ int block_exclusive_sum(int v, int* scratch, int& tot
 }
 
 // Single-CTA radix select of the budget-th largest key (8 digits of 8 bits, most
-// significant first), then a stable compaction in block order: every key above the
-// threshold plus the lowest-index keys equal to it. Writes sel ascending.
+// significant first; keys held in shared memory when they fit), then a stable
+// compaction in block order: every key above the threshold plus the lowest-index keys
+// equal to it, which writes sel ascending. With kRank the same CTA also writes rank by
+// counting: position of selected i = #{j : key_j > key_i} + #{j < i : key_j == key_i}.
 constexpr int kSelThreads = 1024;
+constexpr int kRankInCtaMax = 1024;        // budgets up to this are ranked in the CTA
+constexpr size_t kSelSmemKeysMax = 160 * 1024;
 
-__global__ void __launch_bounds__(kSelThreads) k_topk_select(const double* __restrict__ delta, int B, int budget,
-                                                             int32_t* __restrict__ sel) {
+template <bool kSmemKeys, bool kRank>
+__global__ void __launch_bounds__(kSelThreads) k_topk(const double* __restrict__ delta, int B, int budget,
+                                                      int32_t* __restrict__ sel, int32_t* __restrict__ rank) {
+    griddep_wait();
+    griddep_launch();
+    extern __shared__ __align__(16) uint64_t dyn[];
+    uint64_t* keys = dyn;                                   // [B] when kSmemKeys
+    uint64_t* selkey = dyn + (kSmemKeys ? B : 0);           // [budget] when kRank
+    int32_t* selidx = reinterpret_cast<int32_t*>(selkey + (kRank ? budget : 0));
     __shared__ unsigned hist[256];
     __shared__ uint64_t s_prefix, s_mask;
     __shared__ int s_need;
     __shared__ int scratch[32];
-    if (threadIdx.x == 0) { s_prefix = 0; s_mask = 0; s_need = budget; }
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    if (kSmemKeys)
+        for (int i = tid; i < B; i += kSelThreads) keys[i] = order_key(delta[i]);
+    if (tid == 0) { s_prefix = 0; s_mask = 0; s_need = budget; }
     __syncthreads();
+    auto key_of = [&](int i) -> uint64_t { return kSmemKeys ? keys[i] : order_key(delta[i]); };
 #pragma unroll 1
     for (int shift = 56; shift >= 0; shift -= 8) {
-        for (int i = threadIdx.x; i < 256; i += kSelThreads) hist[i] = 0;
+        if (tid < 256) hist[tid] = 0;
         __syncthreads();
         const uint64_t prefix = s_prefix, mask = s_mask;
-        for (int i = threadIdx.x; i < B; i += kSelThreads) {
-            const uint64_t key = order_key(delta[i]);
-            if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+        // warp-aggregated histogram: lanes with the same digit add once (the keys share
+        // their leading digits, so per-lane atomics would all hit one bin)
+        for (int i0 = tid - lane; i0 < B; i0 += kSelThreads) {
+            const int i = i0 + lane;
+            unsigned digit = 256u;  // not counted
+            if (i < B) {
+                const uint64_t key = key_of(i);
+                if ((key & mask) == prefix) digit = (unsigned)(key >> shift) & 255u;
+            }
+            const unsigned peers = __match_any_sync(0xffffffffu, digit);
+            if (digit < 256u && lane == __ffs(peers) - 1) atomicAdd(&hist[digit], (unsigned)__popc(peers));
         }
         __syncthreads();
-        if (threadIdx.x == 0) {
-            int need = s_need;
-            unsigned cum = 0;
-            int digit = 0;
-            for (int d = 255; d >= 0; --d) {
-                if (cum + hist[d] >= (unsigned)need) { digit = d; break; }
-                cum += hist[d];
+        if (warp == 0) {
+            // lane l scans bins 255-8l down to 248-8l; find the bin where the count of
+            // keys from the top reaches `need`
+            unsigned cnt[8], tot = 0;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) { cnt[j] = hist[255 - 8 * lane - j]; tot += cnt[j]; }
+            unsigned incl = tot;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const unsigned y = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += y;
             }
-            s_need = need - (int)cum;
-            s_prefix = prefix | ((uint64_t)digit << shift);
-            s_mask = mask | ((uint64_t)255 << shift);
+            const int need = s_need;
+            const unsigned hit = __ballot_sync(0xffffffffu, incl >= (unsigned)need);
+            const int first = __ffs(hit) - 1;
+            if (lane == first) {
+                unsigned cum = incl - tot;
+                int digit = 0;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    if (cum + cnt[j] >= (unsigned)need) { digit = 255 - 8 * lane - j; break; }
+                    cum += cnt[j];
+                }
+                s_need = need - (int)cum;
+                s_prefix = prefix | ((uint64_t)digit << shift);
+                s_mask = mask | ((uint64_t)255 << shift);
+            }
         }
         __syncthreads();
     }
     const uint64_t T = s_prefix;
     const int need_eq = s_need;  // how many keys equal to T are taken (lowest b first)
     const int chunk = (B + kSelThreads - 1) / kSelThreads;
-    const int lo = min(B, (int)threadIdx.x * chunk), hi = min(B, lo + chunk);
+    const int lo = min(B, tid * chunk), hi = min(B, lo + chunk);
     int gt = 0, eq = 0;
     for (int i = lo; i < hi; ++i) {
-        const uint64_t key = order_key(delta[i]);
+        const uint64_t key = key_of(i);
         gt += key > T;
         eq += key == T;
     }
@@ -155,10 +248,264 @@ __global__ void __launch_bounds__(kSelThreads) k_topk_select(const double* __res
     int out = block_exclusive_sum<kSelThreads>(gt + eq_take, scratch, total);
     int eq_seen = eq_before;
     for (int i = lo; i < hi; ++i) {
-        const uint64_t key = order_key(delta[i]);
+        const uint64_t key = key_of(i);
         bool take = key > T;
         if (key == T) take = eq_seen++ < need_eq;
-        if (take) sel[out++] = i;
+        if (take) {
+            sel[out] = i;
+            if (kRank) { selkey[out] = key; selidx[out] = i; }
+            ++out;
+        }
+    }
+    if (kRank) {
+        // position of selected i, counted in `parts` slices of j by different threads
+        __shared__ int pos_s[kRankInCtaMax];
+        for (int i = tid; i < budget; i += kSelThreads) pos_s[i] = 0;
+        __syncthreads();
+        const int parts = max(1, kSelThreads / budget);
+        const int span = (budget + parts - 1) / parts;
+        for (int w = tid; w < budget * parts; w += kSelThreads) {
+            const int i = w / parts, part = w % parts;
+            const uint64_t mine = selkey[i];
+            const int j0 = part * span, j1 = min(budget, j0 + span);
+            int pos = 0;
+            for (int j = j0; j < j1; ++j) {
+                const uint64_t kj = selkey[j];
+                pos += (kj > mine) | ((kj == mine) & (j < i));
+            }
+            atomicAdd(&pos_s[i], pos);
+        }
+        __syncthreads();
+        for (int i = tid; i < budget; i += kSelThreads) rank[pos_s[i]] = selidx[i];
+    }
+}
+
+// Top-K for budgets up to kSmallBudget, one CTA:
+//  1. keys (order-preserving 64-bit images of Delta) and their common leading bits;
+//  2. 8-bit radix passes below the common prefix until at most kCandMax keys share the
+//     bucket that holds the budget-th largest key (warp-uniform digits add once);
+//  3. the keys of higher buckets (all selected) and the candidates of that bucket go
+//     into one list, sorted by (key descending, block index ascending), a strict total
+//     order: its first `budget` entries are rank; sel is the same set in ascending block
+//     index, from a bitmap scan.
+// If the keys tie beyond kCandMax candidates (the bucket is resolved to a single key
+// value), the selected set is compacted in block order instead (every key above the
+// value, then the lowest-index keys equal to it) and then sorted for rank.
+constexpr int kSmallBudget = 1024;
+constexpr int kCandMax = 512;
+constexpr int kSortCap = 2048;  // budget + candidates, a power of two
+
+__device__ __forceinline__ bool before(uint64_t ka, int ia, uint64_t kb, int ib) {
+    return ka > kb || (ka == kb && ia < ib);
+}
+
+// Bitonic sort of n2 (power of two, <= 2 * blockDim.x) (key, idx) pairs in shared memory
+// by (key descending, idx ascending). Pair p belongs to thread p; a warp's pairs cover 64
+// consecutive elements for strides below 64, which then need only __syncwarp.
+__device__ __forceinline__ void block_sort_desc(uint64_t* key, int32_t* idx, int n2) {
+    const int p = threadIdx.x;
+    const bool act = p < (n2 >> 1);
+    for (int k = 2, lk = 1; k <= n2; k <<= 1, ++lk) {
+        for (int j = k >> 1, lj = lk - 1; j > 0; j >>= 1, --lj) {
+            if (act) {
+                const int i = ((p >> lj) << (lj + 1)) | (p & (j - 1)), q = i + j;
+                const bool desc = (i & k) == 0;
+                const uint64_t ki = key[i], kq = key[q];
+                const int ii = idx[i], iq = idx[q];
+                if (before(kq, iq, ki, ii) == desc) {
+                    key[i] = kq;
+                    key[q] = ki;
+                    idx[i] = iq;
+                    idx[q] = ii;
+                }
+            }
+            const int jn = j > 1 ? (j >> 1) : k;  // the next stage's stride
+            if (j >= 64 || jn >= 64) __syncthreads();
+            else __syncwarp();
+        }
+    }
+}
+
+__device__ __forceinline__ uint64_t warp_and64(uint64_t v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v &= __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+__device__ __forceinline__ uint64_t warp_or64(uint64_t v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v |= __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+template <bool kSmemKeys>
+__global__ void __launch_bounds__(kSelThreads) k_topk_small(const double* __restrict__ delta, int B, int budget,
+                                                            int32_t* __restrict__ rank, int32_t* __restrict__ sel) {
+    extern __shared__ __align__(16) uint64_t dyn[];
+    uint64_t* keys = dyn;                                         // [B] when kSmemKeys
+    uint64_t* skey = dyn + (kSmemKeys ? B : 0);                   // [kSortCap]
+    int32_t* sidx = reinterpret_cast<int32_t*>(skey + kSortCap);  // [kSortCap]
+    uint32_t* bits = reinterpret_cast<uint32_t*>(sidx + kSortCap); // [ceil(B / 32)]
+    __shared__ unsigned hist[256];
+    __shared__ uint64_t s_and[32], s_or[32];
+    __shared__ uint64_t s_prefix;
+    __shared__ int s_pos, s_need, s_cand, s_nsel;
+    __shared__ int scratch[32];
+    griddep_wait();  // Delta comes from the previous kernel
+    griddep_launch();
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int nw = (B + 31) / 32;
+    auto key_of = [&](int i) -> uint64_t { return kSmemKeys ? keys[i] : order_key(delta[i]); };
+
+    uint64_t a = ~0ull, o = 0ull;
+    for (int i = tid; i < B; i += kSelThreads) {
+        const uint64_t k = order_key(delta[i]);
+        if (kSmemKeys) keys[i] = k;
+        a &= k;
+        o |= k;
+    }
+    for (int w = tid; w < nw; w += kSelThreads) bits[w] = 0u;
+    a = warp_and64(a);
+    o = warp_or64(o);
+    if (lane == 0) { s_and[warp] = a; s_or[warp] = o; }
+    __syncthreads();
+    if (warp == 0) {
+        a = s_and[lane];
+        o = s_or[lane];
+        a = warp_and64(a);
+        o = warp_or64(o);
+        if (lane == 0) {
+            const int cp = (a ^ o) ? __clzll((long long)(a ^ o)) : 64;  // common leading bits
+            s_pos = 64 - cp;
+            s_prefix = cp ? (a & (~0ull << (64 - cp))) : 0ull;
+            s_need = budget;
+            s_cand = B;
+            s_nsel = 0;
+        }
+    }
+    __syncthreads();
+    // radix passes below the common prefix
+    while (s_pos > 0 && s_cand > kCandMax) {
+        const int pos = s_pos, w = pos < 8 ? pos : 8, shift = pos - w;
+        const uint64_t prefix = s_prefix, hi = pos >= 64 ? 0ull : (~0ull << pos);
+        if (tid < 256) hist[tid] = 0;
+        __syncthreads();
+        for (int i0 = tid - lane; i0 < B; i0 += kSelThreads) {
+            const int i = i0 + lane;
+            unsigned digit = 256u;
+            if (i < B) {
+                const uint64_t k = key_of(i);
+                if ((k & hi) == prefix) digit = (unsigned)(k >> shift) & ((1u << w) - 1u);
+            }
+            const bool uniform = __all_sync(0xffffffffu, digit == __shfl_sync(0xffffffffu, digit, 0));
+            if (uniform) {
+                if (lane == 0 && digit < 256u) atomicAdd(&hist[digit], 32u);
+            } else if (digit < 256u) {
+                atomicAdd(&hist[digit], 1u);
+            }
+        }
+        __syncthreads();
+        if (warp == 0) {
+            // bins from the top: lane l holds bins 255-8l .. 248-8l
+            unsigned cnt[8], tot = 0;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) { cnt[j] = hist[255 - 8 * lane - j]; tot += cnt[j]; }
+            unsigned incl = tot;
+#pragma unroll
+            for (int d = 1; d < 32; d <<= 1) {
+                const unsigned y = __shfl_up_sync(0xffffffffu, incl, d);
+                if (lane >= d) incl += y;
+            }
+            const int need = s_need;
+            const unsigned hit = __ballot_sync(0xffffffffu, incl >= (unsigned)need);
+            const int first = __ffs(hit) - 1;
+            if (lane == first) {
+                unsigned cum = incl - tot;
+                int digit = 0;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    if (cum + cnt[j] >= (unsigned)need) {
+                        digit = 255 - 8 * lane - j;
+                        s_cand = (int)cnt[j];
+                        break;
+                    }
+                    cum += cnt[j];
+                }
+                s_need = need - (int)cum;
+                s_prefix = prefix | ((uint64_t)digit << shift);
+                s_pos = shift;
+            }
+        }
+        __syncthreads();
+    }
+    const int pos = s_pos, need = s_need;
+    const uint64_t prefix = s_prefix, hi = pos >= 64 ? 0ull : (~0ull << pos);
+    if (s_cand <= kCandMax) {
+        // every key above the bucket plus the bucket's candidates, then one sort
+        for (int i = tid; i < B; i += kSelThreads) {
+            const uint64_t k = key_of(i);
+            const uint64_t kh = k & hi;
+            if (kh >= prefix) {
+                const int slot = atomicAdd(&s_nsel, 1);
+                skey[slot] = k;
+                sidx[slot] = i;
+            }
+        }
+        __syncthreads();
+        const int nsel = s_nsel;
+        int n2 = 2;
+        while (n2 < nsel) n2 <<= 1;
+        for (int e = nsel + tid; e < n2; e += kSelThreads) { skey[e] = 0ull; sidx[e] = 0x7FFFFFFF - e; }
+        __syncthreads();
+        block_sort_desc(skey, sidx, n2);
+    } else {
+        // the bucket is a single key value T shared by more than kCandMax keys: keys above
+        // T and the lowest-index `need` keys equal to T, compacted in block order
+        const uint64_t T = prefix;
+        const int chunk = (B + kSelThreads - 1) / kSelThreads;
+        const int lo = min(B, tid * chunk), hi2 = min(B, lo + chunk);
+        int gt = 0, eq = 0;
+        for (int i = lo; i < hi2; ++i) {
+            const uint64_t k = key_of(i);
+            gt += k > T;
+            eq += k == T;
+        }
+        int total;
+        const int eq_before = block_exclusive_sum<kSelThreads>(eq, scratch, total);
+        const int eq_take = max(0, min(eq, need - eq_before));
+        int out = block_exclusive_sum<kSelThreads>(gt + eq_take, scratch, total);
+        int eq_seen = eq_before;
+        for (int i = lo; i < hi2; ++i) {
+            const uint64_t k = key_of(i);
+            bool take = k > T;
+            if (k == T) take = eq_seen++ < need;
+            if (take) { skey[out] = k; sidx[out] = i; ++out; }
+        }
+        __syncthreads();
+        int n2 = 2;
+        while (n2 < budget) n2 <<= 1;
+        for (int e = budget + tid; e < n2; e += kSelThreads) { skey[e] = 0ull; sidx[e] = 0x7FFFFFFF - e; }
+        __syncthreads();
+        block_sort_desc(skey, sidx, n2);
+    }
+    for (int e = tid; e < budget; e += kSelThreads) {
+        rank[e] = sidx[e];
+        atomicOr(&bits[sidx[e] >> 5], 1u << (sidx[e] & 31));
+    }
+    __syncthreads();
+    // sel: the set bits in index order (each thread scans a run of bitmap words)
+    const int per = (nw + kSelThreads - 1) / kSelThreads;
+    const int w0 = min(nw, tid * per), w1 = min(nw, w0 + per);
+    int cnt = 0;
+    for (int w = w0; w < w1; ++w) cnt += __popc(bits[w]);
+    int total;
+    int out = block_exclusive_sum<kSelThreads>(cnt, scratch, total);
+    for (int w = w0; w < w1; ++w) {
+        uint32_t b = bits[w];
+        while (b) {
+            const int t = __ffs(b) - 1;
+            b &= b - 1;
+            sel[out++] = w * 32 + t;
+        }
     }
 }
 
@@ -166,6 +513,8 @@ __global__ void __launch_bounds__(kSelThreads) k_topk_select(const double* __res
 // (sel is ascending, so a lower list index is a lower block index).
 __global__ void __launch_bounds__(256) k_topk_rank(const double* __restrict__ delta, const int32_t* __restrict__ sel,
                                                    int budget, int32_t* __restrict__ rank) {
+    griddep_wait();
+    griddep_launch();
     __shared__ uint64_t keys[2048];
     const int i = blockIdx.x * blockDim.x + threadIdx.x;
     const uint64_t mine = i < budget ? order_key(delta[sel[i]]) : 0;
@@ -194,6 +543,8 @@ __global__ void __launch_bounds__(256) k_pack(const uint8_t* __restrict__ rcodes
                                               uint8_t* __restrict__ blk_codes, uint8_t* __restrict__ blk_sf,
                                               int32_t* __restrict__ blk_kt, int32_t* __restrict__ tile_ptr,
                                               uint32_t* __restrict__ bitmap) {
+    griddep_wait();
+    griddep_launch();
     const int KB = K / 64, NBr = N / 64, KW = (KB + 31) / 32;
     if ((int)blockIdx.x < budget) {
         const int i = blockIdx.x;
@@ -247,15 +598,54 @@ __global__ void __launch_bounds__(256) k_pack(const uint8_t* __restrict__ rcodes
 cudaError_t launch_delta(const uint16_t* W, int N, int K, const float* H, const float* g, double* delta,
                          cudaStream_t s) {
     const int B = (N / 64) * (K / 64);
-    k_delta<<<B, 256, 0, s>>>(W, N, K, H, g, delta);
-    return cudaGetLastError();
+    return launch_pdl(k_delta, dim3(B), dim3(128), 0, s, 1, W, N, K, H, g, delta);
+}
+
+cudaError_t launch_quant_delta(const uint16_t* W, int N, int K, const float* H, uint8_t* codes, uint8_t* sf,
+                               uint8_t* sf_swz, float* g, uint8_t* rcodes, uint8_t* rsf, double* delta,
+                               float* partial, cudaStream_t s) {
+    cudaError_t e = launch_amax(W, (int64_t)N * K, partial, s);
+    if (e != cudaSuccess) return e;
+    const int B = (N / 64) * (K / 64);
+    return launch_pdl(k_quant_delta, dim3(B), dim3(128), 0, s, 1, W, N, K, H, (const float*)partial, codes, sf,
+                      sf_swz, g, rcodes, rsf, delta);
 }
 
 cudaError_t launch_topk(const double* delta, int B, int budget, int32_t* rank, int32_t* sel, cudaStream_t s) {
     if (budget <= 0) return cudaSuccess;
-    k_topk_select<<<1, kSelThreads, 0, s>>>(delta, B, budget, sel);
-    k_topk_rank<<<(budget + 255) / 256, 256, 0, s>>>(delta, sel, budget, rank);
-    return cudaGetLastError();
+    if (budget <= kSmallBudget) {
+        const size_t tail = (size_t)kSortCap * 12 + (size_t)((B + 31) / 32) * 4;
+        const bool smem_keys = (size_t)B * 8 + tail <= kSelSmemKeysMax;
+        const size_t smem = (smem_keys ? (size_t)B * 8 : 0) + tail;
+        static bool attr[2] = {false, false};
+        auto go = [&](auto kern, int which) -> cudaError_t {
+            if (!attr[which]) {
+                cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                     (int)kSelSmemKeysMax + 16 * 1024);
+                if (e != cudaSuccess) return e;
+                attr[which] = true;
+            }
+            return launch_pdl(kern, dim3(1), dim3(kSelThreads), smem, s, 1, delta, B, budget, rank, sel);
+        };
+        return smem_keys ? go(k_topk_small<true>, 0) : go(k_topk_small<false>, 1);
+    }
+    // larger budgets: radix select and compaction, then a separate counting rank kernel
+    const bool smem_keys = (size_t)B * 8 <= kSelSmemKeysMax;
+    const size_t smem = smem_keys ? (size_t)B * 8 : 0;
+    static bool attr2[2] = {false, false};
+    auto go2 = [&](auto kern, int which) -> cudaError_t {
+        if (!attr2[which]) {
+            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 (int)kSelSmemKeysMax + 16 * 1024);
+            if (e != cudaSuccess) return e;
+            attr2[which] = true;
+        }
+        return launch_pdl(kern, dim3(1), dim3(kSelThreads), smem, s, 1, delta, B, budget, sel, rank);
+    };
+    cudaError_t e = smem_keys ? go2(k_topk<true, false>, 0) : go2(k_topk<false, false>, 1);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(k_topk_rank, dim3((budget + 255) / 256), dim3(256), 0, s, 1, delta, (const int32_t*)sel, budget,
+                      rank);
 }
 
 cudaError_t launch_pack(const uint8_t* rcodes, const uint8_t* rsf, int N, int K, const int32_t* sel, int budget,
@@ -263,8 +653,8 @@ cudaError_t launch_pack(const uint8_t* rcodes, const uint8_t* rsf, int N, int K,
                         cudaStream_t s) {
     const int NBr = N / 64;
     const int grid = budget + (NBr + 255) / 256;
-    k_pack<<<grid, 256, 0, s>>>(rcodes, rsf, N, K, sel, budget, blk_codes, blk_sf, blk_kt, tile_ptr, bitmap);
-    return cudaGetLastError();
+    return launch_pdl(k_pack, dim3(grid), dim3(256), 0, s, 1, rcodes, rsf, N, K, sel, budget, blk_codes, blk_sf,
+                      blk_kt, tile_ptr, bitmap);
 }
 
 }  // namespace mq

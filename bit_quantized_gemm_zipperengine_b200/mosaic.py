@@ -26,7 +26,7 @@ EXPORTED = (
     "mq_sf_swz_bytes", "mq_budget_blocks", "mq_quantize_weight_workspace_bytes", "mq_delta_topk_workspace_bytes",
     "mq_gemm_workspace_bytes", "mq_quantize_weight", "mq_hessian_diag", "mq_delta_score_topk", "mq_pack_residual",
     "mq_quantize_act", "mq_gemm", "mq_run_layer", "mq_get_error", "mq_status_string", "mq_launch_count",
-    "mq_gemm_noalloc", "mq_gemm_noalloc_scratch_limit",
+    "mq_gemm_noalloc", "mq_gemm_noalloc_scratch_limit", "mq_quantize_weight_delta", "mq_topk_blocks",
 )
 
 
@@ -88,6 +88,10 @@ def lib():
     L.mq_gemm_noalloc.restype = i32
     L.mq_gemm_noalloc_scratch_limit.argtypes = []
     L.mq_gemm_noalloc_scratch_limit.restype = sz
+    L.mq_quantize_weight_delta.argtypes = [vp, i32, i32, vp, P(NVFP4Mat), P(NVFP4Mat), vp, vp, sz, vp]
+    L.mq_quantize_weight_delta.restype = i32
+    L.mq_topk_blocks.argtypes = [vp, i32, i32, vp, vp, vp]
+    L.mq_topk_blocks.restype = i32
     L.mq_get_error.argtypes = [vp]
     L.mq_status_string.argtypes = [i32]
     L.mq_status_string.restype = ctypes.c_char_p
@@ -166,6 +170,19 @@ def mq_quantize_weight(W: torch.Tensor, base: dict, resid: dict, ws: torch.Tenso
     N, K = W.shape
     _check(lib().mq_quantize_weight(_ptr(W), N, K, ctypes.byref(mat(base)), ctypes.byref(mat(resid)), _ptr(ws),
                                     ws.numel() * ws.element_size(), _stream(stream)), "mq_quantize_weight")
+
+
+def mq_quantize_weight_delta(W: torch.Tensor, H: torch.Tensor, base: dict, resid: dict, delta: torch.Tensor,
+                             ws: torch.Tensor, stream=None):
+    N, K = W.shape
+    _check(lib().mq_quantize_weight_delta(_ptr(W), N, K, _ptr(H), ctypes.byref(mat(base)), ctypes.byref(mat(resid)),
+                                          _ptr(delta), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
+           "mq_quantize_weight_delta")
+
+
+def mq_topk_blocks(delta: torch.Tensor, budget: int, rank, sel, stream=None):
+    _check(lib().mq_topk_blocks(_ptr(delta), delta.numel(), budget, _ptr(rank), _ptr(sel), _stream(stream)),
+           "mq_topk_blocks")
 
 
 def mq_hessian_diag(Xcal: torch.Tensor, H: torch.Tensor, stream=None):
@@ -252,9 +269,17 @@ class Layer:
         self._act = {}
 
     def prepare(self, W: torch.Tensor, Xcal: torch.Tensor, stream=None):
+        """A1..A5 through the separate calls (quantize, H, Delta + top-K, pack)."""
         mq_quantize_weight(W, self.base, self.resid, self.qws, stream)
         mq_hessian_diag(Xcal, self.H, stream)
         mq_delta_score_topk(W, self.H, self.base, None, self.budget, self.delta, self.rank, self.sel, None, stream)
+        mq_pack_residual(self.resid, self.sel, self.budget, self.packed, stream)
+
+    def prepare_fused(self, W: torch.Tensor, Xcal: torch.Tensor, stream=None):
+        """A1..A5 with quantization and Delta in one pass over W (as mq_run_layer)."""
+        mq_hessian_diag(Xcal, self.H, stream)
+        mq_quantize_weight_delta(W, self.H, self.base, self.resid, self.delta, self.qws, stream)
+        mq_topk_blocks(self.delta, self.budget, self.rank, self.sel, stream)
         mq_pack_residual(self.resid, self.sel, self.budget, self.packed, stream)
 
     def act_buffers(self, M: int, flags: int = 0):

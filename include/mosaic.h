@@ -11,8 +11,8 @@
  * Number format (NVFP4): E2M1 values {0, 0.5, 1, 1.5, 2, 3, 4, 6} with a sign bit, one
  * E4M3 scale per 16 consecutive K elements, and an fp32 tensor scale g (one per weight
  * matrix, one per token for activations). g = amax / 2688 (1 if amax = 0). Per group:
- * s = amax_group / (6 g); sf = E4M3_rne_satfinite(s); d = dec(sf) * g;
- * code_i = E2M1_rne_satfinite(a_i / d) (a signed zero when d = 0). All fp32 IEEE
+ * s = amax_group / (6 g); sf = E4M3_rne_satfinite(s); d = dec(sf) * g; r = 1 / d;
+ * code_i = E2M1_rne_satfinite(a_i * r) (a signed zero when d = 0). All fp32 IEEE
  * operations, no fused multiply-add; codes and scales are bit-exact with the CPU oracle.
  *
  * Conventions for every call:
@@ -162,6 +162,22 @@ mq_status mq_hessian_diag(const mq_bf16* Xcal, int T, int K, float* H, mq_stream
 mq_status mq_delta_score_topk(const mq_bf16* W, const float* H, const mq_nvfp4_mat* base,
                               const mq_nvfp4_mat* resid_full, int budget, double* delta, int32_t* rank,
                               int32_t* sel, void* ws, size_t ws_bytes, mq_stream stream);
+
+/*
+ * A1 + A3 in one pass over W (same results as mq_quantize_weight followed by the
+ * Delta part of mq_delta_score_topk): base and full residual NVFP4 codes and scales, the
+ * tensor scale, and Delta [(N/64)*(K/64)] (fp64), with H from mq_hessian_diag.
+ * Buffers and workspace as in mq_quantize_weight; base->sf may be NULL.
+ */
+mq_status mq_quantize_weight_delta(const mq_bf16* W, int N, int K, const float* H, mq_nvfp4_mat* base,
+                                   mq_nvfp4_mat* resid_full, double* delta, void* ws, size_t ws_bytes,
+                                   mq_stream stream);
+
+/*
+ * A4 alone: order nblk blocks by (Delta descending, block index ascending); rank gets the
+ * first `budget` indices in that order, sel the same set ascending. 0 <= budget <= nblk.
+ */
+mq_status mq_topk_blocks(const double* delta, int nblk, int budget, int32_t* rank, int32_t* sel, mq_stream stream);
 
 /*
  * A5. Pack the selected residual blocks (the sparse residual of section 1, stored per

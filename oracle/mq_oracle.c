@@ -28,7 +28,8 @@
  * 16-element blocks and an E2M1 mantissa ("Problem" section of that page).
  *
  * Arithmetic: fp32 IEEE operations exactly as written (compile with
- * -ffp-contract=off, no fast-math), fp64 where stated. Rounding is RNE throughout.
+ * -ffp-contract=off, no fast-math; the one fused multiply-add is an explicit fmaf),
+ * fp64 where stated. Rounding is RNE throughout.
  *
  * Parity pins (tests/test_oracle_*.py): grid round trips and tie tables against a
  * brute-force nearest-value search, torch's float8 conversion, closed-form error
@@ -120,7 +121,10 @@ float orc_global_scale_f32(const float* a, int64_t n) {
 
 /* One 16-element group with tensor scale g, fp32 ops in this order:
  *   amax = max|a_i|;  g6 = 6*g;  s = amax / g6;  sf = E4M3(s);  d = dec(sf) * g;
- *   code_i = E2M1(a_i / d) if d > 0, else a signed zero;  deq_i = val(code_i) * d.
+ *   r = 1 / d;  code_i = E2M1(a_i * r) if d > 0, else a signed zero;
+ *   deq_i = val(code_i) * d.
+ * The scaled value is a_i times the group's reciprocal (one division per group, the
+ * usual form of a block-scaled quantizer), not a per-element division.
  * Writes 16 codes (one per byte, unpacked), the scale byte and the dequantized values. */
 static void nvfp4_group(const float* a, float g, uint8_t* codes, uint8_t* sf, float* deq) {
     float amax = 0.0f;
@@ -130,8 +134,9 @@ static void nvfp4_group(const float* a, float g, uint8_t* codes, uint8_t* sf, fl
     uint8_t sfc = orc_e4m3_encode(s_raw);
     float sd = (float)orc_e4m3_value(sfc);
     float d = sd * g;
+    float r = (d > 0.0f) ? 1.0f / d : 0.0f;
     for (int i = 0; i < 16; ++i) {
-        uint8_t c = (d > 0.0f) ? orc_e2m1_encode(a[i] / d) : (uint8_t)(signbit(a[i]) ? 8 : 0);
+        uint8_t c = (d > 0.0f) ? orc_e2m1_encode(a[i] * r) : (uint8_t)(signbit(a[i]) ? 8 : 0);
         codes[i] = c;
         deq[i] = (float)orc_e2m1_value(c) * d;
     }
@@ -225,6 +230,12 @@ void orc_hessian_diag(const uint16_t* Xcal, int T, int K, float* H) {
 }
 
 /* Pairwise tree over 64 values: v[i] += v[i+32] (i<32), then +16, +8, +4, +2, +1. */
+static float tree64f(float* v) {
+    for (int h = 32; h >= 1; h >>= 1)
+        for (int i = 0; i < h; ++i) v[i] = v[i] + v[i + h];
+    return v[0];
+}
+
 static double tree64(double* v) {
     for (int h = 32; h >= 1; h >>= 1)
         for (int i = 0; i < h; ++i) v[i] = v[i] + v[i + h];
@@ -235,10 +246,10 @@ static double tree64(double* v) {
  * Delta-score (A3) for every 64x64 block b = nt*(K/64) + kt:
  *   e   = R = fp32(W - deq Q(W))            (base quantization error)
  *   e'  = fp32(R - deq R)                   (error left after the residual)
- *   tau = fp64(e)^2 - fp64(e')^2            (squares exact in fp64)
- *   c_k = tree64 over the block's 64 rows of tau
- *   p_k = fp64(H_k) * c_k
- *   Delta_b = tree64 over the block's 64 columns of p_k
+ *   tau = fp32( e*e - fp32(e'*e') )         (one fused multiply-add, fp32)
+ *   c_k = tree64 over the block's 64 rows of tau, in fp32
+ *   p_k = fp64(H_k) * fp64(c_k)
+ *   Delta_b = tree64 over the block's 64 columns of p_k, in fp64
  */
 void orc_delta_score(const uint16_t* W, int N, int K, const float* H, const uint8_t* base_codes,
                      const uint8_t* base_sf, float g_w, const uint8_t* res_codes, const uint8_t* res_sf,
@@ -252,16 +263,18 @@ void orc_delta_score(const uint16_t* W, int N, int K, const float* H, const uint
 #pragma omp parallel for schedule(static)
     for (int b = 0; b < NBr * KB; ++b) {
         int nt = b / KB, kt = b % KB;
-        double p[64], col[64];
+        double p[64];
+        float col[64];
         for (int c = 0; c < 64; ++c) {
             int k = kt * 64 + c;
             for (int r = 0; r < 64; ++r) {
                 int64_t i = (int64_t)(nt * 64 + r) * K + k;
                 float e = bf16_to_f32(W[i]) - dq[i];
                 float e2 = e - dr[i];
-                col[r] = (double)e * (double)e - (double)e2 * (double)e2;
+                float e2sq = e2 * e2;
+                col[r] = fmaf(e, e, -e2sq);
             }
-            p[c] = (double)H[k] * tree64(col);
+            p[c] = (double)H[k] * (double)tree64f(col);
         }
         delta[b] = tree64(p);
     }

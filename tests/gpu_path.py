@@ -13,15 +13,16 @@ def to_dev(bits: np.ndarray, dev) -> torch.Tensor:
     return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
 
 
-def gpu_run(L: dict, budget: int, dev, flags: int = 0, X_bits=None):
-    """Whole path on the GPU for layer inputs L (bf16 bits); returns numpy copies."""
+def gpu_run(L: dict, budget: int, dev, flags: int = 0, X_bits=None, fused: bool = False):
+    """Whole path on the GPU for layer inputs L (bf16 bits); returns numpy copies.
+    fused=True quantizes and scores W in one pass (mq_quantize_weight_delta)."""
     from bit_quantized_gemm_zipperengine_b200 import mosaic
     N, K = L["N"], L["K"]
     W = to_dev(L["W"], dev)
     Xc = to_dev(L["Xcal"], dev)
     X = to_dev(L["X"] if X_bits is None else X_bits, dev)
     layer = mosaic.Layer(N, K, budget, dev)
-    layer.prepare(W, Xc)
+    (layer.prepare_fused if fused else layer.prepare)(W, Xc)
     Y = layer.forward(X, flags)
     xq = layer.act_buffers(X.shape[0], flags)[0]
     torch.cuda.synchronize()

@@ -41,9 +41,10 @@ def test_size_helpers(L):
     assert L.mq_budget_blocks(28672, 8192, 0.05) == 2867
     assert L.mq_budget_blocks(256, 512, 1.5) == -1
     assert L.mq_quantize_weight_workspace_bytes(4096, 4096) >= 4 * 148 * 8
-    # decode GEMM at M=16, N=K=4096: 32 weight tiles x 4 K splits -> fp32 partials + counters
-    ws = L.mq_gemm_workspace_bytes(16, 4096, 4096, 0)
-    assert ws == 4 * 16 * 4096 * 4 + 32 * 4
+    # decode GEMM at M=16, N=K=4096: 32 weight tiles x 4 K splits reduced inside a cluster
+    assert L.mq_gemm_workspace_bytes(16, 4096, 4096, 0) == 0
+    # a narrow layer (8 weight tiles) splits K 16 ways: fp32 partials + tile counters
+    assert L.mq_gemm_workspace_bytes(16, 1024, 4096, 0) == 16 * 16 * 1024 * 4 + 8 * 4
 
 
 def test_host_validation_rejects_bad_arguments(L):
@@ -60,6 +61,8 @@ def test_host_validation_rejects_bad_arguments(L):
     wm2 = mosaic.NVFP4Mat(4096, 4096, fake, None, fake, fake)
     assert L.mq_gemm(ctypes.byref(xm), ctypes.byref(wm2), None, fake, 16, 4096, 4096,
                      mosaic.MQ_GEMM_BASE_ONLY | mosaic.MQ_GEMM_RESIDUAL_ONLY, None, 0, None) == 1
-    # decode split-K needs its workspace
-    assert L.mq_gemm(ctypes.byref(xm), ctypes.byref(wm2), None, fake, 16, 4096, 4096, 0, None, 0, None) == 3
+    # a split-K problem on the workspace path needs its workspace
+    xm1 = mosaic.NVFP4Mat(16, 4096, fake, None, fake, fake)
+    wm1 = mosaic.NVFP4Mat(1024, 4096, fake, None, fake, fake)
+    assert L.mq_gemm(ctypes.byref(xm1), ctypes.byref(wm1), None, fake, 16, 1024, 4096, 0, None, 0, None) == 3
     assert L.mq_status_string(3) == b"workspace missing or too small"

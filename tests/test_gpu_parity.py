@@ -20,23 +20,28 @@ def dev():
 
 
 _cache = {}
+_oracle = {}
 
 
-def _pair(name, dev, M=None):
-    key = (name, M)
+def _pair(name, dev, M=None, fused=False):
+    key = (name, M, fused)
     if key not in _cache:
         L = synth.layer(name, M=M)
         budget = synth.budget_blocks(L["N"], L["K"], 0.10)
-        _cache[key] = (L, budget, gpu_run(L, budget, dev), oracle_ref(L, budget))
+        if (name, M) not in _oracle:
+            _oracle[(name, M)] = oracle_ref(L, budget)
+        _cache[key] = (L, budget, gpu_run(L, budget, dev, fused=fused), _oracle[(name, M)])
     return _cache[key]
 
 
 WORKLOADS = ["tiny", "llama3_8b_qproj_decode"]
+PATHS = [pytest.param(False, id="separate"), pytest.param(True, id="fused")]
 
 
+@pytest.mark.parametrize("fused", PATHS)
 @pytest.mark.parametrize("name", WORKLOADS)
-def test_quantize_weight_bit_exact(name, dev):
-    L, budget, g, o = _pair(name, dev)
+def test_quantize_weight_bit_exact(name, fused, dev):
+    L, budget, g, o = _pair(name, dev, fused=fused)
     wq = o["wq"]
     assert g["g"] == wq["g"]
     assert np.array_equal(g["codes"], wq["codes"])
@@ -46,23 +51,26 @@ def test_quantize_weight_bit_exact(name, dev):
     assert np.array_equal(g["r_sf"], wq["r_sf"])
 
 
+@pytest.mark.parametrize("fused", PATHS)
 @pytest.mark.parametrize("name", WORKLOADS)
-def test_hessian_bit_exact(name, dev):
-    L, budget, g, o = _pair(name, dev)
+def test_hessian_bit_exact(name, fused, dev):
+    L, budget, g, o = _pair(name, dev, fused=fused)
     assert np.array_equal(g["H"].view(np.uint32), o["H"].view(np.uint32))
 
 
+@pytest.mark.parametrize("fused", PATHS)
 @pytest.mark.parametrize("name", WORKLOADS)
-def test_delta_and_selection_bit_exact(name, dev):
-    L, budget, g, o = _pair(name, dev)
+def test_delta_and_selection_bit_exact(name, fused, dev):
+    L, budget, g, o = _pair(name, dev, fused=fused)
     assert np.array_equal(g["delta"].view(np.uint64), o["delta"].view(np.uint64))
     assert np.array_equal(g["rank"], o["rank"])
     assert np.array_equal(g["sel"], o["sel"])
 
 
+@pytest.mark.parametrize("fused", PATHS)
 @pytest.mark.parametrize("name", WORKLOADS)
-def test_pack_bit_exact(name, dev):
-    L, budget, g, o = _pair(name, dev)
+def test_pack_bit_exact(name, fused, dev):
+    L, budget, g, o = _pair(name, dev, fused=fused)
     for k in ("blk_codes", "blk_sf", "blk_kt", "tile_ptr"):
         assert np.array_equal(g["packed"][k], o["packed"][k]), k
     assert np.array_equal(g["packed"]["bitmap"].view(np.uint32), o["packed"]["bitmap"])
@@ -77,9 +85,10 @@ def test_quantize_act_bit_exact(name, dev):
     assert np.array_equal(g["xq_swz"], oracle.sf_tile(xq["sf"], L["M"], L["K"]))
 
 
+@pytest.mark.parametrize("fused", PATHS)
 @pytest.mark.parametrize("name", WORKLOADS)
-def test_gemm_fused_within_tolerance(name, dev):
-    L, budget, g, o = _pair(name, dev)
+def test_gemm_fused_within_tolerance(name, fused, dev):
+    L, budget, g, o = _pair(name, dev, fused=fused)
     check_gemm(g["Y"], o["y"], o["yabs"], name)
 
 
@@ -93,6 +102,23 @@ def test_gemm_ragged_token_counts(M, dev):
     o = oracle_ref(L, budget)
     assert np.array_equal(g["xq_codes"], o["xq"]["codes"])
     check_gemm(g["Y"], o["y"], o["yabs"], f"M={M}")
+
+
+@pytest.mark.parametrize("M", [16, 100, 128])
+def test_gemm_narrow_layer_workspace_split_k(M, dev):
+    """A 1024 x 4096 layer: 8 weight tiles, so K is split 16 ways and the partials are
+    added through the global workspace (the path above the cluster size)."""
+    from bit_quantized_gemm_zipperengine_b200 import mosaic
+    N, K = 1024, 4096
+    L = {"N": N, "K": K, "M": M, "T": 128,
+         "W": synth.weight(N, K, 801, 804, 0.02, int(0.005 * N * K), 51, 20.0),
+         "X": synth.act(M, K, 802, 804, 40, 30.0), "Xcal": synth.act(128, K, 803, 804, 40, 30.0)}
+    budget = synth.budget_blocks(N, K, 0.10)
+    assert mosaic.lib().mq_gemm_workspace_bytes(M, N, K, 0) > 0
+    g = gpu_run(L, budget, dev, fused=True)
+    o = oracle_ref(L, budget)
+    assert np.array_equal(g["sel"], o["sel"])
+    check_gemm(g["Y"], o["y"], o["yabs"], f"narrow M={M}")
 
 
 def test_gemm_base_only_paths_identical(dev):
@@ -142,3 +168,50 @@ def test_repeat_calls_deterministic(dev):
         assert np.array_equal(g[k], g2[k]), k
     assert np.array_equal(g["delta"].view(np.uint64), g2["delta"].view(np.uint64))
     assert np.array_equal(g["Y"], g2["Y"])
+
+
+def test_topk_blocks_alone_and_large_budgets(dev):
+    """A4 alone on many blocks and budgets (in-CTA rank and the separate rank kernel,
+    shared-memory and global keys), with ties, against the oracle's sort."""
+    from bit_quantized_gemm_zipperengine_b200 import mosaic
+    rng = np.random.default_rng(12)
+    for B, budgets in ((32, (0, 1, 3, 32)), (4096, (409, 1024, 1025)), (57344, (2867, 11468))):
+        d = rng.standard_normal(B) * np.exp2(rng.integers(-20, 5, B))
+        d[rng.choice(B, B // 10, replace=False)] = 0.0      # ties at zero
+        d[rng.choice(B, B // 50, replace=False)] = d[0]     # ties at an arbitrary value
+        d[:3] = -0.0
+        dd = torch.from_numpy(d).to(dev)
+        for k in budgets:
+            rank = torch.empty(max(k, 1), dtype=torch.int32, device=dev)
+            sel = torch.empty(max(k, 1), dtype=torch.int32, device=dev)
+            mosaic.mq_topk_blocks(dd, k, rank, sel)
+            torch.cuda.synchronize()
+            r_ref, s_ref = oracle.topk(d, k)
+            assert np.array_equal(rank[:k].cpu().numpy(), r_ref), (B, k)
+            assert np.array_equal(sel[:k].cpu().numpy(), s_ref), (B, k)
+
+
+@pytest.mark.parametrize("host", [False, True])
+def test_run_layer_whole_path(host, dev):
+    """mq_run_layer (the whole path in one C call), with device buffers and with pinned
+    host buffers copied inside the call, against the oracle."""
+    from bit_quantized_gemm_zipperengine_b200 import mosaic
+    L = synth.layer("llama3_8b_qproj_decode")
+    M, N, K, T = L["M"], L["N"], L["K"], L["T"]
+    budget = synth.budget_blocks(N, K, 0.10)
+    o = _oracle.get(("llama3_8b_qproj_decode", None)) or oracle_ref(L, budget)
+    layer = mosaic.Layer(N, K, budget, dev, with_sf=False)
+    buf = layer.buffers(M, T, staging=host)
+    if host:
+        W = torch.from_numpy(L["W"].view(np.int16)).view(torch.bfloat16).pin_memory()
+        X = torch.from_numpy(L["X"].view(np.int16)).view(torch.bfloat16).pin_memory()
+        C = torch.from_numpy(L["Xcal"].view(np.int16)).view(torch.bfloat16).pin_memory()
+        Y = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
+    else:
+        W, X, C = to_dev(L["W"], dev), to_dev(L["X"], dev), to_dev(L["Xcal"], dev)
+        Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    mosaic.mq_run_layer(W, X, C, Y, M, N, K, T, budget, 0, host, buf)
+    torch.cuda.synchronize()
+    assert mosaic.mq_get_error() == 0
+    assert np.array_equal(layer.sel[:budget].cpu().numpy(), o["sel"])
+    check_gemm(Y.float().cpu().numpy().astype(np.float64), o["y"], o["yabs"], f"run_layer host={host}")

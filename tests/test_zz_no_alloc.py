@@ -26,11 +26,22 @@ def dev():
     return torch.device("cuda:0")
 
 
-@pytest.mark.parametrize("name,M", [("llama3_8b_qproj_decode", 16), ("tiny", 37)])
-def test_noalloc_matches_workspace_gemm_twice(name, M, dev):
+def _narrow_layer(M):
+    """A 1024 x 4096 layer: 8 weight tiles, so the decode GEMM splits K 16 ways and its
+    partials go through scratch memory (the case this entry point exists for)."""
+    N, K = 1024, 4096
+    return {"N": N, "K": K, "M": M, "T": 128,
+            "W": synth.weight(N, K, 901, 904, 0.02, int(0.005 * N * K), 51, 20.0),
+            "X": synth.act(M, K, 902, 904, 40, 30.0), "Xcal": synth.act(128, K, 903, 904, 40, 30.0)}
+
+
+@pytest.mark.parametrize("M", [16, 64])
+def test_noalloc_matches_workspace_gemm_twice(M, dev):
     from bit_quantized_gemm_zipperengine_b200 import mosaic
-    L = synth.layer(name, M=M)
+    L = _narrow_layer(M)
     N, K = L["N"], L["K"]
+    name = f"narrow M={M}"
+    assert mosaic.lib().mq_gemm_workspace_bytes(M, N, K, 0) > 0  # the scratch is really used
     budget = synth.budget_blocks(N, K, 0.10)
     layer = mosaic.Layer(N, K, budget, dev)
     layer.prepare(to_dev(L["W"], dev), to_dev(L["Xcal"], dev))
@@ -55,11 +66,11 @@ def test_noalloc_refuses_problems_beyond_the_static_scratch(dev):
     Lb = mosaic.lib()
     limit = Lb.mq_gemm_noalloc_scratch_limit()
     assert limit == 8 << 20
-    # M=128, N=5120, K=25600 needs 3 splits x 128 x 5120 fp32 partials = 7.5 MiB (fits);
-    # M=128, N=9216, K=25600 needs 2 x 128 x 9216 x 4 B = 9 MiB and must be refused
-    # before any launch.
-    assert Lb.mq_gemm_workspace_bytes(128, 5120, 25600, 0) <= limit
-    M, N, K = 128, 9216, 25600
+    # M=16, N=1024, K=16384 needs 16 splits x 16 x 1024 fp32 partials = 1 MiB (fits);
+    # M=128, N=1024, K=16384 needs 16 x 128 x 1024 x 4 B = 8 MiB plus the tile counters
+    # and must be refused before any launch.
+    assert 0 < Lb.mq_gemm_workspace_bytes(16, 1024, 16384, 0) <= limit
+    M, N, K = 128, 1024, 16384
     assert Lb.mq_gemm_workspace_bytes(M, N, K, 0) > limit
     fake = ctypes.c_void_p(0x10000)
     xm = mosaic.NVFP4Mat(M, K, fake, None, fake, fake)
