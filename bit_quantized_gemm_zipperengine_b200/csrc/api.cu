@@ -16,11 +16,11 @@ cudaError_t launch_quant_weight(const uint16_t* W, int N, int K, uint8_t* codes,
 cudaError_t launch_quant_act(const uint16_t* X, int M, int K, uint8_t* codes, uint8_t* sf, uint8_t* sf_swz,
                              float* g, cudaStream_t s);
 cudaError_t launch_hessian(const uint16_t* X, int T, int K, float* H, cudaStream_t s);
-cudaError_t launch_delta(const uint16_t* W, int N, int K, const float* H, const float* g, double* delta,
-                         cudaStream_t s);
-cudaError_t launch_quant_delta(const uint16_t* W, int N, int K, const float* H, uint8_t* codes, uint8_t* sf,
-                               uint8_t* sf_swz, float* g, uint8_t* rcodes, uint8_t* rsf, double* delta,
-                               float* partial, cudaStream_t s);
+cudaError_t launch_delta(const CUtensorMap& tw, int N, int K, const float* H, const float* g, double* delta,
+                         int* err, cudaStream_t s);
+cudaError_t launch_quant_delta(const uint16_t* W, const CUtensorMap& tw, int N, int K, const float* H,
+                               uint8_t* codes, uint8_t* sf, uint8_t* sf_swz, float* g, uint8_t* rcodes, uint8_t* rsf,
+                               double* delta, float* partial, int* err, cudaStream_t s);
 cudaError_t launch_topk(const double* delta, int B, int budget, int32_t* rank, int32_t* sel, cudaStream_t s);
 cudaError_t launch_pack(const uint8_t* rcodes, const uint8_t* rsf, int N, int K, const int32_t* sel, int budget,
                         uint8_t* blk_codes, uint8_t* blk_sf, int32_t* blk_kt, int32_t* tile_ptr, uint32_t* bitmap,
@@ -64,6 +64,33 @@ static bool make_tmap_bytes(CUtensorMap* map, const void* base, uint64_t row_byt
     return r == CUDA_SUCCESS;
 }
 
+// bf16 matrix [rows][cols] in 64 x 64 boxes with the 128-byte swizzle (one Delta block).
+static bool make_tmap_bf16_blocks(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * 2};
+    cuuint32_t box[2] = {64, 64};
+    cuuint32_t es[2] = {1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<void*>(base), dims, strides, box, es,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// Device address of the library's error word (looked up once per device).
+static int* err_word() {
+    static int* ptrs[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    if (!ptrs[dev]) {
+        int* p = nullptr;
+        if (error_word(&p) != cudaSuccess) return nullptr;
+        ptrs[dev] = p;
+    }
+    return ptrs[dev];
+}
+
 static inline cudaStream_t as_stream(mq_stream s) { return reinterpret_cast<cudaStream_t>(s); }
 
 static inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
@@ -103,9 +130,11 @@ size_t mq_delta_topk_workspace_bytes(int N, int K, int budget) {
 }
 
 size_t mq_gemm_workspace_bytes(int M, int N, int K, unsigned flags) {
-    (void)flags;
     if (M <= 0 || N <= 0 || K <= 0 || N % 128 || K % 256) return 0;
-    return decode_workspace_bytes(M, N, K);
+    bool prefill = M > 128 && N % 256 == 0;
+    if (flags & MQ_GEMM_DECODE) prefill = false;
+    if (flags & MQ_GEMM_PREFILL) prefill = true;
+    return prefill ? 0 : decode_workspace_bytes(M, N, K);
 }
 
 mq_status mq_quantize_weight(const mq_bf16* W, int N, int K, mq_nvfp4_mat* base, mq_nvfp4_mat* resid_full,
@@ -142,7 +171,10 @@ mq_status mq_delta_score_topk(const mq_bf16* W, const float* H, const mq_nvfp4_m
     if (budget < 0 || budget > B) return MQ_ERR_INVALID_ARG;
     if (budget > 0 && (!rank || !sel)) return MQ_ERR_INVALID_ARG;
     cudaStream_t s = as_stream(stream);
-    cudaError_t e = launch_delta(W, N, K, H, base->gscale, delta, s);
+    CUtensorMap tw;
+    int* err = err_word();
+    if (!err || !make_tmap_bf16_blocks(&tw, W, (uint64_t)K, (uint64_t)N)) return MQ_ERR_CUDA;
+    cudaError_t e = launch_delta(tw, N, K, H, base->gscale, delta, err, s);
     if (e != cudaSuccess) return MQ_ERR_CUDA;
     g_launches.fetch_add(1);
     return launched(launch_topk(delta, B, budget, rank, sel, s), budget <= 0 ? 0 : budget <= 1024 ? 1 : 2);
@@ -160,8 +192,12 @@ mq_status mq_quantize_weight_delta(const mq_bf16* W, int N, int K, const float* 
         !aligned(resid_full->sf, 4) || (base->sf && !aligned(base->sf, 4)))
         return MQ_ERR_INVALID_ARG;
     if (!ws || ws_bytes < mq_quantize_weight_workspace_bytes(N, K)) return MQ_ERR_WORKSPACE;
-    cudaError_t e = launch_quant_delta(W, N, K, H, base->codes, base->sf, base->sf_swz, base->gscale, resid_full->codes,
-                                       resid_full->sf, delta, static_cast<float*>(ws), as_stream(stream));
+    CUtensorMap tw;
+    int* err = err_word();
+    if (!err || !make_tmap_bf16_blocks(&tw, W, (uint64_t)K, (uint64_t)N)) return MQ_ERR_CUDA;
+    cudaError_t e = launch_quant_delta(W, tw, N, K, H, base->codes, base->sf, base->sf_swz, base->gscale,
+                                       resid_full->codes, resid_full->sf, delta, static_cast<float*>(ws), err,
+                                       as_stream(stream));
     return launched(e, 2);
 }
 
@@ -210,14 +246,13 @@ mq_status mq_gemm(const mq_nvfp4_mat* xq, const mq_nvfp4_mat* wq, const mq_resid
             return MQ_ERR_INVALID_ARG;
         if (!aligned(r->blk_codes, 16) || !aligned(r->blk_sf, 16)) return MQ_ERR_INVALID_ARG;
     }
-    DecodePlan d = plan_decode(M, N, K);
-    const size_t need = decode_workspace_bytes(M, N, K);
-    if (need > 0 && (!ws || ws_bytes < need || !aligned(ws, 16))) return MQ_ERR_WORKSPACE;
-
-    CUtensorMap tw, tx;
-    if (!make_tmap_bytes(&tw, wq->codes, (uint64_t)K / 2, (uint64_t)N, 128, 128)) return MQ_ERR_CUDA;
-    if (!make_tmap_bytes(&tx, xq->codes, (uint64_t)K / 2, (uint64_t)M, 128, (uint32_t)d.BN)) return MQ_ERR_CUDA;
-
+    // kernel choice: the prefill kernel tiles 256 weight rows, the decode kernel 128
+    bool prefill = M > 128 && N % 256 == 0;
+    if (flags & MQ_GEMM_DECODE) prefill = false;
+    if (flags & MQ_GEMM_PREFILL) {
+        if (N % 256) return MQ_ERR_UNSUPPORTED_SHAPE;
+        prefill = true;
+    }
     GemmParams p;
     memset(&p, 0, sizeof p);
     p.w_sf = wq->sf_swz;
@@ -236,6 +271,17 @@ mq_status mq_gemm(const mq_nvfp4_mat* xq, const mq_nvfp4_mat* wq, const mq_resid
     p.N = N;
     p.K = K;
     p.mode = (flags & MQ_GEMM_BASE_ONLY) ? 1 : (flags & MQ_GEMM_RESIDUAL_ONLY) ? 2 : 0;
+    CUtensorMap tw, tx;
+    if (prefill) {
+        if (!make_tmap_bytes(&tw, wq->codes, (uint64_t)K / 2, (uint64_t)N, 128, 256)) return MQ_ERR_CUDA;
+        if (!make_tmap_bytes(&tx, xq->codes, (uint64_t)K / 2, (uint64_t)M, 128, 128)) return MQ_ERR_CUDA;
+        return launched(launch_gemm_prefill(tw, tx, p, as_stream(stream)), 1);
+    }
+    DecodePlan d = plan_decode(M, N, K);
+    const size_t need = decode_workspace_bytes(M, N, K);
+    if (need > 0 && (!ws || ws_bytes < need || !aligned(ws, 16))) return MQ_ERR_WORKSPACE;
+    if (!make_tmap_bytes(&tw, wq->codes, (uint64_t)K / 2, (uint64_t)N, 128, 128)) return MQ_ERR_CUDA;
+    if (!make_tmap_bytes(&tx, xq->codes, (uint64_t)K / 2, (uint64_t)M, 128, (uint32_t)d.BN)) return MQ_ERR_CUDA;
     if (need > 0) {
         size_t part = (size_t)d.splits * d.tiles_m * d.BN * N * sizeof(float);  // workspace path only
         part = (part + 255) & ~size_t(255);

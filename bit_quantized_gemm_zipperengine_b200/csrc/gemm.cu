@@ -394,6 +394,262 @@ __global__ void __launch_bounds__(192, 1)
     }
 }
 
+// ------------------------------------------------------------------ prefill kernel
+// Large M: the tokens are the MMA's M side (128 per tile, A = X) and the weight its N
+// side (256 rows per tile, B = W), K = 256 per pipeline stage. CTAs are persistent and
+// walk the tiles m-fastest, so CTAs running at the same time share W tiles through L2.
+// A selected residual block (64 weight rows x 64 K) is one N = 64 MMA written into its
+// 64-column slice of the same fp32 accumulator: exactly the block's work. Residual
+// blocks stream through their own ring of shared-memory slots.
+// Warps: 0 producer (TMA / bulk copies), 1 MMA issuer (one thread), 2-9 epilogue (two
+// warps per 32-lane quarter of tensor memory, 128 accumulator columns each). The
+// epilogue copies the accumulator to registers and releases it before scaling and
+// storing, so the next tile's MMAs overlap the stores.
+struct PrefillCfg {
+    static constexpr int kStages = 3;
+    static constexpr int kOffX = 0;                    // 128 rows x 128 B, swizzled
+    static constexpr int kOffW = 16384;                // 256 rows x 128 B, swizzled
+    static constexpr int kOffSFX = kOffW + 32768;      // 4 x 512 B
+    static constexpr int kOffSFW = kOffSFX + 2048;     // 2 row tiles x 4 x 512 B
+    static constexpr int kStageBytes = kOffSFW + 4096; // 55296
+    static constexpr int kRSlots = 8;                  // residual ring: 2048 B codes + 512 B scales
+    static constexpr int kRSlotBytes = 2560;
+    static constexpr int kOffRing = kStages * kStageBytes;
+    static constexpr int kCtrlOff = kOffRing + kRSlots * kRSlotBytes;
+    static constexpr int kCtrlBytes = 512;
+    static constexpr int kSmemBytes = kCtrlOff + kCtrlBytes + 1024;
+    static constexpr int kThreads = 320;
+    static constexpr uint32_t kTmemCols = 512;
+    static constexpr int kSfCol0 = 256;                // after the 256-column accumulator
+    static constexpr int kSfStageCols = 48;            // X: 4 x 4, W: 4 x 8
+    static constexpr int kRSfCol0 = kSfCol0 + kStages * kSfStageCols;
+    static_assert(kStageBytes % 1024 == 0, "stage alignment");
+    static_assert(kSmemBytes <= 232448, "shared memory budget");
+    static_assert(kRSfCol0 + kRSlots * 4 <= 512, "tensor memory budget");
+};
+
+// Which 64-column slices of a tile's accumulator receive an MMA (bit h: weight rows
+// 64h..64h+63)? All of them unless only the residual is computed, in which case a slice
+// is written only if its block row has selected blocks.
+__device__ __forceinline__ uint32_t prefill_tile_slices(const GemmParams& p, int n_tile) {
+    if (p.mode != 2) return 0xFu;
+    if (!p.has_resid) return 0u;
+    uint32_t m = 0;
+    for (int h = 0; h < 4; ++h)
+        if (__ldg(p.tile_ptr + n_tile * 4 + h + 1) > __ldg(p.tile_ptr + n_tile * 4 + h)) m |= 1u << h;
+    return m;
+}
+
+__global__ void __launch_bounds__(320, 1)
+    k_gemm_prefill(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
+                   const GemmParams p) {
+    using C = PrefillCfg;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kCtrlOff);
+    uint64_t* empty = full + C::kStages;
+    uint64_t* rfull = empty + C::kStages;
+    uint64_t* rempty = rfull + C::kRSlots;
+    uint64_t* accf = rempty + C::kRSlots;
+    uint64_t* acce = accf + 1;
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(acce + 1);
+    uint32_t* rmask = tmem_holder + 1;  // [kStages]: bit 4*kk + h
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int KS = p.K / 256, KS64 = p.K / 64;
+    const int tiles_m = (p.M + 127) / 128, tiles_n = p.N / 256;
+    const int ntiles = tiles_m * tiles_n;
+
+    if (warp == 0 && lane == 0) {
+        for (int s = 0; s < C::kStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int r = 0; r < C::kRSlots; ++r) {
+            mbar_init(&rfull[r], 1);
+            mbar_init(&rempty[r], 1);
+        }
+        mbar_init(accf, 1);
+        mbar_init(acce, 8);
+        mbar_fence_init();
+        tma_prefetch_desc(&tmap_w);
+        tma_prefetch_desc(&tmap_x);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_holder, C::kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ------------------------------------------------ producer
+            griddep_wait();
+            int sc = 0, rc = 0;  // stage and residual-slot use counters
+            bool ok = true;
+            for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+                const int m_tile = t % tiles_m, n_tile = t / tiles_m;
+                RowCursor cur[4];
+                if (p.has_resid)
+#pragma unroll
+                    for (int h = 0; h < 4; ++h) cur[h] = row_cursor(p, n_tile * 4 + h, 0);
+                for (int ks = 0; ks < KS && ok; ++ks, ++sc) {
+                    const int s = sc % C::kStages;
+                    if (!mbar_wait(&empty[s], ((sc / C::kStages) & 1) ^ 1)) { ok = false; break; }
+                    uint32_t m = 0;
+                    int idx[4][4];
+                    if (p.has_resid)
+#pragma unroll
+                        for (int h = 0; h < 4; ++h) {
+                            const uint32_t mb = row_step(cur[h], ks * 4, idx[h]);
+#pragma unroll
+                            for (int kk = 0; kk < 4; ++kk) m |= ((mb >> kk) & 1u) << (4 * kk + h);
+                        }
+                    rmask[s] = m;
+                    uint8_t* st = smem + s * C::kStageBytes;
+                    mbar_arrive_expect_tx(&full[s], 16384 + 32768 + 2048 + 4096);
+                    tma_load_2d(st + C::kOffX, &tmap_x, &full[s], ks * 128, m_tile * 128);
+                    tma_load_2d(st + C::kOffW, &tmap_w, &full[s], ks * 128, n_tile * 256);
+                    bulk_load(st + C::kOffSFX, p.x_sf + ((int64_t)m_tile * KS64 + ks * 4) * 512, 2048, &full[s]);
+#pragma unroll
+                    for (int h2 = 0; h2 < 2; ++h2)
+                        bulk_load(st + C::kOffSFW + h2 * 2048,
+                                  p.w_sf + ((int64_t)(n_tile * 2 + h2) * KS64 + ks * 4) * 512, 2048, &full[s]);
+                    // residual blocks of this stage, in (kk, h) order
+#pragma unroll 1
+                    for (int j = 0; j < 16 && ok; ++j) {
+                        if (!((m >> j) & 1u)) continue;
+                        const int kk = j >> 2, h = j & 3;
+                        const int r = rc % C::kRSlots;
+                        if (!mbar_wait(&rempty[r], ((rc / C::kRSlots) & 1) ^ 1)) { ok = false; break; }
+                        uint8_t* slot = smem + C::kOffRing + r * C::kRSlotBytes;
+                        const int bi = idx[h][kk];
+                        mbar_arrive_expect_tx(&rfull[r], 2560);
+                        bulk_load(slot, p.blk_codes + (int64_t)bi * 2048, 2048, &rfull[r]);
+                        bulk_load(slot + 2048, p.blk_sf + (int64_t)bi * 512, 512, &rfull[r]);
+                        ++rc;
+                    }
+                }
+            }
+            // Do not leave while copies into this CTA's shared memory are in flight:
+            // wait for the last uses of every stage and residual slot.
+            for (int u = max(0, sc - C::kStages); u < sc; ++u) mbar_wait(&full[u % C::kStages], (u / C::kStages) & 1);
+            for (int u = max(0, rc - C::kRSlots); u < rc; ++u) mbar_wait(&rfull[u % C::kRSlots], (u / C::kRSlots) & 1);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // ------------------------------------------------ MMA issuer
+            constexpr uint32_t idesc_d = idesc_mxf4nvf4(128, 256);
+            constexpr uint32_t idesc_r = idesc_mxf4nvf4(128, 64);
+            int sc = 0, rc = 0, tc = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++tc) {
+                if (!mbar_wait(acce, (tc & 1) ^ 1)) break;  // the epilogue has read the previous tile
+                tc_fence_after();
+                uint32_t acc4 = 0;  // bit h: the tile's slice h already holds a partial sum
+                for (int ks = 0; ks < KS; ++ks, ++sc) {
+                    const int s = sc % C::kStages;
+                    if (!mbar_wait(&full[s], (sc / C::kStages) & 1)) { ok = false; break; }
+                    tc_fence_after();
+                    uint8_t* st = smem + s * C::kStageBytes;
+                    const uint32_t sfc = tmem + C::kSfCol0 + s * C::kSfStageCols;
+                    const uint32_t m = p.mode != 1 ? rmask[s] : 0u;
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk) {
+                        tc_cp_sf_chunk(sfc + 4 * kk, smem_desc(smem_u32(st + C::kOffSFX + kk * 512), 0, 128, 0));
+                        tc_cp_sf_chunk(sfc + 16 + 8 * kk, smem_desc(smem_u32(st + C::kOffSFW + kk * 512), 0, 128, 0));
+                        tc_cp_sf_chunk(sfc + 16 + 8 * kk + 4,
+                                       smem_desc(smem_u32(st + C::kOffSFW + 2048 + kk * 512), 0, 128, 0));
+                    }
+                    const uint32_t ax = smem_u32(st + C::kOffX), bw = smem_u32(st + C::kOffW);
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk) {
+                        const uint64_t adesc = smem_desc(ax + 32 * kk, 16, 1024, 2);
+                        if (p.mode != 2) {
+                            mma_mxf4nvf4(tmem, adesc, smem_desc(bw + 32 * kk, 16, 1024, 2), idesc_d, sfc + 4 * kk,
+                                         sfc + 16 + 8 * kk, acc4 == 0xFu);
+                            acc4 = 0xFu;
+                        }
+#pragma unroll 1
+                        for (int h = 0; h < 4; ++h) {
+                            if (!((m >> (4 * kk + h)) & 1u)) continue;
+                            const int r = rc % C::kRSlots;
+                            if (!mbar_wait(&rfull[r], (rc / C::kRSlots) & 1)) { ok = false; break; }
+                            tc_fence_after();
+                            uint8_t* slot = smem + C::kOffRing + r * C::kRSlotBytes;
+                            const uint32_t rsf = tmem + C::kRSfCol0 + 4 * r;
+                            tc_cp_sf_chunk(rsf, smem_desc(smem_u32(slot + 2048), 0, 128, 0));
+                            mma_mxf4nvf4(tmem + 64 * h, adesc, smem_desc(smem_u32(slot), 128, 256, 0), idesc_r,
+                                         sfc + 4 * kk, rsf + 2 * (h & 1), (acc4 >> h) & 1u);
+                            acc4 |= 1u << h;
+                            tc_commit(&rempty[r]);
+                            ++rc;
+                        }
+                        if (!ok) break;
+                    }
+                    // when the dense half was skipped a stage may carry no MMA: still release it
+                    tc_commit(&empty[s]);
+                    if (!ok) break;
+                }
+                tc_commit(accf);
+            }
+        }
+    } else {
+        // ---------------------------------------------------- epilogue (warps 2..9)
+        const int q = warp & 3, half = (warp - 2) >> 2;
+        griddep_wait();  // g_x and Y follow the previous kernel
+        const float gw = __ldg(p.g_w);
+        int tc = 0;
+        for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++tc) {
+            const int m_tile = t % tiles_m, n_tile = t / tiles_m;
+            const bool waited = mbar_wait(accf, tc & 1);
+            tc_fence_after();
+            const uint32_t slices = waited ? prefill_tile_slices(p, n_tile) : 0u;
+            float acc[128];
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                // columns 128*half + 16c .. +15 lie in slice 2*half + c/4
+                if ((slices >> (2 * half + (c >> 2))) & 1u) {
+                    tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + 128 * half + 16 * c, acc + 16 * c);
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) acc[16 * c + j] = 0.0f;
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(acce);  // accumulator free for the next tile
+            const int mm = m_tile * 128 + 32 * q + lane;
+            if (waited && mm < p.M) {
+                const float sc = __fmul_rn(__ldg(p.g_x + mm), gw);
+                uint16_t* yrow = p.Y + (int64_t)mm * p.N + n_tile * 256 + 128 * half;
+#pragma unroll
+                for (int c = 0; c < 16; ++c) {
+                    uint32_t w[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const __nv_bfloat16 lo = __float2bfloat16_rn(__fmul_rn(acc[8 * c + 2 * u], sc));
+                        const __nv_bfloat16 hi = __float2bfloat16_rn(__fmul_rn(acc[8 * c + 2 * u + 1], sc));
+                        w[u] = (uint32_t)(*reinterpret_cast<const uint16_t*>(&lo)) |
+                               ((uint32_t)(*reinterpret_cast<const uint16_t*>(&hi)) << 16);
+                    }
+                    *reinterpret_cast<uint4*>(yrow + 8 * c) = make_uint4(w[0], w[1], w[2], w[3]);
+                }
+            }
+            if (!waited) break;
+        }
+    }
+    griddep_launch();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::kTmemCols);
+    }
+}
+
 // ------------------------------------------------------------------ host side
 DecodePlan plan_decode(int M, int N, int K) {
     DecodePlan d;
@@ -447,6 +703,27 @@ cudaError_t launch_gemm_decode(const CUtensorMap& tw, const CUtensorMap& tx, Gem
         case 64: return launch_decode_bn<64>(tw, tx, p, d, s);
         default: return launch_decode_bn<128>(tw, tx, p, d, s);
     }
+}
+
+// Device address of the error word (for kernels of other translation units).
+cudaError_t error_word(int** ptr) { return cudaGetSymbolAddress(reinterpret_cast<void**>(ptr), g_error); }
+
+cudaError_t launch_gemm_prefill(const CUtensorMap& tw, const CUtensorMap& tx, const GemmParams& p, cudaStream_t s) {
+    static bool attr_set[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(k_gemm_prefill, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             PrefillCfg::kSmemBytes);
+        if (e != cudaSuccess) return e;
+        attr_set[dev] = true;
+    }
+    int sms = 148;
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int ntiles = ((p.M + 127) / 128) * (p.N / 256);
+    const int grid = ntiles < sms ? ntiles : sms;
+    return launch_pdl(k_gemm_prefill, dim3(grid), dim3(PrefillCfg::kThreads), PrefillCfg::kSmemBytes, s, 1, tw, tx,
+                      p);
 }
 
 cudaError_t read_clear_error(int* value) {

@@ -38,6 +38,8 @@ DecodePlan plan_decode(int M, int N, int K);
 size_t decode_workspace_bytes(int M, int N, int K);
 cudaError_t launch_gemm_decode(const CUtensorMap& tw, const CUtensorMap& tx, GemmParams p, const DecodePlan& d,
                                cudaStream_t s);
+cudaError_t launch_gemm_prefill(const CUtensorMap& tw, const CUtensorMap& tx, const GemmParams& p, cudaStream_t s);
 cudaError_t read_clear_error(int* value);
+cudaError_t error_word(int** ptr);
 
 }  // namespace mq

@@ -8,30 +8,45 @@
 namespace mq {
 
 // ------------------------------------------------------------------ Delta-score
-// One CTA (4 warps) per 64x64 block (nt, kt). Warp q owns group column q (16 K
-// elements); lane r owns block rows r and r+32, so the first level of the fixed
-// pairwise row tree (v[i] += v[i+32]) happens in registers. The remaining levels
-// (+16, +8, +4, +2, +1) run as a butterfly over the lanes that at each level also
-// halves the set of columns a lane keeps: the adds are exactly the tree's pairs, and
-// at the end lanes 2c and 2c+1 hold column c of the group. e and e' are recomputed
-// from W and the tensor scale with the weight quantizer's arithmetic, so they are
-// bit-identical to the stored codes. tau = fma(e, e, -fp32(e'^2)) (fp32); the column
-// sums are widened to fp64 for p_k = H_k c_k and the 64-column tree.
+// Persistent CTAs (4 warps) walk over the 64x64 blocks (nt, kt); TMA stages each block's
+// bf16 tile (64 rows x 128 bytes, 128-byte swizzle) into a ring of shared-memory buffers
+// ahead of the arithmetic. Warp q owns group column q (16 K elements); lane r owns block
+// rows r and r+32, so the first level of the fixed pairwise row tree (v[i] += v[i+32])
+// happens in registers. The remaining levels (+16, +8, +4, +2, +1) run as a butterfly
+// over the lanes that at each level also halves the set of columns a lane keeps: the
+// adds are exactly the tree's pairs, and at the end lanes 2c and 2c+1 hold column c of
+// the group. e and e' are recomputed from W and the tensor scale with the weight
+// quantizer's arithmetic, so they are bit-identical to the stored codes.
+// tau = fma(e, e, -fp32(e'^2)) (fp32); the column sums are widened to fp64 for
+// p_k = H_k c_k and the 64-column tree.
+constexpr int kQDStages = 3;
+constexpr int kQDTile = 64 * 128;  // bytes of one staged block
+
+// 16 values of row rl, group q of a staged tile (16-byte chunk c of a row sits at
+// chunk position c ^ (rl % 8): the TMA 128-byte swizzle).
+__device__ __forceinline__ void tile_group(const uint8_t* tile, int rl, int q, float (&a)[16]) {
+    const uint4* row = reinterpret_cast<const uint4*>(tile + rl * 128);
+    const uint4 v0 = row[(2 * q) ^ (rl & 7)], v1 = row[(2 * q + 1) ^ (rl & 7)];
+    const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        a[2 * i] = bf16_bits_to_f32(w[i] & 0xFFFFu);
+        a[2 * i + 1] = bf16_bits_to_f32(w[i] >> 16);
+    }
+}
+
 template <bool kWriteCodes>
-__device__ __forceinline__ void quant_delta_block(const uint16_t* __restrict__ W, int K, const float* __restrict__ H,
-                                                  float g, int nt, int kt, uint8_t* __restrict__ codes,
+__device__ __forceinline__ void quant_delta_block(const uint8_t* tile, int K, const float* __restrict__ H, float g,
+                                                  int nt, int kt, uint8_t* __restrict__ codes,
                                                   uint8_t* __restrict__ sf, uint8_t* __restrict__ sf_swz,
                                                   uint8_t* __restrict__ rcodes, uint8_t* __restrict__ rsf,
-                                                  double* __restrict__ delta_out) {
-    __shared__ double pcol[64];
-    __shared__ uint32_t sf_s[64], rsf_s[64];  // the 4 group scales of each block row
+                                                  double* __restrict__ delta_out, double* pcol, uint32_t* sf_s,
+                                                  uint32_t* rsf_s) {
     const int q = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const float g6 = __fmul_rn(6.0f, g);
-    // both rows' loads first, so 64 bytes per thread are in flight before any arithmetic
     float a2[2][16];
 #pragma unroll
-    for (int h = 0; h < 2; ++h)
-        load16_bf16(W + ((int64_t)nt * 64 + lane + 32 * h) * K + kt * 64 + q * 16, a2[h]);
+    for (int h = 0; h < 2; ++h) tile_group(tile, lane + 32 * h, q, a2[h]);
     float v[16];
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
@@ -91,31 +106,55 @@ __device__ __forceinline__ void quant_delta_block(const uint16_t* __restrict__ W
     }
 }
 
-// A3: Delta-score from W, H and the tensor scale (no codes written).
-__global__ void __launch_bounds__(128) k_delta(const uint16_t* __restrict__ W, int N, int K,
-                                               const float* __restrict__ H, const float* __restrict__ gptr,
-                                               double* __restrict__ delta) {
-    griddep_wait();
-    griddep_launch();
-    const int KB = K / 64, b = blockIdx.x;
-    quant_delta_block<false>(W, K, H, __ldg(gptr), b / KB, b % KB, nullptr, nullptr, nullptr, nullptr, nullptr,
-                             delta + b);
-}
-
-// A1 + A3 in one pass over W: base and residual codes/scales and the Delta-score of
-// every block, with the tensor scale from the |W| maximum pass.
-__global__ void __launch_bounds__(128) k_quant_delta(const uint16_t* __restrict__ W, int N, int K,
-                                                     const float* __restrict__ H, const float* __restrict__ partial,
+// A3 (kWriteCodes = false: Delta only, tensor scale read from g_in) and A1 + A3 in one
+// pass over W (kWriteCodes = true: codes, scales and Delta, tensor scale from the |W|
+// maximum partials). Persistent: CTA c handles blocks c, c + gridDim.x, ...
+template <bool kWriteCodes>
+__global__ void __launch_bounds__(128) k_quant_delta(const __grid_constant__ CUtensorMap tmap_w, int N, int K,
+                                                     const float* __restrict__ H, const float* __restrict__ g_in,
                                                      uint8_t* __restrict__ codes, uint8_t* __restrict__ sf,
                                                      uint8_t* __restrict__ sf_swz, float* __restrict__ g_out,
                                                      uint8_t* __restrict__ rcodes, uint8_t* __restrict__ rsf,
-                                                     double* __restrict__ delta) {
+                                                     double* __restrict__ delta, int* __restrict__ err) {
+    extern __shared__ uint8_t qd_raw[];
+    uint8_t* tiles = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(qd_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(tiles + kQDStages * kQDTile);
+    __shared__ double pcol[64];
+    __shared__ uint32_t sf_s[64], rsf_s[64];
     griddep_wait();
     griddep_launch();
-    const float g = tensor_scale(partial);
-    if (blockIdx.x == 0 && threadIdx.x == 0) *g_out = g;
-    const int KB = K / 64, b = blockIdx.x;
-    quant_delta_block<true>(W, K, H, g, b / KB, b % KB, codes, sf, sf_swz, rcodes, rsf, delta + b);
+    const float g = kWriteCodes ? tensor_scale(g_in) : __ldg(g_in);
+    if (kWriteCodes && blockIdx.x == 0 && threadIdx.x == 0) *g_out = g;
+    const int KB = K / 64, NB = (N / 64) * KB;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kQDStages; ++s) mbar_init(&full[s], 1);
+        mbar_fence_init();
+        tma_prefetch_desc(&tmap_w);
+    }
+    __syncthreads();
+    auto issue = [&](int i) {  // block number i of this CTA into stage i % kQDStages
+        const int b = blockIdx.x + i * gridDim.x;
+        if (b < NB) {
+            const int s = i % kQDStages;
+            mbar_arrive_expect_tx(&full[s], kQDTile);
+            tma_load_2d_u16(tiles + s * kQDTile, &tmap_w, &full[s], (b % KB) * 64, (b / KB) * 64);
+        }
+    };
+    if (threadIdx.x == 0)
+        for (int i = 0; i < kQDStages; ++i) issue(i);
+    bool ok = true;
+    for (int i = 0;; ++i) {
+        const int b = blockIdx.x + i * gridDim.x;
+        if (b >= NB) break;
+        const int s = i % kQDStages;
+        if (ok) ok = mbar_wait_err(&full[s], (i / kQDStages) & 1, err);
+        if (ok)
+            quant_delta_block<kWriteCodes>(tiles + s * kQDTile, K, H, g, b / KB, b % KB, codes, sf, sf_swz, rcodes,
+                                           rsf, delta + b, pcol, sf_s, rsf_s);
+        __syncthreads();  // stage s and the block's shared scratch are free again
+        // every copy issued here is waited for by a later iteration of this loop
+        if (threadIdx.x == 0 && ok) issue(i + kQDStages);
+    }
 }
 
 // ------------------------------------------------------------------ top-K
@@ -595,20 +634,39 @@ __global__ void __launch_bounds__(256) k_pack(const uint8_t* __restrict__ rcodes
 }
 
 // ------------------------------------------------------------------ launchers
-cudaError_t launch_delta(const uint16_t* W, int N, int K, const float* H, const float* g, double* delta,
-                         cudaStream_t s) {
-    const int B = (N / 64) * (K / 64);
-    return launch_pdl(k_delta, dim3(B), dim3(128), 0, s, 1, W, N, K, H, g, delta);
+static int quant_delta_grid(int NB) {
+    static int per_sm = 0;
+    if (!per_sm) {
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_quant_delta<true>, 128,
+                                                          kQDStages * kQDTile + 1024 + 64) != cudaSuccess ||
+            per_sm < 1)
+            per_sm = 4;
+    }
+    int sms = 148;
+    int dev = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int grid = per_sm * sms;
+    return NB < grid ? NB : grid;
 }
 
-cudaError_t launch_quant_delta(const uint16_t* W, int N, int K, const float* H, uint8_t* codes, uint8_t* sf,
-                               uint8_t* sf_swz, float* g, uint8_t* rcodes, uint8_t* rsf, double* delta,
-                               float* partial, cudaStream_t s) {
+static const size_t kQDSmem = kQDStages * kQDTile + 1024 + 64;
+
+cudaError_t launch_delta(const CUtensorMap& tw, int N, int K, const float* H, const float* g, double* delta,
+                         int* err, cudaStream_t s) {
+    const int NB = (N / 64) * (K / 64);
+    return launch_pdl(k_quant_delta<false>, dim3(quant_delta_grid(NB)), dim3(128), kQDSmem, s, 1, tw, N, K, H, g,
+                      (uint8_t*)nullptr, (uint8_t*)nullptr, (uint8_t*)nullptr, (float*)nullptr, (uint8_t*)nullptr,
+                      (uint8_t*)nullptr, delta, err);
+}
+
+cudaError_t launch_quant_delta(const uint16_t* W, const CUtensorMap& tw, int N, int K, const float* H,
+                               uint8_t* codes, uint8_t* sf, uint8_t* sf_swz, float* g, uint8_t* rcodes, uint8_t* rsf,
+                               double* delta, float* partial, int* err, cudaStream_t s) {
     cudaError_t e = launch_amax(W, (int64_t)N * K, partial, s);
     if (e != cudaSuccess) return e;
-    const int B = (N / 64) * (K / 64);
-    return launch_pdl(k_quant_delta, dim3(B), dim3(128), 0, s, 1, W, N, K, H, (const float*)partial, codes, sf,
-                      sf_swz, g, rcodes, rsf, delta);
+    const int NB = (N / 64) * (K / 64);
+    return launch_pdl(k_quant_delta<true>, dim3(quant_delta_grid(NB)), dim3(128), kQDSmem, s, 1, tw, N, K, H,
+                      (const float*)partial, codes, sf, sf_swz, g, rcodes, rsf, delta, err);
 }
 
 cudaError_t launch_topk(const double* delta, int B, int budget, int32_t* rank, int32_t* sel, cudaStream_t s) {

@@ -50,9 +50,9 @@ typedef enum {
 
 /* GEMM flags. */
 enum {
-    MQ_GEMM_AUTO = 0,          /* pick the decode or prefill kernel from M */
+    MQ_GEMM_AUTO = 0,          /* prefill kernel for M > 128 and N % 256 == 0, else decode */
     MQ_GEMM_DECODE = 1,        /* small-M kernel: W as the MMA's M side, split-K */
-    MQ_GEMM_PREFILL = 2,       /* large-M kernel: X as the MMA's M side */
+    MQ_GEMM_PREFILL = 2,       /* large-M kernel: X as the MMA's M side; needs N % 256 == 0 */
     MQ_GEMM_BASE_ONLY = 4,     /* skip the residual blocks (dense-only reference) */
     MQ_GEMM_RESIDUAL_ONLY = 8  /* only the residual blocks (linearity check) */
 };

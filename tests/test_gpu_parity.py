@@ -104,6 +104,51 @@ def test_gemm_ragged_token_counts(M, dev):
     check_gemm(g["Y"], o["y"], o["yabs"], f"M={M}")
 
 
+@pytest.mark.parametrize("M", [129, 256, 300, 1000])
+@pytest.mark.parametrize("flags_name", ["AUTO", "PREFILL", "DECODE"])
+def test_gemm_prefill_kernel(M, flags_name, dev):
+    """Large token counts through the prefill kernel (tokens as the MMA's M side, 256-row
+    weight tiles, N = 64 residual MMAs), with a ragged last token tile; the decode kernel
+    forced on the same inputs must agree with the oracle too."""
+    from bit_quantized_gemm_zipperengine_b200 import mosaic
+    N, K = 512, 1024
+    L = {"N": N, "K": K, "M": M, "T": 128,
+         "W": synth.weight(N, K, 701, 704, 0.02, int(0.005 * N * K), 6, 20.0),
+         "X": synth.act(M, K, 702, 704, 10, 30.0), "Xcal": synth.act(128, K, 703, 704, 10, 30.0)}
+    budget = synth.budget_blocks(N, K, 0.10)
+    flags = getattr(mosaic, "MQ_GEMM_" + flags_name)
+    g = gpu_run(L, budget, dev, flags=flags, fused=True)
+    o = oracle_ref(L, budget)
+    check_gemm(g["Y"], o["y"], o["yabs"], f"M={M} {flags_name}")
+
+
+def test_gemm_prefill_modes(dev):
+    """Prefill kernel: base-only equals the oracle's dense base; residual-only the
+    oracle's residual; r = NULL equals base-only bit for bit."""
+    from bit_quantized_gemm_zipperengine_b200 import mosaic
+    N, K, M = 512, 1024, 384
+    L = {"N": N, "K": K, "M": M, "T": 128,
+         "W": synth.weight(N, K, 711, 714, 0.02, int(0.005 * N * K), 6, 20.0),
+         "X": synth.act(M, K, 712, 714, 10, 30.0), "Xcal": synth.act(128, K, 713, 714, 10, 30.0)}
+    budget = synth.budget_blocks(N, K, 0.10)
+    g = gpu_run(L, budget, dev, fused=True)
+    o = oracle_ref(L, budget)
+    layer = g["layer"]
+    xq = layer.act_buffers(M)[0]
+    outs = {}
+    for name, flags, packed in (("base", mosaic.MQ_GEMM_BASE_ONLY, layer.packed), ("none", 0, None),
+                                ("resid", mosaic.MQ_GEMM_RESIDUAL_ONLY, layer.packed)):
+        Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        mosaic.mq_gemm(xq, layer.base, packed, Y, M, N, K, flags | mosaic.MQ_GEMM_PREFILL, None)
+        outs[name] = Y
+    torch.cuda.synchronize()
+    assert torch.equal(outs["base"], outs["none"])
+    yb, yba = oracle.gemm_rows(o["xq"], o["wq"], o["sel"], M, N, K, 1)
+    check_gemm(outs["base"].float().cpu().numpy().astype(np.float64), yb, yba, "prefill base only")
+    yr, yra = oracle.gemm_rows(o["xq"], o["wq"], o["sel"], M, N, K, 2)
+    check_gemm(outs["resid"].float().cpu().numpy().astype(np.float64), yr, yra, "prefill residual only")
+
+
 @pytest.mark.parametrize("M", [16, 100, 128])
 def test_gemm_narrow_layer_workspace_split_k(M, dev):
     """A 1024 x 4096 layer: 8 weight tiles, so K is split 16 ways and the partials are
