@@ -54,6 +54,25 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
     }
 }
 
+// One lane of a converged warp (the same lane every time the full warp calls it).
+__device__ __forceinline__ bool elect_one() {
+    uint32_t pred;
+    asm volatile(
+        "{\n\t.reg .pred P;\n\t.reg .b32 r;\n\t"
+        "elect.sync r|P, 0xffffffff;\n\t"
+        "selp.u32 %0, 1, 0, P;\n\t}"
+        : "=r"(pred));
+    return pred != 0;
+}
+
+// Bounded wait by a whole warp: all lanes poll, and leave together with lane 0's verdict.
+// Role loops (producer, MMA issuer) run converged and let one elected lane issue:
+// a loop run by a single lane of an otherwise waiting warp issues far more slowly.
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity) {
+    const bool ok = mbar_wait(bar, parity);
+    return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+}
+
 constexpr int kMaxSplits = 16;        // split-K factor bound of the decode plan
 constexpr int kMaxClusterSplits = 8;  // splits reduced through a thread-block cluster
 
@@ -171,117 +190,138 @@ __global__ void __launch_bounds__(192, 1)
     const uint32_t tmem = *tmem_holder;
 
     if (warp == 0) {
-        if (lane == 0) {
-            // ------------------------------------------------ producer
-            const uint8_t* xsf_tile = p.x_sf + (int64_t)(m0 / 128) * KS64 * 512;
-            const uint8_t* wsf_tile = p.w_sf + (int64_t)n_tile * KS64 * 512;
-            // W tile and W scales: written by earlier kernels, loaded before the wait
-            auto issue_w = [&](int it) {
-                const int st_i = it % C::kStages, ks = ks_begin + it;
-                uint8_t* st = smem + st_i * C::kStageBytes;
-                mbar_arrive_expect_tx(&full[st_i], 16384 + BN * 128 + 2048 + 2048);
-                tma_load_2d(st + C::kOffW, &tmap_w, &full[st_i], ks * 128, n0);
-                bulk_load(st + C::kOffSFW, wsf_tile + (int64_t)ks * 4 * 512, 2048, &full[st_i]);
-            };
-            // X tile and X scales: written by the previous kernel
-            auto issue_x = [&](int it) {
-                const int st_i = it % C::kStages, ks = ks_begin + it;
-                uint8_t* st = smem + st_i * C::kStageBytes;
-                tma_load_2d(st + C::kOffX, &tmap_x, &full[st_i], ks * 128, m0);
-                bulk_load(st + C::kOffSFX, xsf_tile + (int64_t)ks * 4 * 512, 2048, &full[st_i]);
-            };
-            RowCursor cur0, cur1;
-            auto issue_resid = [&](int it) {
-                const int s = it % C::kStages, ks = ks_begin + it;
-                uint8_t* st = smem + s * C::kStageBytes;
-                uint32_t m = 0;
-                int idx0[4] = {0, 0, 0, 0}, idx1[4] = {0, 0, 0, 0};
-                if (p.has_resid) {
-                    const uint32_t m0b = row_step(cur0, ks * 4, idx0);
-                    const uint32_t m1b = row_step(cur1, ks * 4, idx1);
+        // ---------------------------------------------------- producer (converged warp, one lane issues)
+        const uint8_t* xsf_tile = p.x_sf + (int64_t)(m0 / 128) * KS64 * 512;
+        const uint8_t* wsf_tile = p.w_sf + (int64_t)n_tile * KS64 * 512;
+        // W tile and W scales: written by earlier kernels, loaded before the wait
+        auto issue_w = [&](int it) {
+            const int st_i = it % C::kStages, ks = ks_begin + it;
+            uint8_t* st = smem + st_i * C::kStageBytes;
+            mbar_arrive_expect_tx(&full[st_i], 16384 + BN * 128 + 2048 + 2048);
+            tma_load_2d(st + C::kOffW, &tmap_w, &full[st_i], ks * 128, n0);
+            bulk_load(st + C::kOffSFW, wsf_tile + (int64_t)ks * 4 * 512, 2048, &full[st_i]);
+        };
+        // X tile and X scales: written by the previous kernel
+        auto issue_x = [&](int it) {
+            const int st_i = it % C::kStages, ks = ks_begin + it;
+            uint8_t* st = smem + st_i * C::kStageBytes;
+            tma_load_2d(st + C::kOffX, &tmap_x, &full[st_i], ks * 128, m0);
+            bulk_load(st + C::kOffSFX, xsf_tile + (int64_t)ks * 4 * 512, 2048, &full[st_i]);
+        };
+        RowCursor cur0, cur1;
+        // selected residual blocks of a stage (bit 2*kk + h) and their packed indices
+        auto resid_mask = [&](int it, int (&idx0)[4], int (&idx1)[4]) -> uint32_t {
+            uint32_t m = 0;
+            if (p.has_resid) {
+                const int ks = ks_begin + it;
+                const uint32_t m0b = row_step(cur0, ks * 4, idx0);
+                const uint32_t m1b = row_step(cur1, ks * 4, idx1);
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        m |= (((m0b >> kk) & 1u) << (2 * kk)) | (((m1b >> kk) & 1u) << (2 * kk + 1));
-                }
-                rmask[s] = m;
-                mbar_arrive_expect_tx(&rfull[s], __popc(m) * (2048 + 512));
-#pragma unroll 1
-                for (int j = 0; j < 8; ++j) {
-                    if (!((m >> j) & 1u)) continue;
-                    const int kk = j >> 1, h = j & 1;
-                    const int idx = h ? idx1[kk] : idx0[kk];
-                    bulk_load(st + C::kOffRC + kk * 4096 + h * 2048, p.blk_codes + (int64_t)idx * 2048, 2048,
-                              &rfull[s]);
-                    bulk_load(st + C::kOffRSF + j * 512, p.blk_sf + (int64_t)idx * 512, 512, &rfull[s]);
-                }
-            };
-            const int first = min(C::kStages, n_iters);
-            for (int it = 0; it < first; ++it) issue_w(it);  // nothing to wait for yet
-            if (p.has_resid && n_iters > 0) {
-                cur0 = row_cursor(p, n_tile * 2 + 0, ks_begin * 4);
-                cur1 = row_cursor(p, n_tile * 2 + 1, ks_begin * 4);
+                for (int kk = 0; kk < 4; ++kk)
+                    m |= (((m0b >> kk) & 1u) << (2 * kk)) | (((m1b >> kk) & 1u) << (2 * kk + 1));
             }
-            for (int it = 0; it < first; ++it) issue_resid(it);
-            griddep_wait();
+            return m;
+        };
+        auto issue_resid = [&](int it, uint32_t m, const int (&idx0)[4], const int (&idx1)[4]) {
+            const int s = it % C::kStages;
+            uint8_t* st = smem + s * C::kStageBytes;
+            rmask[s] = m;
+            mbar_arrive_expect_tx(&rfull[s], __popc(m) * (2048 + 512));
+            for (uint32_t mm = m; mm; mm &= mm - 1) {
+                const int j = __ffs(mm) - 1, kk = j >> 1, h = j & 1;
+                int idx = 0;
+#pragma unroll
+                for (int a = 0; a < 4; ++a)
+                    if (a == kk) idx = h ? idx1[a] : idx0[a];
+                bulk_load(st + C::kOffRC + kk * 4096 + h * 2048, p.blk_codes + (int64_t)idx * 2048, 2048,
+                          &rfull[s]);
+                bulk_load(st + C::kOffRSF + j * 512, p.blk_sf + (int64_t)idx * 512, 512, &rfull[s]);
+            }
+        };
+        const int first = min(C::kStages, n_iters);
+        if (elect_one())
+            for (int it = 0; it < first; ++it) issue_w(it);  // nothing to wait for yet
+        __syncwarp();
+        if (p.has_resid && n_iters > 0) {
+            cur0 = row_cursor(p, n_tile * 2 + 0, ks_begin * 4);
+            cur1 = row_cursor(p, n_tile * 2 + 1, ks_begin * 4);
+        }
+        for (int it = 0; it < first; ++it) {
+            int idx0[4] = {0, 0, 0, 0}, idx1[4] = {0, 0, 0, 0};
+            const uint32_t m = resid_mask(it, idx0, idx1);
+            if (elect_one()) issue_resid(it, m, idx0, idx1);
+            __syncwarp();
+        }
+        griddep_wait();
+        if (elect_one())
             for (int it = 0; it < first; ++it) issue_x(it);
-            int issued = first;
-            for (int it = first; it < n_iters; ++it) {
-                const int st_i = it % C::kStages;
-                if (!mbar_wait(&empty[st_i], ((it / C::kStages) - 1) & 1)) break;
+        __syncwarp();
+        int issued = first;
+        for (int it = first; it < n_iters; ++it) {
+            const int st_i = it % C::kStages;
+            if (!mbar_wait_warp(&empty[st_i], ((it / C::kStages) - 1) & 1)) break;
+            int idx0[4] = {0, 0, 0, 0}, idx1[4] = {0, 0, 0, 0};
+            const uint32_t m = resid_mask(it, idx0, idx1);
+            if (elect_one()) {
                 issue_w(it);
                 issue_x(it);
-                issue_resid(it);
-                ++issued;
+                issue_resid(it, m, idx0, idx1);
             }
-            // Do not leave while copies into this CTA's shared memory are in flight.
-            for (int it = max(0, issued - C::kStages); it < issued; ++it) {
-                mbar_wait(&full[it % C::kStages], (it / C::kStages) & 1);
-                mbar_wait(&rfull[it % C::kStages], (it / C::kStages) & 1);
-            }
+            __syncwarp();
+            ++issued;
+        }
+        // Do not leave while copies into this CTA's shared memory are in flight.
+        for (int it = max(0, issued - C::kStages); it < issued; ++it) {
+            mbar_wait_warp(&full[it % C::kStages], (it / C::kStages) & 1);
+            mbar_wait_warp(&rfull[it % C::kStages], (it / C::kStages) & 1);
         }
     } else if (warp == 1) {
-        if (lane == 0) {
-            // ------------------------------------------------ MMA issuer
-            constexpr uint32_t idesc = idesc_mxf4nvf4(128, BN);
-            uint32_t acc = 0;
-            for (int it = 0; it < n_iters; ++it) {
-                const int s = it % C::kStages;
-                const uint32_t par = (it / C::kStages) & 1;
-                if (!mbar_wait(&full[s], par)) break;
-                tc_fence_after();
-                uint8_t* st = smem + s * C::kStageBytes;
-                const uint32_t sfc = tmem + C::kSfCol0 + s * 64;
-                const uint32_t aw = smem_u32(st + C::kOffW), bx = smem_u32(st + C::kOffX);
+        // ---------------------------------------------------- MMA issuer (converged warp, one lane issues)
+        constexpr uint32_t idesc = idesc_mxf4nvf4(128, BN);
+        uint32_t acc = 0;
+        for (int it = 0; it < n_iters; ++it) {
+            const int s = it % C::kStages;
+            const uint32_t par = (it / C::kStages) & 1;
+            if (!mbar_wait_warp(&full[s], par)) break;
+            tc_fence_after();
+            const uint32_t st = smem_u32(smem + s * C::kStageBytes);
+            const uint32_t sfc = tmem + C::kSfCol0 + s * 64;
+            if (elect_one()) {
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) {
-                    tc_cp_sf_chunk(sfc + 4 * kk, smem_desc(smem_u32(st + C::kOffSFW + kk * 512), 0, 128, 0));
-                    tc_cp_sf_chunk(sfc + 16 + 4 * kk, smem_desc(smem_u32(st + C::kOffSFX + kk * 512), 0, 128, 0));
+                    tc_cp_sf_chunk(sfc + 4 * kk, smem_desc(st + C::kOffSFW + kk * 512, 0, 128, 0));
+                    tc_cp_sf_chunk(sfc + 16 + 4 * kk, smem_desc(st + C::kOffSFX + kk * 512, 0, 128, 0));
                 }
                 if (p.mode != 2) {
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk) {
-                        mma_mxf4nvf4(tmem, smem_desc(aw + 32 * kk, 16, 1024, 2), smem_desc(bx + 32 * kk, 16, 1024, 2),
-                                     idesc, sfc + 4 * kk, sfc + 16 + 4 * kk, acc);
-                        acc = 1;
-                    }
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_mxf4nvf4(tmem, smem_desc(st + C::kOffW + 32 * kk, 16, 1024, 2),
+                                     smem_desc(st + C::kOffX + 32 * kk, 16, 1024, 2), idesc, sfc + 4 * kk,
+                                     sfc + 16 + 4 * kk, (acc | kk) != 0);
+                    acc = 1;
                 }
-                if (!mbar_wait(&rfull[s], par)) break;
-                tc_fence_after();
-                const uint32_t m = p.mode != 1 ? rmask[s] : 0u;
-#pragma unroll 1
-                for (int j = 0; j < 8; ++j) {
-                    if (!((m >> j) & 1u)) continue;
-                    const int kk = j >> 1;
-                    tc_cp_sf_chunk(sfc + 32 + 4 * j, smem_desc(smem_u32(st + C::kOffRSF + j * 512), 0, 128, 0));
-                    mma_mxf4nvf4(tmem, smem_desc(smem_u32(st + C::kOffRC + kk * 4096), 128, 256, 0),
-                                 smem_desc(bx + 32 * kk, 16, 1024, 2), idesc, sfc + 32 + 4 * j, sfc + 16 + 4 * kk,
-                                 acc);
+            }
+            __syncwarp();
+            acc = __shfl_sync(0xffffffffu, acc, 0);
+            if (!mbar_wait_warp(&rfull[s], par)) break;
+            tc_fence_after();
+            const uint32_t m = p.mode != 1 ? rmask[s] : 0u;
+            if (elect_one()) {
+                for (uint32_t mm = m; mm; mm &= mm - 1) {
+                    const int j = __ffs(mm) - 1, kk = j >> 1;
+                    tc_cp_sf_chunk(sfc + 32 + 4 * j, smem_desc(st + C::kOffRSF + j * 512, 0, 128, 0));
+                    mma_mxf4nvf4(tmem, smem_desc(st + C::kOffRC + kk * 4096, 128, 256, 0),
+                                 smem_desc(st + C::kOffX + 32 * kk, 16, 1024, 2), idesc, sfc + 32 + 4 * j,
+                                 sfc + 16 + 4 * kk, acc);
                     acc = 1;
                 }
                 tc_commit(&empty[s]);
             }
-            tc_commit(accf);
+            __syncwarp();
+            acc = __shfl_sync(0xffffffffu, acc, 0);
         }
+        if (elect_one()) tc_commit(accf);
+        __syncwarp();
     } else {
         // ---------------------------------------------------- epilogue (warps 2..5)
         const int q = warp & 3;
@@ -399,12 +439,14 @@ __global__ void __launch_bounds__(192, 1)
 // side (256 rows per tile, B = W), K = 256 per pipeline stage. CTAs are persistent and
 // walk the tiles m-fastest, so CTAs running at the same time share W tiles through L2.
 // A selected residual block (64 weight rows x 64 K) is one N = 64 MMA written into its
-// 64-column slice of the same fp32 accumulator: exactly the block's work. Residual
-// blocks stream through their own ring of shared-memory slots.
-// Warps: 0 producer (TMA / bulk copies), 1 MMA issuer (one thread), 2-9 epilogue (two
-// warps per 32-lane quarter of tensor memory, 128 accumulator columns each). The
-// epilogue copies the accumulator to registers and releases it before scaling and
-// storing, so the next tile's MMAs overlap the stores.
+// 64-column slice of the same fp32 accumulator: exactly the block's work. The residual
+// blocks of a stage land in a ring of shared-memory slots on the stage's own barrier,
+// and the stage's release frees them with it.
+// Warps: 0 producer (TMA / bulk copies), 1 MMA issuer, 2-9 epilogue (two warps per
+// 32-lane quarter of tensor memory, 128 accumulator columns each). Producer and MMA
+// warps run their loops converged and let one elected lane issue. The epilogue copies
+// the accumulator to registers and releases it before scaling and storing, so the next
+// tile's MMAs overlap the stores.
 struct PrefillCfg {
     static constexpr int kStages = 3;
     static constexpr int kOffX = 0;                    // 128 rows x 128 B, swizzled
@@ -412,7 +454,8 @@ struct PrefillCfg {
     static constexpr int kOffSFX = kOffW + 32768;      // 4 x 512 B
     static constexpr int kOffSFW = kOffSFX + 2048;     // 2 row tiles x 4 x 512 B
     static constexpr int kStageBytes = kOffSFW + 4096; // 55296
-    static constexpr int kRSlots = 8;                  // residual ring: 2048 B codes + 512 B scales
+    static constexpr int kBaseTx = kStageBytes;        // bytes a stage's base operands bring
+    static constexpr int kRSlots = 16;                 // residual ring: 2048 B codes + 512 B scales
     static constexpr int kRSlotBytes = 2560;
     static constexpr int kOffRing = kStages * kStageBytes;
     static constexpr int kCtrlOff = kOffRing + kRSlots * kRSlotBytes;
@@ -426,6 +469,7 @@ struct PrefillCfg {
     static_assert(kStageBytes % 1024 == 0, "stage alignment");
     static_assert(kSmemBytes <= 232448, "shared memory budget");
     static_assert(kRSfCol0 + kRSlots * 4 <= 512, "tensor memory budget");
+    static_assert(kRSlots >= 16, "a stage may carry 16 residual blocks");
 };
 
 // Which 64-column slices of a tile's accumulator receive an MMA (bit h: weight rows
@@ -440,17 +484,31 @@ __device__ __forceinline__ uint32_t prefill_tile_slices(const GemmParams& p, int
     return m;
 }
 
+// Element i of a small per-stage register array (unrolled select, no local memory).
+template <int N>
+__device__ __forceinline__ int pick(const int (&a)[N], int i) {
+    int v = a[0];
+#pragma unroll
+    for (int j = 1; j < N; ++j)
+        if (i == j) v = a[j];
+    return v;
+}
+template <int N>
+__device__ __forceinline__ void put(int (&a)[N], int i, int v) {
+#pragma unroll
+    for (int j = 0; j < N; ++j)
+        if (i == j) a[j] = v;
+}
+
 __global__ void __launch_bounds__(320, 1)
     k_gemm_prefill(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
                    const GemmParams p) {
     using C = PrefillCfg;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kCtrlOff);
-    uint64_t* empty = full + C::kStages;
-    uint64_t* rfull = empty + C::kStages;
-    uint64_t* rempty = rfull + C::kRSlots;
-    uint64_t* accf = rempty + C::kRSlots;
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kCtrlOff);  // base operands + residual blocks landed
+    uint64_t* empty = full + C::kStages;                                // stage (and its ring slots) consumed
+    uint64_t* accf = empty + C::kStages;
     uint64_t* acce = accf + 1;
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(acce + 1);
     uint32_t* rmask = tmem_holder + 1;  // [kStages]: bit 4*kk + h
@@ -459,15 +517,12 @@ __global__ void __launch_bounds__(320, 1)
     const int KS = p.K / 256, KS64 = p.K / 64;
     const int tiles_m = (p.M + 127) / 128, tiles_n = p.N / 256;
     const int ntiles = tiles_m * tiles_n;
+    const bool resid = p.has_resid && p.mode != 1;
 
     if (warp == 0 && lane == 0) {
         for (int s = 0; s < C::kStages; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
-        }
-        for (int r = 0; r < C::kRSlots; ++r) {
-            mbar_init(&rfull[r], 1);
-            mbar_init(&rempty[r], 1);
         }
         mbar_init(accf, 1);
         mbar_init(acce, 8);
@@ -483,119 +538,136 @@ __global__ void __launch_bounds__(320, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
+    const uint32_t sbase = smem_u32(smem);
 
     if (warp == 0) {
-        if (lane == 0) {
-            // ------------------------------------------------ producer
-            griddep_wait();
-            int sc = 0, rc = 0;  // stage and residual-slot use counters
-            bool ok = true;
-            for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-                const int m_tile = t % tiles_m, n_tile = t / tiles_m;
-                RowCursor cur[4];
-                if (p.has_resid)
+        // ---------------------------------------------------- producer
+        griddep_wait();
+        int sc = 0, rc = 0;  // stages and residual blocks issued so far
+        int rdone = 0;       // residual blocks known consumed (ring slots below it are free)
+        int ends[C::kStages] = {};  // rc after the latest stage held by each stage buffer
+        bool ok = true;
+        for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+            const int m_tile = t % tiles_m, n_tile = t / tiles_m;
+            RowCursor cur[4];
+            if (resid)
 #pragma unroll
-                    for (int h = 0; h < 4; ++h) cur[h] = row_cursor(p, n_tile * 4 + h, 0);
-                for (int ks = 0; ks < KS && ok; ++ks, ++sc) {
-                    const int s = sc % C::kStages;
-                    if (!mbar_wait(&empty[s], ((sc / C::kStages) & 1) ^ 1)) { ok = false; break; }
-                    uint32_t m = 0;
-                    int idx[4][4];
-                    if (p.has_resid)
+                for (int h = 0; h < 4; ++h) cur[h] = row_cursor(p, n_tile * 4 + h, 0);
+            for (int ks = 0; ks < KS && ok; ++ks, ++sc) {
+                const int s = sc % C::kStages;
+                if (sc >= C::kStages) {
+                    if (!mbar_wait_warp(&empty[s], ((sc / C::kStages) & 1) ^ 1)) { ok = false; break; }
+                    rdone = max(rdone, pick(ends, s));
+                }
+                uint32_t m = 0;
+                int idx[4][4];
+                if (resid)
 #pragma unroll
-                        for (int h = 0; h < 4; ++h) {
-                            const uint32_t mb = row_step(cur[h], ks * 4, idx[h]);
+                    for (int h = 0; h < 4; ++h) {
+                        const uint32_t mb = row_step(cur[h], ks * 4, idx[h]);
 #pragma unroll
-                            for (int kk = 0; kk < 4; ++kk) m |= ((mb >> kk) & 1u) << (4 * kk + h);
-                        }
+                        for (int kk = 0; kk < 4; ++kk) m |= ((mb >> kk) & 1u) << (4 * kk + h);
+                    }
+                const int n = __popc(m);
+                // ring slots [rc, rc + n) must be free: wait for younger stages until they are
+                for (int u = sc - C::kStages + 1; rc + n - C::kRSlots > rdone && u < sc && ok; ++u) {
+                    if (u < 0) continue;
+                    ok = mbar_wait_warp(&empty[u % C::kStages], (u / C::kStages) & 1);
+                    rdone = max(rdone, pick(ends, u % C::kStages));
+                }
+                if (!ok) break;
+                const uint32_t st = sbase + s * C::kStageBytes;
+                if (elect_one()) {
                     rmask[s] = m;
-                    uint8_t* st = smem + s * C::kStageBytes;
-                    mbar_arrive_expect_tx(&full[s], 16384 + 32768 + 2048 + 4096);
-                    tma_load_2d(st + C::kOffX, &tmap_x, &full[s], ks * 128, m_tile * 128);
-                    tma_load_2d(st + C::kOffW, &tmap_w, &full[s], ks * 128, n_tile * 256);
-                    bulk_load(st + C::kOffSFX, p.x_sf + ((int64_t)m_tile * KS64 + ks * 4) * 512, 2048, &full[s]);
+                    mbar_arrive_expect_tx(&full[s], C::kBaseTx + n * C::kRSlotBytes);
+                    tma_load_2d(smem + s * C::kStageBytes + C::kOffX, &tmap_x, &full[s], ks * 128, m_tile * 128);
+                    tma_load_2d(smem + s * C::kStageBytes + C::kOffW, &tmap_w, &full[s], ks * 128, n_tile * 256);
+                    bulk_load_s(st + C::kOffSFX, p.x_sf + ((int64_t)m_tile * KS64 + ks * 4) * 512, 2048, &full[s]);
+                    bulk_load_s(st + C::kOffSFW, p.w_sf + ((int64_t)(n_tile * 2) * KS64 + ks * 4) * 512, 2048,
+                                &full[s]);
+                    bulk_load_s(st + C::kOffSFW + 2048, p.w_sf + ((int64_t)(n_tile * 2 + 1) * KS64 + ks * 4) * 512,
+                                2048, &full[s]);
+                    // residual blocks of the stage in (kk, h) order, into consecutive ring slots
+                    int r = rc;
+                    for (uint32_t mm = m; mm; mm &= mm - 1, ++r) {
+                        const int j = __ffs(mm) - 1, kk = j >> 2, h = j & 3;
+                        int bi = 0;
 #pragma unroll
-                    for (int h2 = 0; h2 < 2; ++h2)
-                        bulk_load(st + C::kOffSFW + h2 * 2048,
-                                  p.w_sf + ((int64_t)(n_tile * 2 + h2) * KS64 + ks * 4) * 512, 2048, &full[s]);
-                    // residual blocks of this stage, in (kk, h) order
-#pragma unroll 1
-                    for (int j = 0; j < 16 && ok; ++j) {
-                        if (!((m >> j) & 1u)) continue;
-                        const int kk = j >> 2, h = j & 3;
-                        const int r = rc % C::kRSlots;
-                        if (!mbar_wait(&rempty[r], ((rc / C::kRSlots) & 1) ^ 1)) { ok = false; break; }
-                        uint8_t* slot = smem + C::kOffRing + r * C::kRSlotBytes;
-                        const int bi = idx[h][kk];
-                        mbar_arrive_expect_tx(&rfull[r], 2560);
-                        bulk_load(slot, p.blk_codes + (int64_t)bi * 2048, 2048, &rfull[r]);
-                        bulk_load(slot + 2048, p.blk_sf + (int64_t)bi * 512, 512, &rfull[r]);
-                        ++rc;
+                        for (int a = 0; a < 4; ++a)
+#pragma unroll
+                            for (int b = 0; b < 4; ++b)
+                                if (a == h && b == kk) bi = idx[a][b];
+                        const uint32_t slot = sbase + C::kOffRing + (r % C::kRSlots) * C::kRSlotBytes;
+                        bulk_load_s(slot, p.blk_codes + (int64_t)bi * 2048, 2048, &full[s]);
+                        bulk_load_s(slot + 2048, p.blk_sf + (int64_t)bi * 512, 512, &full[s]);
                     }
                 }
+                __syncwarp();
+                rc += n;
+                put(ends, s, rc);
             }
-            // Do not leave while copies into this CTA's shared memory are in flight:
-            // wait for the last uses of every stage and residual slot.
-            for (int u = max(0, sc - C::kStages); u < sc; ++u) mbar_wait(&full[u % C::kStages], (u / C::kStages) & 1);
-            for (int u = max(0, rc - C::kRSlots); u < rc; ++u) mbar_wait(&rfull[u % C::kRSlots], (u / C::kRSlots) & 1);
         }
+        // Do not leave while copies into this CTA's shared memory are in flight.
+        for (int u = max(0, sc - C::kStages); u < sc; ++u) mbar_wait_warp(&full[u % C::kStages], (u / C::kStages) & 1);
     } else if (warp == 1) {
-        if (lane == 0) {
-            // ------------------------------------------------ MMA issuer
-            constexpr uint32_t idesc_d = idesc_mxf4nvf4(128, 256);
-            constexpr uint32_t idesc_r = idesc_mxf4nvf4(128, 64);
-            int sc = 0, rc = 0, tc = 0;
-            bool ok = true;
-            for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++tc) {
-                if (!mbar_wait(acce, (tc & 1) ^ 1)) break;  // the epilogue has read the previous tile
+        // ---------------------------------------------------- MMA issuer
+        constexpr uint32_t idesc_d = idesc_mxf4nvf4(128, 256);
+        constexpr uint32_t idesc_r = idesc_mxf4nvf4(128, 64);
+        int sc = 0, rc = 0, tc = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++tc) {
+            if (!mbar_wait_warp(acce, (tc & 1) ^ 1)) break;  // the epilogue has read the previous tile
+            tc_fence_after();
+            uint32_t acc4 = 0;  // bit h: the tile's slice h already holds a partial sum
+            for (int ks = 0; ks < KS; ++ks, ++sc) {
+                const int s = sc % C::kStages;
+                if (!mbar_wait_warp(&full[s], (sc / C::kStages) & 1)) { ok = false; break; }
                 tc_fence_after();
-                uint32_t acc4 = 0;  // bit h: the tile's slice h already holds a partial sum
-                for (int ks = 0; ks < KS; ++ks, ++sc) {
-                    const int s = sc % C::kStages;
-                    if (!mbar_wait(&full[s], (sc / C::kStages) & 1)) { ok = false; break; }
-                    tc_fence_after();
-                    uint8_t* st = smem + s * C::kStageBytes;
-                    const uint32_t sfc = tmem + C::kSfCol0 + s * C::kSfStageCols;
-                    const uint32_t m = p.mode != 1 ? rmask[s] : 0u;
+                const uint32_t st = sbase + s * C::kStageBytes;
+                const uint32_t sfc = tmem + C::kSfCol0 + s * C::kSfStageCols;
+                const uint32_t m = resid ? rmask[s] : 0u;
+                if (elect_one()) {
+                    if (p.mode != 2 || m) {
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk) {
-                        tc_cp_sf_chunk(sfc + 4 * kk, smem_desc(smem_u32(st + C::kOffSFX + kk * 512), 0, 128, 0));
-                        tc_cp_sf_chunk(sfc + 16 + 8 * kk, smem_desc(smem_u32(st + C::kOffSFW + kk * 512), 0, 128, 0));
-                        tc_cp_sf_chunk(sfc + 16 + 8 * kk + 4,
-                                       smem_desc(smem_u32(st + C::kOffSFW + 2048 + kk * 512), 0, 128, 0));
+                        for (int kk = 0; kk < 4; ++kk)
+                            tc_cp_sf_chunk(sfc + 4 * kk, smem_desc(st + C::kOffSFX + kk * 512, 0, 128, 0));
                     }
-                    const uint32_t ax = smem_u32(st + C::kOffX), bw = smem_u32(st + C::kOffW);
+                    if (p.mode != 2) {
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk) {
-                        const uint64_t adesc = smem_desc(ax + 32 * kk, 16, 1024, 2);
-                        if (p.mode != 2) {
-                            mma_mxf4nvf4(tmem, adesc, smem_desc(bw + 32 * kk, 16, 1024, 2), idesc_d, sfc + 4 * kk,
-                                         sfc + 16 + 8 * kk, acc4 == 0xFu);
-                            acc4 = 0xFu;
+                        for (int kk = 0; kk < 4; ++kk) {
+                            tc_cp_sf_chunk(sfc + 16 + 8 * kk, smem_desc(st + C::kOffSFW + kk * 512, 0, 128, 0));
+                            tc_cp_sf_chunk(sfc + 16 + 8 * kk + 4,
+                                           smem_desc(st + C::kOffSFW + 2048 + kk * 512, 0, 128, 0));
                         }
-#pragma unroll 1
-                        for (int h = 0; h < 4; ++h) {
-                            if (!((m >> (4 * kk + h)) & 1u)) continue;
-                            const int r = rc % C::kRSlots;
-                            if (!mbar_wait(&rfull[r], (rc / C::kRSlots) & 1)) { ok = false; break; }
-                            tc_fence_after();
-                            uint8_t* slot = smem + C::kOffRing + r * C::kRSlotBytes;
-                            const uint32_t rsf = tmem + C::kRSfCol0 + 4 * r;
-                            tc_cp_sf_chunk(rsf, smem_desc(smem_u32(slot + 2048), 0, 128, 0));
-                            mma_mxf4nvf4(tmem + 64 * h, adesc, smem_desc(smem_u32(slot), 128, 256, 0), idesc_r,
-                                         sfc + 4 * kk, rsf + 2 * (h & 1), (acc4 >> h) & 1u);
-                            acc4 |= 1u << h;
-                            tc_commit(&rempty[r]);
-                            ++rc;
-                        }
-                        if (!ok) break;
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk)
+                            mma_mxf4nvf4(tmem, smem_desc(st + C::kOffX + 32 * kk, 16, 1024, 2),
+                                         smem_desc(st + C::kOffW + 32 * kk, 16, 1024, 2), idesc_d, sfc + 4 * kk,
+                                         sfc + 16 + 8 * kk, (acc4 | kk) != 0);
+                        acc4 = 0xFu;
                     }
-                    // when the dense half was skipped a stage may carry no MMA: still release it
+                    // residual blocks in (kk, h) order: block (kk, h) adds into accumulator slice h
+                    int r = rc;
+                    for (uint32_t mm = m; mm; mm &= mm - 1, ++r) {
+                        const int j = __ffs(mm) - 1, kk = j >> 2, h = j & 3;
+                        const int slot_i = r % C::kRSlots;
+                        const uint32_t slot = sbase + C::kOffRing + slot_i * C::kRSlotBytes;
+                        const uint32_t rsf = tmem + C::kRSfCol0 + 4 * slot_i;
+                        tc_cp_sf_chunk(rsf, smem_desc(slot + 2048, 0, 128, 0));
+                        mma_mxf4nvf4(tmem + 64 * h, smem_desc(st + C::kOffX + 32 * kk, 16, 1024, 2),
+                                     smem_desc(slot, 128, 256, 0), idesc_r, sfc + 4 * kk, rsf + 2 * (h & 1),
+                                     (acc4 >> h) & 1u);
+                        acc4 |= 1u << h;
+                    }
+                    // releases the stage and its ring slots once every MMA above has completed
                     tc_commit(&empty[s]);
-                    if (!ok) break;
                 }
-                tc_commit(accf);
+                __syncwarp();
+                acc4 = __shfl_sync(0xffffffffu, acc4, 0);
+                rc += __popc(m);
             }
+            if (elect_one()) tc_commit(accf);
+            __syncwarp();
         }
     } else {
         // ---------------------------------------------------- epilogue (warps 2..9)
@@ -605,7 +677,7 @@ __global__ void __launch_bounds__(320, 1)
         int tc = 0;
         for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++tc) {
             const int m_tile = t % tiles_m, n_tile = t / tiles_m;
-            const bool waited = mbar_wait(accf, tc & 1);
+            const bool waited = mbar_wait_warp(accf, tc & 1);
             tc_fence_after();
             const uint32_t slices = waited ? prefill_tile_slices(p, n_tile) : 0u;
             float acc[128];
