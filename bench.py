@@ -51,12 +51,12 @@ def step_bytes(M: int, N: int, K: int, T: int, nblk: int) -> dict:
     idx = 4 * (NBr + 1) + 4 * NBr * KW
     return {
         "hessian_diag": 2 * T * K + 4 * K,
-        # W, H in; base codes + tiled scales + g, residual codes + scales, Delta out
-        "quantize_weight_delta": 2 * NK + 4 * K + NK // 2 + NK // 16 + 4 + NK // 2 + NK // 16 + 8 * B,
+        # W, H in; base codes + tiled scales + g, Delta out (the full residual is not stored)
+        "quantize_weight_delta": 2 * NK + 4 * K + NK // 2 + NK // 16 + 4 + 8 * B,
         # Delta in; rank + sel out
         "topk_blocks": 8 * B + 8 * nblk,
-        # selected residual codes + scales + sel in; packed blocks + kt + index out
-        "pack_residual": nblk * (2048 + 256 + 4) + nblk * (2048 + 512 + 4) + idx,
+        # selected W blocks (bf16) + g + sel in; packed residual blocks + kt + index out
+        "pack_residual": nblk * (8192 + 4) + 4 + nblk * (2048 + 512 + 4) + idx,
         "quantize_act": 2 * M * K + M * K // 2 + Mp * K // 16 + 4 * M,
         # NVFP4 W (codes + scales) + residual blocks (codes + scales) + index + X (codes + scales
         # + per-token scale) + bf16 Y
@@ -230,13 +230,13 @@ def isolated_profile(sets, calls, M, N, K, budget, reps, stream):
         layer = s["layer"]
         xq, Yb, ws = layer.act_buffers(M)
         if c == "quantize_weight_delta":
-            mosaic.mq_quantize_weight_delta(s["W"], layer.H, layer.base, layer.resid, layer.delta, layer.qws)
+            mosaic.mq_quantize_weight_delta(s["W"], layer.H, layer.base, None, layer.delta, layer.qws)
         elif c == "hessian_diag":
             mosaic.mq_hessian_diag(s["Xcal"], layer.H)
         elif c == "topk_blocks":
             mosaic.mq_topk_blocks(layer.delta, budget, layer.rank, layer.sel)
         elif c == "pack_residual":
-            mosaic.mq_pack_residual(layer.resid, layer.sel, budget, layer.packed)
+            mosaic.mq_pack_residual_weight(s["W"], layer.base, layer.sel, budget, layer.packed)
         elif c == "quantize_act":
             mosaic.mq_quantize_act(s["X"], xq)
         else:
@@ -337,10 +337,9 @@ def main():
         layer = s["layer"]
         xq, Yb, ws = layer.act_buffers(M)
         ops = [lambda: mosaic.mq_hessian_diag(s["Xcal"], layer.H),
-               lambda: mosaic.mq_quantize_weight_delta(s["W"], layer.H, layer.base, layer.resid, layer.delta,
-                                                       layer.qws),
+               lambda: mosaic.mq_quantize_weight_delta(s["W"], layer.H, layer.base, None, layer.delta, layer.qws),
                lambda: mosaic.mq_topk_blocks(layer.delta, budget, layer.rank, layer.sel),
-               lambda: mosaic.mq_pack_residual(layer.resid, layer.sel, budget, layer.packed),
+               lambda: mosaic.mq_pack_residual_weight(s["W"], layer.base, layer.sel, budget, layer.packed),
                lambda: mosaic.mq_quantize_act(s["X"], xq),
                lambda: mosaic.mq_gemm(xq, layer.base, layer.packed, Yb, M, N, K, 0, ws)]
         for j, op in enumerate(ops):

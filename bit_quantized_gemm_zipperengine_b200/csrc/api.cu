@@ -25,6 +25,9 @@ cudaError_t launch_topk(const double* delta, int B, int budget, int32_t* rank, i
 cudaError_t launch_pack(const uint8_t* rcodes, const uint8_t* rsf, int N, int K, const int32_t* sel, int budget,
                         uint8_t* blk_codes, uint8_t* blk_sf, int32_t* blk_kt, int32_t* tile_ptr, uint32_t* bitmap,
                         cudaStream_t s);
+cudaError_t launch_pack_w(const uint16_t* W, int N, int K, const float* g_w, const int32_t* sel, int budget,
+                          uint8_t* blk_codes, uint8_t* blk_sf, int32_t* blk_kt, int32_t* tile_ptr, uint32_t* bitmap,
+                          cudaStream_t s);
 
 }  // namespace mq
 
@@ -64,13 +67,14 @@ static bool make_tmap_bytes(CUtensorMap* map, const void* base, uint64_t row_byt
     return r == CUDA_SUCCESS;
 }
 
-// bf16 matrix [rows][cols] in 64 x 64 boxes with the 128-byte swizzle (one Delta block).
+// bf16 matrix [rows][cols] in 64-column x 128-row boxes with the 128-byte swizzle (two
+// stacked Delta blocks); rows outside the matrix read as zero.
 static bool make_tmap_bf16_blocks(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     cuuint64_t dims[2] = {cols, rows};
     cuuint64_t strides[1] = {cols * 2};
-    cuuint32_t box[2] = {64, 64};
+    cuuint32_t box[2] = {64, 128};
     cuuint32_t es[2] = {1, 1};
     CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<void*>(base), dims, strides, box, es,
                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -183,21 +187,22 @@ mq_status mq_delta_score_topk(const mq_bf16* W, const float* H, const mq_nvfp4_m
 mq_status mq_quantize_weight_delta(const mq_bf16* W, int N, int K, const float* H, mq_nvfp4_mat* base,
                                    mq_nvfp4_mat* resid_full, double* delta, void* ws, size_t ws_bytes,
                                    mq_stream stream) {
-    if (!W || !H || !delta || !base || !resid_full || !nvfp4_shape_ok(N, K) || N % 64) return MQ_ERR_INVALID_ARG;
-    if (!base->codes || !base->sf_swz || !base->gscale || !resid_full->codes || !resid_full->sf)
+    if (!W || !H || !delta || !base || !nvfp4_shape_ok(N, K) || N % 64) return MQ_ERR_INVALID_ARG;
+    if (!base->codes || !base->sf_swz || !base->gscale) return MQ_ERR_INVALID_ARG;
+    if (base->rows != N || base->cols != K) return MQ_ERR_INVALID_ARG;
+    if (resid_full && (!resid_full->codes || !resid_full->sf || resid_full->rows != N || resid_full->cols != K))
         return MQ_ERR_INVALID_ARG;
-    if (base->rows != N || base->cols != K || resid_full->rows != N || resid_full->cols != K)
+    if (!aligned(W, 16) || !aligned(base->codes, 16) || !aligned(base->sf_swz, 16) ||
+        (base->sf && !aligned(base->sf, 4)))
         return MQ_ERR_INVALID_ARG;
-    if (!aligned(W, 16) || !aligned(base->codes, 8) || !aligned(resid_full->codes, 8) || !aligned(base->sf_swz, 4) ||
-        !aligned(resid_full->sf, 4) || (base->sf && !aligned(base->sf, 4)))
-        return MQ_ERR_INVALID_ARG;
+    if (resid_full && (!aligned(resid_full->codes, 16) || !aligned(resid_full->sf, 4))) return MQ_ERR_INVALID_ARG;
     if (!ws || ws_bytes < mq_quantize_weight_workspace_bytes(N, K)) return MQ_ERR_WORKSPACE;
     CUtensorMap tw;
     int* err = err_word();
     if (!err || !make_tmap_bf16_blocks(&tw, W, (uint64_t)K, (uint64_t)N)) return MQ_ERR_CUDA;
     cudaError_t e = launch_quant_delta(W, tw, N, K, H, base->codes, base->sf, base->sf_swz, base->gscale,
-                                       resid_full->codes, resid_full->sf, delta, static_cast<float*>(ws), err,
-                                       as_stream(stream));
+                                       resid_full ? resid_full->codes : nullptr, resid_full ? resid_full->sf : nullptr,
+                                       delta, static_cast<float*>(ws), err, as_stream(stream));
     return launched(e, 2);
 }
 
@@ -220,6 +225,27 @@ mq_status mq_pack_residual(const mq_nvfp4_mat* resid_full, const int32_t* sel, i
     if (budget > 0 && (!aligned(out->blk_codes, 16) || !aligned(out->blk_sf, 16))) return MQ_ERR_INVALID_ARG;
     return launched(launch_pack(resid_full->codes, resid_full->sf, N, K, sel, budget, out->blk_codes, out->blk_sf,
                                 out->blk_kt, out->tile_ptr, out->bitmap, as_stream(stream)),
+                    1);
+}
+
+static mq_status check_packed(const mq_residual_packed* out, int N, int K, const int32_t* sel, int budget) {
+    if (!out || out->N != N || out->K != K || out->nblk != budget || budget < 0 || budget > (N / 64) * (K / 64))
+        return MQ_ERR_INVALID_ARG;
+    if (!out->tile_ptr || !out->bitmap) return MQ_ERR_INVALID_ARG;
+    if (budget > 0 && (!sel || !out->blk_codes || !out->blk_sf || !out->blk_kt)) return MQ_ERR_INVALID_ARG;
+    if (budget > 0 && (!aligned(out->blk_codes, 16) || !aligned(out->blk_sf, 16))) return MQ_ERR_INVALID_ARG;
+    return MQ_OK;
+}
+
+mq_status mq_pack_residual_weight(const mq_bf16* W, const mq_nvfp4_mat* base, const int32_t* sel, int budget,
+                                  mq_residual_packed* out, mq_stream stream) {
+    if (!W || !base || !base->gscale) return MQ_ERR_INVALID_ARG;
+    const int N = base->rows, K = base->cols;
+    if (!nvfp4_shape_ok(N, K) || N % 64 || !aligned(W, 16)) return MQ_ERR_INVALID_ARG;
+    const mq_status st = check_packed(out, N, K, sel, budget);
+    if (st != MQ_OK) return st;
+    return launched(launch_pack_w(W, N, K, base->gscale, sel, budget, out->blk_codes, out->blk_sf, out->blk_kt,
+                                  out->tile_ptr, out->bitmap, as_stream(stream)),
                     1);
 }
 
@@ -310,12 +336,12 @@ mq_status mq_run_layer(const mq_bf16* W, const mq_bf16* X, const mq_bf16* Xcal, 
     }
     mq_status st;
     if ((st = mq_hessian_diag(xc, T, K, buf->H, stream)) != MQ_OK) return st;
-    if ((st = mq_quantize_weight_delta(w, N, K, buf->H, &buf->base, &buf->resid_full, buf->delta, buf->ws_quant,
+    if ((st = mq_quantize_weight_delta(w, N, K, buf->H, &buf->base, nullptr, buf->delta, buf->ws_quant,
                                        buf->ws_quant_bytes, stream)) != MQ_OK)
         return st;
     if ((st = mq_topk_blocks(buf->delta, (N / 64) * (K / 64), budget, buf->rank, buf->sel, stream)) != MQ_OK)
         return st;
-    if ((st = mq_pack_residual(&buf->resid_full, buf->sel, budget, &buf->packed, stream)) != MQ_OK) return st;
+    if ((st = mq_pack_residual_weight(w, &buf->base, buf->sel, budget, &buf->packed, stream)) != MQ_OK) return st;
     if ((st = mq_quantize_act(x, M, K, &buf->xq, stream)) != MQ_OK) return st;
     if ((st = mq_gemm(&buf->xq, &buf->base, &buf->packed, y, M, N, K, flags, buf->ws_gemm, buf->ws_gemm_bytes,
                       stream)) != MQ_OK)

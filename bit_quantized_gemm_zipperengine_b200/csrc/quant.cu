@@ -16,9 +16,13 @@ __device__ __forceinline__ float warp_max(float v) {
 
 // Per-CTA maxima of |W| over a grid-stride range of 8-element vectors (kAmaxBlocks
 // CTAs, 4 independent 16-byte loads in flight per thread).
+// W is an input of the call, never written by the preceding kernel, so the kernel lets
+// its dependent start and reads W at once: it overlaps the preceding kernel (the Hessian
+// estimate, which it does not use). It waits for that kernel only at its end, so that
+// its own completion still implies the predecessor's. The partials it overwrites are
+// read by the quantizers before they let their dependents start.
 __global__ void __launch_bounds__(512) k_amax_partial(const uint16_t* __restrict__ W, int64_t n8,
                                                       float* __restrict__ partial) {
-    griddep_wait();
     griddep_launch();
     float m = 0.0f;
     const uint4* v = reinterpret_cast<const uint4*>(W);
@@ -52,6 +56,7 @@ __global__ void __launch_bounds__(512) k_amax_partial(const uint16_t* __restrict
         t = warp_max(t);
         if (threadIdx.x == 0) partial[blockIdx.x] = t;
     }
+    griddep_wait();
 }
 
 // Gathers the scale bytes of 4 consecutive groups (lanes l..l+3, l % 4 == 0) into one
@@ -65,21 +70,23 @@ __device__ __forceinline__ uint32_t gather4(uint32_t b) {
 
 // A1: base NVFP4(W, g) and residual NVFP4(W - deq Q(W), g) for every group.
 // One thread per group; the group count is a multiple of 32 (K % 64 == 0 and
-// N % 64 == 0), so whole warps stay together for the 4-group scale gather.
+// N % 64 == 0), so whole warps stay together for the 4-group scale gather. The groups of
+// the rows past N up to the next multiple of 128 write zero tiled scales.
 __global__ void __launch_bounds__(256) k_quant_weight(const uint16_t* __restrict__ W, int N, int K,
                                                       const float* __restrict__ partial,
                                                       uint8_t* __restrict__ codes, uint8_t* __restrict__ sf,
                                                       uint8_t* __restrict__ sf_swz, float* __restrict__ g_out,
                                                       uint8_t* __restrict__ rcodes, uint8_t* __restrict__ rsf) {
     griddep_wait();
-    griddep_launch();
     const float g = tensor_scale(partial);
     if (blockIdx.x == 0 && threadIdx.x == 0) *g_out = g;
+    griddep_launch();  // once every CTA has read the partials
     const float g6 = __fmul_rn(6.0f, g);
     const int G = K / 16;
     const int64_t ngrp = (int64_t)N * G;
+    const int64_t ngrp_pad = (int64_t)((N + 127) / 128 * 128) * G;  // rows past N: zero tiled scales
     const int lane = threadIdx.x & 31;
-    for (int64_t grp = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; grp - lane < ngrp;
+    for (int64_t grp = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; grp - lane < ngrp_pad;
          grp += (int64_t)gridDim.x * blockDim.x) {
         const bool live = grp < ngrp;
         float a[16], deq[16];
@@ -91,7 +98,7 @@ __global__ void __launch_bounds__(256) k_quant_weight(const uint16_t* __restrict
             if (sf) sf[grp] = (uint8_t)sfb;
         }
         const uint32_t word = gather4(sfb);
-        if (live && (lane & 3) == 0) {
+        if (grp < ngrp_pad && (lane & 3) == 0) {
             const int64_t r = grp / G, q = grp % G;
             *reinterpret_cast<uint32_t*>(sf_swz + sf_swz_offset(r, q, K)) = word;
         }

@@ -8,19 +8,33 @@
 namespace mq {
 
 // ------------------------------------------------------------------ Delta-score
-// Persistent CTAs (4 warps) walk over the 64x64 blocks (nt, kt); TMA stages each block's
-// bf16 tile (64 rows x 128 bytes, 128-byte swizzle) into a ring of shared-memory buffers
-// ahead of the arithmetic. Warp q owns group column q (16 K elements); lane r owns block
-// rows r and r+32, so the first level of the fixed pairwise row tree (v[i] += v[i+32])
-// happens in registers. The remaining levels (+16, +8, +4, +2, +1) run as a butterfly
-// over the lanes that at each level also halves the set of columns a lane keeps: the
-// adds are exactly the tree's pairs, and at the end lanes 2c and 2c+1 hold column c of
-// the group. e and e' are recomputed from W and the tensor scale with the weight
-// quantizer's arithmetic, so they are bit-identical to the stored codes.
+// Persistent CTAs (8 warps) walk over strips of two vertically adjacent 64x64 blocks
+// (block rows 2i and 2i+1, block column kt); TMA stages each strip's bf16 tile (128 rows
+// x 128 bytes, 128-byte swizzle; rows past N read as zero) into a ring of shared-memory
+// buffers ahead of the arithmetic. Warp w works on block w / 4 of the strip and its group
+// column q = w % 4 (16 K elements); lane r owns the block's rows r and r+32, so the first
+// level of the fixed pairwise row tree (v[i] += v[i+32]) happens in registers. The
+// remaining levels (+16, +8, +4, +2, +1) run as a butterfly over the lanes that at each
+// level also halves the set of columns a lane keeps: the adds are exactly the tree's
+// pairs, and at the end lanes 2c and 2c+1 hold column c of the group. e and e' are
+// recomputed from W and the tensor scale with the weight quantizer's arithmetic, so they
+// are bit-identical to the stored codes.
 // tau = fma(e, e, -fp32(e'^2)) (fp32); the column sums are widened to fp64 for
 // p_k = H_k c_k and the 64-column tree.
+// Codes and scales are gathered in shared memory and written as whole 32-byte sectors:
+// a strip's 128 rows x 32 bytes of codes, and its 512-byte chunk of the GEMM's tiled scale
+// layout (one 128-row tile x 4 groups) at once.
 constexpr int kQDStages = 3;
-constexpr int kQDTile = 64 * 128;  // bytes of one staged block
+constexpr int kQDRows = 128;                   // rows of a strip
+constexpr int kQDTile = kQDRows * 128;         // bytes of one staged strip
+constexpr int kQDThreads = 256;
+constexpr int kQDStageOff = kQDStages * kQDTile;
+// staging after the tiles: codes [128][32], residual codes [128][32], tiled scales [512],
+// linear scales [128][4] and residual linear scales [128][4], column products [2][64]
+constexpr int kQDOffC = kQDStageOff, kQDOffRC = kQDOffC + 4096, kQDOffSw = kQDOffRC + 4096;
+constexpr int kQDOffSl = kQDOffSw + 512, kQDOffRSl = kQDOffSl + 512, kQDOffP = kQDOffRSl + 512;
+constexpr int kQDOffBar = kQDOffP + 2 * 64 * 8;
+constexpr size_t kQDSmem = kQDOffBar + 64 + 1024;
 
 // 16 values of row rl, group q of a staged tile (16-byte chunk c of a row sits at
 // chunk position c ^ (rl % 8): the TMA 128-byte swizzle).
@@ -35,34 +49,39 @@ __device__ __forceinline__ void tile_group(const uint8_t* tile, int rl, int q, f
     }
 }
 
-template <bool kWriteCodes>
-__device__ __forceinline__ void quant_delta_block(const uint8_t* tile, int K, const float* __restrict__ H, float g,
-                                                  int nt, int kt, uint8_t* __restrict__ codes,
-                                                  uint8_t* __restrict__ sf, uint8_t* __restrict__ sf_swz,
-                                                  uint8_t* __restrict__ rcodes, uint8_t* __restrict__ rsf,
-                                                  double* __restrict__ delta_out, double* pcol, uint32_t* sf_s,
-                                                  uint32_t* rsf_s) {
-    const int q = threadIdx.x >> 5, lane = threadIdx.x & 31;
+// One strip: quantization (when kWriteCodes), Delta of its one or two blocks, and the
+// coalesced stores. `nblk_rows` = N / 64.
+template <bool kWriteCodes, bool kWriteResid>
+__device__ __forceinline__ void quant_delta_strip(const uint8_t* tile, uint8_t* st, int K, int nblk_rows,
+                                                  const float* __restrict__ H, float g, int si, int kt,
+                                                  uint8_t* __restrict__ codes, uint8_t* __restrict__ sf,
+                                                  uint8_t* __restrict__ sf_swz, uint8_t* __restrict__ rcodes,
+                                                  uint8_t* __restrict__ rsf, double* __restrict__ delta) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int blk = warp >> 2, q = warp & 3;
+    const int KB = K / 64;
     const float g6 = __fmul_rn(6.0f, g);
-    float a2[2][16];
-#pragma unroll
-    for (int h = 0; h < 2; ++h) tile_group(tile, lane + 32 * h, q, a2[h]);
+    double* pcol = reinterpret_cast<double*>(st + kQDOffP) + blk * 64;
     float v[16];
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-        const int rl = lane + 32 * h;
-        const int64_t row = (int64_t)nt * 64 + rl;
+        const int rl = blk * 64 + lane + 32 * h;  // strip row
+        float a[16];
+        tile_group(tile, rl, q, a);
         float deq[16], R[16], rdeq[16];
         uint32_t lo, hi, rlo, rhi;
-        const uint32_t sfb = nvfp4_group(a2[h], g, g6, lo, hi, deq);
+        const uint32_t sfb = nvfp4_group(a, g, g6, lo, hi, deq);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) R[i] = __fsub_rn(a2[h][i], deq[i]);
+        for (int i = 0; i < 16; ++i) R[i] = __fsub_rn(a[i], deq[i]);
         const uint32_t rsb = nvfp4_group(R, g, g6, rlo, rhi, rdeq);
         if (kWriteCodes) {
-            *reinterpret_cast<uint2*>(codes + row * (K / 2) + kt * 32 + q * 8) = make_uint2(lo, hi);
-            *reinterpret_cast<uint2*>(rcodes + row * (K / 2) + kt * 32 + q * 8) = make_uint2(rlo, rhi);
-            reinterpret_cast<uint8_t*>(sf_s)[rl * 4 + q] = (uint8_t)sfb;
-            reinterpret_cast<uint8_t*>(rsf_s)[rl * 4 + q] = (uint8_t)rsb;
+            *reinterpret_cast<uint2*>(st + kQDOffC + rl * 32 + q * 8) = make_uint2(lo, hi);
+            st[kQDOffSw + (rl & 31) * 16 + (rl >> 5) * 4 + q] = (uint8_t)sfb;
+            st[kQDOffSl + rl * 4 + q] = (uint8_t)sfb;
+        }
+        if (kWriteResid) {
+            *reinterpret_cast<uint2*>(st + kQDOffRC + rl * 32 + q * 8) = make_uint2(rlo, rhi);
+            st[kQDOffRSl + rl * 4 + q] = (uint8_t)rsb;
         }
         // tau = fma(e, e, -fp32(e'^2)) with e = R, e' = R - deqR; the squares of e' are
         // taken in pairs
@@ -91,67 +110,87 @@ __device__ __forceinline__ void quant_delta_block(const uint8_t* tile, int K, co
     const int c = (lane >> 1) & 15;
     if ((lane & 1) == 0) pcol[q * 16 + c] = __dmul_rn((double)__ldg(H + kt * 64 + q * 16 + c), (double)colsum);
     __syncthreads();
-    if (q == 0) {
+    const int nt = 2 * si + blk;
+    if (q == 0 && nt < nblk_rows) {  // warps 0 and 4: the 64-column tree of their block
         double d = __dadd_rn(pcol[lane], pcol[lane + 32]);
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) d = __dadd_rn(d, __shfl_down_sync(0xffffffffu, d, o));
-        if (lane == 0) *delta_out = d;
+        if (lane == 0) delta[(int64_t)nt * KB + kt] = d;
     }
-    if (kWriteCodes && threadIdx.x < 64) {
-        const int64_t row = (int64_t)nt * 64 + threadIdx.x;
-        const uint32_t wsf = sf_s[threadIdx.x], wr = rsf_s[threadIdx.x];
-        if (sf) *reinterpret_cast<uint32_t*>(sf + row * (K / 16) + kt * 4) = wsf;
-        *reinterpret_cast<uint32_t*>(rsf + row * (K / 16) + kt * 4) = wr;
-        *reinterpret_cast<uint32_t*>(sf_swz + sf_swz_offset(row, (int64_t)kt * 4, K)) = wsf;
+    const int rows = min(kQDRows, (nblk_rows - 2 * si) * 64);  // rows of the strip inside W
+    const int t = threadIdx.x;
+    if (kWriteCodes) {
+        {   // codes: thread t writes half t % 2 of row t / 2 (two lanes make one sector)
+            const int r = t >> 1;
+            if (r < rows)
+                *reinterpret_cast<uint4*>(codes + (int64_t)(si * kQDRows + r) * (K / 2) + kt * 32 + 16 * (t & 1)) =
+                    *reinterpret_cast<const uint4*>(st + kQDOffC + r * 32 + 16 * (t & 1));
+        }
+        if (t < 32)  // the strip's 512-byte chunk of the tiled layout (rows past N: scale 0)
+            *reinterpret_cast<uint4*>(sf_swz + ((int64_t)si * KB + kt) * 512 + 16 * t) =
+                *reinterpret_cast<const uint4*>(st + kQDOffSw + 16 * t);
+        if (sf && t < rows)
+            *reinterpret_cast<uint32_t*>(sf + (int64_t)(si * kQDRows + t) * (K / 16) + kt * 4) =
+                *reinterpret_cast<const uint32_t*>(st + kQDOffSl + 4 * t);
+    }
+    if (kWriteResid) {
+        const int r = t >> 1;
+        if (r < rows)
+            *reinterpret_cast<uint4*>(rcodes + (int64_t)(si * kQDRows + r) * (K / 2) + kt * 32 + 16 * (t & 1)) =
+                *reinterpret_cast<const uint4*>(st + kQDOffRC + r * 32 + 16 * (t & 1));
+        if (t < rows)
+            *reinterpret_cast<uint32_t*>(rsf + (int64_t)(si * kQDRows + t) * (K / 16) + kt * 4) =
+                *reinterpret_cast<const uint32_t*>(st + kQDOffRSl + 4 * t);
     }
 }
 
-// A3 (kWriteCodes = false: Delta only, tensor scale read from g_in) and A1 + A3 in one
-// pass over W (kWriteCodes = true: codes, scales and Delta, tensor scale from the |W|
-// maximum partials). Persistent: CTA c handles blocks c, c + gridDim.x, ...
-template <bool kWriteCodes>
-__global__ void __launch_bounds__(128) k_quant_delta(const __grid_constant__ CUtensorMap tmap_w, int N, int K,
-                                                     const float* __restrict__ H, const float* __restrict__ g_in,
-                                                     uint8_t* __restrict__ codes, uint8_t* __restrict__ sf,
-                                                     uint8_t* __restrict__ sf_swz, float* __restrict__ g_out,
-                                                     uint8_t* __restrict__ rcodes, uint8_t* __restrict__ rsf,
-                                                     double* __restrict__ delta, int* __restrict__ err) {
+// kWriteCodes = false: Delta only, tensor scale read from g_in. kWriteCodes = true: base
+// codes and scales, Delta, and (kWriteResid) the full residual, in one pass over W; the
+// tensor scale comes from the |W| maximum partials. Persistent: CTA c handles strips c,
+// c + gridDim.x, ... in (strip row, kt) order, kt fastest.
+template <bool kWriteCodes, bool kWriteResid>
+__global__ void __launch_bounds__(kQDThreads, 3) k_quant_delta(const __grid_constant__ CUtensorMap tmap_w, int N, int K,
+                                                            const float* __restrict__ H, const float* __restrict__ g_in,
+                                                            uint8_t* __restrict__ codes, uint8_t* __restrict__ sf,
+                                                            uint8_t* __restrict__ sf_swz, float* __restrict__ g_out,
+                                                            uint8_t* __restrict__ rcodes, uint8_t* __restrict__ rsf,
+                                                            double* __restrict__ delta, int* __restrict__ err) {
     extern __shared__ uint8_t qd_raw[];
-    uint8_t* tiles = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(qd_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t* full = reinterpret_cast<uint64_t*>(tiles + kQDStages * kQDTile);
-    __shared__ double pcol[64];
-    __shared__ uint32_t sf_s[64], rsf_s[64];
-    griddep_wait();
-    griddep_launch();
-    const float g = kWriteCodes ? tensor_scale(g_in) : __ldg(g_in);
-    if (kWriteCodes && blockIdx.x == 0 && threadIdx.x == 0) *g_out = g;
-    const int KB = K / 64, NB = (N / 64) * KB;
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(qd_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(sm + kQDOffBar);
+    const int KB = K / 64, nbr = N / 64, nstrips = ((nbr + 1) / 2) * KB;
     if (threadIdx.x == 0) {
         for (int s = 0; s < kQDStages; ++s) mbar_init(&full[s], 1);
         mbar_fence_init();
         tma_prefetch_desc(&tmap_w);
     }
     __syncthreads();
-    auto issue = [&](int i) {  // block number i of this CTA into stage i % kQDStages
+    auto issue = [&](int i) {  // strip number i of this CTA into stage i % kQDStages
         const int b = blockIdx.x + i * gridDim.x;
-        if (b < NB) {
+        if (b < nstrips) {
             const int s = i % kQDStages;
             mbar_arrive_expect_tx(&full[s], kQDTile);
-            tma_load_2d_u16(tiles + s * kQDTile, &tmap_w, &full[s], (b % KB) * 64, (b / KB) * 64);
+            tma_load_2d_u16(sm + s * kQDTile, &tmap_w, &full[s], (b % KB) * 64, (b / KB) * kQDRows);
         }
     };
+    // W is an input of the call (never written by the preceding kernels): start loading
     if (threadIdx.x == 0)
         for (int i = 0; i < kQDStages; ++i) issue(i);
+    griddep_wait();
+    const float g = kWriteCodes ? tensor_scale(g_in) : __ldg(g_in);
+    if (kWriteCodes && blockIdx.x == 0 && threadIdx.x == 0) *g_out = g;
+    // the next kernel may start once every CTA has read the tensor-scale partials
+    griddep_launch();
     bool ok = true;
     for (int i = 0;; ++i) {
         const int b = blockIdx.x + i * gridDim.x;
-        if (b >= NB) break;
+        if (b >= nstrips) break;
         const int s = i % kQDStages;
         if (ok) ok = mbar_wait_err(&full[s], (i / kQDStages) & 1, err);
         if (ok)
-            quant_delta_block<kWriteCodes>(tiles + s * kQDTile, K, H, g, b / KB, b % KB, codes, sf, sf_swz, rcodes,
-                                           rsf, delta + b, pcol, sf_s, rsf_s);
-        __syncthreads();  // stage s and the block's shared scratch are free again
+            quant_delta_strip<kWriteCodes, kWriteResid>(sm + s * kQDTile, sm, K, nbr, H, g, b / KB, b % KB, codes,
+                                                        sf, sf_swz, rcodes, rsf, delta);
+        __syncthreads();  // stage s and the strip's staging are free again
         // every copy issued here is waited for by a later iteration of this loop
         if (threadIdx.x == 0 && ok) issue(i + kQDStages);
     }
@@ -319,50 +358,22 @@ __global__ void __launch_bounds__(kSelThreads) k_topk(const double* __restrict__
     }
 }
 
-// Top-K for budgets up to kSmallBudget, one CTA:
+// Top-K for budgets up to kSmallBudget, one CTA of 1024 threads:
 //  1. keys (order-preserving 64-bit images of Delta) and their common leading bits;
-//  2. 8-bit radix passes below the common prefix until at most kCandMax keys share the
-//     bucket that holds the budget-th largest key (warp-uniform digits add once);
-//  3. the keys of higher buckets (all selected) and the candidates of that bucket go
-//     into one list, sorted by (key descending, block index ascending), a strict total
-//     order: its first `budget` entries are rank; sel is the same set in ascending block
-//     index, from a bitmap scan.
-// If the keys tie beyond kCandMax candidates (the bucket is resolved to a single key
-// value), the selected set is compacted in block order instead (every key above the
-// value, then the lowest-index keys equal to it) and then sorted for rank.
+//  2. radix passes of up to 11 bits below the common prefix narrow the bucket that holds
+//     the budget-th largest key until it has at most kCandMax keys (or is one key value);
+//  3. every key above the bucket is selected; the bucket's candidates are ordered among
+//     themselves by (key descending, block index ascending) by counting, and the first
+//     `need` are selected (a bucket of one key value takes its lowest block indices);
+//  4. the `budget` selected pairs, one per thread, are sorted by the same strict order
+//     with a bitonic network (lane shuffles below stride 32, shared memory above): thread
+//     p then holds rank p. sel is the same set in ascending block index (bitmap scan).
 constexpr int kSmallBudget = 1024;
-constexpr int kCandMax = 512;
-constexpr int kSortCap = 2048;  // budget + candidates, a power of two
+constexpr int kCandMax = 64;
+constexpr int kDigitBits = 11;
 
 __device__ __forceinline__ bool before(uint64_t ka, int ia, uint64_t kb, int ib) {
     return ka > kb || (ka == kb && ia < ib);
-}
-
-// Bitonic sort of n2 (power of two, <= 2 * blockDim.x) (key, idx) pairs in shared memory
-// by (key descending, idx ascending). Pair p belongs to thread p; a warp's pairs cover 64
-// consecutive elements for strides below 64, which then need only __syncwarp.
-__device__ __forceinline__ void block_sort_desc(uint64_t* key, int32_t* idx, int n2) {
-    const int p = threadIdx.x;
-    const bool act = p < (n2 >> 1);
-    for (int k = 2, lk = 1; k <= n2; k <<= 1, ++lk) {
-        for (int j = k >> 1, lj = lk - 1; j > 0; j >>= 1, --lj) {
-            if (act) {
-                const int i = ((p >> lj) << (lj + 1)) | (p & (j - 1)), q = i + j;
-                const bool desc = (i & k) == 0;
-                const uint64_t ki = key[i], kq = key[q];
-                const int ii = idx[i], iq = idx[q];
-                if (before(kq, iq, ki, ii) == desc) {
-                    key[i] = kq;
-                    key[q] = ki;
-                    idx[i] = iq;
-                    idx[q] = ii;
-                }
-            }
-            const int jn = j > 1 ? (j >> 1) : k;  // the next stage's stride
-            if (j >= 64 || jn >= 64) __syncthreads();
-            else __syncwarp();
-        }
-    }
 }
 
 __device__ __forceinline__ uint64_t warp_and64(uint64_t v) {
@@ -376,18 +387,50 @@ __device__ __forceinline__ uint64_t warp_or64(uint64_t v) {
     return v;
 }
 
+// Bitonic sort of n2 (a power of two, <= blockDim.x) pairs by (key descending, idx
+// ascending); thread p holds pair p before and after. Every thread of the CTA calls it.
+__device__ __forceinline__ void block_bitonic(uint64_t& key, int& idx, int n2, uint64_t* skey, int* sidx) {
+    const int p = threadIdx.x;
+    for (int k = 2; k <= n2; k <<= 1) {
+        for (int j = k >> 1; j > 0; j >>= 1) {
+            uint64_t pk;
+            int pi;
+            if (j >= 32) {
+                skey[p] = key;
+                sidx[p] = idx;
+                __syncthreads();
+                pk = skey[p ^ j];
+                pi = sidx[p ^ j];
+                __syncthreads();
+            } else {
+                pk = __shfl_xor_sync(0xffffffffu, key, j);
+                pi = __shfl_xor_sync(0xffffffffu, idx, j);
+            }
+            // in a block sorted first-to-last the lower position keeps the earlier pair
+            const bool want_first = ((p & j) == 0) == ((p & k) == 0);
+            const bool partner_first = before(pk, pi, key, idx);
+            if (p < n2 && partner_first == want_first) {
+                key = pk;
+                idx = pi;
+            }
+        }
+    }
+}
+
 template <bool kSmemKeys>
 __global__ void __launch_bounds__(kSelThreads) k_topk_small(const double* __restrict__ delta, int B, int budget,
                                                             int32_t* __restrict__ rank, int32_t* __restrict__ sel) {
     extern __shared__ __align__(16) uint64_t dyn[];
-    uint64_t* keys = dyn;                                         // [B] when kSmemKeys
-    uint64_t* skey = dyn + (kSmemKeys ? B : 0);                   // [kSortCap]
-    int32_t* sidx = reinterpret_cast<int32_t*>(skey + kSortCap);  // [kSortCap]
-    uint32_t* bits = reinterpret_cast<uint32_t*>(sidx + kSortCap); // [ceil(B / 32)]
-    __shared__ unsigned hist[256];
+    uint64_t* keys = dyn;                                           // [B] when kSmemKeys
+    uint64_t* skey = dyn + (kSmemKeys ? B : 0);                     // [kSelThreads]
+    int32_t* sidx = reinterpret_cast<int32_t*>(skey + kSelThreads); // [kSelThreads]
+    uint32_t* bits = reinterpret_cast<uint32_t*>(sidx + kSelThreads); // [ceil(B / 32)]
+    __shared__ unsigned hist[1 << kDigitBits];
     __shared__ uint64_t s_and[32], s_or[32];
     __shared__ uint64_t s_prefix;
-    __shared__ int s_pos, s_need, s_cand, s_nsel;
+    __shared__ int s_pos, s_need, s_cand, s_nsel, s_ncand;
+    __shared__ uint64_t ckey[kCandMax];
+    __shared__ int cidx[kCandMax];
     __shared__ int scratch[32];
     griddep_wait();  // Delta comes from the previous kernel
     griddep_launch();
@@ -408,10 +451,8 @@ __global__ void __launch_bounds__(kSelThreads) k_topk_small(const double* __rest
     if (lane == 0) { s_and[warp] = a; s_or[warp] = o; }
     __syncthreads();
     if (warp == 0) {
-        a = s_and[lane];
-        o = s_or[lane];
-        a = warp_and64(a);
-        o = warp_or64(o);
+        a = warp_and64(s_and[lane]);
+        o = warp_or64(s_or[lane]);
         if (lane == 0) {
             const int cp = (a ^ o) ? __clzll((long long)(a ^ o)) : 64;  // common leading bits
             s_pos = 64 - cp;
@@ -419,83 +460,67 @@ __global__ void __launch_bounds__(kSelThreads) k_topk_small(const double* __rest
             s_need = budget;
             s_cand = B;
             s_nsel = 0;
+            s_ncand = 0;
         }
     }
     __syncthreads();
-    // radix passes below the common prefix
+    // radix passes: the bucket (keys sharing the bits above s_pos with s_prefix) holds
+    // the budget-th largest key; s_need of its keys are still to be taken
     while (s_pos > 0 && s_cand > kCandMax) {
-        const int pos = s_pos, w = pos < 8 ? pos : 8, shift = pos - w;
+        const int pos = s_pos, w = pos < kDigitBits ? pos : kDigitBits, shift = pos - w;
         const uint64_t prefix = s_prefix, hi = pos >= 64 ? 0ull : (~0ull << pos);
-        if (tid < 256) hist[tid] = 0;
+        const int need = s_need;  // read before the owner of the bucket rewrites it
+        const int nb = 1 << w;
+        for (int b = tid; b < nb; b += kSelThreads) hist[b] = 0;
         __syncthreads();
-        for (int i0 = tid - lane; i0 < B; i0 += kSelThreads) {
-            const int i = i0 + lane;
-            unsigned digit = 256u;
-            if (i < B) {
-                const uint64_t k = key_of(i);
-                if ((k & hi) == prefix) digit = (unsigned)(k >> shift) & ((1u << w) - 1u);
-            }
-            const bool uniform = __all_sync(0xffffffffu, digit == __shfl_sync(0xffffffffu, digit, 0));
-            if (uniform) {
-                if (lane == 0 && digit < 256u) atomicAdd(&hist[digit], 32u);
-            } else if (digit < 256u) {
-                atomicAdd(&hist[digit], 1u);
-            }
+        for (int i = tid; i < B; i += kSelThreads) {
+            const uint64_t k = key_of(i);
+            if ((k & hi) == prefix) atomicAdd(&hist[(unsigned)(k >> shift) & (nb - 1)], 1u);
         }
         __syncthreads();
-        if (warp == 0) {
-            // bins from the top: lane l holds bins 255-8l .. 248-8l
-            unsigned cnt[8], tot = 0;
-#pragma unroll
-            for (int j = 0; j < 8; ++j) { cnt[j] = hist[255 - 8 * lane - j]; tot += cnt[j]; }
-            unsigned incl = tot;
-#pragma unroll
-            for (int d = 1; d < 32; d <<= 1) {
-                const unsigned y = __shfl_up_sync(0xffffffffu, incl, d);
-                if (lane >= d) incl += y;
-            }
-            const int need = s_need;
-            const unsigned hit = __ballot_sync(0xffffffffu, incl >= (unsigned)need);
-            const int first = __ffs(hit) - 1;
-            if (lane == first) {
-                unsigned cum = incl - tot;
-                int digit = 0;
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    if (cum + cnt[j] >= (unsigned)need) {
-                        digit = 255 - 8 * lane - j;
-                        s_cand = (int)cnt[j];
-                        break;
-                    }
-                    cum += cnt[j];
-                }
-                s_need = need - (int)cum;
-                s_prefix = prefix | ((uint64_t)digit << shift);
-                s_pos = shift;
-            }
+        // thread t owns the bins nb-1-2t and nb-2-2t (from the top)
+        const int b0 = nb - 1 - 2 * tid;
+        const unsigned c0 = b0 >= 0 ? hist[b0] : 0u, c1 = b0 - 1 >= 0 ? hist[b0 - 1] : 0u;
+        int total;
+        const int above = block_exclusive_sum<kSelThreads>((int)(c0 + c1), scratch, total);
+        if (b0 >= 0 && above < need && above + (int)(c0 + c1) >= need) {
+            const bool first = above + (int)c0 >= need;
+            const int digit = first ? b0 : b0 - 1;
+            s_need = need - (first ? above : above + (int)c0);
+            s_cand = (int)(first ? c0 : c1);
+            s_prefix = prefix | ((uint64_t)digit << shift);
+            s_pos = shift;
         }
         __syncthreads();
     }
     const int pos = s_pos, need = s_need;
     const uint64_t prefix = s_prefix, hi = pos >= 64 ? 0ull : (~0ull << pos);
     if (s_cand <= kCandMax) {
-        // every key above the bucket plus the bucket's candidates, then one sort
+        // keys above the bucket are selected; the bucket's keys are candidates
         for (int i = tid; i < B; i += kSelThreads) {
-            const uint64_t k = key_of(i);
-            const uint64_t kh = k & hi;
-            if (kh >= prefix) {
+            const uint64_t k = key_of(i), kh = k & hi;
+            if (kh > prefix) {
                 const int slot = atomicAdd(&s_nsel, 1);
                 skey[slot] = k;
                 sidx[slot] = i;
+            } else if (kh == prefix) {
+                const int slot = atomicAdd(&s_ncand, 1);
+                ckey[slot] = k;
+                cidx[slot] = i;
             }
         }
         __syncthreads();
-        const int nsel = s_nsel;
-        int n2 = 2;
-        while (n2 < nsel) n2 <<= 1;
-        for (int e = nsel + tid; e < n2; e += kSelThreads) { skey[e] = 0ull; sidx[e] = 0x7FFFFFFF - e; }
-        __syncthreads();
-        block_sort_desc(skey, sidx, n2);
+        const int nsel = s_nsel, nc = s_ncand;
+        if (tid < nc) {
+            const uint64_t mk = ckey[tid];
+            const int mi = cidx[tid];
+            int r = 0;
+            for (int j = 0; j < nc; ++j) r += before(ckey[j], cidx[j], mk, mi);
+            if (r < need) {
+                skey[nsel + r] = mk;
+                sidx[nsel + r] = mi;
+            }
+        }
     } else {
         // the bucket is a single key value T shared by more than kCandMax keys: keys above
         // T and the lowest-index `need` keys equal to T, compacted in block order
@@ -519,18 +544,21 @@ __global__ void __launch_bounds__(kSelThreads) k_topk_small(const double* __rest
             if (k == T) take = eq_seen++ < need;
             if (take) { skey[out] = k; sidx[out] = i; ++out; }
         }
-        __syncthreads();
-        int n2 = 2;
-        while (n2 < budget) n2 <<= 1;
-        for (int e = budget + tid; e < n2; e += kSelThreads) { skey[e] = 0ull; sidx[e] = 0x7FFFFFFF - e; }
-        __syncthreads();
-        block_sort_desc(skey, sidx, n2);
-    }
-    for (int e = tid; e < budget; e += kSelThreads) {
-        rank[e] = sidx[e];
-        atomicOr(&bits[sidx[e] >> 5], 1u << (sidx[e] & 31));
     }
     __syncthreads();
+    // exactly `budget` selected pairs in skey/sidx: sort them, one per thread
+    int n2 = 32;
+    while (n2 < budget) n2 <<= 1;
+    uint64_t key = 0ull;
+    int idx = 0x7FFFFFFF - tid;  // padding sorts after every block
+    if (tid < budget) {
+        key = skey[tid];
+        idx = sidx[tid];
+        atomicOr(&bits[idx >> 5], 1u << (idx & 31));
+    }
+    __syncthreads();
+    block_bitonic(key, idx, n2, skey, sidx);
+    if (tid < budget) rank[tid] = idx;
     // sel: the set bits in index order (each thread scans a run of bitmap words)
     const int per = (nw + kSelThreads - 1) / kSelThreads;
     const int w0 = min(nw, tid * per), w1 = min(nw, w0 + per);
@@ -574,39 +602,11 @@ __global__ void __launch_bounds__(256) k_topk_rank(const double* __restrict__ de
 }
 
 // ------------------------------------------------------------------ pack
-// CTAs [0, budget): copy selected block i into the MMA's no-swizzle K-major layout and
-// its scales into the 128-row scale chunk of its band. The remaining CTAs build the
-// per-block-row CSR and bitmap (one thread per block row).
-__global__ void __launch_bounds__(256) k_pack(const uint8_t* __restrict__ rcodes, const uint8_t* __restrict__ rsf,
-                                              int N, int K, const int32_t* __restrict__ sel, int budget,
-                                              uint8_t* __restrict__ blk_codes, uint8_t* __restrict__ blk_sf,
-                                              int32_t* __restrict__ blk_kt, int32_t* __restrict__ tile_ptr,
-                                              uint32_t* __restrict__ bitmap) {
-    griddep_wait();
-    griddep_launch();
-    const int KB = K / 64, NBr = N / 64, KW = (KB + 31) / 32;
-    if ((int)blockIdx.x < budget) {
-        const int i = blockIdx.x;
-        const int b = __ldg(sel + i), nt = b / KB, kt = b % KB;
-        const int t = threadIdx.x;
-        {   // codes: row r, bytes 8*c8 .. 8*c8+7 of the block row
-            const int r = t >> 2, c8 = t & 3, j = 8 * c8;
-            const uint2 v = __ldg(reinterpret_cast<const uint2*>(rcodes + (int64_t)(nt * 64 + r) * (K / 2) + kt * 32 + j));
-            const int off = (r >> 3) * 256 + (j >> 4) * 128 + (r & 7) * 16 + (j & 15);
-            *reinterpret_cast<uint2*>(blk_codes + (int64_t)i * 2048 + off) = v;
-        }
-        if (t < 128) {  // scales: the block's 64 rows, zeros for the other half of the band
-            const int half = nt & 1;
-            const int tr = t;  // tile row 0..127
-            uint32_t v = 0;
-            if ((tr >> 6) == half)
-                v = __ldg(reinterpret_cast<const uint32_t*>(rsf + (int64_t)(nt * 64 + (tr & 63)) * (K / 16) + kt * 4));
-            *reinterpret_cast<uint32_t*>(blk_sf + (int64_t)i * 512 + (tr & 31) * 16 + (tr >> 5) * 4) = v;
-        }
-        if (t == 0) blk_kt[i] = kt;
-        return;
-    }
-    const int nt = (blockIdx.x - budget) * blockDim.x + threadIdx.x;
+// Per-block-row CSR (tile_ptr) and selection bitmap of the ascending selection `sel`, one
+// thread per block row nt.
+__device__ __forceinline__ void pack_rows(int nt, int NBr, int KB, const int32_t* __restrict__ sel, int budget,
+                                          int32_t* __restrict__ tile_ptr, uint32_t* __restrict__ bitmap) {
+    const int KW = (KB + 31) / 32;
     if (nt >= NBr) return;
     auto lower_bound = [&](int key) {
         int lo = 0, hi = budget;
@@ -633,30 +633,119 @@ __global__ void __launch_bounds__(256) k_pack(const uint8_t* __restrict__ rcodes
     }
 }
 
+// Byte offset of packed byte j (0..31) of block row r in the MMA's no-swizzle K-major
+// operand layout (8-row x 16-byte core matrices).
+__device__ __forceinline__ int core_offset(int r, int j) { return (r >> 3) * 256 + (j >> 4) * 128 + (r & 7) * 16 + (j & 15); }
+
+// CTAs [0, budget): copy selected block i into the MMA's no-swizzle K-major layout and
+// its scales into the 128-row scale chunk of its band. The remaining CTAs build the
+// per-block-row CSR and bitmap (one thread per block row).
+__global__ void __launch_bounds__(256) k_pack(const uint8_t* __restrict__ rcodes, const uint8_t* __restrict__ rsf,
+                                              int N, int K, const int32_t* __restrict__ sel, int budget,
+                                              uint8_t* __restrict__ blk_codes, uint8_t* __restrict__ blk_sf,
+                                              int32_t* __restrict__ blk_kt, int32_t* __restrict__ tile_ptr,
+                                              uint32_t* __restrict__ bitmap) {
+    griddep_wait();
+    griddep_launch();
+    const int KB = K / 64;
+    if ((int)blockIdx.x < budget) {
+        const int i = blockIdx.x;
+        const int b = __ldg(sel + i), nt = b / KB, kt = b % KB;
+        const int t = threadIdx.x;
+        {   // codes: row r, bytes 8*c8 .. 8*c8+7 of the block row
+            const int r = t >> 2, j = 8 * (t & 3);
+            const uint2 v = __ldg(reinterpret_cast<const uint2*>(rcodes + (int64_t)(nt * 64 + r) * (K / 2) + kt * 32 + j));
+            *reinterpret_cast<uint2*>(blk_codes + (int64_t)i * 2048 + core_offset(r, j)) = v;
+        }
+        if (t < 128) {  // scales: the block's 64 rows, zeros for the other half of the band
+            const int half = nt & 1;
+            const int tr = t;  // tile row 0..127
+            uint32_t v = 0;
+            if ((tr >> 6) == half)
+                v = __ldg(reinterpret_cast<const uint32_t*>(rsf + (int64_t)(nt * 64 + (tr & 63)) * (K / 16) + kt * 4));
+            *reinterpret_cast<uint32_t*>(blk_sf + (int64_t)i * 512 + (tr & 31) * 16 + (tr >> 5) * 4) = v;
+        }
+        if (t == 0) blk_kt[i] = kt;
+        return;
+    }
+    pack_rows((blockIdx.x - budget) * blockDim.x + threadIdx.x, N / 64, KB, sel, budget, tile_ptr, bitmap);
+}
+
+// Pack straight from W: CTAs [0, budget) recompute the residual of selected block i with
+// the weight quantizer's arithmetic (base group, R = W - deq, NVFP4(R) with the same
+// tensor scale), bit-identical to packing the full residual; the full residual is never
+// stored. Warp q handles group column q, lane r the block rows r and r+32. The remaining
+// CTAs build the CSR and bitmap.
+__global__ void __launch_bounds__(128) k_pack_w(const uint16_t* __restrict__ W, int N, int K,
+                                                const float* __restrict__ g_w, const int32_t* __restrict__ sel,
+                                                int budget, uint8_t* __restrict__ blk_codes,
+                                                uint8_t* __restrict__ blk_sf, int32_t* __restrict__ blk_kt,
+                                                int32_t* __restrict__ tile_ptr, uint32_t* __restrict__ bitmap) {
+    griddep_wait();
+    griddep_launch();
+    const int KB = K / 64;
+    if ((int)blockIdx.x >= budget) {
+        pack_rows((blockIdx.x - budget) * blockDim.x + threadIdx.x, N / 64, KB, sel, budget, tile_ptr, bitmap);
+        return;
+    }
+    __shared__ __align__(16) uint32_t chunk[128];  // the block's positioned 512-byte scale chunk
+    const int i = blockIdx.x, t = threadIdx.x, q = t >> 5, lane = t & 31;
+    const int b = __ldg(sel + i), nt = b / KB, kt = b % KB;
+    const float g = __ldg(g_w), g6 = __fmul_rn(6.0f, g);
+    chunk[t] = 0u;
+    __syncthreads();
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const int r = lane + 32 * h;
+        const uint4* src = reinterpret_cast<const uint4*>(W + (int64_t)(nt * 64 + r) * K + kt * 64 + q * 16);
+        const uint4 v0 = __ldg(src), v1 = __ldg(src + 1);
+        const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+        float a[16], deq[16], R[16], rdeq[16];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            a[2 * j] = bf16_bits_to_f32(w[j] & 0xFFFFu);
+            a[2 * j + 1] = bf16_bits_to_f32(w[j] >> 16);
+        }
+        uint32_t lo, hi, rlo, rhi;
+        nvfp4_group(a, g, g6, lo, hi, deq);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) R[j] = __fsub_rn(a[j], deq[j]);
+        const uint32_t rsb = nvfp4_group(R, g, g6, rlo, rhi, rdeq);
+        *reinterpret_cast<uint2*>(blk_codes + (int64_t)i * 2048 + core_offset(r, 8 * q)) = make_uint2(rlo, rhi);
+        const int tr = 64 * (nt & 1) + r;
+        reinterpret_cast<uint8_t*>(chunk)[(tr & 31) * 16 + (tr >> 5) * 4 + q] = (uint8_t)rsb;
+    }
+    __syncthreads();
+    if (t < 32) reinterpret_cast<uint4*>(blk_sf + (int64_t)i * 512)[t] = reinterpret_cast<const uint4*>(chunk)[t];
+    if (t == 0) blk_kt[i] = kt;
+}
+
 // ------------------------------------------------------------------ launchers
-static int quant_delta_grid(int NB) {
+static int quant_delta_grid(int nstrips) {
     static int per_sm = 0;
     if (!per_sm) {
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_quant_delta<true>, 128,
-                                                          kQDStages * kQDTile + 1024 + 64) != cudaSuccess ||
+        cudaFuncSetAttribute(k_quant_delta<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kQDSmem);
+        cudaFuncSetAttribute(k_quant_delta<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kQDSmem);
+        cudaFuncSetAttribute(k_quant_delta<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kQDSmem);
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_quant_delta<true, true>, kQDThreads, kQDSmem) !=
+                cudaSuccess ||
             per_sm < 1)
-            per_sm = 4;
+            per_sm = 2;
     }
     int sms = 148;
     int dev = 0;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int grid = per_sm * sms;
-    return NB < grid ? NB : grid;
+    return nstrips < grid ? nstrips : grid;
 }
 
-static const size_t kQDSmem = kQDStages * kQDTile + 1024 + 64;
+static int qd_strips(int N, int K) { return ((N / 64 + 1) / 2) * (K / 64); }
 
 cudaError_t launch_delta(const CUtensorMap& tw, int N, int K, const float* H, const float* g, double* delta,
                          int* err, cudaStream_t s) {
-    const int NB = (N / 64) * (K / 64);
-    return launch_pdl(k_quant_delta<false>, dim3(quant_delta_grid(NB)), dim3(128), kQDSmem, s, 1, tw, N, K, H, g,
-                      (uint8_t*)nullptr, (uint8_t*)nullptr, (uint8_t*)nullptr, (float*)nullptr, (uint8_t*)nullptr,
-                      (uint8_t*)nullptr, delta, err);
+    return launch_pdl(k_quant_delta<false, false>, dim3(quant_delta_grid(qd_strips(N, K))), dim3(kQDThreads),
+                      kQDSmem, s, 1, tw, N, K, H, g, (uint8_t*)nullptr, (uint8_t*)nullptr, (uint8_t*)nullptr,
+                      (float*)nullptr, (uint8_t*)nullptr, (uint8_t*)nullptr, delta, err);
 }
 
 cudaError_t launch_quant_delta(const uint16_t* W, const CUtensorMap& tw, int N, int K, const float* H,
@@ -664,15 +753,18 @@ cudaError_t launch_quant_delta(const uint16_t* W, const CUtensorMap& tw, int N, 
                                double* delta, float* partial, int* err, cudaStream_t s) {
     cudaError_t e = launch_amax(W, (int64_t)N * K, partial, s);
     if (e != cudaSuccess) return e;
-    const int NB = (N / 64) * (K / 64);
-    return launch_pdl(k_quant_delta<true>, dim3(quant_delta_grid(NB)), dim3(128), kQDSmem, s, 1, tw, N, K, H,
-                      (const float*)partial, codes, sf, sf_swz, g, rcodes, rsf, delta, err);
+    const dim3 grid(quant_delta_grid(qd_strips(N, K)));
+    if (rcodes)
+        return launch_pdl(k_quant_delta<true, true>, grid, dim3(kQDThreads), kQDSmem, s, 1, tw, N, K, H,
+                          (const float*)partial, codes, sf, sf_swz, g, rcodes, rsf, delta, err);
+    return launch_pdl(k_quant_delta<true, false>, grid, dim3(kQDThreads), kQDSmem, s, 1, tw, N, K, H,
+                      (const float*)partial, codes, sf, sf_swz, g, (uint8_t*)nullptr, (uint8_t*)nullptr, delta, err);
 }
 
 cudaError_t launch_topk(const double* delta, int B, int budget, int32_t* rank, int32_t* sel, cudaStream_t s) {
     if (budget <= 0) return cudaSuccess;
     if (budget <= kSmallBudget) {
-        const size_t tail = (size_t)kSortCap * 12 + (size_t)((B + 31) / 32) * 4;
+        const size_t tail = (size_t)kSelThreads * 12 + (size_t)((B + 31) / 32) * 4;
         const bool smem_keys = (size_t)B * 8 + tail <= kSelSmemKeysMax;
         const size_t smem = (smem_keys ? (size_t)B * 8 : 0) + tail;
         static bool attr[2] = {false, false};
@@ -713,6 +805,15 @@ cudaError_t launch_pack(const uint8_t* rcodes, const uint8_t* rsf, int N, int K,
     const int grid = budget + (NBr + 255) / 256;
     return launch_pdl(k_pack, dim3(grid), dim3(256), 0, s, 1, rcodes, rsf, N, K, sel, budget, blk_codes, blk_sf,
                       blk_kt, tile_ptr, bitmap);
+}
+
+cudaError_t launch_pack_w(const uint16_t* W, int N, int K, const float* g_w, const int32_t* sel, int budget,
+                          uint8_t* blk_codes, uint8_t* blk_sf, int32_t* blk_kt, int32_t* tile_ptr, uint32_t* bitmap,
+                          cudaStream_t s) {
+    const int NBr = N / 64;
+    const int grid = budget + (NBr + 127) / 128;
+    return launch_pdl(k_pack_w, dim3(grid), dim3(128), 0, s, 1, W, N, K, g_w, sel, budget, blk_codes, blk_sf, blk_kt,
+                      tile_ptr, bitmap);
 }
 
 }  // namespace mq

@@ -27,6 +27,7 @@ EXPORTED = (
     "mq_gemm_workspace_bytes", "mq_quantize_weight", "mq_hessian_diag", "mq_delta_score_topk", "mq_pack_residual",
     "mq_quantize_act", "mq_gemm", "mq_run_layer", "mq_get_error", "mq_status_string", "mq_launch_count",
     "mq_gemm_noalloc", "mq_gemm_noalloc_scratch_limit", "mq_quantize_weight_delta", "mq_topk_blocks",
+    "mq_pack_residual_weight",
 )
 
 
@@ -92,6 +93,8 @@ def lib():
     L.mq_quantize_weight_delta.restype = i32
     L.mq_topk_blocks.argtypes = [vp, i32, i32, vp, vp, vp]
     L.mq_topk_blocks.restype = i32
+    L.mq_pack_residual_weight.argtypes = [vp, P(NVFP4Mat), vp, i32, P(ResidualPacked), vp]
+    L.mq_pack_residual_weight.restype = i32
     L.mq_get_error.argtypes = [vp]
     L.mq_status_string.argtypes = [i32]
     L.mq_status_string.restype = ctypes.c_char_p
@@ -172,10 +175,12 @@ def mq_quantize_weight(W: torch.Tensor, base: dict, resid: dict, ws: torch.Tenso
                                     ws.numel() * ws.element_size(), _stream(stream)), "mq_quantize_weight")
 
 
-def mq_quantize_weight_delta(W: torch.Tensor, H: torch.Tensor, base: dict, resid: dict, delta: torch.Tensor,
+def mq_quantize_weight_delta(W: torch.Tensor, H: torch.Tensor, base: dict, resid: dict | None, delta: torch.Tensor,
                              ws: torch.Tensor, stream=None):
+    """resid None: the full residual is not stored (see mq_pack_residual_weight)."""
     N, K = W.shape
-    _check(lib().mq_quantize_weight_delta(_ptr(W), N, K, _ptr(H), ctypes.byref(mat(base)), ctypes.byref(mat(resid)),
+    r = None if resid is None else ctypes.byref(mat(resid))
+    _check(lib().mq_quantize_weight_delta(_ptr(W), N, K, _ptr(H), ctypes.byref(mat(base)), r,
                                           _ptr(delta), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
            "mq_quantize_weight_delta")
 
@@ -200,6 +205,12 @@ def mq_delta_score_topk(W, H, base: dict, resid: dict | None, budget: int, delta
 def mq_pack_residual(resid: dict, sel, budget: int, packed: dict, stream=None):
     _check(lib().mq_pack_residual(ctypes.byref(mat(resid)), _ptr(sel), budget, ctypes.byref(packed_struct(packed)),
                                   _stream(stream)), "mq_pack_residual")
+
+
+def mq_pack_residual_weight(W: torch.Tensor, base: dict, sel, budget: int, packed: dict, stream=None):
+    _check(lib().mq_pack_residual_weight(_ptr(W), ctypes.byref(mat(base)), _ptr(sel), budget,
+                                         ctypes.byref(packed_struct(packed)), _stream(stream)),
+           "mq_pack_residual_weight")
 
 
 def mq_quantize_act(X: torch.Tensor, xq: dict, stream=None):
@@ -276,11 +287,20 @@ class Layer:
         mq_pack_residual(self.resid, self.sel, self.budget, self.packed, stream)
 
     def prepare_fused(self, W: torch.Tensor, Xcal: torch.Tensor, stream=None):
-        """A1..A5 with quantization and Delta in one pass over W (as mq_run_layer)."""
+        """A1..A5 with quantization and Delta in one pass over W; the full residual is stored
+        and the selected blocks packed from it."""
         mq_hessian_diag(Xcal, self.H, stream)
         mq_quantize_weight_delta(W, self.H, self.base, self.resid, self.delta, self.qws, stream)
         mq_topk_blocks(self.delta, self.budget, self.rank, self.sel, stream)
         mq_pack_residual(self.resid, self.sel, self.budget, self.packed, stream)
+
+    def prepare_path(self, W: torch.Tensor, Xcal: torch.Tensor, stream=None):
+        """A1..A5 as mq_run_layer: the full residual is not stored; the selected blocks are
+        recomputed from W when packed."""
+        mq_hessian_diag(Xcal, self.H, stream)
+        mq_quantize_weight_delta(W, self.H, self.base, None, self.delta, self.qws, stream)
+        mq_topk_blocks(self.delta, self.budget, self.rank, self.sel, stream)
+        mq_pack_residual_weight(W, self.base, self.sel, self.budget, self.packed, stream)
 
     def act_buffers(self, M: int, flags: int = 0):
         key = (M, flags)

@@ -165,9 +165,13 @@ mq_status mq_delta_score_topk(const mq_bf16* W, const float* H, const mq_nvfp4_m
 
 /*
  * A1 + A3 in one pass over W (same results as mq_quantize_weight followed by the
- * Delta part of mq_delta_score_topk): base and full residual NVFP4 codes and scales, the
- * tensor scale, and Delta [(N/64)*(K/64)] (fp64), with H from mq_hessian_diag.
- * Buffers and workspace as in mq_quantize_weight; base->sf may be NULL.
+ * Delta part of mq_delta_score_topk): base NVFP4 codes and scales, the tensor scale,
+ * Delta [(N/64)*(K/64)] (fp64) with H from mq_hessian_diag, and, if resid_full is not
+ * NULL, the full residual's codes and sf. resid_full == NULL skips storing the residual
+ * (mq_pack_residual_weight recomputes the selected blocks from W). base->sf may be NULL.
+ * W is read before the call waits for the preceding kernel in the stream (it must not be
+ * written by a kernel that lets its dependents start early). Buffers and workspace as in
+ * mq_quantize_weight; base->codes and sf_swz 16-byte aligned.
  */
 mq_status mq_quantize_weight_delta(const mq_bf16* W, int N, int K, const float* H, mq_nvfp4_mat* base,
                                    mq_nvfp4_mat* resid_full, double* delta, void* ws, size_t ws_bytes,
@@ -187,6 +191,18 @@ mq_status mq_topk_blocks(const double* delta, int nblk, int budget, int32_t* ran
  */
 mq_status mq_pack_residual(const mq_nvfp4_mat* resid_full, const int32_t* sel, int budget,
                            mq_residual_packed* out, mq_stream stream);
+
+/*
+ * A5 straight from W: the selected blocks' residual is recomputed with the weight
+ * quantizer's arithmetic (base group, R = W - deq Q(W), NVFP4(R) with the tensor scale
+ * base->gscale) and written packed; the result is bit-identical to mq_pack_residual on
+ * mq_quantize_weight's resid_full, and the full residual never has to be stored.
+ * W: bf16 [N][K] (16-byte aligned). base: rows = N, cols = K, gscale (from
+ * mq_quantize_weight or mq_quantize_weight_delta); its codes are not read.
+ * sel: ascending block indices [budget]. out: as in mq_pack_residual.
+ */
+mq_status mq_pack_residual_weight(const mq_bf16* W, const mq_nvfp4_mat* base, const int32_t* sel, int budget,
+                                  mq_residual_packed* out, mq_stream stream);
 
 /*
  * A6. Activation quantization (summary, "Methodology", section 3: quantization inside
@@ -218,7 +234,7 @@ mq_status mq_gemm(const mq_nvfp4_mat* xq, const mq_nvfp4_mat* wq, const mq_resid
  */
 typedef struct {
     mq_nvfp4_mat base;        /* sf may be NULL */
-    mq_nvfp4_mat resid_full;  /* codes and sf */
+    mq_nvfp4_mat resid_full;  /* not used by mq_run_layer (may be all zero) */
     mq_nvfp4_mat xq;          /* codes, sf_swz, gscale [M] */
     float* H;                 /* [K] */
     double* delta;            /* [(N/64)*(K/64)] */
@@ -236,12 +252,14 @@ typedef struct {
 } mq_layer_buffers;
 
 /*
- * The whole path for one layer in the method's order: A1 quantize W, A2 H from the T
- * calibration tokens, A3+A4 Delta and top-`budget` selection, A5 pack, A6 quantize X,
- * A7+A8 fused GEMM into Y. With host == 0, W, X, Xcal and Y are device pointers. With
- * host != 0 they are HOST pointers (page-locked for the copies to be asynchronous):
- * the inputs are copied into buf->W_dev, X_dev, Xcal_dev and the result from buf->Y_dev
- * back to Y, all on `stream`. Errors as the individual calls.
+ * The whole path for one layer in the method's order: A2 H from the T calibration
+ * tokens, A1+A3 quantize W and score every block (mq_quantize_weight_delta, residual not
+ * stored), A4 top-`budget` selection, A5 pack the selected residual from W
+ * (mq_pack_residual_weight), A6 quantize X, A7+A8 fused GEMM into Y. With host == 0, W,
+ * X, Xcal and Y are device pointers. With host != 0 they are HOST pointers
+ * (page-locked for the copies to be asynchronous): the inputs are copied into
+ * buf->W_dev, X_dev, Xcal_dev and the result from buf->Y_dev back to Y, all on
+ * `stream`. Errors as the individual calls.
  */
 mq_status mq_run_layer(const mq_bf16* W, const mq_bf16* X, const mq_bf16* Xcal, mq_bf16* Y, int M, int N, int K,
                        int T, int budget, unsigned flags, int host, mq_layer_buffers* buf, mq_stream stream);

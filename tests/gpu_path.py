@@ -13,16 +13,27 @@ def to_dev(bits: np.ndarray, dev) -> torch.Tensor:
     return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
 
 
-def gpu_run(L: dict, budget: int, dev, flags: int = 0, X_bits=None, fused: bool = False):
+def prepare(layer, W, Xc, fused):
+    """fused: False = separate calls, True = one quantize+Delta pass with the full residual
+    stored and packed from it, "path" = as mq_run_layer (residual packed from W)."""
+    if fused == "path":
+        layer.prepare_path(W, Xc)
+    elif fused:
+        layer.prepare_fused(W, Xc)
+    else:
+        layer.prepare(W, Xc)
+
+
+def gpu_run(L: dict, budget: int, dev, flags: int = 0, X_bits=None, fused=False):
     """Whole path on the GPU for layer inputs L (bf16 bits); returns numpy copies.
-    fused=True quantizes and scores W in one pass (mq_quantize_weight_delta)."""
+    fused: see prepare()."""
     from bit_quantized_gemm_zipperengine_b200 import mosaic
     N, K = L["N"], L["K"]
     W = to_dev(L["W"], dev)
     Xc = to_dev(L["Xcal"], dev)
     X = to_dev(L["X"] if X_bits is None else X_bits, dev)
     layer = mosaic.Layer(N, K, budget, dev)
-    (layer.prepare_fused if fused else layer.prepare)(W, Xc)
+    prepare(layer, W, Xc, fused)
     Y = layer.forward(X, flags)
     xq = layer.act_buffers(X.shape[0], flags)[0]
     torch.cuda.synchronize()

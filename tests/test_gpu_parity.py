@@ -7,7 +7,7 @@ import torch
 
 import oracle
 import synth
-from gpu_path import check_gemm, gpu_run, oracle_ref, to_dev
+from gpu_path import check_gemm, gpu_run, oracle_ref, prepare, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -35,7 +35,7 @@ def _pair(name, dev, M=None, fused=False):
 
 
 WORKLOADS = ["tiny", "llama3_8b_qproj_decode"]
-PATHS = [pytest.param(False, id="separate"), pytest.param(True, id="fused")]
+PATHS = [pytest.param(False, id="separate"), pytest.param(True, id="fused"), pytest.param("path", id="path")]
 
 
 @pytest.mark.parametrize("fused", PATHS)
@@ -47,8 +47,9 @@ def test_quantize_weight_bit_exact(name, fused, dev):
     assert np.array_equal(g["codes"], wq["codes"])
     assert np.array_equal(g["sf"], wq["sf"])
     assert np.array_equal(g["sf_swz"], oracle.sf_tile(wq["sf"], L["N"], L["K"]))
-    assert np.array_equal(g["r_codes"], wq["r_codes"])
-    assert np.array_equal(g["r_sf"], wq["r_sf"])
+    if fused != "path":  # the run_layer route does not store the full residual
+        assert np.array_equal(g["r_codes"], wq["r_codes"])
+        assert np.array_equal(g["r_sf"], wq["r_sf"])
 
 
 @pytest.mark.parametrize("fused", PATHS)
@@ -260,3 +261,34 @@ def test_run_layer_whole_path(host, dev):
     assert mosaic.mq_get_error() == 0
     assert np.array_equal(layer.sel[:budget].cpu().numpy(), o["sel"])
     check_gemm(Y.float().cpu().numpy().astype(np.float64), o["y"], o["yabs"], f"run_layer host={host}")
+
+
+@pytest.mark.parametrize("fused", PATHS)
+def test_odd_block_rows_bit_exact(fused, dev):
+    """N / 64 odd (5 block rows): the quantize+Delta pass works on strips of two block rows,
+    and the last strip holds a single block; codes, tiled scales, Delta, the selection and
+    the packed store must still match the oracle bit for bit."""
+    from bit_quantized_gemm_zipperengine_b200 import mosaic
+    N, K, T = 320, 512, 64
+    Wb = synth.weight(N, K, 801, 804, 0.02, int(0.005 * N * K), 4, 20.0)
+    Cb = synth.act(T, K, 803, 804, 8, 30.0)
+    budget = synth.budget_blocks(N, K, 0.10)
+    wq = oracle.quantize_weight(Wb)
+    H = oracle.hessian_diag(Cb)
+    delta = oracle.delta_score(Wb, H, wq)
+    rank, sel = oracle.topk(delta, budget)
+    packed = oracle.pack_residual(wq, sel, N, K)
+    layer = mosaic.Layer(N, K, budget, dev)
+    prepare(layer, to_dev(Wb, dev), to_dev(Cb, dev), fused)
+    torch.cuda.synchronize()
+    assert mosaic.mq_get_error() == 0
+    assert layer.base["gscale"].cpu().numpy()[0] == wq["g"]
+    assert np.array_equal(layer.base["codes"].cpu().numpy(), wq["codes"])
+    assert np.array_equal(layer.base["sf_swz"].cpu().numpy(), oracle.sf_tile(wq["sf"], N, K))
+    assert np.array_equal(layer.delta.cpu().numpy().view(np.uint64), delta.ravel().view(np.uint64))
+    assert np.array_equal(layer.rank[:budget].cpu().numpy(), rank)
+    assert np.array_equal(layer.sel[:budget].cpu().numpy(), sel)
+    for k in ("blk_codes", "blk_sf", "blk_kt"):
+        assert np.array_equal(layer.packed[k][:budget].cpu().numpy(), packed[k]), k
+    assert np.array_equal(layer.packed["tile_ptr"].cpu().numpy(), packed["tile_ptr"])
+    assert np.array_equal(layer.packed["bitmap"].cpu().numpy().view(np.uint32), packed["bitmap"])
