@@ -22,6 +22,7 @@ cudaError_t launch_quant_delta(const uint16_t* W, const CUtensorMap& tw, int N, 
                                uint8_t* codes, uint8_t* sf, uint8_t* sf_swz, float* g, uint8_t* rcodes, uint8_t* rsf,
                                double* delta, float* partial, int* err, cudaStream_t s);
 cudaError_t launch_topk(const double* delta, int B, int budget, int32_t* rank, int32_t* sel, cudaStream_t s);
+int topk_launches(int budget);
 cudaError_t launch_pack(const uint8_t* rcodes, const uint8_t* rsf, int N, int K, const int32_t* sel, int budget,
                         uint8_t* blk_codes, uint8_t* blk_sf, int32_t* blk_kt, int32_t* tile_ptr, uint32_t* bitmap,
                         cudaStream_t s);
@@ -181,7 +182,7 @@ mq_status mq_delta_score_topk(const mq_bf16* W, const float* H, const mq_nvfp4_m
     cudaError_t e = launch_delta(tw, N, K, H, base->gscale, delta, err, s);
     if (e != cudaSuccess) return MQ_ERR_CUDA;
     g_launches.fetch_add(1);
-    return launched(launch_topk(delta, B, budget, rank, sel, s), budget <= 0 ? 0 : budget <= 1024 ? 1 : 2);
+    return launched(launch_topk(delta, B, budget, rank, sel, s), topk_launches(budget));
 }
 
 mq_status mq_quantize_weight_delta(const mq_bf16* W, int N, int K, const float* H, mq_nvfp4_mat* base,
@@ -209,8 +210,7 @@ mq_status mq_quantize_weight_delta(const mq_bf16* W, int N, int K, const float* 
 mq_status mq_topk_blocks(const double* delta, int nblk, int budget, int32_t* rank, int32_t* sel, mq_stream stream) {
     if (!delta || nblk <= 0 || budget < 0 || budget > nblk) return MQ_ERR_INVALID_ARG;
     if (budget > 0 && (!rank || !sel)) return MQ_ERR_INVALID_ARG;
-    const int kernels = budget <= 0 ? 0 : budget <= 1024 ? 1 : 2;
-    return launched(launch_topk(delta, nblk, budget, rank, sel, as_stream(stream)), kernels);
+    return launched(launch_topk(delta, nblk, budget, rank, sel, as_stream(stream)), topk_launches(budget));
 }
 
 mq_status mq_pack_residual(const mq_nvfp4_mat* resid_full, const int32_t* sel, int budget, mq_residual_packed* out,

@@ -242,6 +242,12 @@ __global__ void __launch_bounds__(192, 1)
         if (elect_one())
             for (int it = 0; it < first; ++it) issue_w(it);  // nothing to wait for yet
         __syncwarp();
+        griddep_wait();
+        if (elect_one())
+            for (int it = 0; it < first; ++it) issue_x(it);
+        __syncwarp();
+        // the residual lookups (dependent index loads) run while W and X are in flight;
+        // the base MMAs of a stage do not wait for its residual blocks
         if (p.has_resid && n_iters > 0) {
             cur0 = row_cursor(p, n_tile * 2 + 0, ks_begin * 4);
             cur1 = row_cursor(p, n_tile * 2 + 1, ks_begin * 4);
@@ -252,10 +258,6 @@ __global__ void __launch_bounds__(192, 1)
             if (elect_one()) issue_resid(it, m, idx0, idx1);
             __syncwarp();
         }
-        griddep_wait();
-        if (elect_one())
-            for (int it = 0; it < first; ++it) issue_x(it);
-        __syncwarp();
         int issued = first;
         for (int it = first; it < n_iters; ++it) {
             const int st_i = it % C::kStages;
@@ -412,15 +414,35 @@ __global__ void __launch_bounds__(192, 1)
             const int r0 = (int)(r * 128 / S), r1 = (int)((r + 1) * 128 / S), rows = r1 - r0;
             const float* red = reinterpret_cast<const float*>(smem);
             const float gw = __ldg(p.g_w);
-            for (int e = threadIdx.x - 64; e < rows * BN; e += 128) {
-                const int j = e / rows, nl = r0 + e % rows;
-                const int mm = m0 + j;
-                float sum = ld_dsmem_f32(red + j * 128 + nl, 0);
-                for (uint32_t s2 = 1; s2 < S; ++s2) sum = __fadd_rn(sum, ld_dsmem_f32(red + j * 128 + nl, s2));
-                if (mm < p.M) {
-                    const float sc = __fmul_rn(__ldg(p.g_x + mm), gw);
-                    const __nv_bfloat16 y = __float2bfloat16_rn(__fmul_rn(sum, sc));
-                    p.Y[(int64_t)mm * p.N + n0 + nl] = *reinterpret_cast<const uint16_t*>(&y);
+            // kU elements per thread at a time: all their peers' partials are requested
+            // before the first add, then added in split order
+            constexpr int kU = 4;
+            const int total = rows * BN;
+            for (int e0 = threadIdx.x - 64; e0 < total; e0 += 128 * kU) {
+                float v[kU][kMaxClusterSplits];
+#pragma unroll
+                for (int u = 0; u < kU; ++u) {
+                    const int e = min(e0 + 128 * u, total - 1);
+                    const int j = e / rows, nl = r0 + e % rows;
+#pragma unroll
+                    for (uint32_t s2 = 0; s2 < (uint32_t)kMaxClusterSplits; ++s2)
+                        if (s2 < S) v[u][s2] = ld_dsmem_f32(red + j * 128 + nl, s2);
+                }
+#pragma unroll
+                for (int u = 0; u < kU; ++u) {
+                    const int e = e0 + 128 * u;
+                    if (e >= total) break;
+                    const int j = e / rows, nl = r0 + e % rows;
+                    const int mm = m0 + j;
+                    float sum = v[u][0];
+#pragma unroll
+                    for (uint32_t s2 = 1; s2 < (uint32_t)kMaxClusterSplits; ++s2)
+                        if (s2 < S) sum = __fadd_rn(sum, v[u][s2]);
+                    if (mm < p.M) {
+                        const float sc = __fmul_rn(__ldg(p.g_x + mm), gw);
+                        const __nv_bfloat16 y = __float2bfloat16_rn(__fmul_rn(sum, sc));
+                        p.Y[(int64_t)mm * p.N + n0 + nl] = *reinterpret_cast<const uint16_t*>(&y);
+                    }
                 }
             }
         }

@@ -362,15 +362,19 @@ __global__ void __launch_bounds__(kSelThreads) k_topk(const double* __restrict__
 //  1. keys (order-preserving 64-bit images of Delta) and their common leading bits;
 //  2. radix passes of up to 11 bits below the common prefix narrow the bucket that holds
 //     the budget-th largest key until it has at most kCandMax keys (or is one key value);
-//  3. every key above the bucket is selected; the bucket's candidates are ordered among
-//     themselves by (key descending, block index ascending) by counting, and the first
-//     `need` are selected (a bucket of one key value takes its lowest block indices);
-//  4. the `budget` selected pairs, one per thread, are sorted by the same strict order
-//     with a bitonic network (lane shuffles below stride 32, shared memory above): thread
-//     p then holds rank p. sel is the same set in ascending block index (bitmap scan).
-constexpr int kSmallBudget = 1024;
-constexpr int kCandMax = 64;
+//  3. every key above the bucket and every key in it (at most budget + kCandMax <= 1024)
+//     are sorted by (key descending, block index ascending), a strict total order: the
+//     first `budget` are rank. (A bucket of one key value shared by more than kCandMax
+//     keys takes its lowest block indices instead, and only the `budget` selected keys
+//     are sorted.) sel is the same set in ascending block index (bitmap scan).
+// The sort: each warp sorts 32 pairs in registers (bitonic network over lane shuffles),
+// then sorted runs are merged pairwise: a pair's place in the merged run is its place in
+// its own run plus the number of pairs of the partner run that come before it (binary
+// search), so every pair moves once per merge level.
+constexpr int kSmallBudget = 768;
+constexpr int kCandMax = 256;
 constexpr int kDigitBits = 11;
+static_assert(kSmallBudget + kCandMax <= 1024, "one pair per thread");
 
 __device__ __forceinline__ bool before(uint64_t ka, int ia, uint64_t kb, int ib) {
     return ka > kb || (ka == kb && ia < ib);
@@ -387,33 +391,58 @@ __device__ __forceinline__ uint64_t warp_or64(uint64_t v) {
     return v;
 }
 
-// Bitonic sort of n2 (a power of two, <= blockDim.x) pairs by (key descending, idx
-// ascending); thread p holds pair p before and after. Every thread of the CTA calls it.
-__device__ __forceinline__ void block_bitonic(uint64_t& key, int& idx, int n2, uint64_t* skey, int* sidx) {
-    const int p = threadIdx.x;
-    for (int k = 2; k <= n2; k <<= 1) {
-        for (int j = k >> 1; j > 0; j >>= 1) {
-            uint64_t pk;
-            int pi;
-            if (j >= 32) {
-                skey[p] = key;
-                sidx[p] = idx;
-                __syncthreads();
-                pk = skey[p ^ j];
-                pi = sidx[p ^ j];
-                __syncthreads();
-            } else {
-                pk = __shfl_xor_sync(0xffffffffu, key, j);
-                pi = __shfl_xor_sync(0xffffffffu, idx, j);
+// Sorts the n (<= blockDim.x) pairs skey/sidx[0, n) of the CTA by (key descending, idx
+// ascending). Thread p starts with pair p (padding past n sorts last) and ends holding
+// the pair at position `pos` of the sorted order, in registers; tkey/tidx are scratch of
+// the same size. Every thread of the CTA calls it.
+__device__ __forceinline__ void block_merge_sort(uint64_t* skey, int32_t* sidx, uint64_t* tkey, int32_t* tidx, int n,
+                                                 uint64_t& key, int& idx, int& pos) {
+    const int p = threadIdx.x, lane = p & 31;
+    const int total = (n + 31) & ~31;  // whole warps
+    const bool act = p < total;
+    key = p < n ? skey[p] : 0ull;
+    idx = p < n ? sidx[p] : 0x7FFFFFFF - p;
+    if (act) {
+        for (int k = 2; k <= 32; k <<= 1)
+            for (int j = k >> 1; j > 0; j >>= 1) {
+                const uint64_t pk = __shfl_xor_sync(0xffffffffu, key, j);
+                const int pi = __shfl_xor_sync(0xffffffffu, idx, j);
+                const bool want_first = ((lane & j) == 0) == ((lane & k) == 0);
+                if (before(pk, pi, key, idx) == want_first) {
+                    key = pk;
+                    idx = pi;
+                }
             }
-            // in a block sorted first-to-last the lower position keeps the earlier pair
-            const bool want_first = ((p & j) == 0) == ((p & k) == 0);
-            const bool partner_first = before(pk, pi, key, idx);
-            if (p < n2 && partner_first == want_first) {
-                key = pk;
-                idx = pi;
+    }
+    pos = p;
+    __syncthreads();  // every thread has read its input pair
+    if (act) {
+        skey[p] = key;
+        sidx[p] = idx;
+    }
+    __syncthreads();
+    uint64_t* ck = skey;
+    int32_t* ci = sidx;
+    uint64_t* ok = tkey;
+    int32_t* oi = tidx;
+    for (int len = 32; len < total; len <<= 1) {
+        if (act) {
+            const int run = pos / len, start = run * len;
+            const int pstart = (run ^ 1) * len;
+            const int plen = max(0, min(len, total - pstart));
+            int lo = 0, hi = plen;
+            while (lo < hi) {
+                const int mid = (lo + hi) >> 1;
+                if (before(ck[pstart + mid], ci[pstart + mid], key, idx)) lo = mid + 1;
+                else hi = mid;
             }
+            pos = (run & ~1) * len + (pos - start) + lo;
+            ok[pos] = key;
+            oi[pos] = idx;
         }
+        __syncthreads();
+        uint64_t* tk = ck; ck = ok; ok = tk;
+        int32_t* ti = ci; ci = oi; oi = ti;
     }
 }
 
@@ -421,16 +450,16 @@ template <bool kSmemKeys>
 __global__ void __launch_bounds__(kSelThreads) k_topk_small(const double* __restrict__ delta, int B, int budget,
                                                             int32_t* __restrict__ rank, int32_t* __restrict__ sel) {
     extern __shared__ __align__(16) uint64_t dyn[];
-    uint64_t* keys = dyn;                                           // [B] when kSmemKeys
-    uint64_t* skey = dyn + (kSmemKeys ? B : 0);                     // [kSelThreads]
-    int32_t* sidx = reinterpret_cast<int32_t*>(skey + kSelThreads); // [kSelThreads]
-    uint32_t* bits = reinterpret_cast<uint32_t*>(sidx + kSelThreads); // [ceil(B / 32)]
+    uint64_t* keys = dyn;                                             // [B] when kSmemKeys
+    uint64_t* skey = dyn + (kSmemKeys ? B : 0);                       // [kSelThreads]
+    uint64_t* tkey = skey + kSelThreads;                              // [kSelThreads]
+    int32_t* sidx = reinterpret_cast<int32_t*>(tkey + kSelThreads);   // [kSelThreads]
+    int32_t* tidx = sidx + kSelThreads;                               // [kSelThreads]
+    uint32_t* bits = reinterpret_cast<uint32_t*>(tidx + kSelThreads); // [ceil(B / 32)]
     __shared__ unsigned hist[1 << kDigitBits];
     __shared__ uint64_t s_and[32], s_or[32];
     __shared__ uint64_t s_prefix;
-    __shared__ int s_pos, s_need, s_cand, s_nsel, s_ncand;
-    __shared__ uint64_t ckey[kCandMax];
-    __shared__ int cidx[kCandMax];
+    __shared__ int s_pos, s_need, s_cand, s_n;
     __shared__ int scratch[32];
     griddep_wait();  // Delta comes from the previous kernel
     griddep_launch();
@@ -459,8 +488,7 @@ __global__ void __launch_bounds__(kSelThreads) k_topk_small(const double* __rest
             s_prefix = cp ? (a & (~0ull << (64 - cp))) : 0ull;
             s_need = budget;
             s_cand = B;
-            s_nsel = 0;
-            s_ncand = 0;
+            s_n = 0;
         }
     }
     __syncthreads();
@@ -473,9 +501,17 @@ __global__ void __launch_bounds__(kSelThreads) k_topk_small(const double* __rest
         const int nb = 1 << w;
         for (int b = tid; b < nb; b += kSelThreads) hist[b] = 0;
         __syncthreads();
-        for (int i = tid; i < B; i += kSelThreads) {
-            const uint64_t k = key_of(i);
-            if ((k & hi) == prefix) atomicAdd(&hist[(unsigned)(k >> shift) & (nb - 1)], 1u);
+        // warp-aggregated histogram: lanes with the same digit add once (keys of similar
+        // magnitude share their leading digits, so per-lane atomics would pile up on a bin)
+        for (int i0 = tid - lane; i0 < B; i0 += kSelThreads) {
+            const int i = i0 + lane;
+            unsigned digit = 1u << kDigitBits;  // not counted
+            if (i < B) {
+                const uint64_t k = key_of(i);
+                if ((k & hi) == prefix) digit = (unsigned)(k >> shift) & (nb - 1);
+            }
+            const unsigned peers = __match_any_sync(0xffffffffu, digit);
+            if (digit < (1u << kDigitBits) && lane == __ffs(peers) - 1) atomicAdd(&hist[digit], (unsigned)__popc(peers));
         }
         __syncthreads();
         // thread t owns the bins nb-1-2t and nb-2-2t (from the top)
@@ -495,32 +531,26 @@ __global__ void __launch_bounds__(kSelThreads) k_topk_small(const double* __rest
     }
     const int pos = s_pos, need = s_need;
     const uint64_t prefix = s_prefix, hi = pos >= 64 ? 0ull : (~0ull << pos);
+    int n;
     if (s_cand <= kCandMax) {
-        // keys above the bucket are selected; the bucket's keys are candidates
-        for (int i = tid; i < B; i += kSelThreads) {
-            const uint64_t k = key_of(i), kh = k & hi;
-            if (kh > prefix) {
-                const int slot = atomicAdd(&s_nsel, 1);
+        // the keys above the bucket and the bucket's keys (slots reserved once per warp)
+        const unsigned lt = (1u << lane) - 1u;
+        for (int i0 = tid - lane; i0 < B; i0 += kSelThreads) {
+            const int i = i0 + lane;
+            const uint64_t k = i < B ? key_of(i) : 0ull;
+            const bool take = i < B && (k & hi) >= prefix;
+            const unsigned mt = __ballot_sync(0xffffffffu, take);
+            int base = 0;
+            if (lane == 0 && mt) base = atomicAdd(&s_n, __popc(mt));
+            base = __shfl_sync(0xffffffffu, base, 0);
+            if (take) {
+                const int slot = base + __popc(mt & lt);
                 skey[slot] = k;
                 sidx[slot] = i;
-            } else if (kh == prefix) {
-                const int slot = atomicAdd(&s_ncand, 1);
-                ckey[slot] = k;
-                cidx[slot] = i;
             }
         }
         __syncthreads();
-        const int nsel = s_nsel, nc = s_ncand;
-        if (tid < nc) {
-            const uint64_t mk = ckey[tid];
-            const int mi = cidx[tid];
-            int r = 0;
-            for (int j = 0; j < nc; ++j) r += before(ckey[j], cidx[j], mk, mi);
-            if (r < need) {
-                skey[nsel + r] = mk;
-                sidx[nsel + r] = mi;
-            }
-        }
+        n = s_n;
     } else {
         // the bucket is a single key value T shared by more than kCandMax keys: keys above
         // T and the lowest-index `need` keys equal to T, compacted in block order
@@ -544,21 +574,17 @@ __global__ void __launch_bounds__(kSelThreads) k_topk_small(const double* __rest
             if (k == T) take = eq_seen++ < need;
             if (take) { skey[out] = k; sidx[out] = i; ++out; }
         }
+        __syncthreads();
+        n = budget;
     }
-    __syncthreads();
-    // exactly `budget` selected pairs in skey/sidx: sort them, one per thread
-    int n2 = 32;
-    while (n2 < budget) n2 <<= 1;
-    uint64_t key = 0ull;
-    int idx = 0x7FFFFFFF - tid;  // padding sorts after every block
-    if (tid < budget) {
-        key = skey[tid];
-        idx = sidx[tid];
+    uint64_t key;
+    int idx, at;
+    block_merge_sort(skey, sidx, tkey, tidx, n, key, idx, at);
+    if (at < budget) {
+        rank[at] = idx;
         atomicOr(&bits[idx >> 5], 1u << (idx & 31));
     }
     __syncthreads();
-    block_bitonic(key, idx, n2, skey, sidx);
-    if (tid < budget) rank[tid] = idx;
     // sel: the set bits in index order (each thread scans a run of bitmap words)
     const int per = (nw + kSelThreads - 1) / kSelThreads;
     const int w0 = min(nw, tid * per), w1 = min(nw, w0 + per);
@@ -761,10 +787,12 @@ cudaError_t launch_quant_delta(const uint16_t* W, const CUtensorMap& tw, int N, 
                       (const float*)partial, codes, sf, sf_swz, g, (uint8_t*)nullptr, (uint8_t*)nullptr, delta, err);
 }
 
+int topk_launches(int budget) { return budget <= 0 ? 0 : budget <= kSmallBudget ? 1 : 2; }
+
 cudaError_t launch_topk(const double* delta, int B, int budget, int32_t* rank, int32_t* sel, cudaStream_t s) {
     if (budget <= 0) return cudaSuccess;
     if (budget <= kSmallBudget) {
-        const size_t tail = (size_t)kSelThreads * 12 + (size_t)((B + 31) / 32) * 4;
+        const size_t tail = (size_t)kSelThreads * 24 + (size_t)((B + 31) / 32) * 4;
         const bool smem_keys = (size_t)B * 8 + tail <= kSelSmemKeysMax;
         const size_t smem = (smem_keys ? (size_t)B * 8 : 0) + tail;
         static bool attr[2] = {false, false};

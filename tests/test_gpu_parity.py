@@ -217,15 +217,25 @@ def test_repeat_calls_deterministic(dev):
 
 
 def test_topk_blocks_alone_and_large_budgets(dev):
-    """A4 alone on many blocks and budgets (in-CTA rank and the separate rank kernel,
-    shared-memory and global keys), with ties, against the oracle's sort."""
+    """A4 alone on many blocks and budgets (the one-CTA select-and-sort path up to its
+    budget limit, the radix select with the separate rank kernel above it, keys in shared
+    or global memory), with ties, against the oracle's sort."""
     from bit_quantized_gemm_zipperengine_b200 import mosaic
     rng = np.random.default_rng(12)
-    for B, budgets in ((32, (0, 1, 3, 32)), (4096, (409, 1024, 1025)), (57344, (2867, 11468))):
+    cases = [(32, (0, 1, 3, 32), False), (4096, (409, 767, 768, 769, 1024, 1025), False),
+             (57344, (500, 2867, 11468), False), (4096, (300, 500, 700), True)]
+    for B, budgets, many_ties in cases:
         d = rng.standard_normal(B) * np.exp2(rng.integers(-20, 5, B))
         d[rng.choice(B, B // 10, replace=False)] = 0.0      # ties at zero
         d[rng.choice(B, B // 50, replace=False)] = d[0]     # ties at an arbitrary value
         d[:3] = -0.0
+        if many_ties:
+            # mostly negative, ~400 positive, 1000 zeros: a threshold inside a bucket of one
+            # value shared by far more keys than the candidate list holds
+            d = -np.abs(d)
+            d[rng.choice(B, 400, replace=False)] *= -1.0
+            z = rng.choice(np.flatnonzero(d < 0), 1000, replace=False)
+            d[z] = 0.0
         dd = torch.from_numpy(d).to(dev)
         for k in budgets:
             rank = torch.empty(max(k, 1), dtype=torch.int32, device=dev)
