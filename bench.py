@@ -243,34 +243,113 @@ def isolated_profile(sets, calls, M, N, K, budget, reps, stream):
             mosaic.mq_gemm(xq, layer.base, layer.packed, Yb, M, N, K, 0, ws)
 
     out = {}
+    inner = 4  # passes over the sets per graph, so graph launch gaps are amortised
     for c in calls:
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g):
-            for s in sets:
-                issue(c, s)
+            for _ in range(inner):
+                for s in sets:
+                    issue(c, s)
         g.replay()
         torch.cuda.synchronize()
-        n = max(1, reps // len(sets))
+        n = max(1, reps // (inner * len(sets)))
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
         for _ in range(n):
             g.replay()
         b.record(stream)
         torch.cuda.synchronize()
-        out[c] = a.elapsed_time(b) / (n * len(sets)) * reps
+        out[c] = a.elapsed_time(b) / (n * inner * len(sets)) * reps
+    return out
+
+
+# ------------------------------------------------------------------ GEMM vs M
+SWEEP = (("qwen3_32b", "q", (1, 16, 128, 1024, 8192)), ("qwen3_32b", "up", (16, 1024, 8192)),
+         ("llama3_8b_mlp_prefill", "up", (2048,)))
+
+
+def gemm_sweep(peaks: dict, reps: int = 20) -> list:
+    """The fused GEMM alone (and dense-only) across token counts: device time per call from
+    CUDA events around graphs of back-to-back calls over enough rotating copies of the
+    quantized weight, residual and activations that every call reads them from HBM."""
+    import numpy as np
+    import torch
+
+    import synth
+    from bit_quantized_gemm_zipperengine_b200 import mosaic
+
+    dev = torch.device("cuda", torch.cuda.current_device())
+    fp4_sus = peaks["bf16_tflops_sustained"] * FP4_PER_BF16
+    fp4_burst = peaks["bf16_tflops"] * FP4_PER_BF16
+    out = []
+    for wl, mat, Ms in SWEEP:
+        L = synth.layer(wl, matrix=mat, M=max(Ms))
+        N, K = L["N"], L["K"]
+        budget = synth.budget_blocks(N, K, 0.10)
+        layer = mosaic.Layer(N, K, budget, dev, with_sf=False)
+        W = torch.from_numpy(L["W"].view(np.int16)).view(torch.bfloat16).to(dev)
+        C = torch.from_numpy(L["Xcal"].view(np.int16)).view(torch.bfloat16).to(dev)
+        Xall = torch.from_numpy(L["X"].view(np.int16)).view(torch.bfloat16).to(dev)
+        layer.prepare_path(W, C)
+        del W, C
+        for M in Ms:
+            X = Xall[:M].contiguous()
+            xq, Y, ws = layer.act_buffers(M)
+            mosaic.mq_quantize_act(X, xq)
+            per_call = N * K * 0.5625 + budget * 2304 + M * K * 0.5625 + 4 * M + 2 * M * N
+            R = max(2, int(np.ceil(3 * 126e6 / per_call)))
+            copies = []
+            for _ in range(R):
+                b = {k: (v.clone() if isinstance(v, torch.Tensor) else v) for k, v in layer.base.items()}
+                p = {k: (v.clone() if isinstance(v, torch.Tensor) else v) for k, v in layer.packed.items()}
+                a = {k: (v.clone() if isinstance(v, torch.Tensor) else v) for k, v in xq.items()}
+                copies.append((b, p, a, torch.empty_like(Y), None if ws is None else ws.clone()))
+            res = {}
+            for flags, lab in ((0, "fused"), (mosaic.MQ_GEMM_BASE_ONLY, "base")):
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g):
+                    for b, p, a, y, w in copies:
+                        mosaic.mq_gemm(a, b, p, y, M, N, K, flags, w)
+                g.replay()
+                torch.cuda.synchronize()
+                n = max(1, reps * 4 // R)
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record()
+                for _ in range(n):
+                    g.replay()
+                e1.record()
+                torch.cuda.synchronize()
+                res[lab] = e0.elapsed_time(e1) * 1e3 / (n * R)
+            del copies
+            fl = 2.0 * M * N * K + 2.0 * M * 4096 * budget
+            us = res["fused"]
+            tf = fl / (us * 1e-6) / 1e12
+            gbs = per_call / (us * 1e-6) / 1e9
+            out.append({"workload": wl, "matrix": mat, "M": M, "N": N, "K": K, "budget_blocks": budget,
+                        "kernel": "prefill" if (M > 128 and N % 256 == 0) else "decode", "us": round(us, 3),
+                        "us_dense_only": round(res["base"], 3),
+                        "residual_overhead": round(us / res["base"] - 1.0, 4),
+                        "tflops_executed": round(tf, 1), "gbs": round(gbs, 1),
+                        "frac_fp4_sustained": round(tf / fp4_sus, 4), "frac_fp4_burst": round(tf / fp4_burst, 4),
+                        "frac_hbm": round(gbs / peaks["hbm_gbs"], 4),
+                        "bound": "hbm" if M <= 316 else "tensor", "rotating_copies": R})
+        del layer, Xall
+        torch.cuda.empty_cache()
+    assert mosaic.mq_get_error() == 0
     return out
 
 
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--steps", type=int, default=10000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--sets", type=int, default=6, help="rotating input sets (L2 defeat)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-sweep", action="store_true", help="skip the GEMM-vs-M sweep")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -399,11 +478,15 @@ def main():
     bytes_step = sum(per_call.values())
     value = bytes_step * world / (ms_step * 1e-3) / 1e9
 
-    # per-call device time inside the step (event nodes in the captured graph); if the
-    # runtime cannot time captured events, time each call alone in graphs of R launches
+    # per-call device time: each call replayed back to back over the R rotating input sets
+    # (CUDA events around graphs of R launches; programmatic dependent launch hides the
+    # launch latency between them, so this is the kernel's own duration). The same calls
+    # timed inside the step graph (event nodes between calls, which serialise them and
+    # add the launch gap to every call) are reported beside it as in_step_us.
     prof_reps = min(args.steps, 300)
-    acc = {c: 0.0 for c in calls}
-    profile_mode = "in-step (event nodes in the step graph)"
+    profile_mode = f"isolated (each call replayed back to back, {R} rotating sets)"
+    acc = isolated_profile(sets, calls, M, N, K, budget, prof_reps, stream)
+    in_step = {c: 0.0 for c in calls}
     try:
         for r in range(prof_reps):
             i = r % R
@@ -411,19 +494,19 @@ def main():
             torch.cuda.synchronize()
             e = evs[i]
             for j, c in enumerate(calls):
-                acc[c] += e[j].elapsed_time(e[j + 1])
+                in_step[c] += e[j].elapsed_time(e[j + 1])
     except RuntimeError:
-        profile_mode = f"isolated (each call alone, {R} rotating sets)"
-        acc = isolated_profile(sets, calls, M, N, K, budget, prof_reps, stream)
+        in_step = None
     peaks = load_peaks()
     kern = {}
     for c in calls:
         us = acc[c] / prof_reps * 1e3
         gbs = per_call[c] / (us * 1e-6) / 1e9
         kern[c] = {"us": round(us, 3), "alg_bytes": per_call[c], "gbs": round(gbs, 1),
-                   "frac_hbm": round(gbs / peaks["hbm_gbs"], 4), "traffic": dram_traffic(c)}
+                   "frac_hbm": round(gbs / peaks["hbm_gbs"], 4), "traffic": dram_traffic(c),
+                   "in_step_us": None if in_step is None else round(in_step[c] / prof_reps * 1e3, 3)}
     dom = max(calls, key=lambda c: kern[c]["us"])
-    roofline = {"bound": "hbm", "kernel": dom, "timing": profile_mode + "; step time from graphs without event nodes", "achieved": kern[dom]["gbs"], "peak": peaks["hbm_gbs"], "unit": "GB/s",
+    roofline = {"bound": "hbm", "kernel": dom, "timing": profile_mode, "achieved": kern[dom]["gbs"], "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": kern[dom]["frac_hbm"], "traffic": kern[dom]["traffic"],
                 "peak_source": f"{peaks['source']} (copy bandwidth)"}
     fl_exec, fl_dense = gemm_flops(M, N, K, budget)
@@ -469,6 +552,16 @@ def main():
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(args.workload, M)
 
+    sweep = None
+    if world == 1 and not args.no_sweep:
+        for st in sets:
+            st.clear()
+        sets.clear()
+        graphs.clear()
+        pgraphs.clear()
+        torch.cuda.empty_cache()
+        sweep = gemm_sweep(load_peaks())
+
     if world > 1:
         graphs.clear()
         pgraphs.clear()
@@ -483,7 +576,7 @@ def main():
             "config": {"workload": args.workload, "M": M, "N": N, "K": K, "T": T, "budget_frac": 0.10,
                        "budget_blocks": budget, "parallelism": f"replicas x{world}",
                        "l2": f"{R} rotating input sets (~{R * 57} MB touched) > 2x L2; no flush"},
-            "roofline": roofline, "gemm": gemm, "kernels": kern, "cpu_baseline": cpu, "e2e": e2e,
+            "roofline": roofline, "gemm": gemm, "gemm_vs_M": sweep, "kernels": kern, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": int(launches_per_step * args.steps), "clocks": clocks}
     print(json.dumps(line), flush=True)
 
