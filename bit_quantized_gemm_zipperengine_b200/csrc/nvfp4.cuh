@@ -27,11 +27,19 @@ __device__ __forceinline__ float e4m3_value(uint32_t c) {
     return e == 0 ? __fmul_rn((float)m, 0.001953125f) : __uint_as_float(((e + 120u) << 23) | (m << 20));
 }
 
+// Maximum of three fp32 values (sm_100 three-input max; exact).
+__device__ __forceinline__ float max3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
 // Packed fp32 multiply (sm_100 mul.rn.f32x2): each lane is one IEEE fp32 multiply with
 // round-to-nearest-even, bit-identical to __fmul_rn (a product's sign, zeros included,
 // is the xor of the operands' signs). Packed add/sub/fma are not used: on B200,
-// sub.rn.f32x2 returned -0 for (-x) - (-x), where IEEE round-to-nearest gives +0, and
-// the sign of a zero residual is part of its code.
+// sub.rn.f32x2 returned -0 for (-x) - (-x), where IEEE round-to-nearest gives +0 (the sign
+// of a zero residual is part of its code), and Delta values computed with it for e' =
+// R - deqR (only ever squared) differed from the IEEE scalar path.
 __device__ __forceinline__ float2 mul2(float2 a, float2 b) {
     float2 d;
     asm("{\n\t.reg .b64 a, b, d;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
@@ -93,9 +101,10 @@ __device__ __forceinline__ uint32_t sign_nibbles8(const float* a) {
 // Returns the scale byte; codes (element 2j in the low nibble of byte j) in lo/hi.
 __device__ __forceinline__ uint32_t nvfp4_group(const float (&a)[16], float g, float g6, uint32_t& lo, uint32_t& hi,
                                                 float (&deq)[16]) {
-    float amax = 0.0f;
+    float amax = max3(fabsf(a[0]), fabsf(a[1]), fabsf(a[2]));
 #pragma unroll
-    for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(a[i]));
+    for (int i = 3; i < 15; i += 2) amax = max3(amax, fabsf(a[i]), fabsf(a[i + 1]));
+    amax = fmaxf(amax, fabsf(a[15]));
     const float s = __fdiv_rn(amax, g6);
     const uint32_t sf = e4m3_encode_nonneg(s);
     const float d = __fmul_rn(e4m3_value(sf), g);

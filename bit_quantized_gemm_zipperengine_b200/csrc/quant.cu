@@ -8,6 +8,15 @@
 
 namespace mq {
 
+// 16-byte read-only streaming load (not kept in L1).
+__device__ __forceinline__ uint4 ld_stream16(const uint4* p) {
+    uint4 r;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+                 : "l"(p));
+    return r;
+}
+
 __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
@@ -15,25 +24,34 @@ __device__ __forceinline__ float warp_max(float v) {
 }
 
 // Per-CTA maxima of |W| over a grid-stride range of 8-element vectors (kAmaxBlocks
-// CTAs, 4 independent 16-byte loads in flight per thread).
+// CTAs of 512 threads, 8 independent 16-byte loads in flight per thread: 64 KB per SM,
+// about what HBM needs in flight to run at full rate).
 // W is an input of the call, never written by the preceding kernel, so the kernel lets
 // its dependent start and reads W at once: it overlaps the preceding kernel (the Hessian
 // estimate, which it does not use). It waits for that kernel only at its end, so that
 // its own completion still implies the predecessor's. The partials it overwrites are
 // read by the quantizers before they let their dependents start.
-__global__ void __launch_bounds__(512) k_amax_partial(const uint16_t* __restrict__ W, int64_t n8,
+__global__ void __launch_bounds__(512, 1) k_amax_partial(const uint16_t* __restrict__ W, int64_t n8,
                                                       float* __restrict__ partial) {
     griddep_launch();
     float m = 0.0f;
     const uint4* v = reinterpret_cast<const uint4*>(W);
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
-    for (; i + 3 * stride < n8; i += 4 * stride) {
-        uint4 x[4];
+    for (; i + 7 * stride < n8; i += 8 * stride) {
+        uint4 x[8];
+        // volatile: the eight loads are issued before any of them is used
 #pragma unroll
-        for (int u = 0; u < 4; ++u) x[u] = __ldg(v + i + u * stride);
+        for (int u = 0; u < 8; ++u) x[u] = ld_stream16(v + i + u * stride);
+        // every loaded word is an operand here, so all eight loads precede the first use
+        asm volatile("" : "+r"(x[0].x), "+r"(x[0].y), "+r"(x[0].z), "+r"(x[0].w), "+r"(x[1].x), "+r"(x[1].y),
+                     "+r"(x[1].z), "+r"(x[1].w), "+r"(x[2].x), "+r"(x[2].y), "+r"(x[2].z), "+r"(x[2].w),
+                     "+r"(x[3].x), "+r"(x[3].y), "+r"(x[3].z), "+r"(x[3].w));
+        asm volatile("" : "+r"(x[4].x), "+r"(x[4].y), "+r"(x[4].z), "+r"(x[4].w), "+r"(x[5].x), "+r"(x[5].y),
+                     "+r"(x[5].z), "+r"(x[5].w), "+r"(x[6].x), "+r"(x[6].y), "+r"(x[6].z), "+r"(x[6].w),
+                     "+r"(x[7].x), "+r"(x[7].y), "+r"(x[7].z), "+r"(x[7].w));
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
+        for (int u = 0; u < 8; ++u) {
             const uint32_t w[4] = {x[u].x, x[u].y, x[u].z, x[u].w};
 #pragma unroll
             for (int j = 0; j < 4; ++j) m = fmaxf(m, fmaxf(fabsf(bf16_bits_to_f32(w[j] & 0xFFFFu)),
