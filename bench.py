@@ -305,7 +305,8 @@ def gemm_sweep(peaks: dict, reps: int = 20) -> list:
                 a = {k: (v.clone() if isinstance(v, torch.Tensor) else v) for k, v in xq.items()}
                 copies.append((b, p, a, torch.empty_like(Y), None if ws is None else ws.clone()))
             res = {}
-            for flags, lab in ((0, "fused"), (mosaic.MQ_GEMM_BASE_ONLY, "base")):
+            for flags, lab in ((0, "fused"), (mosaic.MQ_GEMM_BASE_ONLY, "base"),
+                               (mosaic.MQ_GEMM_RESIDUAL_ONLY, "resid")):
                 g = torch.cuda.CUDAGraph()
                 with torch.cuda.graph(g):
                     for b, p, a, y, w in copies:
@@ -320,7 +321,25 @@ def gemm_sweep(peaks: dict, reps: int = 20) -> list:
                 e1.record()
                 torch.cuda.synchronize()
                 res[lab] = e0.elapsed_time(e1) * 1e3 / (n * R)
-            del copies
+            # the unfused design the pages argue against: dense GEMM, a separate residual-block
+            # GEMM (it reads X again), then an elementwise merge of the two outputs (a torch
+            # add here: this ablation is not part of the path)
+            g = torch.cuda.CUDAGraph()
+            ys = [torch.empty_like(Y) for _ in range(2)]
+            with torch.cuda.graph(g):
+                for _ in range(R):
+                    ys[0].add_(ys[1])
+            g.replay()
+            torch.cuda.synchronize()
+            n = max(1, reps * 4 // R)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(n):
+                g.replay()
+            e1.record()
+            torch.cuda.synchronize()
+            res["merge"] = e0.elapsed_time(e1) * 1e3 / (n * R)
+            del copies, ys
             fl = 2.0 * M * N * K + 2.0 * M * 4096 * budget
             us = res["fused"]
             tf = fl / (us * 1e-6) / 1e12
@@ -329,6 +348,8 @@ def gemm_sweep(peaks: dict, reps: int = 20) -> list:
                         "kernel": "prefill" if (M > 128 and N % 256 == 0) else "decode", "us": round(us, 3),
                         "us_dense_only": round(res["base"], 3),
                         "residual_overhead": round(us / res["base"] - 1.0, 4),
+                        "us_residual_only": round(res["resid"], 3),
+                        "us_unfused": round(res["base"] + res["resid"] + res["merge"], 3),
                         "tflops_executed": round(tf, 1), "gbs": round(gbs, 1),
                         "frac_fp4_sustained": round(tf / fp4_sus, 4), "frac_fp4_burst": round(tf / fp4_burst, 4),
                         "frac_hbm": round(gbs / peaks["hbm_gbs"], 4),

@@ -194,12 +194,16 @@ __global__ void __launch_bounds__(192, 1)
         const uint8_t* xsf_tile = p.x_sf + (int64_t)(m0 / 128) * KS64 * 512;
         const uint8_t* wsf_tile = p.w_sf + (int64_t)n_tile * KS64 * 512;
         // W tile and W scales: written by earlier kernels, loaded before the wait
+        // (only the residual computed: the dense W tile is not needed)
+        const bool dense = p.mode != 2;
         auto issue_w = [&](int it) {
             const int st_i = it % C::kStages, ks = ks_begin + it;
             uint8_t* st = smem + st_i * C::kStageBytes;
-            mbar_arrive_expect_tx(&full[st_i], 16384 + BN * 128 + 2048 + 2048);
-            tma_load_2d(st + C::kOffW, &tmap_w, &full[st_i], ks * 128, n0);
-            bulk_load(st + C::kOffSFW, wsf_tile + (int64_t)ks * 4 * 512, 2048, &full[st_i]);
+            mbar_arrive_expect_tx(&full[st_i], (dense ? 16384 + 2048 : 0) + BN * 128 + 2048);
+            if (dense) {
+                tma_load_2d(st + C::kOffW, &tmap_w, &full[st_i], ks * 128, n0);
+                bulk_load(st + C::kOffSFW, wsf_tile + (int64_t)ks * 4 * 512, 2048, &full[st_i]);
+            }
         };
         // X tile and X scales: written by the previous kernel
         auto issue_x = [&](int it) {
@@ -291,7 +295,7 @@ __global__ void __launch_bounds__(192, 1)
             if (elect_one()) {
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) {
-                    tc_cp_sf_chunk(sfc + 4 * kk, smem_desc(st + C::kOffSFW + kk * 512, 0, 128, 0));
+                    if (p.mode != 2) tc_cp_sf_chunk(sfc + 4 * kk, smem_desc(st + C::kOffSFW + kk * 512, 0, 128, 0));
                     tc_cp_sf_chunk(sfc + 16 + 4 * kk, smem_desc(st + C::kOffSFX + kk * 512, 0, 128, 0));
                 }
                 if (p.mode != 2) {
@@ -601,14 +605,24 @@ __global__ void __launch_bounds__(320, 1)
                 const uint32_t st = sbase + s * C::kStageBytes;
                 if (elect_one()) {
                     rmask[s] = m;
-                    mbar_arrive_expect_tx(&full[s], C::kBaseTx + n * C::kRSlotBytes);
-                    tma_load_2d(smem + s * C::kStageBytes + C::kOffX, &tmap_x, &full[s], ks * 128, m_tile * 128);
-                    tma_load_2d(smem + s * C::kStageBytes + C::kOffW, &tmap_w, &full[s], ks * 128, n_tile * 256);
-                    bulk_load_s(st + C::kOffSFX, p.x_sf + ((int64_t)m_tile * KS64 + ks * 4) * 512, 2048, &full[s]);
-                    bulk_load_s(st + C::kOffSFW, p.w_sf + ((int64_t)(n_tile * 2) * KS64 + ks * 4) * 512, 2048,
-                                &full[s]);
-                    bulk_load_s(st + C::kOffSFW + 2048, p.w_sf + ((int64_t)(n_tile * 2 + 1) * KS64 + ks * 4) * 512,
-                                2048, &full[s]);
+                    // only the residual computed: no dense W tile, and no X tile for a stage
+                    // without residual blocks (its barrier completes on the plain arrive)
+                    const bool dense = p.mode != 2, xneed = dense || n > 0;
+                    mbar_arrive_expect_tx(&full[s], (dense ? C::kBaseTx : xneed ? 16384 + 2048 : 0) +
+                                                        n * C::kRSlotBytes);
+                    if (xneed) {
+                        tma_load_2d(smem + s * C::kStageBytes + C::kOffX, &tmap_x, &full[s], ks * 128,
+                                    m_tile * 128);
+                        bulk_load_s(st + C::kOffSFX, p.x_sf + ((int64_t)m_tile * KS64 + ks * 4) * 512, 2048,
+                                    &full[s]);
+                    }
+                    if (dense) {
+                        tma_load_2d(smem + s * C::kStageBytes + C::kOffW, &tmap_w, &full[s], ks * 128, n_tile * 256);
+                        bulk_load_s(st + C::kOffSFW, p.w_sf + ((int64_t)(n_tile * 2) * KS64 + ks * 4) * 512, 2048,
+                                    &full[s]);
+                        bulk_load_s(st + C::kOffSFW + 2048,
+                                    p.w_sf + ((int64_t)(n_tile * 2 + 1) * KS64 + ks * 4) * 512, 2048, &full[s]);
+                    }
                     // residual blocks of the stage in (kk, h) order, into consecutive ring slots
                     int r = rc;
                     for (uint32_t mm = m; mm; mm &= mm - 1, ++r) {

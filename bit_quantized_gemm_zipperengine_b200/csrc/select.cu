@@ -380,28 +380,28 @@ __device__ __forceinline__ bool before(uint64_t ka, int ia, uint64_t kb, int ib)
     return ka > kb || (ka == kb && ia < ib);
 }
 
-__device__ __forceinline__ uint64_t warp_and64(uint64_t v) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v &= __shfl_xor_sync(0xffffffffu, v, o);
-    return v;
-}
-__device__ __forceinline__ uint64_t warp_or64(uint64_t v) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v |= __shfl_xor_sync(0xffffffffu, v, o);
-    return v;
+// A (key, block index) pair in one 16-byte shared-memory word.
+__device__ __forceinline__ ulonglong2 kpair(uint64_t key, int idx) {
+    return make_ulonglong2(key, (unsigned long long)(unsigned)idx);
 }
 
-// Sorts the n (<= blockDim.x) pairs skey/sidx[0, n) of the CTA by (key descending, idx
+// Sorts the n (<= blockDim.x) pairs s[0, n) of the CTA by (key descending, idx
 // ascending). Thread p starts with pair p (padding past n sorts last) and ends holding
-// the pair at position `pos` of the sorted order, in registers; tkey/tidx are scratch of
-// the same size. Every thread of the CTA calls it.
-__device__ __forceinline__ void block_merge_sort(uint64_t* skey, int32_t* sidx, uint64_t* tkey, int32_t* tidx, int n,
-                                                 uint64_t& key, int& idx, int& pos) {
+// the pair at position `pos` of the sorted order, in registers; t is scratch of the same
+// size. Every thread of the CTA calls it.
+__device__ __forceinline__ void block_merge_sort(ulonglong2* s, ulonglong2* t, int n, uint64_t& key, int& idx,
+                                                 int& pos) {
     const int p = threadIdx.x, lane = p & 31;
     const int total = (n + 31) & ~31;  // whole warps
     const bool act = p < total;
-    key = p < n ? skey[p] : 0ull;
-    idx = p < n ? sidx[p] : 0x7FFFFFFF - p;
+    if (p < n) {
+        const ulonglong2 v = s[p];
+        key = v.x;
+        idx = (int)v.y;
+    } else {
+        key = 0ull;
+        idx = 0x7FFFFFFF - p;
+    }
     if (act) {
         for (int k = 2; k <= 32; k <<= 1)
             for (int j = k >> 1; j > 0; j >>= 1) {
@@ -416,15 +416,10 @@ __device__ __forceinline__ void block_merge_sort(uint64_t* skey, int32_t* sidx, 
     }
     pos = p;
     __syncthreads();  // every thread has read its input pair
-    if (act) {
-        skey[p] = key;
-        sidx[p] = idx;
-    }
+    if (act) s[p] = kpair(key, idx);
     __syncthreads();
-    uint64_t* ck = skey;
-    int32_t* ci = sidx;
-    uint64_t* ok = tkey;
-    int32_t* oi = tidx;
+    ulonglong2* cur = s;
+    ulonglong2* out = t;
     for (int len = 32; len < total; len <<= 1) {
         if (act) {
             const int run = pos / len, start = run * len;
@@ -433,31 +428,47 @@ __device__ __forceinline__ void block_merge_sort(uint64_t* skey, int32_t* sidx, 
             int lo = 0, hi = plen;
             while (lo < hi) {
                 const int mid = (lo + hi) >> 1;
-                if (before(ck[pstart + mid], ci[pstart + mid], key, idx)) lo = mid + 1;
+                const ulonglong2 v = cur[pstart + mid];
+                if (before(v.x, (int)v.y, key, idx)) lo = mid + 1;
                 else hi = mid;
             }
             pos = (run & ~1) * len + (pos - start) + lo;
-            ok[pos] = key;
-            oi[pos] = idx;
+            out[pos] = kpair(key, idx);
         }
         __syncthreads();
-        uint64_t* tk = ck; ck = ok; ok = tk;
-        int32_t* ti = ci; ci = oi; oi = ti;
+        ulonglong2* tmp = cur; cur = out; out = tmp;
     }
+}
+
+// Exclusive prefix sum over the CTA's threads in thread order (kThreads <= 1024), with
+// one barrier: a shuffle scan inside each warp, the warp totals through `wsum`, and the
+// sum of the lower warps' totals by a warp reduction. `wsum` must not be reused before
+// the next barrier.
+template <int kThreads>
+__device__ __forceinline__ int block_excl_sum_1bar(int v, int* wsum) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    if (lane == 31) wsum[warp] = x;
+    __syncthreads();
+    const int ws = (lane < kThreads / 32 && lane < warp) ? wsum[lane] : 0;
+    return (int)__reduce_add_sync(0xffffffffu, (unsigned)ws) + x - v;
 }
 
 template <bool kSmemKeys>
 __global__ void __launch_bounds__(kSelThreads) k_topk_small(const double* __restrict__ delta, int B, int budget,
                                                             int32_t* __restrict__ rank, int32_t* __restrict__ sel) {
     extern __shared__ __align__(16) uint64_t dyn[];
-    uint64_t* keys = dyn;                                             // [B] when kSmemKeys
-    uint64_t* skey = dyn + (kSmemKeys ? B : 0);                       // [kSelThreads]
-    uint64_t* tkey = skey + kSelThreads;                              // [kSelThreads]
-    int32_t* sidx = reinterpret_cast<int32_t*>(tkey + kSelThreads);   // [kSelThreads]
-    int32_t* tidx = sidx + kSelThreads;                               // [kSelThreads]
-    uint32_t* bits = reinterpret_cast<uint32_t*>(tidx + kSelThreads); // [ceil(B / 32)]
+    uint64_t* keys = dyn;                                                        // [B] when kSmemKeys
+    ulonglong2* spair = reinterpret_cast<ulonglong2*>(dyn + (kSmemKeys ? (B + 1) & ~1 : 0));  // [kSelThreads]
+    ulonglong2* tpair = spair + kSelThreads;                                     // [kSelThreads]
+    uint32_t* bits = reinterpret_cast<uint32_t*>(tpair + kSelThreads);           // [ceil(B / 32)]
     __shared__ unsigned hist[1 << kDigitBits];
-    __shared__ uint64_t s_and[32], s_or[32];
+    __shared__ uint32_t s_and[64], s_or[64];
     __shared__ uint64_t s_prefix;
     __shared__ int s_pos, s_need, s_cand, s_n;
     __shared__ int scratch[32];
@@ -475,13 +486,26 @@ __global__ void __launch_bounds__(kSelThreads) k_topk_small(const double* __rest
         o |= k;
     }
     for (int w = tid; w < nw; w += kSelThreads) bits[w] = 0u;
-    a = warp_and64(a);
-    o = warp_or64(o);
-    if (lane == 0) { s_and[warp] = a; s_or[warp] = o; }
+    {
+        const uint32_t ah = __reduce_and_sync(0xffffffffu, (uint32_t)(a >> 32));
+        const uint32_t al = __reduce_and_sync(0xffffffffu, (uint32_t)a);
+        const uint32_t oh = __reduce_or_sync(0xffffffffu, (uint32_t)(o >> 32));
+        const uint32_t ol = __reduce_or_sync(0xffffffffu, (uint32_t)o);
+        if (lane == 0) {
+            s_and[2 * warp] = ah;
+            s_and[2 * warp + 1] = al;
+            s_or[2 * warp] = oh;
+            s_or[2 * warp + 1] = ol;
+        }
+    }
     __syncthreads();
     if (warp == 0) {
-        a = warp_and64(s_and[lane]);
-        o = warp_or64(s_or[lane]);
+        const uint32_t ah = __reduce_and_sync(0xffffffffu, s_and[2 * lane]);
+        const uint32_t al = __reduce_and_sync(0xffffffffu, s_and[2 * lane + 1]);
+        const uint32_t oh = __reduce_or_sync(0xffffffffu, s_or[2 * lane]);
+        const uint32_t ol = __reduce_or_sync(0xffffffffu, s_or[2 * lane + 1]);
+        a = ((uint64_t)ah << 32) | al;
+        o = ((uint64_t)oh << 32) | ol;
         if (lane == 0) {
             const int cp = (a ^ o) ? __clzll((long long)(a ^ o)) : 64;  // common leading bits
             s_pos = 64 - cp;
@@ -517,8 +541,7 @@ __global__ void __launch_bounds__(kSelThreads) k_topk_small(const double* __rest
         // thread t owns the bins nb-1-2t and nb-2-2t (from the top)
         const int b0 = nb - 1 - 2 * tid;
         const unsigned c0 = b0 >= 0 ? hist[b0] : 0u, c1 = b0 - 1 >= 0 ? hist[b0 - 1] : 0u;
-        int total;
-        const int above = block_exclusive_sum<kSelThreads>((int)(c0 + c1), scratch, total);
+        const int above = block_excl_sum_1bar<kSelThreads>((int)(c0 + c1), scratch);
         if (b0 >= 0 && above < need && above + (int)(c0 + c1) >= need) {
             const bool first = above + (int)c0 >= need;
             const int digit = first ? b0 : b0 - 1;
@@ -543,11 +566,7 @@ __global__ void __launch_bounds__(kSelThreads) k_topk_small(const double* __rest
             int base = 0;
             if (lane == 0 && mt) base = atomicAdd(&s_n, __popc(mt));
             base = __shfl_sync(0xffffffffu, base, 0);
-            if (take) {
-                const int slot = base + __popc(mt & lt);
-                skey[slot] = k;
-                sidx[slot] = i;
-            }
+            if (take) spair[base + __popc(mt & lt)] = kpair(k, i);
         }
         __syncthreads();
         n = s_n;
@@ -572,14 +591,14 @@ __global__ void __launch_bounds__(kSelThreads) k_topk_small(const double* __rest
             const uint64_t k = key_of(i);
             bool take = k > T;
             if (k == T) take = eq_seen++ < need;
-            if (take) { skey[out] = k; sidx[out] = i; ++out; }
+            if (take) spair[out++] = kpair(k, i);
         }
         __syncthreads();
         n = budget;
     }
     uint64_t key;
     int idx, at;
-    block_merge_sort(skey, sidx, tkey, tidx, n, key, idx, at);
+    block_merge_sort(spair, tpair, n, key, idx, at);
     if (at < budget) {
         rank[at] = idx;
         atomicOr(&bits[idx >> 5], 1u << (idx & 31));
@@ -792,9 +811,10 @@ int topk_launches(int budget) { return budget <= 0 ? 0 : budget <= kSmallBudget 
 cudaError_t launch_topk(const double* delta, int B, int budget, int32_t* rank, int32_t* sel, cudaStream_t s) {
     if (budget <= 0) return cudaSuccess;
     if (budget <= kSmallBudget) {
-        const size_t tail = (size_t)kSelThreads * 24 + (size_t)((B + 31) / 32) * 4;
-        const bool smem_keys = (size_t)B * 8 + tail <= kSelSmemKeysMax;
-        const size_t smem = (smem_keys ? (size_t)B * 8 : 0) + tail;
+        const size_t tail = (size_t)kSelThreads * 32 + (size_t)((B + 31) / 32) * 4;
+        const size_t keys_bytes = (size_t)((B + 1) & ~1) * 8;  // keeps the pairs 16-byte aligned
+        const bool smem_keys = keys_bytes + tail <= kSelSmemKeysMax;
+        const size_t smem = (smem_keys ? keys_bytes : 0) + tail;
         static bool attr[2] = {false, false};
         auto go = [&](auto kern, int which) -> cudaError_t {
             if (!attr[which]) {
