@@ -428,9 +428,10 @@ def main():
     torch.cuda.synchronize()
     assert mosaic.mq_get_error() == 0
 
-    # per input set: a clean step graph (timed; consecutive kernels overlap through
-    # programmatic dependent launch) and a profiling graph with event nodes between calls
-    # (which serialize them) for per-call device times
+    # per input set: the timed step graph is one mq_run_layer call (the whole path as a
+    # user issues it; consecutive kernels overlap through programmatic dependent launch),
+    # and a profiling graph issues the same steps as separate public calls with event
+    # nodes between them (which serialise them) for the in-step per-call times
     calls = ["hessian_diag", "quantize_weight_delta", "topk_blocks", "pack_residual", "quantize_act", "gemm"]
 
     def issue_step(s, events=None, cs=None):
@@ -453,7 +454,7 @@ def main():
     for i in range(R):
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g):
-            issue_step(sets[i])
+            step(i)
         graphs.append(g)
         e = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(len(calls) + 1)]
         pg = torch.cuda.CUDAGraph()

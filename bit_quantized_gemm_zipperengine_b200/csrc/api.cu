@@ -256,8 +256,12 @@ mq_status mq_quantize_act(const mq_bf16* X, int M, int K, mq_nvfp4_mat* xq, mq_s
     return launched(launch_quant_act(X, M, K, xq->codes, xq->sf, xq->sf_swz, xq->gscale, as_stream(stream)), 1);
 }
 
-mq_status mq_gemm(const mq_nvfp4_mat* xq, const mq_nvfp4_mat* wq, const mq_residual_packed* r, mq_bf16* Y, int M,
-                  int N, int K, unsigned flags, void* ws, size_t ws_bytes, mq_stream stream) {
+// prefetch: the caller guarantees wq was complete before the kernel preceding the GEMM in
+// the stream started (the whole-path call's order), so the decode kernel may load it
+// before waiting for that kernel.
+static mq_status gemm_impl(const mq_nvfp4_mat* xq, const mq_nvfp4_mat* wq, const mq_residual_packed* r, mq_bf16* Y,
+                           int M, int N, int K, unsigned flags, void* ws, size_t ws_bytes, bool prefetch,
+                           mq_stream stream) {
     if (!xq || !wq || !Y || M <= 0 || N <= 0 || K <= 0 || N % 64 || K % 64) return MQ_ERR_INVALID_ARG;
     if (N % 128 || K % 256) return MQ_ERR_UNSUPPORTED_SHAPE;
     if (!xq->codes || !xq->sf_swz || !xq->gscale || !wq->codes || !wq->sf_swz || !wq->gscale)
@@ -297,6 +301,7 @@ mq_status mq_gemm(const mq_nvfp4_mat* xq, const mq_nvfp4_mat* wq, const mq_resid
     p.N = N;
     p.K = K;
     p.mode = (flags & MQ_GEMM_BASE_ONLY) ? 1 : (flags & MQ_GEMM_RESIDUAL_ONLY) ? 2 : 0;
+    p.prefetch = prefetch ? 1 : 0;
     CUtensorMap tw, tx;
     if (prefill) {
         if (!make_tmap_bytes(&tw, wq->codes, (uint64_t)K / 2, (uint64_t)N, 128, 256)) return MQ_ERR_CUDA;
@@ -317,6 +322,11 @@ mq_status mq_gemm(const mq_nvfp4_mat* xq, const mq_nvfp4_mat* wq, const mq_resid
     return launched(launch_gemm_decode(tw, tx, p, d, as_stream(stream)), 1);
 }
 
+mq_status mq_gemm(const mq_nvfp4_mat* xq, const mq_nvfp4_mat* wq, const mq_residual_packed* r, mq_bf16* Y, int M,
+                  int N, int K, unsigned flags, void* ws, size_t ws_bytes, mq_stream stream) {
+    return gemm_impl(xq, wq, r, Y, M, N, K, flags, ws, ws_bytes, false, stream);
+}
+
 mq_status mq_run_layer(const mq_bf16* W, const mq_bf16* X, const mq_bf16* Xcal, mq_bf16* Y, int M, int N, int K,
                        int T, int budget, unsigned flags, int host, mq_layer_buffers* buf, mq_stream stream) {
     if (!W || !X || !Xcal || !Y || !buf || M <= 0 || N <= 0 || K <= 0 || T <= 0) return MQ_ERR_INVALID_ARG;
@@ -334,6 +344,10 @@ mq_status mq_run_layer(const mq_bf16* W, const mq_bf16* X, const mq_bf16* Xcal, 
         xc = buf->Xcal_dev;
         y = buf->Y_dev;
     }
+    // The method's order. Every kernel waits for its predecessor before reading its
+    // outputs (and lets its dependent start right after), so when the GEMM starts, the
+    // quantize+Delta kernel has long completed and the GEMM requests W before waiting
+    // for the activation quantizer (prefetch).
     mq_status st;
     if ((st = mq_hessian_diag(xc, T, K, buf->H, stream)) != MQ_OK) return st;
     if ((st = mq_quantize_weight_delta(w, N, K, buf->H, &buf->base, nullptr, buf->delta, buf->ws_quant,
@@ -343,8 +357,8 @@ mq_status mq_run_layer(const mq_bf16* W, const mq_bf16* X, const mq_bf16* Xcal, 
         return st;
     if ((st = mq_pack_residual_weight(w, &buf->base, buf->sel, budget, &buf->packed, stream)) != MQ_OK) return st;
     if ((st = mq_quantize_act(x, M, K, &buf->xq, stream)) != MQ_OK) return st;
-    if ((st = mq_gemm(&buf->xq, &buf->base, &buf->packed, y, M, N, K, flags, buf->ws_gemm, buf->ws_gemm_bytes,
-                      stream)) != MQ_OK)
+    if ((st = gemm_impl(&buf->xq, &buf->base, &buf->packed, y, M, N, K, flags, buf->ws_gemm, buf->ws_gemm_bytes, true,
+                        stream)) != MQ_OK)
         return st;
     if (host && cudaMemcpyAsync(Y, buf->Y_dev, (size_t)M * N * 2, cudaMemcpyDeviceToHost, s) != cudaSuccess)
         return MQ_ERR_CUDA;

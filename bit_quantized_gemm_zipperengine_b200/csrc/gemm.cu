@@ -17,9 +17,11 @@
 // order, then scales by g_x[m] * g_w and stores bf16. Above 8 splits (narrow layers) the
 // partials go through a global workspace instead, added in the same order by the last
 // CTA of the tile (a tile counter).
-// The kernel is launched with programmatic dependent launch: its prologue and the W,
-// W-scale and residual loads (written by earlier kernels) overlap the preceding kernel;
-// it waits for that kernel before loading X and its scales.
+// The kernel is launched with programmatic dependent launch: its prologue overlaps the
+// preceding kernel. It waits for that kernel before its loads, unless the caller
+// guarantees that W was complete before that kernel started (GemmParams::prefetch, set by
+// the whole-path call, where the activation quantizer precedes the GEMM): then the first
+// stages' W is requested before the wait.
 #include <cuda_bf16.h>
 
 #include "common.cuh"
@@ -193,7 +195,7 @@ __global__ void __launch_bounds__(192, 1)
         // ---------------------------------------------------- producer (converged warp, one lane issues)
         const uint8_t* xsf_tile = p.x_sf + (int64_t)(m0 / 128) * KS64 * 512;
         const uint8_t* wsf_tile = p.w_sf + (int64_t)n_tile * KS64 * 512;
-        // W tile and W scales: written by earlier kernels, loaded before the wait
+        // W tile and W scales (the stage's expected bytes are armed here, X's included)
         // (only the residual computed: the dense W tile is not needed)
         const bool dense = p.mode != 2;
         auto issue_w = [&](int it) {
@@ -205,7 +207,7 @@ __global__ void __launch_bounds__(192, 1)
                 bulk_load(st + C::kOffSFW, wsf_tile + (int64_t)ks * 4 * 512, 2048, &full[st_i]);
             }
         };
-        // X tile and X scales: written by the previous kernel
+        // X tile and X scales
         auto issue_x = [&](int it) {
             const int st_i = it % C::kStages, ks = ks_begin + it;
             uint8_t* st = smem + st_i * C::kStageBytes;
@@ -243,10 +245,15 @@ __global__ void __launch_bounds__(192, 1)
             }
         };
         const int first = min(C::kStages, n_iters);
+        // W normally comes from an earlier kernel of the stream, so it is loaded after the
+        // wait for the preceding kernel; a caller that guarantees it was complete before
+        // that kernel started (p.prefetch) lets the first stages' W load at once. X (the
+        // activation quantizer's output) always waits.
+        if (!p.prefetch) griddep_wait();
         if (elect_one())
-            for (int it = 0; it < first; ++it) issue_w(it);  // nothing to wait for yet
+            for (int it = 0; it < first; ++it) issue_w(it);
         __syncwarp();
-        griddep_wait();
+        if (p.prefetch) griddep_wait();
         if (elect_one())
             for (int it = 0; it < first; ++it) issue_x(it);
         __syncwarp();

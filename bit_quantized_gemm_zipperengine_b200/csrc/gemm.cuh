@@ -25,6 +25,8 @@ struct GemmParams {
     int mode;                // 0 fused, 1 base only, 2 residual only
     int has_resid;
     int cluster;             // split-K reduced through the cluster's shared memory
+    int prefetch;            // W was complete before the preceding kernel started, so the
+                             // decode kernel may load it before waiting for that kernel
 };
 
 // Decode kernel tiling: token tile BN, grid tiles_n x splits x tiles_m, `iters`

@@ -133,6 +133,51 @@ __device__ __forceinline__ uint32_t nvfp4_group(const float (&a)[16], float g, f
     return sf;
 }
 
+// The dequantization step d = fp32(dec(sf) * g) and its reciprocal r = fp32(1 / d) (0 when
+// d = 0) of every E4M3 scale code 0..127 for tensor scale g, as (d, r) pairs: the same
+// operations nvfp4_group performs per group, done once per CTA. The CTA's threads fill it
+// (the caller synchronizes before use).
+__device__ __forceinline__ void nvfp4_scale_table(float g, float2* tab) {
+    for (int c = threadIdx.x; c < 128; c += blockDim.x) {
+        const float d = __fmul_rn(e4m3_value((uint32_t)c), g);
+        tab[c] = make_float2(d, d > 0.0f ? __frcp_rn(d) : 0.0f);
+    }
+}
+
+// nvfp4_group with d and r looked up in a table from nvfp4_scale_table (bit-identical).
+__device__ __forceinline__ uint32_t nvfp4_group_tab(const float (&a)[16], float g6, const float2* tab, uint32_t& lo,
+                                                    uint32_t& hi, float (&deq)[16]) {
+    float amax = max3(fabsf(a[0]), fabsf(a[1]), fabsf(a[2]));
+#pragma unroll
+    for (int i = 3; i < 15; i += 2) amax = max3(amax, fabsf(a[i]), fabsf(a[i + 1]));
+    amax = fmaxf(amax, fabsf(a[15]));
+    const uint32_t sf = e4m3_encode_nonneg(__fdiv_rn(amax, g6));
+    const float2 dr = tab[sf];
+    const float d = dr.x;
+    if (d > 0.0f) {
+        const float2 rr = make_float2(dr.y, dr.y);
+        float2 q[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) q[j] = mul2(make_float2(a[2 * j], a[2 * j + 1]), rr);
+        lo = e2m1x8(q[0].x, q[0].y, q[1].x, q[1].y, q[2].x, q[2].y, q[3].x, q[3].y);
+        hi = e2m1x8(q[4].x, q[4].y, q[5].x, q[5].y, q[6].x, q[6].y, q[7].x, q[7].y);
+    } else {
+        lo = sign_nibbles8(a);
+        hi = sign_nibbles8(a + 8);
+    }
+    float v[16];
+    e2m1x8_values(lo, v);
+    e2m1x8_values(hi, v + 8);
+    const float2 dd = make_float2(d, d);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const float2 t = mul2(make_float2(v[2 * j], v[2 * j + 1]), dd);
+        deq[2 * j] = t.x;
+        deq[2 * j + 1] = t.y;
+    }
+    return sf;
+}
+
 // Byte offset of (row r, group q) in the GEMM's tiled scale layout of a matrix with
 // `cols` columns: 512-byte chunks per (128-row tile, 4 groups), (t%32)*16 + (t/32)*4 + q%4.
 __device__ __forceinline__ int64_t sf_swz_offset(int64_t r, int64_t q, int cols) {

@@ -53,7 +53,8 @@ __device__ __forceinline__ void tile_group(const uint8_t* tile, int rl, int q, f
 // coalesced stores. `nblk_rows` = N / 64.
 template <bool kWriteCodes, bool kWriteResid>
 __device__ __forceinline__ void quant_delta_strip(const uint8_t* tile, uint8_t* st, int K, int nblk_rows,
-                                                  const float* __restrict__ H, float g, int si, int kt,
+                                                  const float* __restrict__ H, float g, const float2* tab, int si,
+                                                  int kt,
                                                   uint8_t* __restrict__ codes, uint8_t* __restrict__ sf,
                                                   uint8_t* __restrict__ sf_swz, uint8_t* __restrict__ rcodes,
                                                   uint8_t* __restrict__ rsf, double* __restrict__ delta) {
@@ -70,10 +71,10 @@ __device__ __forceinline__ void quant_delta_strip(const uint8_t* tile, uint8_t* 
         tile_group(tile, rl, q, a);
         float deq[16], R[16], rdeq[16];
         uint32_t lo, hi, rlo, rhi;
-        const uint32_t sfb = nvfp4_group(a, g, g6, lo, hi, deq);
+        const uint32_t sfb = nvfp4_group_tab(a, g6, tab, lo, hi, deq);
 #pragma unroll
         for (int i = 0; i < 16; ++i) R[i] = __fsub_rn(a[i], deq[i]);
-        const uint32_t rsb = nvfp4_group(R, g, g6, rlo, rhi, rdeq);
+        const uint32_t rsb = nvfp4_group_tab(R, g6, tab, rlo, rhi, rdeq);
         if (kWriteCodes) {
             *reinterpret_cast<uint2*>(st + kQDOffC + rl * 32 + q * 8) = make_uint2(lo, hi);
             st[kQDOffSw + (rl & 31) * 16 + (rl >> 5) * 4 + q] = (uint8_t)sfb;
@@ -179,6 +180,9 @@ __global__ void __launch_bounds__(kQDThreads, 3) k_quant_delta(const __grid_cons
     griddep_wait();
     const float g = kWriteCodes ? tensor_scale(g_in) : __ldg(g_in);
     if (kWriteCodes && blockIdx.x == 0 && threadIdx.x == 0) *g_out = g;
+    __shared__ float2 s_tab[128];  // (d, 1/d) of every scale code for this tensor scale
+    nvfp4_scale_table(g, s_tab);
+    __syncthreads();
     // the next kernel may start once every CTA has read the tensor-scale partials
     griddep_launch();
     bool ok = true;
@@ -188,7 +192,7 @@ __global__ void __launch_bounds__(kQDThreads, 3) k_quant_delta(const __grid_cons
         const int s = i % kQDStages;
         if (ok) ok = mbar_wait_err(&full[s], (i / kQDStages) & 1, err);
         if (ok)
-            quant_delta_strip<kWriteCodes, kWriteResid>(sm + s * kQDTile, sm, K, nbr, H, g, b / KB, b % KB, codes,
+            quant_delta_strip<kWriteCodes, kWriteResid>(sm + s * kQDTile, sm, K, nbr, H, g, s_tab, b / KB, b % KB, codes,
                                                         sf, sf_swz, rcodes, rsf, delta);
         __syncthreads();  // stage s and the strip's staging are free again
         // every copy issued here is waited for by a later iteration of this loop

@@ -255,11 +255,11 @@ typedef struct {
  * The whole path for one layer in the method's order: A2 H from the T calibration
  * tokens, A1+A3 quantize W and score every block (mq_quantize_weight_delta, residual not
  * stored), A4 top-`budget` selection, A5 pack the selected residual from W
- * (mq_pack_residual_weight), A6 quantize X, A7+A8 fused GEMM into Y. With host == 0, W,
- * X, Xcal and Y are device pointers. With host != 0 they are HOST pointers
- * (page-locked for the copies to be asynchronous): the inputs are copied into
- * buf->W_dev, X_dev, Xcal_dev and the result from buf->Y_dev back to Y, all on
- * `stream`. Errors as the individual calls.
+ * (mq_pack_residual_weight), A6 quantize X, A7+A8 fused GEMM into Y; results are those of
+ * the individual calls in this order. With host == 0, W, X, Xcal and Y are device
+ * pointers. With host != 0 they are HOST pointers (page-locked for the copies to be
+ * asynchronous): the inputs are copied into buf->W_dev, X_dev, Xcal_dev and the result
+ * from buf->Y_dev back to Y, all on `stream`. Errors as the individual calls.
  */
 mq_status mq_run_layer(const mq_bf16* W, const mq_bf16* X, const mq_bf16* Xcal, mq_bf16* Y, int M, int N, int K,
                        int T, int budget, unsigned flags, int host, mq_layer_buffers* buf, mq_stream stream);
