@@ -321,6 +321,38 @@ def gemm_sweep(peaks: dict, reps: int = 20) -> list:
                 e1.record()
                 torch.cuda.synchronize()
                 res[lab] = e0.elapsed_time(e1) * 1e3 / (n * R)
+            # the decode kernel quantizing the bf16 activations itself (mq_gemm_act)
+            if M <= 128:
+                ga = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(ga):
+                    for b, p, a, y, w in copies:
+                        mosaic.mq_gemm_act(X, b, p, y, M, N, K, 0, w)
+                ga.replay()
+                torch.cuda.synchronize()
+                n = max(1, reps * 4 // R)
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record()
+                for _ in range(n):
+                    ga.replay()
+                e1.record()
+                torch.cuda.synchronize()
+                res["act_fused"] = e0.elapsed_time(e1) * 1e3 / (n * R)
+                del ga
+                # the same with the separate activation quantizer in front
+                gs = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(gs):
+                    for b, p, a, y, w in copies:
+                        mosaic.mq_quantize_act(X, a)
+                        mosaic.mq_gemm(a, b, p, y, M, N, K, 0, w)
+                gs.replay()
+                torch.cuda.synchronize()
+                e0.record()
+                for _ in range(n):
+                    gs.replay()
+                e1.record()
+                torch.cuda.synchronize()
+                res["act_separate"] = e0.elapsed_time(e1) * 1e3 / (n * R)
+                del gs
             # the unfused design the pages argue against: dense GEMM, a separate residual-block
             # GEMM (it reads X again), then an elementwise merge of the two outputs (a torch
             # add here: this ablation is not part of the path)
@@ -350,6 +382,8 @@ def gemm_sweep(peaks: dict, reps: int = 20) -> list:
                         "residual_overhead": round(us / res["base"] - 1.0, 4),
                         "us_residual_only": round(res["resid"], 3),
                         "us_unfused": round(res["base"] + res["resid"] + res["merge"], 3),
+                        "us_quantize_act_then_gemm": round(res["act_separate"], 3) if "act_separate" in res else None,
+                        "us_gemm_act": round(res["act_fused"], 3) if "act_fused" in res else None,
                         "tflops_executed": round(tf, 1), "gbs": round(gbs, 1),
                         "frac_fp4_sustained": round(tf / fp4_sus, 4), "frac_fp4_burst": round(tf / fp4_burst, 4),
                         "frac_hbm": round(gbs / peaks["hbm_gbs"], 4),

@@ -327,6 +327,60 @@ mq_status mq_gemm(const mq_nvfp4_mat* xq, const mq_nvfp4_mat* wq, const mq_resid
     return gemm_impl(xq, wq, r, Y, M, N, K, flags, ws, ws_bytes, false, stream);
 }
 
+// Decode kernel with the activation quantization inside it (X bf16).
+static mq_status gemm_act_impl(const mq_bf16* X, const mq_nvfp4_mat* wq, const mq_residual_packed* r, mq_bf16* Y,
+                               int M, int N, int K, unsigned flags, void* ws, size_t ws_bytes, float* gx_out,
+                               bool prefetch, mq_stream stream) {
+    if (!X || !wq || !Y || M <= 0 || N <= 0 || K <= 0 || N % 64 || K % 64) return MQ_ERR_INVALID_ARG;
+    if (N % 128 || K % 256 || (flags & MQ_GEMM_PREFILL)) return MQ_ERR_UNSUPPORTED_SHAPE;
+    if (!wq->codes || !wq->sf_swz || !wq->gscale || wq->rows != N || wq->cols != K) return MQ_ERR_INVALID_ARG;
+    if ((flags & MQ_GEMM_BASE_ONLY) && (flags & MQ_GEMM_RESIDUAL_ONLY)) return MQ_ERR_INVALID_ARG;
+    if (!aligned(X, 16) || !aligned(wq->codes, 16) || !aligned(wq->sf_swz, 16)) return MQ_ERR_INVALID_ARG;
+    const bool has_r = r && r->nblk > 0 && !(flags & MQ_GEMM_BASE_ONLY);
+    if (r && r->nblk > 0) {
+        if (r->N != N || r->K != K || !r->blk_codes || !r->blk_sf || !r->tile_ptr || !r->bitmap)
+            return MQ_ERR_INVALID_ARG;
+        if (!aligned(r->blk_codes, 16) || !aligned(r->blk_sf, 16)) return MQ_ERR_INVALID_ARG;
+    }
+    GemmParams p;
+    memset(&p, 0, sizeof p);
+    p.w_sf = wq->sf_swz;
+    p.g_w = wq->gscale;
+    if (has_r) {
+        p.blk_codes = r->blk_codes;
+        p.blk_sf = r->blk_sf;
+        p.tile_ptr = r->tile_ptr;
+        p.bitmap = r->bitmap;
+    }
+    p.has_resid = has_r ? 1 : 0;
+    p.Y = Y;
+    p.M = M;
+    p.N = N;
+    p.K = K;
+    p.mode = (flags & MQ_GEMM_BASE_ONLY) ? 1 : (flags & MQ_GEMM_RESIDUAL_ONLY) ? 2 : 0;
+    p.prefetch = prefetch ? 1 : 0;
+    p.x_bf16 = X;
+    p.gx_out = gx_out;
+    DecodePlan d = plan_decode(M, N, K);
+    const size_t need = decode_workspace_bytes(M, N, K);
+    if (need > 0 && (!ws || ws_bytes < need || !aligned(ws, 16))) return MQ_ERR_WORKSPACE;
+    CUtensorMap tw;
+    if (!make_tmap_bytes(&tw, wq->codes, (uint64_t)K / 2, (uint64_t)N, 128, 128)) return MQ_ERR_CUDA;
+    if (need > 0) {
+        size_t part = (size_t)d.splits * d.tiles_m * d.BN * N * sizeof(float);
+        part = (part + 255) & ~size_t(255);
+        p.partial = static_cast<float*>(ws);
+        p.counters = reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + part);
+    }
+    // the X tensor map is not used in this mode
+    return launched(launch_gemm_decode(tw, tw, p, d, as_stream(stream)), 1);
+}
+
+mq_status mq_gemm_act(const mq_bf16* X, const mq_nvfp4_mat* wq, const mq_residual_packed* r, mq_bf16* Y, int M, int N,
+                      int K, unsigned flags, void* ws, size_t ws_bytes, float* gx_out, mq_stream stream) {
+    return gemm_act_impl(X, wq, r, Y, M, N, K, flags, ws, ws_bytes, gx_out, false, stream);
+}
+
 mq_status mq_run_layer(const mq_bf16* W, const mq_bf16* X, const mq_bf16* Xcal, mq_bf16* Y, int M, int N, int K,
                        int T, int budget, unsigned flags, int host, mq_layer_buffers* buf, mq_stream stream) {
     if (!W || !X || !Xcal || !Y || !buf || M <= 0 || N <= 0 || K <= 0 || T <= 0) return MQ_ERR_INVALID_ARG;
@@ -347,7 +401,7 @@ mq_status mq_run_layer(const mq_bf16* W, const mq_bf16* X, const mq_bf16* Xcal, 
     // The method's order. Every kernel waits for its predecessor before reading its
     // outputs (and lets its dependent start right after), so when the GEMM starts, the
     // quantize+Delta kernel has long completed and the GEMM requests W before waiting
-    // for the activation quantizer (prefetch).
+    // for its predecessor (prefetch).
     mq_status st;
     if ((st = mq_hessian_diag(xc, T, K, buf->H, stream)) != MQ_OK) return st;
     if ((st = mq_quantize_weight_delta(w, N, K, buf->H, &buf->base, nullptr, buf->delta, buf->ws_quant,
@@ -356,6 +410,9 @@ mq_status mq_run_layer(const mq_bf16* W, const mq_bf16* X, const mq_bf16* Xcal, 
     if ((st = mq_topk_blocks(buf->delta, (N / 64) * (K / 64), budget, buf->rank, buf->sel, stream)) != MQ_OK)
         return st;
     if ((st = mq_pack_residual_weight(w, &buf->base, buf->sel, budget, &buf->packed, stream)) != MQ_OK) return st;
+    // The activation quantizer runs as its own kernel: on B200 at decode sizes that is
+    // faster than quantizing inside the GEMM (mq_gemm_act), whose per-token maxima must
+    // first be exchanged between the K splits before the first MMA.
     if ((st = mq_quantize_act(x, M, K, &buf->xq, stream)) != MQ_OK) return st;
     if ((st = gemm_impl(&buf->xq, &buf->base, &buf->packed, y, M, N, K, flags, buf->ws_gemm, buf->ws_gemm_bytes, true,
                         stream)) != MQ_OK)

@@ -26,6 +26,7 @@
 
 #include "common.cuh"
 #include "gemm.cuh"
+#include "quant.cuh"
 
 namespace mq {
 
@@ -89,7 +90,11 @@ struct DecodeCfg {
     static constexpr int kOffRSF = kOffRC + 16384;       // 8 x 512 B
     static constexpr int kStageBytes = kOffRSF + 4096;
     static constexpr int kCtrlBytes = 256;  // 3 barriers per stage, accumulator barrier, TMEM address, masks
-    static constexpr int kSmemBytes = kStages * kStageBytes + kCtrlBytes + 1024;
+    // fused activation quantization: per-token partial maxima of every split [8][BN], the
+    // token scales [BN], this CTA's partial maxima [BN], the exchange barrier
+    static constexpr int kOffFused = kStages * kStageBytes + kCtrlBytes;
+    static constexpr int kFusedBytes = (kMaxClusterSplits + 2) * BN * 4 + 16;
+    static constexpr int kSmemBytes = kOffFused + kFusedBytes + 1024;
     static constexpr int kThreads = 192;
     static constexpr uint32_t kTmemCols = 512;
     static constexpr int kSfCol0 = 128;                  // scale columns start after D
@@ -171,16 +176,23 @@ __global__ void __launch_bounds__(192, 1)
     const int ks_end = min(KS, ks_begin + p.iters_per_split);
     const int n_iters = max(0, ks_end - ks_begin);
 
+    // fused activation quantization (p.x_bf16): warps 2-5 quantize X into the stages
+    const bool fused_x = p.x_bf16 != nullptr;
+    float* amax_in = reinterpret_cast<float*>(smem + C::kOffFused);  // [kMaxClusterSplits][BN]
+    float* g_s = amax_in + kMaxClusterSplits * BN;                      // [BN] token scales
+    float* part = g_s + BN;                                             // [BN] this CTA's maxima
+    uint64_t* xg_bar = reinterpret_cast<uint64_t*>(part + BN);          // peers' maxima landed
     if (warp == 0 && lane == 0) {
         for (int s = 0; s < C::kStages; ++s) {
-            mbar_init(&full[s], 1);
+            mbar_init(&full[s], fused_x ? 2 : 1);  // + the quantizer warps' arrival
             mbar_init(&rfull[s], 1);
             mbar_init(&empty[s], 1);
         }
         mbar_init(accf, 1);
+        mbar_init(xg_bar, fused_x && p.cluster ? p.splits : 1);
         mbar_fence_init();
         tma_prefetch_desc(&tmap_w);
-        tma_prefetch_desc(&tmap_x);
+        if (!fused_x) tma_prefetch_desc(&tmap_x);
     }
     if (warp == 1) {
         tmem_alloc(tmem_holder, C::kTmemCols);
@@ -190,6 +202,9 @@ __global__ void __launch_bounds__(192, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
+    // peers write their activation maxima into this CTA's shared memory: every barrier of
+    // the cluster is initialised before any of them starts
+    if (fused_x && p.cluster) cluster_sync();
 
     if (warp == 0) {
         // ---------------------------------------------------- producer (converged warp, one lane issues)
@@ -201,7 +216,7 @@ __global__ void __launch_bounds__(192, 1)
         auto issue_w = [&](int it) {
             const int st_i = it % C::kStages, ks = ks_begin + it;
             uint8_t* st = smem + st_i * C::kStageBytes;
-            mbar_arrive_expect_tx(&full[st_i], (dense ? 16384 + 2048 : 0) + BN * 128 + 2048);
+            mbar_arrive_expect_tx(&full[st_i], (dense ? 16384 + 2048 : 0) + (fused_x ? 0 : BN * 128 + 2048));
             if (dense) {
                 tma_load_2d(st + C::kOffW, &tmap_w, &full[st_i], ks * 128, n0);
                 bulk_load(st + C::kOffSFW, wsf_tile + (int64_t)ks * 4 * 512, 2048, &full[st_i]);
@@ -209,6 +224,7 @@ __global__ void __launch_bounds__(192, 1)
         };
         // X tile and X scales
         auto issue_x = [&](int it) {
+            if (fused_x) return;  // the quantizer warps write X into the stage
             const int st_i = it % C::kStages, ks = ks_begin + it;
             uint8_t* st = smem + st_i * C::kStageBytes;
             tma_load_2d(st + C::kOffX, &tmap_x, &full[st_i], ks * 128, m0);
@@ -339,7 +355,125 @@ __global__ void __launch_bounds__(192, 1)
         // ---------------------------------------------------- epilogue (warps 2..5)
         const int q = warp & 3;
         const int nl = 32 * q + lane, n = n0 + nl;
-        griddep_wait();  // g_x, Y and the workspace follow the previous kernel
+        griddep_wait();  // X, g_x, Y and the workspace follow the previous kernel
+        if (fused_x) {
+            // ---- activation quantization in the pipeline: per-token maxima over this
+            // CTA's K range, exchanged with the cluster's other K splits (or over all of K
+            // when the splits do not form a cluster), then every stage's BN x 256 block of
+            // X quantized straight into the stage's MMA layout, spread over all 128 threads
+            const int tq = threadIdx.x - 64;
+            const bool whole_k = p.splits > 1 && !p.cluster;
+            const int kb = whole_k ? 0 : ks_begin * 256, kspan = whole_k ? p.K : n_iters * 256;
+            {
+                // token t = tq / TPT, TPT threads per token striding over its 16-byte vectors
+                constexpr int TPT = 128 / BN;
+                const int t = tq / TPT, sub = tq % TPT, mm = m0 + t;
+                const int nvec = kspan / 8;
+                float mx = 0.0f;
+                if (mm < p.M) {
+                    const uint4* row = reinterpret_cast<const uint4*>(p.x_bf16 + (int64_t)mm * p.K + kb);
+                    for (int v0 = sub; v0 < nvec; v0 += TPT * 8) {
+                        uint4 x[8];  // eight independent loads in flight
+#pragma unroll
+                        for (int u = 0; u < 8; ++u) {
+                            const int v = v0 + TPT * u;
+                            x[u] = v < nvec ? __ldg(row + v) : make_uint4(0u, 0u, 0u, 0u);
+                        }
+#pragma unroll
+                        for (int u = 0; u < 8; ++u) {
+                            const uint32_t w[4] = {x[u].x, x[u].y, x[u].z, x[u].w};
+#pragma unroll
+                            for (int j = 0; j < 4; ++j)
+                                mx = max3(mx, fabsf(bf16_bits_to_f32(w[j] & 0xFFFFu)),
+                                          fabsf(bf16_bits_to_f32(w[j] >> 16)));
+                        }
+                    }
+                }
+#pragma unroll
+                for (int o = 1; o < TPT; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+                if (sub == 0) part[t] = mx;
+            }
+            // the stages' scale rows of tokens >= BN stay zero
+            for (int i = tq; i < C::kStages * 128; i += 128)
+                reinterpret_cast<uint4*>(smem + (i >> 7) * C::kStageBytes + C::kOffSFX)[i & 127] =
+                    make_uint4(0u, 0u, 0u, 0u);
+            asm volatile("bar.sync 1, 128;" ::: "memory");
+            bool xok = true;
+            if (p.cluster) {
+                // every split's maxima into every CTA of the cluster, then one arrival each
+                const uint32_t S = (uint32_t)p.splits, rank = cluster_ctarank();
+                if (tq < BN)
+                    for (uint32_t r = 0; r < S; ++r)
+                        st_dsmem_f32(mapa_u32(smem_u32(amax_in + rank * BN + tq), r), part[tq]);
+                asm volatile("bar.sync 1, 128;" ::: "memory");
+                if (tq == 0) {
+                    fence_acq_rel_cluster();
+                    for (uint32_t r = 0; r < S; ++r) mbar_arrive_remote(mapa_u32(smem_u32(xg_bar), r));
+                }
+                // bounded wait for the S arrivals
+                if (!mbar_try_wait_cluster(xg_bar, 0)) {
+                    const unsigned long long t0 = globaltimer();
+                    while (!mbar_try_wait_cluster(xg_bar, 0))
+                        if (globaltimer() - t0 > kWaitLimitNs) {
+                            atomicCAS(&g_error, 0, (int)MQ_ERR_TIMEOUT);
+                            xok = false;
+                            break;
+                        }
+                }
+                if (tq < BN) {
+                    float mx = 0.0f;
+                    for (uint32_t r = 0; r < S; ++r) mx = fmaxf(mx, amax_in[r * BN + tq]);
+                    part[tq] = mx;
+                }
+                asm volatile("bar.sync 1, 128;" ::: "memory");
+            }
+            if (tq < BN) {
+                const float mx = part[tq];
+                g_s[tq] = mx == 0.0f ? 1.0f : __fdiv_rn(mx, 2688.0f);
+                if (p.gx_out && n_tile == 0 && split == 0 && m0 + tq < p.M) p.gx_out[m0 + tq] = g_s[tq];
+            }
+            asm volatile("bar.sync 1, 128;" ::: "memory");
+            // group i = tq + 128 j of a stage: token i / 16, group (i % 16) of its 256 K
+            constexpr int GPT = BN * 16 / 128;  // groups per thread and stage
+            for (int it = 0; it < n_iters && xok; ++it) {
+                const int s = it % C::kStages, ks = ks_begin + it;
+                if (it >= C::kStages && !mbar_wait(&empty[s], ((it / C::kStages) - 1) & 1)) { xok = false; break; }
+                uint8_t* st = smem + s * C::kStageBytes;
+                constexpr int kChunk = GPT < 4 ? GPT : 4;  // groups loaded together
+#pragma unroll 1
+                for (int j0 = 0; j0 < GPT; j0 += kChunk) {
+                float a[kChunk][16];
+#pragma unroll
+                for (int jj = 0; jj < kChunk; ++jj) {  // the chunk's loads first
+                    const int i = tq + 128 * (j0 + jj), t = i >> 4, q16 = i & 15, mm = m0 + t;
+                    if (mm < p.M) {
+                        load16_bf16(p.x_bf16 + (int64_t)mm * p.K + ks * 256 + q16 * 16, a[jj]);
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) a[jj][e] = 0.0f;
+                    }
+                }
+#pragma unroll
+                for (int jj = 0; jj < kChunk; ++jj) {
+                    const int j = j0 + jj;
+                    const int i = tq + 128 * j, t = i >> 4, q16 = i & 15, kk = q16 >> 2, gq = q16 & 3;
+                    const float g = g_s[t], g6 = __fmul_rn(6.0f, g);
+                    float deq[16];
+                    uint32_t lo, hi;
+                    const uint32_t sfb = nvfp4_group(a[jj], g, g6, lo, hi, deq);
+                    // 8 bytes of token row t at byte 8*q16 (128-byte swizzle); the scale in
+                    // chunk kk, row t (t < BN <= 128: byte (t%32)*16 + (t/32)*4 + gq)
+                    const int c = q16 >> 1;
+                    *reinterpret_cast<uint2*>(st + C::kOffX + t * 128 + ((c ^ (t & 7)) << 4) + 8 * (q16 & 1)) =
+                        make_uint2(lo, hi);
+                    st[C::kOffSFX + kk * 512 + (t & 31) * 16 + (t >> 5) * 4 + gq] = (uint8_t)sfb;
+                }
+                }
+                fence_proxy_async_smem();  // the MMA reads these through the async proxy
+                asm volatile("bar.sync 1, 128;" ::: "memory");
+                if (tq == 0) mbar_arrive(&full[s]);
+            }
+        }
         const bool waited = mbar_wait(accf, 0);
         tc_fence_after();
         const bool have = waited && tile_has_mma(p, n_tile, ks_begin, ks_end);
@@ -360,7 +494,7 @@ __global__ void __launch_bounds__(192, 1)
                 for (int j = 0; j < 16; ++j) {
                     const int mm = m0 + c0 + j;
                     if (mm < p.M) {
-                        const float sc = __fmul_rn(__ldg(p.g_x + mm), gw);
+                        const float sc = __fmul_rn(fused_x ? g_s[mm - m0] : __ldg(p.g_x + mm), gw);
                         const __nv_bfloat16 y = __float2bfloat16_rn(__fmul_rn(acc[j], sc));
                         p.Y[(int64_t)mm * p.N + n] = *reinterpret_cast<const uint16_t*>(&y);
                     }
@@ -404,7 +538,7 @@ __global__ void __launch_bounds__(192, 1)
                     for (int j = 0; j < 8; ++j) {
                         const int mm = m0 + c0 + j;
                         if (mm < p.M) {
-                            const float sc = __fmul_rn(__ldg(p.g_x + mm), gw);
+                            const float sc = __fmul_rn(fused_x ? g_s[mm - m0] : __ldg(p.g_x + mm), gw);
                             const __nv_bfloat16 y = __float2bfloat16_rn(__fmul_rn(sum[j], sc));
                             p.Y[(int64_t)mm * p.N + n] = *reinterpret_cast<const uint16_t*>(&y);
                         }
@@ -450,7 +584,7 @@ __global__ void __launch_bounds__(192, 1)
                     for (uint32_t s2 = 1; s2 < (uint32_t)kMaxClusterSplits; ++s2)
                         if (s2 < S) sum = __fadd_rn(sum, v[u][s2]);
                     if (mm < p.M) {
-                        const float sc = __fmul_rn(__ldg(p.g_x + mm), gw);
+                        const float sc = __fmul_rn(fused_x ? g_s[mm - m0] : __ldg(p.g_x + mm), gw);
                         const __nv_bfloat16 y = __float2bfloat16_rn(__fmul_rn(sum, sc));
                         p.Y[(int64_t)mm * p.N + n0 + nl] = *reinterpret_cast<const uint16_t*>(&y);
                     }

@@ -27,6 +27,9 @@ struct GemmParams {
     int cluster;             // split-K reduced through the cluster's shared memory
     int prefetch;            // W was complete before the preceding kernel started, so the
                              // decode kernel may load it before waiting for that kernel
+    const uint16_t* x_bf16;  // decode kernel: bf16 X [M][K] quantized inside the kernel
+                             // (x_sf and g_x unused), or null
+    float* gx_out;           // with x_bf16: per-token scales written here if not null
 };
 
 // Decode kernel tiling: token tile BN, grid tiles_n x splits x tiles_m, `iters`

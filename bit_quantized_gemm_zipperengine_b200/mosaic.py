@@ -27,7 +27,7 @@ EXPORTED = (
     "mq_gemm_workspace_bytes", "mq_quantize_weight", "mq_hessian_diag", "mq_delta_score_topk", "mq_pack_residual",
     "mq_quantize_act", "mq_gemm", "mq_run_layer", "mq_get_error", "mq_status_string", "mq_launch_count",
     "mq_gemm_noalloc", "mq_gemm_noalloc_scratch_limit", "mq_quantize_weight_delta", "mq_topk_blocks",
-    "mq_pack_residual_weight",
+    "mq_pack_residual_weight", "mq_gemm_act",
 )
 
 
@@ -95,6 +95,8 @@ def lib():
     L.mq_topk_blocks.restype = i32
     L.mq_pack_residual_weight.argtypes = [vp, P(NVFP4Mat), vp, i32, P(ResidualPacked), vp]
     L.mq_pack_residual_weight.restype = i32
+    L.mq_gemm_act.argtypes = [vp, P(NVFP4Mat), P(ResidualPacked), vp, i32, i32, i32, ctypes.c_uint, vp, sz, vp, vp]
+    L.mq_gemm_act.restype = i32
     L.mq_get_error.argtypes = [vp]
     L.mq_status_string.argtypes = [i32]
     L.mq_status_string.restype = ctypes.c_char_p
@@ -237,6 +239,15 @@ def mq_run_layer(W, X, Xcal, Y, M: int, N: int, K: int, T: int, budget: int, fla
         return _ptr(t)
     _check(lib().mq_run_layer(p(W), p(X), p(Xcal), p(Y), M, N, K, T, budget, flags, 1 if host else 0,
                               ctypes.byref(buf), _stream(stream)), "mq_run_layer")
+
+
+def mq_gemm_act(X: torch.Tensor, wq: dict, packed: dict | None, Y: torch.Tensor, M: int, N: int, K: int,
+                flags: int = 0, ws: torch.Tensor | None = None, gx: torch.Tensor | None = None, stream=None):
+    """Decode-kernel GEMM that quantizes the bf16 activations itself (gx receives g_x)."""
+    ps = packed_struct(packed)
+    nbytes = 0 if ws is None else ws.numel() * ws.element_size()
+    _check(lib().mq_gemm_act(_ptr(X), ctypes.byref(mat(wq)), None if ps is None else ctypes.byref(ps), _ptr(Y), M, N,
+                             K, flags, _ptr(ws), nbytes, _ptr(gx), _stream(stream)), "mq_gemm_act")
 
 
 def mq_gemm_noalloc(xq: dict, wq: dict, packed: dict | None, Y: torch.Tensor, M: int, N: int, K: int,

@@ -228,6 +228,22 @@ mq_status mq_gemm(const mq_nvfp4_mat* xq, const mq_nvfp4_mat* wq, const mq_resid
                   int M, int N, int K, unsigned flags, void* ws, size_t ws_bytes, mq_stream stream);
 
 /*
+ * A6 + A7 + A8 in one kernel: the activation quantization runs inside the fused GEMM's
+ * pipeline ("quantization ... scheduled concurrently" with the dense and sparse MMAs and
+ * the reduce-sum: summary, "Methodology", section 3), for the decode kernel. X: bf16
+ * [M][K] (16-byte aligned). Each CTA quantizes the tokens of its tile over its K range
+ * straight into the MMA's operand layout; the per-token scale g_x[m] = amax(X[m,:])/2688
+ * (1 if 0) comes from maxima exchanged between the K splits of a tile through the
+ * thread-block cluster's shared memory (or, for more than 8 splits, each CTA reads the
+ * whole row). Codes, scales and Y are those of mq_quantize_act followed by mq_gemm with
+ * the decode kernel (bit-identical). gx_out: [M] fp32, receives g_x, or NULL. Other
+ * arguments, flags and workspace as in mq_gemm; MQ_GEMM_PREFILL returns
+ * MQ_ERR_UNSUPPORTED_SHAPE (the large-M kernel takes a quantized X).
+ */
+mq_status mq_gemm_act(const mq_bf16* X, const mq_nvfp4_mat* wq, const mq_residual_packed* r, mq_bf16* Y, int M, int N,
+                      int K, unsigned flags, void* ws, size_t ws_bytes, float* gx_out, mq_stream stream);
+
+/*
  * Device buffers of one layer for mq_run_layer (all caller-owned; sizes as in the
  * individual calls above). W_dev, X_dev, Xcal_dev and Y_dev are staging buffers used
  * only when mq_run_layer is given host pointers.
@@ -255,8 +271,8 @@ typedef struct {
  * The whole path for one layer in the method's order: A2 H from the T calibration
  * tokens, A1+A3 quantize W and score every block (mq_quantize_weight_delta, residual not
  * stored), A4 top-`budget` selection, A5 pack the selected residual from W
- * (mq_pack_residual_weight), A6 quantize X, A7+A8 fused GEMM into Y; results are those of
- * the individual calls in this order. With host == 0, W, X, Xcal and Y are device
+ * (mq_pack_residual_weight), A6 quantize X (mq_quantize_act), A7+A8 fused GEMM into Y.
+ * Results are those of the individual calls. With host == 0, W, X, Xcal and Y are device
  * pointers. With host != 0 they are HOST pointers (page-locked for the copies to be
  * asynchronous): the inputs are copied into buf->W_dev, X_dev, Xcal_dev and the result
  * from buf->Y_dev back to Y, all on `stream`. Errors as the individual calls.

@@ -302,3 +302,39 @@ def test_odd_block_rows_bit_exact(fused, dev):
         assert np.array_equal(layer.packed[k][:budget].cpu().numpy(), packed[k]), k
     assert np.array_equal(layer.packed["tile_ptr"].cpu().numpy(), packed["tile_ptr"])
     assert np.array_equal(layer.packed["bitmap"].cpu().numpy().view(np.uint32), packed["bitmap"])
+
+
+@pytest.mark.parametrize("N,K", [(4096, 4096), (1024, 4096), (512, 1024), (25600, 512)])
+@pytest.mark.parametrize("M", [1, 5, 16, 37, 64, 100, 128])
+def test_gemm_act_fused_quantization(N, K, M, dev):
+    """The decode GEMM quantizing bf16 X itself (A6 inside the pipeline) against
+    mq_quantize_act + mq_gemm: per-token scales bit-exact with the oracle and Y bit-exact
+    with the two-call path, across token tiles and the three split-K regimes (no split:
+    N = 25600; split in a cluster: N = 4096 and 512; more than 8 splits through the
+    workspace: N = 1024), plus the oracle within the GEMM tolerance."""
+    from bit_quantized_gemm_zipperengine_b200 import mosaic
+    Wb = synth.weight(N, K, 901, 904, 0.02, int(0.005 * N * K), max(1, (N // 64) * (K // 64) // 20), 20.0)
+    Xb = synth.act(M, K, 902, 904, max(1, K // 100), 30.0)
+    Cb = synth.act(64, K, 903, 904, max(1, K // 100), 30.0)
+    budget = synth.budget_blocks(N, K, 0.10)
+    layer = mosaic.Layer(N, K, budget, dev, with_sf=False)
+    layer.prepare_path(to_dev(Wb, dev), to_dev(Cb, dev))
+    X = to_dev(Xb, dev)
+    flags = mosaic.MQ_GEMM_DECODE
+    xq, Y2, ws = layer.act_buffers(M, flags)
+    mosaic.mq_quantize_act(X, xq)
+    mosaic.mq_gemm(xq, layer.base, layer.packed, Y2, M, N, K, flags, ws)
+    Y1 = torch.empty_like(Y2)
+    gx = torch.empty(M, dtype=torch.float32, device=dev)
+    ws1 = mosaic.gemm_workspace(M, N, K, flags, dev)
+    for _ in range(2):  # twice: the scratch counters reset themselves
+        mosaic.mq_gemm_act(X, layer.base, layer.packed, Y1, M, N, K, flags, ws1, gx)
+    torch.cuda.synchronize()
+    assert mosaic.mq_get_error() == 0
+    xo = oracle.quantize_act(Xb)
+    assert np.array_equal(gx.cpu().numpy().view(np.uint32), xo["g"].view(np.uint32))
+    assert torch.equal(Y1.view(torch.int16), Y2.view(torch.int16))
+    wq = oracle.quantize_weight(Wb)
+    sel = layer.sel[:budget].cpu().numpy()
+    y_ref, yabs = oracle.gemm_rows(xo, wq, sel, M, N, K)
+    check_gemm(Y1.float().cpu().numpy().astype(np.float64), y_ref, yabs, f"gemm_act N={N} K={K} M={M}")
