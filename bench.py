@@ -466,16 +466,16 @@ def main():
     # user issues it; consecutive kernels overlap through programmatic dependent launch),
     # and a profiling graph issues the same steps as separate public calls with event
     # nodes between them (which serialise them) for the in-step per-call times
-    calls = ["hessian_diag", "quantize_weight_delta", "topk_blocks", "pack_residual", "quantize_act", "gemm"]
+    calls = ["hessian_diag", "quantize_weight_delta", "quantize_act", "topk_blocks", "pack_residual", "gemm"]
 
     def issue_step(s, events=None, cs=None):
         layer = s["layer"]
         xq, Yb, ws = layer.act_buffers(M)
         ops = [lambda: mosaic.mq_hessian_diag(s["Xcal"], layer.H),
                lambda: mosaic.mq_quantize_weight_delta(s["W"], layer.H, layer.base, None, layer.delta, layer.qws),
+               lambda: mosaic.mq_quantize_act(s["X"], xq),
                lambda: mosaic.mq_topk_blocks(layer.delta, budget, layer.rank, layer.sel),
                lambda: mosaic.mq_pack_residual_weight(s["W"], layer.base, layer.sel, budget, layer.packed),
-               lambda: mosaic.mq_quantize_act(s["X"], xq),
                lambda: mosaic.mq_gemm(xq, layer.base, layer.packed, Yb, M, N, K, 0, ws)]
         for j, op in enumerate(ops):
             if events is not None:

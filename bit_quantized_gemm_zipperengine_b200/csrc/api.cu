@@ -14,8 +14,9 @@ int amax_grid(int64_t n8);
 cudaError_t launch_quant_weight(const uint16_t* W, int N, int K, uint8_t* codes, uint8_t* sf, uint8_t* sf_swz,
                                 float* g, uint8_t* rcodes, uint8_t* rsf, float* partial, cudaStream_t s);
 cudaError_t launch_quant_act(const uint16_t* X, int M, int K, uint8_t* codes, uint8_t* sf, uint8_t* sf_swz,
-                             float* g, cudaStream_t s);
+                             float* g, bool early, cudaStream_t s);
 cudaError_t launch_hessian(const uint16_t* X, int T, int K, float* H, cudaStream_t s);
+int hessian_max_tokens();
 cudaError_t launch_delta(const CUtensorMap& tw, int N, int K, const float* H, const float* g, double* delta,
                          int* err, cudaStream_t s);
 cudaError_t launch_quant_delta(const uint16_t* W, const CUtensorMap& tw, int N, int K, const float* H,
@@ -159,7 +160,8 @@ mq_status mq_quantize_weight(const mq_bf16* W, int N, int K, mq_nvfp4_mat* base,
 }
 
 mq_status mq_hessian_diag(const mq_bf16* Xcal, int T, int K, float* H, mq_stream stream) {
-    if (!Xcal || !H || T <= 0 || K <= 0 || K % 64) return MQ_ERR_INVALID_ARG;
+    if (!Xcal || !H || T <= 0 || K <= 0 || K % 64 || !aligned(Xcal, 16)) return MQ_ERR_INVALID_ARG;
+    if (T > hessian_max_tokens()) return MQ_ERR_UNSUPPORTED_SHAPE;
     return launched(launch_hessian(Xcal, T, K, H, as_stream(stream)), 1);
 }
 
@@ -253,7 +255,19 @@ mq_status mq_quantize_act(const mq_bf16* X, int M, int K, mq_nvfp4_mat* xq, mq_s
     if (!X || !xq || !xq->codes || !xq->sf_swz || !xq->gscale || !nvfp4_shape_ok(M, K)) return MQ_ERR_INVALID_ARG;
     if (xq->rows != M || xq->cols != K || !aligned(X, 16) || !aligned(xq->codes, 8) || !aligned(xq->sf_swz, 4))
         return MQ_ERR_INVALID_ARG;
-    return launched(launch_quant_act(X, M, K, xq->codes, xq->sf, xq->sf_swz, xq->gscale, as_stream(stream)), 1);
+    if (K > 65536) return MQ_ERR_UNSUPPORTED_SHAPE;
+    return launched(launch_quant_act(X, M, K, xq->codes, xq->sf, xq->sf_swz, xq->gscale, false, as_stream(stream)), 1);
+}
+
+// The whole-path call's activation quantizer: it quantizes X before waiting for the
+// kernel preceding it (X is an input of that call, and the previous readers of xq are
+// complete by the time any kernel of the call after the first one starts).
+static mq_status quantize_act_early(const mq_bf16* X, int M, int K, mq_nvfp4_mat* xq, mq_stream stream) {
+    if (!X || !xq || !xq->codes || !xq->sf_swz || !xq->gscale || !nvfp4_shape_ok(M, K)) return MQ_ERR_INVALID_ARG;
+    if (xq->rows != M || xq->cols != K || !aligned(X, 16) || !aligned(xq->codes, 8) || !aligned(xq->sf_swz, 4))
+        return MQ_ERR_INVALID_ARG;
+    if (K > 65536) return MQ_ERR_UNSUPPORTED_SHAPE;
+    return launched(launch_quant_act(X, M, K, xq->codes, xq->sf, xq->sf_swz, xq->gscale, true, as_stream(stream)), 1);
 }
 
 // prefetch: the caller guarantees wq was complete before the kernel preceding the GEMM in
@@ -398,22 +412,23 @@ mq_status mq_run_layer(const mq_bf16* W, const mq_bf16* X, const mq_bf16* Xcal, 
         xc = buf->Xcal_dev;
         y = buf->Y_dev;
     }
-    // The method's order. Every kernel waits for its predecessor before reading its
-    // outputs (and lets its dependent start right after), so when the GEMM starts, the
-    // quantize+Delta kernel has long completed and the GEMM requests W before waiting
-    // for its predecessor (prefetch).
+    // The method's order, with the activation quantizer moved ahead of top-K. Every kernel
+    // but that one and the weight maxima pass waits for its predecessor before reading
+    // its outputs and lets its dependent start right after; those two read only inputs of
+    // this call, do their work first and wait at their end. So when the GEMM starts, the
+    // quantize+Delta kernel has long completed, and the GEMM requests W before waiting for
+    // its predecessor (prefetch). The activation quantizer runs as its own kernel: on
+    // B200 at decode sizes that is faster than quantizing inside the GEMM (mq_gemm_act),
+    // whose per-token maxima must first be exchanged between the K splits.
     mq_status st;
     if ((st = mq_hessian_diag(xc, T, K, buf->H, stream)) != MQ_OK) return st;
     if ((st = mq_quantize_weight_delta(w, N, K, buf->H, &buf->base, nullptr, buf->delta, buf->ws_quant,
                                        buf->ws_quant_bytes, stream)) != MQ_OK)
         return st;
+    if ((st = quantize_act_early(x, M, K, &buf->xq, stream)) != MQ_OK) return st;
     if ((st = mq_topk_blocks(buf->delta, (N / 64) * (K / 64), budget, buf->rank, buf->sel, stream)) != MQ_OK)
         return st;
     if ((st = mq_pack_residual_weight(w, &buf->base, buf->sel, budget, &buf->packed, stream)) != MQ_OK) return st;
-    // The activation quantizer runs as its own kernel: on B200 at decode sizes that is
-    // faster than quantizing inside the GEMM (mq_gemm_act), whose per-token maxima must
-    // first be exchanged between the K splits before the first MMA.
-    if ((st = mq_quantize_act(x, M, K, &buf->xq, stream)) != MQ_OK) return st;
     if ((st = gemm_impl(&buf->xq, &buf->base, &buf->packed, y, M, N, K, flags, buf->ws_gemm, buf->ws_gemm_bytes, true,
                         stream)) != MQ_OK)
         return st;

@@ -136,11 +136,9 @@ __global__ void __launch_bounds__(256) k_quant_weight(const uint16_t* __restrict
 // thread, groups tid + j * blockDim), so the row is read once. Rows >= M only clear
 // their tiled scales.
 template <int kGPT>
-__global__ void __launch_bounds__(1024) k_quant_act(const uint16_t* __restrict__ X, int M, int K,
-                                                    uint8_t* __restrict__ codes, uint8_t* __restrict__ sf,
-                                                    uint8_t* __restrict__ sf_swz, float* __restrict__ g_x) {
-    griddep_wait();
-    griddep_launch();
+__device__ __forceinline__ void quant_act_row(const uint16_t* __restrict__ X, int M, int K,
+                                              uint8_t* __restrict__ codes, uint8_t* __restrict__ sf,
+                                              uint8_t* __restrict__ sf_swz, float* __restrict__ g_x) {
     const int m = blockIdx.x;
     const int G = K / 16;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -193,66 +191,85 @@ __global__ void __launch_bounds__(1024) k_quant_act(const uint16_t* __restrict__
     }
 }
 
-// A2: H_k = fp32( sum_t x_tk^2 / T ), the fp64 sum taken in t order. A CTA owns 32
-// columns; all threads stage 128-row chunks of those columns in shared memory (a ring
-// of kHChunks chunks in flight with cp.async), one warp runs the 32 sequential sums.
-constexpr int kHCols = 32, kHRows = 128, kHChunks = 4, kHThreads = 256;
-
-__device__ __forceinline__ void cp_async16(void* dst, const void* src, bool pred) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(pred ? 16 : 0)
-                 : "memory");
+// early == 0: wait for the preceding kernel, let the dependent start, quantize.
+// early != 0: let the dependent start, quantize, then wait for the preceding kernel before
+// exiting (so this kernel's completion still implies its predecessor's). For a caller
+// whose X and outputs are not touched by the kernels still running before it.
+template <int kGPT>
+__global__ void __launch_bounds__(1024)
+    k_quant_act(const uint16_t* __restrict__ X, int M, int K, uint8_t* __restrict__ codes,
+                uint8_t* __restrict__ sf, uint8_t* __restrict__ sf_swz, float* __restrict__ g_x, int early) {
+    if (!early) griddep_wait();
+    griddep_launch();
+    quant_act_row<kGPT>(X, M, K, codes, sf, sf_swz, g_x);
+    if (early) griddep_wait();
 }
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
-__global__ void __launch_bounds__(kHThreads) k_hessian(const uint16_t* __restrict__ X, int T, int K,
-                                                       float* __restrict__ H) {
+// A2: H_k = fp32(S_k / T), S_k the fp64 sum of the exact squares fp64(x_tk)^2 by a fixed
+// pairwise tree over t: the squares padded with zeros to a power of two P >= T, then
+// v[i] += v[i + h] for h = P/2, ..., 1. Every sum in the tree is >= +0 and x + (+0) == x,
+// so the padding leaves change nothing and any power of two >= T gives the same S_k; the
+// kernel takes P = 512 * NB (NB = 1 for T <= 512, 2 for T <= 1024).
+// A CTA of 8 warps owns 32 columns; lane l of warp w holds the rows i = r0 + 64 j with
+// r0 = 8 (l >> 2) + w and the 8 columns of quad l & 3 (one 16-byte load per row, 64
+// contiguous bytes per row per warp). The tree's levels, in order:
+//   h = P/2 .. 64  rows of one thread: J = 8 NB leaves j, taken as NB batches of 8
+//                  (batch b: j = b + NB m), each the 8-leaf tree over m, then the batches;
+//   h = 32, 16, 8  lanes 16, 8, 4 apart (r0 + 32, + 16, + 8);
+//   h = 4, 2, 1    warps, in shared memory, one thread per column.
+constexpr int kHMaxTokens = 1024;
+template <int NB>
+__global__ void __launch_bounds__(256) k_hessian(const uint16_t* __restrict__ X, int T, int K,
+                                                 float* __restrict__ H) {
     griddep_wait();
     griddep_launch();
-    __shared__ __align__(16) uint16_t buf[kHChunks][kHRows][kHCols];
-    const int k0 = blockIdx.x * kHCols;
-    const int nchunks = (T + kHRows - 1) / kHRows;
-    auto issue = [&](int c) {
-        if (c < nchunks) {
-            // 128 rows x 64 bytes = 512 16-byte pieces, two per thread
+    __shared__ double red[8][33];
+    const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int r0 = 8 * (lane >> 2) + w, c0 = blockIdx.x * 32 + (lane & 3) * 8;
+    uint4 raw[8 * NB];
 #pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                const int piece = threadIdx.x + u * kHThreads;
-                const int r = piece >> 2, part = piece & 3;
-                const int t = c * kHRows + r;
-                const bool ok = t < T;
-                cp_async16(&buf[c % kHChunks][r][part * 8], X + (int64_t)(ok ? t : 0) * K + k0 + part * 8, ok);
-            }
-        }
-        cp_async_commit();
-    };
-#pragma unroll
-    for (int c = 0; c < kHChunks - 1; ++c) issue(c);
-    double s = 0.0;
-    for (int c = 0; c < nchunks; ++c) {
-        issue(c + kHChunks - 1);
-        cp_async_wait<kHChunks - 1>();
-        __syncthreads();
-        if (threadIdx.x < kHCols) {
-            const int rows = min(kHRows, T - c * kHRows);
-            const uint16_t(*b)[kHCols] = buf[c % kHChunks];
-            int r = 0;
-            for (; r + 8 <= rows; r += 8) {
-                double x[8];
-#pragma unroll
-                for (int j = 0; j < 8; ++j) x[j] = (double)bf16_bits_to_f32(b[r + j][threadIdx.x]);
-#pragma unroll
-                for (int j = 0; j < 8; ++j) s = __dadd_rn(s, __dmul_rn(x[j], x[j]));
-            }
-            for (; r < rows; ++r) {
-                const double x = (double)bf16_bits_to_f32(b[r][threadIdx.x]);
-                s = __dadd_rn(s, __dmul_rn(x, x));
-            }
-        }
-        __syncthreads();
+    for (int j = 0; j < 8 * NB; ++j) {
+        const int i = r0 + 64 * j;
+        raw[j] = i < T ? ld_stream16(reinterpret_cast<const uint4*>(X + (int64_t)i * K + c0)) : make_uint4(0, 0, 0, 0);
     }
-    if (threadIdx.x < kHCols) H[k0 + threadIdx.x] = __double2float_rn(__ddiv_rn(s, (double)T));
+    double acc[8];
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+#pragma unroll
+        for (int b = 0; b < NB; ++b) {
+            double u[8];
+#pragma unroll
+            for (int m = 0; m < 8; ++m) {
+                const uint4 r = raw[b + NB * m];
+                const uint32_t wd = c < 2 ? r.x : c < 4 ? r.y : c < 6 ? r.z : r.w;
+                const double x = (double)bf16_bits_to_f32((c & 1) ? wd >> 16 : wd & 0xFFFFu);
+                u[m] = __dmul_rn(x, x);
+            }
+#pragma unroll
+            for (int h = 4; h >= 1; h >>= 1)
+#pragma unroll
+                for (int m = 0; m < h; ++m) u[m] = __dadd_rn(u[m], u[m + h]);
+            acc[c] = b == 0 ? u[0] : __dadd_rn(acc[c], u[0]);
+        }
+    }
+#pragma unroll
+    for (int h = 16; h >= 4; h >>= 1)  // lanes below h end with the sums they need
+#pragma unroll
+        for (int c = 0; c < 8; ++c) acc[c] = __dadd_rn(acc[c], __shfl_down_sync(0xFFFFFFFFu, acc[c], h));
+    if (lane < 4)
+#pragma unroll
+        for (int c = 0; c < 8; ++c) red[w][lane * 8 + c] = acc[c];
+    __syncthreads();
+    if (w == 0) {
+        double u[8];
+#pragma unroll
+        for (int m = 0; m < 8; ++m) u[m] = red[m][lane];
+#pragma unroll
+        for (int h = 4; h >= 1; h >>= 1)
+#pragma unroll
+            for (int m = 0; m < h; ++m) u[m] = __dadd_rn(u[m], u[m + h]);
+        H[blockIdx.x * 32 + lane] = __double2float_rn(__ddiv_rn(u[0], (double)T));
+    }
 }
 
 // ------------------------------------------------------------------ launchers
@@ -272,19 +289,26 @@ cudaError_t launch_quant_weight(const uint16_t* W, int N, int K, uint8_t* codes,
 }
 
 cudaError_t launch_quant_act(const uint16_t* X, int M, int K, uint8_t* codes, uint8_t* sf, uint8_t* sf_swz,
-                             float* g, cudaStream_t s) {
+                             float* g, bool early, cudaStream_t s) {
     const int Mp = (M + 127) / 128 * 128;
     const int G = K / 16;
     const int gpt = G <= 1024 ? 1 : G <= 2048 ? 2 : 4;
+    if (G > 4 * 1024) return cudaErrorInvalidValue;
     int threads = (G + gpt - 1) / gpt;
     threads = (threads + 31) / 32 * 32;
-    if (gpt == 1) return launch_pdl(k_quant_act<1>, dim3(Mp), dim3(threads), 0, s, 1, X, M, K, codes, sf, sf_swz, g);
-    if (gpt == 2) return launch_pdl(k_quant_act<2>, dim3(Mp), dim3(threads), 0, s, 1, X, M, K, codes, sf, sf_swz, g);
-    return launch_pdl(k_quant_act<4>, dim3(Mp), dim3(threads), 0, s, 1, X, M, K, codes, sf, sf_swz, g);
+    const int e = early ? 1 : 0;
+    if (gpt == 1)
+        return launch_pdl(k_quant_act<1>, dim3(Mp), dim3(threads), 0, s, 1, X, M, K, codes, sf, sf_swz, g, e);
+    if (gpt == 2)
+        return launch_pdl(k_quant_act<2>, dim3(Mp), dim3(threads), 0, s, 1, X, M, K, codes, sf, sf_swz, g, e);
+    return launch_pdl(k_quant_act<4>, dim3(Mp), dim3(threads), 0, s, 1, X, M, K, codes, sf, sf_swz, g, e);
 }
 
 cudaError_t launch_hessian(const uint16_t* X, int T, int K, float* H, cudaStream_t s) {
-    return launch_pdl(k_hessian, dim3(K / kHCols), dim3(kHThreads), 0, s, 1, X, T, K, H);
+    if (T > 512) return launch_pdl(k_hessian<2>, dim3(K / 32), dim3(256), 0, s, 1, X, T, K, H);
+    return launch_pdl(k_hessian<1>, dim3(K / 32), dim3(256), 0, s, 1, X, T, K, H);
 }
+
+int hessian_max_tokens() { return kHMaxTokens; }
 
 }  // namespace mq

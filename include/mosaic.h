@@ -139,8 +139,11 @@ mq_status mq_quantize_weight(const mq_bf16* W, int N, int K, mq_nvfp4_mat* base,
 
 /*
  * A2. Diagonal Hessian estimate of the input channels (summary, "Methodology",
- * section 2): H_k = fp32( sum_t fp64(x_tk)^2 / T ), sum in t order. Xcal: bf16 [T][K],
- * H: fp32 [K]. T >= 1, K % 64 == 0.
+ * section 2): H_k = fp32( S_k / T ), S_k the fp64 sum of the squares fp64(x_tk)^2 by a
+ * fixed pairwise tree over t (the T squares padded with zeros to the next power of two
+ * P, then v[i] += v[i+h] for h = P/2, ..., 1). Xcal: bf16 [T][K], H: fp32 [K].
+ * 1 <= T <= 1024 calibration tokens (MQ_ERR_UNSUPPORTED_SHAPE above), K % 64 == 0,
+ * Xcal 16-byte aligned (MQ_ERR_INVALID_ARG otherwise).
  */
 mq_status mq_hessian_diag(const mq_bf16* Xcal, int T, int K, float* H, mq_stream stream);
 
@@ -208,6 +211,7 @@ mq_status mq_pack_residual_weight(const mq_bf16* W, const mq_nvfp4_mat* base, co
  * A6. Activation quantization (summary, "Methodology", section 3: quantization inside
  * the pipeline). X: bf16 [M][K]. Per token m: g_x[m] = amax(X[m,:]) / 2688 (1 if 0),
  * then NVFP4 with that scale. xq: codes, sf_swz and gscale[M] required, sf optional.
+ * K <= 65536 (MQ_ERR_UNSUPPORTED_SHAPE above). X 16-byte aligned, codes 8, sf_swz 4.
  */
 mq_status mq_quantize_act(const mq_bf16* X, int M, int K, mq_nvfp4_mat* xq, mq_stream stream);
 
@@ -268,11 +272,13 @@ typedef struct {
 } mq_layer_buffers;
 
 /*
- * The whole path for one layer in the method's order: A2 H from the T calibration
- * tokens, A1+A3 quantize W and score every block (mq_quantize_weight_delta, residual not
- * stored), A4 top-`budget` selection, A5 pack the selected residual from W
- * (mq_pack_residual_weight), A6 quantize X (mq_quantize_act), A7+A8 fused GEMM into Y.
- * Results are those of the individual calls. With host == 0, W, X, Xcal and Y are device
+ * The whole path for one layer: A2 H from the T calibration tokens, A1+A3 quantize W and
+ * score every block (mq_quantize_weight_delta, residual not stored), A6 quantize X
+ * (mq_quantize_act; it depends on X alone and runs ahead of the selection so that it
+ * overlaps the Delta pass), A4 top-`budget` selection, A5 pack the selected residual from
+ * W (mq_pack_residual_weight), A7+A8 fused GEMM into Y. Results are those of the
+ * individual calls. The call's first kernel waits for the kernel preceding the call in
+ * the stream before the others may start, so no input is read before that kernel ends. With host == 0, W, X, Xcal and Y are device
  * pointers. With host != 0 they are HOST pointers (page-locked for the copies to be
  * asynchronous): the inputs are copied into buf->W_dev, X_dev, Xcal_dev and the result
  * from buf->Y_dev back to Y, all on `stream`. Errors as the individual calls.

@@ -146,7 +146,7 @@ def quantize_act(X: np.ndarray) -> dict:
 
 
 def hessian_diag(Xcal: np.ndarray) -> np.ndarray:
-    """A2: H_k = fp32(sum_t x_tk^2 / T), fp64 sequential sum."""
+    """A2: H_k = fp32(sum_t x_tk^2 / T), fp64 sum by a pairwise tree over t."""
     Xcal = _c(Xcal, np.uint16)
     T, K = Xcal.shape
     H = np.zeros(K, np.float32)

@@ -216,17 +216,25 @@ void orc_quantize_act(const uint16_t* X, int M, int K, uint8_t* codes, uint8_t* 
     free(x);
 }
 
-/* Diagonal Hessian estimate (A2): H_k = fp32( (sum_t fp64(x_tk)^2) / T ), the sum
- * taken sequentially over t in fp64. */
+/* Diagonal Hessian estimate (A2): H_k = fp32( S_k / T ) with S_k the fp64 sum of the
+ * squares fp64(x_tk)^2 (exact: x is bf16) taken by a fixed pairwise tree over t: the T
+ * squares padded with zeros to P = the next power of two, then v[i] += v[i + h] for
+ * h = P/2, P/4, ..., 1. The pages give the mean of squares and no summation order;
+ * the tree is the order the GPU can run in parallel (the same tree as Delta's). */
 void orc_hessian_diag(const uint16_t* Xcal, int T, int K, float* H) {
+    int P = 1;
+    while (P < T) P <<= 1;
+    double* v = (double*)malloc(sizeof(double) * P);
     for (int k = 0; k < K; ++k) {
-        double s = 0.0;
-        for (int t = 0; t < T; ++t) {
-            double x = (double)bf16_to_f32(Xcal[(int64_t)t * K + k]);
-            s += x * x;
+        for (int t = 0; t < P; ++t) {
+            double x = t < T ? (double)bf16_to_f32(Xcal[(int64_t)t * K + k]) : 0.0;
+            v[t] = x * x;
         }
-        H[k] = (float)(s / (double)T);
+        for (int h = P / 2; h >= 1; h >>= 1)
+            for (int i = 0; i < h; ++i) v[i] = v[i] + v[i + h];
+        H[k] = (float)(v[0] / (double)T);
     }
+    free(v);
 }
 
 /* Pairwise tree over 64 values: v[i] += v[i+32] (i<32), then +16, +8, +4, +2, +1. */

@@ -270,6 +270,15 @@ def test_run_layer_whole_path(host, dev):
     torch.cuda.synchronize()
     assert mosaic.mq_get_error() == 0
     assert np.array_equal(layer.sel[:budget].cpu().numpy(), o["sel"])
+    # every intermediate the call leaves behind, bit for bit (the activation quantizer runs
+    # ahead of the selection and quantizes before waiting for the Delta pass)
+    xq_ref = o["xq"]
+    xq = layer.act_buffers(M)[0]
+    assert np.array_equal(xq["codes"].cpu().numpy(), xq_ref["codes"])
+    assert np.array_equal(xq["sf_swz"].cpu().numpy(), oracle.sf_tile(xq_ref["sf"], M, K))
+    assert np.array_equal(xq["gscale"].cpu().numpy().view(np.uint32), xq_ref["g"].view(np.uint32))
+    assert np.array_equal(layer.H.cpu().numpy().view(np.uint32), o["H"].view(np.uint32))
+    assert np.array_equal(layer.rank[:budget].cpu().numpy(), o["rank"])
     check_gemm(Y.float().cpu().numpy().astype(np.float64), o["y"], o["yabs"], f"run_layer host={host}")
 
 
@@ -338,3 +347,21 @@ def test_gemm_act_fused_quantization(N, K, M, dev):
     sel = layer.sel[:budget].cpu().numpy()
     y_ref, yabs = oracle.gemm_rows(xo, wq, sel, M, N, K)
     check_gemm(Y1.float().cpu().numpy().astype(np.float64), y_ref, yabs, f"gemm_act N={N} K={K} M={M}")
+
+
+@pytest.mark.parametrize("T", [1, 7, 16, 33, 128, 500, 512, 513, 1000, 1024])
+def test_hessian_token_counts(T, dev):
+    """A2 alone across calibration token counts (the kernel pads the tree to 512 or 1024
+    leaves, the oracle to the next power of two; rows past T are not read): bit-exact with
+    the oracle; more than 1024 tokens is refused."""
+    from bit_quantized_gemm_zipperengine_b200 import mosaic
+    K = 256
+    Xb = synth.act(T, K, 911, 914, 3, 30.0)
+    H = torch.empty(K, dtype=torch.float32, device=dev)
+    mosaic.mq_hessian_diag(to_dev(Xb, dev), H)
+    torch.cuda.synchronize()
+    assert np.array_equal(H.cpu().numpy().view(np.uint32), oracle.hessian_diag(Xb).view(np.uint32))
+    if T == 1024:
+        big = to_dev(synth.act(1025, K, 915, 914, 3, 30.0), dev)
+        with pytest.raises(mosaic.MosaicError):
+            mosaic.mq_hessian_diag(big, H)

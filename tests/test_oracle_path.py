@@ -69,6 +69,22 @@ def test_hessian_diag_against_numpy(orc):
     assert np.all(orc.hessian_diag(_bf16(c)) == np.float32(2.25))
 
 
+def test_hessian_diag_exact_when_no_rounding(orc):
+    """Values of one binade ([1, 2), bf16): every square has at most 16 significant bits
+    and every partial sum of up to 1024 of them fits in fp64 exactly, so whatever the
+    summation order H_k must equal the exact mean rounded once to fp32 (Fractions)."""
+    from fractions import Fraction
+    rng = np.random.default_rng(7)
+    for T in (1, 3, 100, 513, 1024):
+        x = (1.0 + rng.integers(0, 128, size=(T, 64)) / 128.0).astype(np.float32)  # exact in bf16
+        H = orc.hessian_diag(_bf16(x))
+        for k in range(0, 64, 7):
+            exact = sum(Fraction(float(v)) ** 2 for v in x[:, k]) / T
+            # fp32(fp64(exact)): fp64 rounding of the exact mean, then to fp32 (the oracle's
+            # division is the only rounding step here, in fp64, then the cast)
+            assert H[k] == np.float32(float(exact)), (T, k)
+
+
 def test_residual_is_base_error_and_shares_scale(orc, tiny):
     wq = tiny["wq"]
     w = _f32(tiny["W"])
