@@ -413,13 +413,14 @@ mq_status mq_run_layer(const mq_bf16* W, const mq_bf16* X, const mq_bf16* Xcal, 
         y = buf->Y_dev;
     }
     // The method's order, with the activation quantizer moved ahead of top-K. Every kernel
-    // but that one and the weight maxima pass waits for its predecessor before reading
-    // its outputs and lets its dependent start right after; those two read only inputs of
-    // this call, do their work first and wait at their end. So when the GEMM starts, the
-    // quantize+Delta kernel has long completed, and the GEMM requests W before waiting for
-    // its predecessor (prefetch). The activation quantizer runs as its own kernel: on
-    // B200 at decode sizes that is faster than quantizing inside the GEMM (mq_gemm_act),
-    // whose per-token maxima must first be exchanged between the K splits.
+    // waits for its predecessor before reading its outputs. The weight maxima pass and the
+    // activation quantizer read only inputs of this call: they let their dependent start
+    // at once, do their work and wait at their end (so their completion still implies
+    // their predecessor's). The others let their dependent start right after their wait.
+    // When the GEMM starts, the quantize+Delta kernel has completed, and the GEMM requests
+    // W before waiting for its predecessor (prefetch). The activation quantizer runs as its
+    // own kernel: on B200 at decode sizes that is faster than quantizing inside the GEMM
+    // (mq_gemm_act), whose per-token maxima must first be exchanged between the K splits.
     mq_status st;
     if ((st = mq_hessian_diag(xc, T, K, buf->H, stream)) != MQ_OK) return st;
     if ((st = mq_quantize_weight_delta(w, N, K, buf->H, &buf->base, nullptr, buf->delta, buf->ws_quant,

@@ -483,11 +483,23 @@ __global__ void __launch_bounds__(kSelThreads) k_topk_small(const double* __rest
     auto key_of = [&](int i) -> uint64_t { return kSmemKeys ? keys[i] : order_key(delta[i]); };
 
     uint64_t a = ~0ull, o = 0ull;
-    for (int i = tid; i < B; i += kSelThreads) {
-        const uint64_t k = order_key(delta[i]);
-        if (kSmemKeys) keys[i] = k;
-        a &= k;
-        o |= k;
+    for (int i0 = tid; i0 < B; i0 += 4 * kSelThreads) {
+        double d[4];  // four loads in flight
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int i = i0 + u * kSelThreads;
+            d[u] = i < B ? delta[i] : 0.0;
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int i = i0 + u * kSelThreads;
+            if (i < B) {
+                const uint64_t k = order_key(d[u]);
+                if (kSmemKeys) keys[i] = k;
+                a &= k;
+                o |= k;
+            }
+        }
     }
     for (int w = tid; w < nw; w += kSelThreads) bits[w] = 0u;
     {

@@ -282,6 +282,46 @@ def test_run_layer_whole_path(host, dev):
     check_gemm(Y.float().cpu().numpy().astype(np.float64), o["y"], o["yabs"], f"run_layer host={host}")
 
 
+RUN_LAYER_CASES = [
+    ("qwen3_32b", "q", 1, 0.10),                        # one token
+    ("qwen3_32b", "up", 16, 0.10),                      # wide N
+    ("llama3_70b_mlp", "down", 16, 0.10),               # K = 28672: split-K through the workspace
+    ("llama3_8b_qproj_decode", "q_proj", 128, 0.10),    # 128-token tile
+    ("llama3_8b_qproj_decode", "q_proj", 16, 0.0),      # no budget: no top-K kernel, no residual
+    ("llama3_8b_qproj_decode", "q_proj", 16, 0.50),     # budget past the one-CTA top-K
+    ("llama3_8b_mlp_prefill", "up", 384, 0.10),         # prefill kernel
+]
+
+
+@pytest.mark.parametrize("wl,mat,M,frac", RUN_LAYER_CASES)
+def test_run_layer_shapes(wl, mat, M, frac, dev):
+    """mq_run_layer across the GEMM's kernels and plans, with and without a residual: the
+    whole-path call overlaps the decode GEMM's base pass with top-K and the pack (the
+    residual blocks follow the wait for the pack). Selection and ranking bit for bit, Y on
+    sampled token rows within the GEMM tolerance."""
+    from bit_quantized_gemm_zipperengine_b200 import mosaic
+    L = synth.layer(wl, matrix=mat, M=M)
+    N, K, T = L["N"], L["K"], L["T"]
+    budget = synth.budget_blocks(N, K, frac)
+    rows = np.array(sorted({0, M // 2, M - 1}), dtype=np.int32)
+    o = oracle_ref(L, budget, rows)
+    layer = mosaic.Layer(N, K, budget, dev, with_sf=False)
+    buf = layer.buffers(M, T)
+    W, X, C = to_dev(L["W"], dev), to_dev(L["X"], dev), to_dev(L["Xcal"], dev)
+    Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    for _ in range(2):  # the second call runs behind the first one's kernels
+        mosaic.mq_run_layer(W, X, C, Y, M, N, K, T, budget, 0, False, buf)
+    torch.cuda.synchronize()
+    assert mosaic.mq_get_error() == 0
+    what = f"{wl}/{mat} M={M} budget={budget}"
+    if budget:
+        assert np.array_equal(layer.rank[:budget].cpu().numpy(), o["rank"]), what
+        assert np.array_equal(layer.sel[:budget].cpu().numpy(), o["sel"]), what
+    assert torch.isfinite(Y.float()).all(), what
+    y = Y[torch.from_numpy(rows).long().to(dev)].float().cpu().numpy().astype(np.float64)
+    check_gemm(y, o["y"], o["yabs"], what)
+
+
 @pytest.mark.parametrize("fused", PATHS)
 def test_odd_block_rows_bit_exact(fused, dev):
     """N / 64 odd (5 block rows): the quantize+Delta pass works on strips of two block rows,
