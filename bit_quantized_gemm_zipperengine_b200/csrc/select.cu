@@ -238,129 +238,8 @@ __device__ __forceinline__ int block_exclusive_sum(int v, int* scratch, int& tot
     return before;
 }
 
-// Single-CTA radix select of the budget-th largest key (8 digits of 8 bits, most
-// significant first; keys held in shared memory when they fit), then a stable
-// compaction in block order: every key above the threshold plus the lowest-index keys
-// equal to it, which writes sel ascending. With kRank the same CTA also writes rank by
-// counting: position of selected i = #{j : key_j > key_i} + #{j < i : key_j == key_i}.
 constexpr int kSelThreads = 1024;
-constexpr int kRankInCtaMax = 1024;        // budgets up to this are ranked in the CTA
 constexpr size_t kSelSmemKeysMax = 160 * 1024;
-
-template <bool kSmemKeys, bool kRank>
-__global__ void __launch_bounds__(kSelThreads) k_topk(const double* __restrict__ delta, int B, int budget,
-                                                      int32_t* __restrict__ sel, int32_t* __restrict__ rank) {
-    griddep_wait();
-    griddep_launch();
-    extern __shared__ __align__(16) uint64_t dyn[];
-    uint64_t* keys = dyn;                                   // [B] when kSmemKeys
-    uint64_t* selkey = dyn + (kSmemKeys ? B : 0);           // [budget] when kRank
-    int32_t* selidx = reinterpret_cast<int32_t*>(selkey + (kRank ? budget : 0));
-    __shared__ unsigned hist[256];
-    __shared__ uint64_t s_prefix, s_mask;
-    __shared__ int s_need;
-    __shared__ int scratch[32];
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    if (kSmemKeys)
-        for (int i = tid; i < B; i += kSelThreads) keys[i] = order_key(delta[i]);
-    if (tid == 0) { s_prefix = 0; s_mask = 0; s_need = budget; }
-    __syncthreads();
-    auto key_of = [&](int i) -> uint64_t { return kSmemKeys ? keys[i] : order_key(delta[i]); };
-#pragma unroll 1
-    for (int shift = 56; shift >= 0; shift -= 8) {
-        if (tid < 256) hist[tid] = 0;
-        __syncthreads();
-        const uint64_t prefix = s_prefix, mask = s_mask;
-        // warp-aggregated histogram: lanes with the same digit add once (the keys share
-        // their leading digits, so per-lane atomics would all hit one bin)
-        for (int i0 = tid - lane; i0 < B; i0 += kSelThreads) {
-            const int i = i0 + lane;
-            unsigned digit = 256u;  // not counted
-            if (i < B) {
-                const uint64_t key = key_of(i);
-                if ((key & mask) == prefix) digit = (unsigned)(key >> shift) & 255u;
-            }
-            const unsigned peers = __match_any_sync(0xffffffffu, digit);
-            if (digit < 256u && lane == __ffs(peers) - 1) atomicAdd(&hist[digit], (unsigned)__popc(peers));
-        }
-        __syncthreads();
-        if (warp == 0) {
-            // lane l scans bins 255-8l down to 248-8l; find the bin where the count of
-            // keys from the top reaches `need`
-            unsigned cnt[8], tot = 0;
-#pragma unroll
-            for (int j = 0; j < 8; ++j) { cnt[j] = hist[255 - 8 * lane - j]; tot += cnt[j]; }
-            unsigned incl = tot;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const unsigned y = __shfl_up_sync(0xffffffffu, incl, o);
-                if (lane >= o) incl += y;
-            }
-            const int need = s_need;
-            const unsigned hit = __ballot_sync(0xffffffffu, incl >= (unsigned)need);
-            const int first = __ffs(hit) - 1;
-            if (lane == first) {
-                unsigned cum = incl - tot;
-                int digit = 0;
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    if (cum + cnt[j] >= (unsigned)need) { digit = 255 - 8 * lane - j; break; }
-                    cum += cnt[j];
-                }
-                s_need = need - (int)cum;
-                s_prefix = prefix | ((uint64_t)digit << shift);
-                s_mask = mask | ((uint64_t)255 << shift);
-            }
-        }
-        __syncthreads();
-    }
-    const uint64_t T = s_prefix;
-    const int need_eq = s_need;  // how many keys equal to T are taken (lowest b first)
-    const int chunk = (B + kSelThreads - 1) / kSelThreads;
-    const int lo = min(B, tid * chunk), hi = min(B, lo + chunk);
-    int gt = 0, eq = 0;
-    for (int i = lo; i < hi; ++i) {
-        const uint64_t key = key_of(i);
-        gt += key > T;
-        eq += key == T;
-    }
-    int total;
-    const int eq_before = block_exclusive_sum<kSelThreads>(eq, scratch, total);
-    const int eq_take = max(0, min(eq, need_eq - eq_before));
-    int out = block_exclusive_sum<kSelThreads>(gt + eq_take, scratch, total);
-    int eq_seen = eq_before;
-    for (int i = lo; i < hi; ++i) {
-        const uint64_t key = key_of(i);
-        bool take = key > T;
-        if (key == T) take = eq_seen++ < need_eq;
-        if (take) {
-            sel[out] = i;
-            if (kRank) { selkey[out] = key; selidx[out] = i; }
-            ++out;
-        }
-    }
-    if (kRank) {
-        // position of selected i, counted in `parts` slices of j by different threads
-        __shared__ int pos_s[kRankInCtaMax];
-        for (int i = tid; i < budget; i += kSelThreads) pos_s[i] = 0;
-        __syncthreads();
-        const int parts = max(1, kSelThreads / budget);
-        const int span = (budget + parts - 1) / parts;
-        for (int w = tid; w < budget * parts; w += kSelThreads) {
-            const int i = w / parts, part = w % parts;
-            const uint64_t mine = selkey[i];
-            const int j0 = part * span, j1 = min(budget, j0 + span);
-            int pos = 0;
-            for (int j = j0; j < j1; ++j) {
-                const uint64_t kj = selkey[j];
-                pos += (kj > mine) | ((kj == mine) & (j < i));
-            }
-            atomicAdd(&pos_s[i], pos);
-        }
-        __syncthreads();
-        for (int i = tid; i < budget; i += kSelThreads) rank[pos_s[i]] = selidx[i];
-    }
-}
 
 // Top-K for budgets up to kSmallBudget, one CTA of 1024 threads:
 //  1. keys (order-preserving 64-bit images of Delta) and their common leading bits;
@@ -637,29 +516,242 @@ __global__ void __launch_bounds__(kSelThreads) k_topk_small(const double* __rest
     }
 }
 
-// rank: position of selected block i = #{j : key_j > key_i} + #{j < i : key_j == key_i}
-// (sel is ascending, so a lower list index is a lower block index).
-__global__ void __launch_bounds__(256) k_topk_rank(const double* __restrict__ delta, const int32_t* __restrict__ sel,
-                                                   int budget, int32_t* __restrict__ rank) {
-    griddep_wait();
+// Top-K for larger budgets, one CTA of 1024 threads for the selection:
+//  1. keys and their common leading bits (eight loads in flight per thread when the keys
+//     do not fit in shared memory and are read again from global memory in every pass);
+//  2. radix passes of up to 11 bits below the common prefix narrow the bucket that holds
+//     the budget-th largest key until the bucket is taken whole (its count equals the
+//     keys still needed) or is a single key value;
+//  3. compaction in block order, warp w over the contiguous index range w: every key above
+//     the bucket, and the bucket's keys (all of them, or the lowest-index `need` ones of a
+//     single key value), which writes sel ascending.
+// rank then comes from k_topk_rank_split.
+template <bool kSmemKeys>
+__global__ void __launch_bounds__(kSelThreads) k_topk_large(const double* __restrict__ delta, int B, int budget,
+                                                            int32_t* __restrict__ sel) {
+    extern __shared__ __align__(16) uint64_t dyn[];
+    uint64_t* keys = dyn;  // [B] when kSmemKeys
+    __shared__ unsigned hist[1 << kDigitBits];
+    __shared__ uint32_t s_and[64], s_or[64];
+    __shared__ uint64_t s_prefix;
+    __shared__ int s_pos, s_need, s_cand;
+    __shared__ int s_gt[32], s_eq[32], s_base[32], s_eqb[32];
+    __shared__ int scratch[32];
+    griddep_wait();  // Delta comes from the previous kernel
     griddep_launch();
-    __shared__ uint64_t keys[2048];
-    const int i = blockIdx.x * blockDim.x + threadIdx.x;
-    const uint64_t mine = i < budget ? order_key(delta[sel[i]]) : 0;
-    int pos = 0;
-    for (int base = 0; base < budget; base += 2048) {
-        const int n = min(2048, budget - base);
-        __syncthreads();
-        for (int j = threadIdx.x; j < n; j += blockDim.x) keys[j] = order_key(delta[sel[base + j]]);
-        __syncthreads();
-        if (i < budget) {
-            for (int j = 0; j < n; ++j) {
-                const uint64_t kj = keys[j];
-                pos += (kj > mine) | ((kj == mine) & (base + j < i));
+    constexpr int U = 8;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    auto key_of = [&](int i) -> uint64_t { return kSmemKeys ? keys[i] : order_key(delta[i]); };
+
+    uint64_t a = ~0ull, o = 0ull;
+    for (int i0 = tid; i0 < B; i0 += U * kSelThreads) {
+        double d[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int i = i0 + u * kSelThreads;
+            d[u] = i < B ? delta[i] : 0.0;
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int i = i0 + u * kSelThreads;
+            if (i < B) {
+                const uint64_t k = order_key(d[u]);
+                if (kSmemKeys) keys[i] = k;
+                a &= k;
+                o |= k;
             }
         }
     }
-    if (i < budget) rank[pos] = sel[i];
+    {
+        const uint32_t ah = __reduce_and_sync(0xffffffffu, (uint32_t)(a >> 32));
+        const uint32_t al = __reduce_and_sync(0xffffffffu, (uint32_t)a);
+        const uint32_t oh = __reduce_or_sync(0xffffffffu, (uint32_t)(o >> 32));
+        const uint32_t ol = __reduce_or_sync(0xffffffffu, (uint32_t)o);
+        if (lane == 0) {
+            s_and[2 * warp] = ah;
+            s_and[2 * warp + 1] = al;
+            s_or[2 * warp] = oh;
+            s_or[2 * warp + 1] = ol;
+        }
+    }
+    __syncthreads();
+    if (warp == 0) {
+        const uint32_t ah = __reduce_and_sync(0xffffffffu, s_and[2 * lane]);
+        const uint32_t al = __reduce_and_sync(0xffffffffu, s_and[2 * lane + 1]);
+        const uint32_t oh = __reduce_or_sync(0xffffffffu, s_or[2 * lane]);
+        const uint32_t ol = __reduce_or_sync(0xffffffffu, s_or[2 * lane + 1]);
+        a = ((uint64_t)ah << 32) | al;
+        o = ((uint64_t)oh << 32) | ol;
+        if (lane == 0) {
+            const int cp = (a ^ o) ? __clzll((long long)(a ^ o)) : 64;
+            s_pos = 64 - cp;
+            s_prefix = cp ? (a & (~0ull << (64 - cp))) : 0ull;
+            s_need = budget;
+            s_cand = B;
+        }
+    }
+    __syncthreads();
+    while (s_pos > 0 && s_cand > s_need) {
+        const int pos = s_pos, w = pos < kDigitBits ? pos : kDigitBits, shift = pos - w;
+        const uint64_t prefix = s_prefix, hi = pos >= 64 ? 0ull : (~0ull << pos);
+        const int need = s_need;
+        const int nb = 1 << w;
+        for (int b = tid; b < nb; b += kSelThreads) hist[b] = 0;
+        __syncthreads();
+        for (int i0 = tid - lane; i0 < B; i0 += U * kSelThreads) {  // warp-uniform
+            uint64_t k[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int i = i0 + lane + u * kSelThreads;
+                k[u] = i < B ? key_of(i) : 0ull;
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int i = i0 + lane + u * kSelThreads;
+                unsigned digit = 1u << kDigitBits;  // not counted
+                if (i < B && (k[u] & hi) == prefix) digit = (unsigned)(k[u] >> shift) & (nb - 1);
+                const unsigned peers = __match_any_sync(0xffffffffu, digit);
+                if (digit < (1u << kDigitBits) && lane == __ffs(peers) - 1)
+                    atomicAdd(&hist[digit], (unsigned)__popc(peers));
+            }
+        }
+        __syncthreads();
+        const int b0 = nb - 1 - 2 * tid;
+        const unsigned c0 = b0 >= 0 ? hist[b0] : 0u, c1 = b0 - 1 >= 0 ? hist[b0 - 1] : 0u;
+        const int above = block_excl_sum_1bar<kSelThreads>((int)(c0 + c1), scratch);
+        if (b0 >= 0 && above < need && above + (int)(c0 + c1) >= need) {
+            const bool first = above + (int)c0 >= need;
+            const int digit = first ? b0 : b0 - 1;
+            s_need = need - (first ? above : above + (int)c0);
+            s_cand = (int)(first ? c0 : c1);
+            s_prefix = prefix | ((uint64_t)digit << shift);
+            s_pos = shift;
+        }
+        __syncthreads();
+    }
+    const int pos = s_pos, need = s_need;
+    const bool whole = s_cand == s_need;
+    const uint64_t prefix = s_prefix, hi = pos >= 64 ? 0ull : (~0ull << pos);
+    const int CW = (B + 32 * 32 - 1) / (32 * 32) * 32;  // indices per warp, a multiple of 32
+    const int w0 = min(B, warp * CW), w1 = min(B, w0 + CW);
+    int gt = 0, eq = 0;
+    for (int i0 = w0; i0 < w1; i0 += 32 * U) {
+        uint64_t k[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int i = i0 + lane + 32 * u;
+            k[u] = i < w1 ? key_of(i) : 0ull;
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int i = i0 + lane + 32 * u;
+            if (i < w1) {
+                const uint64_t t = k[u] & hi;
+                gt += t > prefix;
+                eq += t == prefix;
+            }
+        }
+    }
+    gt = (int)__reduce_add_sync(0xffffffffu, (unsigned)gt);
+    eq = (int)__reduce_add_sync(0xffffffffu, (unsigned)eq);
+    if (lane == 0) {
+        s_gt[warp] = gt;
+        s_eq[warp] = eq;
+    }
+    __syncthreads();
+    if (warp == 0) {
+        const int g = s_gt[lane], e = s_eq[lane];
+        int ie = e;
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, ie, d);
+            if (lane >= d) ie += y;
+        }
+        const int eqb = ie - e;
+        const int take = whole ? e : max(0, min(e, need - eqb));
+        int it = g + take;
+        const int t0 = it;
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, it, d);
+            if (lane >= d) it += y;
+        }
+        s_eqb[lane] = eqb;
+        s_base[lane] = it - t0;
+    }
+    __syncthreads();
+    int out = s_base[warp], eq_seen = s_eqb[warp];
+    const unsigned lt = (1u << lane) - 1u;
+    for (int i0 = w0; i0 < w1; i0 += 32 * U) {
+        uint64_t k[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int i = i0 + lane + 32 * u;
+            k[u] = i < w1 ? key_of(i) : 0ull;
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int i = i0 + lane + 32 * u;
+            const bool valid = i < w1;
+            const uint64_t t = k[u] & hi;
+            const bool is_gt = valid && t > prefix, is_eq = valid && t == prefix;
+            const unsigned meq = __ballot_sync(0xffffffffu, is_eq);
+            bool take = is_gt;
+            if (is_eq) take = whole || eq_seen + __popc(meq & lt) < need;
+            eq_seen += __popc(meq);
+            const unsigned mt = __ballot_sync(0xffffffffu, take);
+            if (take) sel[out + __popc(mt & lt)] = i;
+            out += __popc(mt);
+        }
+    }
+}
+
+// rank for the larger budgets: position of selected block i =
+// #{j : key_j > key_i} + #{j < i : key_j == key_i} over the selected set (sel ascending, so a
+// lower list index is a lower block index). A CTA of 128 threads owns 16 selected blocks,
+// eight threads each; it stages the selected keys in tiles of 2048 and each of the eight
+// threads counts every eighth key of a tile.
+constexpr int kRankTile = 2048;
+__global__ void __launch_bounds__(128) k_topk_rank_split(const double* __restrict__ delta,
+                                                         const int32_t* __restrict__ sel, int budget,
+                                                         int32_t* __restrict__ rank) {
+    griddep_wait();
+    griddep_launch();
+    __shared__ uint64_t tk[kRankTile];
+    const int t = threadIdx.x, part = t & 7;
+    const int i = blockIdx.x * 16 + (t >> 3);
+    const uint64_t mine = i < budget ? order_key(delta[__ldg(sel + i)]) : 0ull;
+    int pos = 0;
+    for (int base = 0; base < budget; base += kRankTile) {
+        const int n = min(kRankTile, budget - base);
+        __syncthreads();  // the previous tile is no longer read
+        for (int j0 = t; j0 < n; j0 += 128 * 8) {
+            int sj[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int j = j0 + 128 * u;
+                sj[u] = j < n ? __ldg(sel + base + j) : 0;
+            }
+            double d[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) d[u] = j0 + 128 * u < n ? delta[sj[u]] : 0.0;
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                if (j0 + 128 * u < n) tk[j0 + 128 * u] = order_key(d[u]);
+        }
+        __syncthreads();
+        if (i < budget) {
+            const int lim = i - base;  // tile entries below lim precede i among equal keys
+            for (int j = part; j < n; j += 8) {
+                const uint64_t kj = tk[j];
+                pos += (kj > mine) | ((kj == mine) & (j < lim));
+            }
+        }
+    }
+    pos += __shfl_xor_sync(0xffffffffu, pos, 1);
+    pos += __shfl_xor_sync(0xffffffffu, pos, 2);
+    pos += __shfl_xor_sync(0xffffffffu, pos, 4);
+    if (i < budget && part == 0) rank[pos] = sel[i];
 }
 
 // ------------------------------------------------------------------ pack
@@ -843,7 +935,7 @@ cudaError_t launch_topk(const double* delta, int B, int budget, int32_t* rank, i
         };
         return smem_keys ? go(k_topk_small<true>, 0) : go(k_topk_small<false>, 1);
     }
-    // larger budgets: radix select and compaction, then a separate counting rank kernel
+    // larger budgets: radix select and compaction, then the split counting rank kernel
     const bool smem_keys = (size_t)B * 8 <= kSelSmemKeysMax;
     const size_t smem = smem_keys ? (size_t)B * 8 : 0;
     static bool attr2[2] = {false, false};
@@ -854,12 +946,12 @@ cudaError_t launch_topk(const double* delta, int B, int budget, int32_t* rank, i
             if (e != cudaSuccess) return e;
             attr2[which] = true;
         }
-        return launch_pdl(kern, dim3(1), dim3(kSelThreads), smem, s, 1, delta, B, budget, sel, rank);
+        return launch_pdl(kern, dim3(1), dim3(kSelThreads), smem, s, 1, delta, B, budget, sel);
     };
-    cudaError_t e = smem_keys ? go2(k_topk<true, false>, 0) : go2(k_topk<false, false>, 1);
+    cudaError_t e = smem_keys ? go2(k_topk_large<true>, 0) : go2(k_topk_large<false>, 1);
     if (e != cudaSuccess) return e;
-    return launch_pdl(k_topk_rank, dim3((budget + 255) / 256), dim3(256), 0, s, 1, delta, (const int32_t*)sel, budget,
-                      rank);
+    return launch_pdl(k_topk_rank_split, dim3((budget + 15) / 16), dim3(128), 0, s, 1, delta, (const int32_t*)sel,
+                      budget, rank);
 }
 
 cudaError_t launch_pack(const uint8_t* rcodes, const uint8_t* rsf, int N, int K, const int32_t* sel, int budget,

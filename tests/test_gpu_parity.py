@@ -218,12 +218,14 @@ def test_repeat_calls_deterministic(dev):
 
 def test_topk_blocks_alone_and_large_budgets(dev):
     """A4 alone on many blocks and budgets (the one-CTA select-and-sort path up to its
-    budget limit, the radix select with the separate rank kernel above it, keys in shared
-    or global memory), with ties, against the oracle's sort."""
+    budget limit, the radix select with the split rank kernel above it, keys in shared or
+    global memory, a threshold inside a bucket of one tied value, every block selected),
+    with ties, against the oracle's sort."""
     from bit_quantized_gemm_zipperengine_b200 import mosaic
     rng = np.random.default_rng(12)
     cases = [(32, (0, 1, 3, 32), False), (4096, (409, 767, 768, 769, 1024, 1025), False),
-             (57344, (500, 2867, 11468), False), (4096, (300, 500, 700), True)]
+             (57344, (500, 2867, 11468, 57344), False), (4096, (300, 500, 700), True),
+             (4096, (1000, 2000, 4096), True), (40000, (1300, 6000), True)]
     for B, budgets, many_ties in cases:
         d = rng.standard_normal(B) * np.exp2(rng.integers(-20, 5, B))
         d[rng.choice(B, B // 10, replace=False)] = 0.0      # ties at zero
