@@ -29,7 +29,8 @@ cudaError_t launch_pack(const uint8_t* rcodes, const uint8_t* rsf, int N, int K,
                         cudaStream_t s);
 cudaError_t launch_pack_w(const uint16_t* W, int N, int K, const float* g_w, const int32_t* sel, int budget,
                           uint8_t* blk_codes, uint8_t* blk_sf, int32_t* blk_kt, int32_t* tile_ptr, uint32_t* bitmap,
-                          cudaStream_t s);
+                          const double* delta, int32_t* rank, cudaStream_t s);
+cudaError_t launch_topk_select(const double* delta, int B, int budget, int32_t* sel, cudaStream_t s);
 
 }  // namespace mq
 
@@ -239,16 +240,23 @@ static mq_status check_packed(const mq_residual_packed* out, int N, int K, const
     return MQ_OK;
 }
 
-mq_status mq_pack_residual_weight(const mq_bf16* W, const mq_nvfp4_mat* base, const int32_t* sel, int budget,
-                                  mq_residual_packed* out, mq_stream stream) {
+// delta and rank: with rank != NULL the pack kernel also writes rank from sel and delta.
+static mq_status pack_residual_weight_impl(const mq_bf16* W, const mq_nvfp4_mat* base, const int32_t* sel,
+                                           int budget, mq_residual_packed* out, const double* delta,
+                                           int32_t* rank, mq_stream stream) {
     if (!W || !base || !base->gscale) return MQ_ERR_INVALID_ARG;
     const int N = base->rows, K = base->cols;
     if (!nvfp4_shape_ok(N, K) || N % 64 || !aligned(W, 16)) return MQ_ERR_INVALID_ARG;
     const mq_status st = check_packed(out, N, K, sel, budget);
     if (st != MQ_OK) return st;
     return launched(launch_pack_w(W, N, K, base->gscale, sel, budget, out->blk_codes, out->blk_sf, out->blk_kt,
-                                  out->tile_ptr, out->bitmap, as_stream(stream)),
+                                  out->tile_ptr, out->bitmap, delta, rank, as_stream(stream)),
                     1);
+}
+
+mq_status mq_pack_residual_weight(const mq_bf16* W, const mq_nvfp4_mat* base, const int32_t* sel, int budget,
+                                  mq_residual_packed* out, mq_stream stream) {
+    return pack_residual_weight_impl(W, base, sel, budget, out, nullptr, nullptr, stream);
 }
 
 mq_status mq_quantize_act(const mq_bf16* X, int M, int K, mq_nvfp4_mat* xq, mq_stream stream) {
@@ -427,9 +435,18 @@ mq_status mq_run_layer(const mq_bf16* W, const mq_bf16* X, const mq_bf16* Xcal, 
                                        buf->ws_quant_bytes, stream)) != MQ_OK)
         return st;
     if ((st = quantize_act_early(x, M, K, &buf->xq, stream)) != MQ_OK) return st;
-    if ((st = mq_topk_blocks(buf->delta, (N / 64) * (K / 64), budget, buf->rank, buf->sel, stream)) != MQ_OK)
+    // A4 as two parts: the selection kernel writes sel, and rank (which the GEMM does not
+    // read) is written by extra CTAs of the pack kernel, beside the packing
+    {
+        const int nblk = (N / 64) * (K / 64);
+        if (!buf->delta || budget < 0 || budget > nblk || (budget > 0 && (!buf->rank || !buf->sel)))
+            return MQ_ERR_INVALID_ARG;
+        if ((st = launched(launch_topk_select(buf->delta, nblk, budget, buf->sel, s), budget > 0 ? 1 : 0)) != MQ_OK)
+            return st;
+    }
+    if ((st = pack_residual_weight_impl(w, &buf->base, buf->sel, budget, &buf->packed, buf->delta, buf->rank,
+                                        stream)) != MQ_OK)
         return st;
-    if ((st = mq_pack_residual_weight(w, &buf->base, buf->sel, budget, &buf->packed, stream)) != MQ_OK) return st;
     if ((st = gemm_impl(&buf->xq, &buf->base, &buf->packed, y, M, N, K, flags, buf->ws_gemm, buf->ws_gemm_bytes, true,
                         stream)) != MQ_OK)
         return st;

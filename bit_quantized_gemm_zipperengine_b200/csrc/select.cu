@@ -241,87 +241,7 @@ __device__ __forceinline__ int block_exclusive_sum(int v, int* scratch, int& tot
 constexpr int kSelThreads = 1024;
 constexpr size_t kSelSmemKeysMax = 160 * 1024;
 
-// Top-K for budgets up to kSmallBudget, one CTA of 1024 threads:
-//  1. keys (order-preserving 64-bit images of Delta) and their common leading bits;
-//  2. radix passes of up to 11 bits below the common prefix narrow the bucket that holds
-//     the budget-th largest key until it has at most kCandMax keys (or is one key value);
-//  3. every key above the bucket and every key in it (at most budget + kCandMax <= 1024)
-//     are sorted by (key descending, block index ascending), a strict total order: the
-//     first `budget` are rank. (A bucket of one key value shared by more than kCandMax
-//     keys takes its lowest block indices instead, and only the `budget` selected keys
-//     are sorted.) sel is the same set in ascending block index (bitmap scan).
-// The sort: each warp sorts 32 pairs in registers (bitonic network over lane shuffles),
-// then sorted runs are merged pairwise: a pair's place in the merged run is its place in
-// its own run plus the number of pairs of the partner run that come before it (binary
-// search), so every pair moves once per merge level.
-constexpr int kSmallBudget = 768;
-constexpr int kCandMax = 256;
 constexpr int kDigitBits = 11;
-static_assert(kSmallBudget + kCandMax <= 1024, "one pair per thread");
-
-__device__ __forceinline__ bool before(uint64_t ka, int ia, uint64_t kb, int ib) {
-    return ka > kb || (ka == kb && ia < ib);
-}
-
-// A (key, block index) pair in one 16-byte shared-memory word.
-__device__ __forceinline__ ulonglong2 kpair(uint64_t key, int idx) {
-    return make_ulonglong2(key, (unsigned long long)(unsigned)idx);
-}
-
-// Sorts the n (<= blockDim.x) pairs s[0, n) of the CTA by (key descending, idx
-// ascending). Thread p starts with pair p (padding past n sorts last) and ends holding
-// the pair at position `pos` of the sorted order, in registers; t is scratch of the same
-// size. Every thread of the CTA calls it.
-__device__ __forceinline__ void block_merge_sort(ulonglong2* s, ulonglong2* t, int n, uint64_t& key, int& idx,
-                                                 int& pos) {
-    const int p = threadIdx.x, lane = p & 31;
-    const int total = (n + 31) & ~31;  // whole warps
-    const bool act = p < total;
-    if (p < n) {
-        const ulonglong2 v = s[p];
-        key = v.x;
-        idx = (int)v.y;
-    } else {
-        key = 0ull;
-        idx = 0x7FFFFFFF - p;
-    }
-    if (act) {
-        for (int k = 2; k <= 32; k <<= 1)
-            for (int j = k >> 1; j > 0; j >>= 1) {
-                const uint64_t pk = __shfl_xor_sync(0xffffffffu, key, j);
-                const int pi = __shfl_xor_sync(0xffffffffu, idx, j);
-                const bool want_first = ((lane & j) == 0) == ((lane & k) == 0);
-                if (before(pk, pi, key, idx) == want_first) {
-                    key = pk;
-                    idx = pi;
-                }
-            }
-    }
-    pos = p;
-    __syncthreads();  // every thread has read its input pair
-    if (act) s[p] = kpair(key, idx);
-    __syncthreads();
-    ulonglong2* cur = s;
-    ulonglong2* out = t;
-    for (int len = 32; len < total; len <<= 1) {
-        if (act) {
-            const int run = pos / len, start = run * len;
-            const int pstart = (run ^ 1) * len;
-            const int plen = max(0, min(len, total - pstart));
-            int lo = 0, hi = plen;
-            while (lo < hi) {
-                const int mid = (lo + hi) >> 1;
-                const ulonglong2 v = cur[pstart + mid];
-                if (before(v.x, (int)v.y, key, idx)) lo = mid + 1;
-                else hi = mid;
-            }
-            pos = (run & ~1) * len + (pos - start) + lo;
-            out[pos] = kpair(key, idx);
-        }
-        __syncthreads();
-        ulonglong2* tmp = cur; cur = out; out = tmp;
-    }
-}
 
 // Exclusive prefix sum over the CTA's threads in thread order (kThreads <= 1024), with
 // one barrier: a shuffle scan inside each warp, the warp totals through `wsum`, and the
@@ -342,181 +262,7 @@ __device__ __forceinline__ int block_excl_sum_1bar(int v, int* wsum) {
     return (int)__reduce_add_sync(0xffffffffu, (unsigned)ws) + x - v;
 }
 
-template <bool kSmemKeys>
-__global__ void __launch_bounds__(kSelThreads) k_topk_small(const double* __restrict__ delta, int B, int budget,
-                                                            int32_t* __restrict__ rank, int32_t* __restrict__ sel) {
-    extern __shared__ __align__(16) uint64_t dyn[];
-    uint64_t* keys = dyn;                                                        // [B] when kSmemKeys
-    ulonglong2* spair = reinterpret_cast<ulonglong2*>(dyn + (kSmemKeys ? (B + 1) & ~1 : 0));  // [kSelThreads]
-    ulonglong2* tpair = spair + kSelThreads;                                     // [kSelThreads]
-    uint32_t* bits = reinterpret_cast<uint32_t*>(tpair + kSelThreads);           // [ceil(B / 32)]
-    __shared__ unsigned hist[1 << kDigitBits];
-    __shared__ uint32_t s_and[64], s_or[64];
-    __shared__ uint64_t s_prefix;
-    __shared__ int s_pos, s_need, s_cand, s_n;
-    __shared__ int scratch[32];
-    griddep_wait();  // Delta comes from the previous kernel
-    griddep_launch();
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int nw = (B + 31) / 32;
-    auto key_of = [&](int i) -> uint64_t { return kSmemKeys ? keys[i] : order_key(delta[i]); };
-
-    uint64_t a = ~0ull, o = 0ull;
-    for (int i0 = tid; i0 < B; i0 += 4 * kSelThreads) {
-        double d[4];  // four loads in flight
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int i = i0 + u * kSelThreads;
-            d[u] = i < B ? delta[i] : 0.0;
-        }
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int i = i0 + u * kSelThreads;
-            if (i < B) {
-                const uint64_t k = order_key(d[u]);
-                if (kSmemKeys) keys[i] = k;
-                a &= k;
-                o |= k;
-            }
-        }
-    }
-    for (int w = tid; w < nw; w += kSelThreads) bits[w] = 0u;
-    {
-        const uint32_t ah = __reduce_and_sync(0xffffffffu, (uint32_t)(a >> 32));
-        const uint32_t al = __reduce_and_sync(0xffffffffu, (uint32_t)a);
-        const uint32_t oh = __reduce_or_sync(0xffffffffu, (uint32_t)(o >> 32));
-        const uint32_t ol = __reduce_or_sync(0xffffffffu, (uint32_t)o);
-        if (lane == 0) {
-            s_and[2 * warp] = ah;
-            s_and[2 * warp + 1] = al;
-            s_or[2 * warp] = oh;
-            s_or[2 * warp + 1] = ol;
-        }
-    }
-    __syncthreads();
-    if (warp == 0) {
-        const uint32_t ah = __reduce_and_sync(0xffffffffu, s_and[2 * lane]);
-        const uint32_t al = __reduce_and_sync(0xffffffffu, s_and[2 * lane + 1]);
-        const uint32_t oh = __reduce_or_sync(0xffffffffu, s_or[2 * lane]);
-        const uint32_t ol = __reduce_or_sync(0xffffffffu, s_or[2 * lane + 1]);
-        a = ((uint64_t)ah << 32) | al;
-        o = ((uint64_t)oh << 32) | ol;
-        if (lane == 0) {
-            const int cp = (a ^ o) ? __clzll((long long)(a ^ o)) : 64;  // common leading bits
-            s_pos = 64 - cp;
-            s_prefix = cp ? (a & (~0ull << (64 - cp))) : 0ull;
-            s_need = budget;
-            s_cand = B;
-            s_n = 0;
-        }
-    }
-    __syncthreads();
-    // radix passes: the bucket (keys sharing the bits above s_pos with s_prefix) holds
-    // the budget-th largest key; s_need of its keys are still to be taken
-    while (s_pos > 0 && s_cand > kCandMax) {
-        const int pos = s_pos, w = pos < kDigitBits ? pos : kDigitBits, shift = pos - w;
-        const uint64_t prefix = s_prefix, hi = pos >= 64 ? 0ull : (~0ull << pos);
-        const int need = s_need;  // read before the owner of the bucket rewrites it
-        const int nb = 1 << w;
-        for (int b = tid; b < nb; b += kSelThreads) hist[b] = 0;
-        __syncthreads();
-        // warp-aggregated histogram: lanes with the same digit add once (keys of similar
-        // magnitude share their leading digits, so per-lane atomics would pile up on a bin)
-        for (int i0 = tid - lane; i0 < B; i0 += kSelThreads) {
-            const int i = i0 + lane;
-            unsigned digit = 1u << kDigitBits;  // not counted
-            if (i < B) {
-                const uint64_t k = key_of(i);
-                if ((k & hi) == prefix) digit = (unsigned)(k >> shift) & (nb - 1);
-            }
-            const unsigned peers = __match_any_sync(0xffffffffu, digit);
-            if (digit < (1u << kDigitBits) && lane == __ffs(peers) - 1) atomicAdd(&hist[digit], (unsigned)__popc(peers));
-        }
-        __syncthreads();
-        // thread t owns the bins nb-1-2t and nb-2-2t (from the top)
-        const int b0 = nb - 1 - 2 * tid;
-        const unsigned c0 = b0 >= 0 ? hist[b0] : 0u, c1 = b0 - 1 >= 0 ? hist[b0 - 1] : 0u;
-        const int above = block_excl_sum_1bar<kSelThreads>((int)(c0 + c1), scratch);
-        if (b0 >= 0 && above < need && above + (int)(c0 + c1) >= need) {
-            const bool first = above + (int)c0 >= need;
-            const int digit = first ? b0 : b0 - 1;
-            s_need = need - (first ? above : above + (int)c0);
-            s_cand = (int)(first ? c0 : c1);
-            s_prefix = prefix | ((uint64_t)digit << shift);
-            s_pos = shift;
-        }
-        __syncthreads();
-    }
-    const int pos = s_pos, need = s_need;
-    const uint64_t prefix = s_prefix, hi = pos >= 64 ? 0ull : (~0ull << pos);
-    int n;
-    if (s_cand <= kCandMax) {
-        // the keys above the bucket and the bucket's keys (slots reserved once per warp)
-        const unsigned lt = (1u << lane) - 1u;
-        for (int i0 = tid - lane; i0 < B; i0 += kSelThreads) {
-            const int i = i0 + lane;
-            const uint64_t k = i < B ? key_of(i) : 0ull;
-            const bool take = i < B && (k & hi) >= prefix;
-            const unsigned mt = __ballot_sync(0xffffffffu, take);
-            int base = 0;
-            if (lane == 0 && mt) base = atomicAdd(&s_n, __popc(mt));
-            base = __shfl_sync(0xffffffffu, base, 0);
-            if (take) spair[base + __popc(mt & lt)] = kpair(k, i);
-        }
-        __syncthreads();
-        n = s_n;
-    } else {
-        // the bucket is a single key value T shared by more than kCandMax keys: keys above
-        // T and the lowest-index `need` keys equal to T, compacted in block order
-        const uint64_t T = prefix;
-        const int chunk = (B + kSelThreads - 1) / kSelThreads;
-        const int lo = min(B, tid * chunk), hi2 = min(B, lo + chunk);
-        int gt = 0, eq = 0;
-        for (int i = lo; i < hi2; ++i) {
-            const uint64_t k = key_of(i);
-            gt += k > T;
-            eq += k == T;
-        }
-        int total;
-        const int eq_before = block_exclusive_sum<kSelThreads>(eq, scratch, total);
-        const int eq_take = max(0, min(eq, need - eq_before));
-        int out = block_exclusive_sum<kSelThreads>(gt + eq_take, scratch, total);
-        int eq_seen = eq_before;
-        for (int i = lo; i < hi2; ++i) {
-            const uint64_t k = key_of(i);
-            bool take = k > T;
-            if (k == T) take = eq_seen++ < need;
-            if (take) spair[out++] = kpair(k, i);
-        }
-        __syncthreads();
-        n = budget;
-    }
-    uint64_t key;
-    int idx, at;
-    block_merge_sort(spair, tpair, n, key, idx, at);
-    if (at < budget) {
-        rank[at] = idx;
-        atomicOr(&bits[idx >> 5], 1u << (idx & 31));
-    }
-    __syncthreads();
-    // sel: the set bits in index order (each thread scans a run of bitmap words)
-    const int per = (nw + kSelThreads - 1) / kSelThreads;
-    const int w0 = min(nw, tid * per), w1 = min(nw, w0 + per);
-    int cnt = 0;
-    for (int w = w0; w < w1; ++w) cnt += __popc(bits[w]);
-    int total;
-    int out = block_exclusive_sum<kSelThreads>(cnt, scratch, total);
-    for (int w = w0; w < w1; ++w) {
-        uint32_t b = bits[w];
-        while (b) {
-            const int t = __ffs(b) - 1;
-            b &= b - 1;
-            sel[out++] = w * 32 + t;
-        }
-    }
-}
-
-// Top-K for larger budgets, one CTA of 1024 threads for the selection:
+// Top-K selection, one CTA of 1024 threads:
 //  1. keys and their common leading bits (eight loads in flight per thread when the keys
 //     do not fit in shared memory and are read again from global memory in every pass);
 //  2. radix passes of up to 11 bits below the common prefix narrow the bucket that holds
@@ -525,7 +271,7 @@ __global__ void __launch_bounds__(kSelThreads) k_topk_small(const double* __rest
 //  3. compaction in block order, warp w over the contiguous index range w: every key above
 //     the bucket, and the bucket's keys (all of them, or the lowest-index `need` ones of a
 //     single key value), which writes sel ascending.
-// rank then comes from k_topk_rank_split.
+// rank (the selected blocks in Delta order) comes from the split counting rank CTAs.
 template <bool kSmemKeys>
 __global__ void __launch_bounds__(kSelThreads) k_topk_large(const double* __restrict__ delta, int B, int budget,
                                                             int32_t* __restrict__ sel) {
@@ -610,9 +356,7 @@ __global__ void __launch_bounds__(kSelThreads) k_topk_large(const double* __rest
                 const int i = i0 + lane + u * kSelThreads;
                 unsigned digit = 1u << kDigitBits;  // not counted
                 if (i < B && (k[u] & hi) == prefix) digit = (unsigned)(k[u] >> shift) & (nb - 1);
-                const unsigned peers = __match_any_sync(0xffffffffu, digit);
-                if (digit < (1u << kDigitBits) && lane == __ffs(peers) - 1)
-                    atomicAdd(&hist[digit], (unsigned)__popc(peers));
+                if (digit < (1u << kDigitBits)) atomicAdd(&hist[digit], 1u);
             }
         }
         __syncthreads();
@@ -706,20 +450,17 @@ __global__ void __launch_bounds__(kSelThreads) k_topk_large(const double* __rest
     }
 }
 
-// rank for the larger budgets: position of selected block i =
-// #{j : key_j > key_i} + #{j < i : key_j == key_i} over the selected set (sel ascending, so a
-// lower list index is a lower block index). A CTA of 128 threads owns 16 selected blocks,
-// eight threads each; it stages the selected keys in tiles of 2048 and each of the eight
-// threads counts every eighth key of a tile.
+// rank: position of selected block i = #{j : key_j > key_i} + #{j < i : key_j == key_i}
+// over the selected set (sel ascending, so a lower list index is a lower block index). A
+// CTA of 128 threads owns the 16 selected blocks 16 c .. 16 c + 15, eight threads each; it
+// stages the selected keys in tiles of 2048 and each of the eight threads counts every
+// eighth key of a tile.
 constexpr int kRankTile = 2048;
-__global__ void __launch_bounds__(128) k_topk_rank_split(const double* __restrict__ delta,
-                                                         const int32_t* __restrict__ sel, int budget,
-                                                         int32_t* __restrict__ rank) {
-    griddep_wait();
-    griddep_launch();
+__device__ __forceinline__ void rank_split_cta(const double* __restrict__ delta, const int32_t* __restrict__ sel,
+                                               int budget, int32_t* __restrict__ rank, int c) {
     __shared__ uint64_t tk[kRankTile];
     const int t = threadIdx.x, part = t & 7;
-    const int i = blockIdx.x * 16 + (t >> 3);
+    const int i = c * 16 + (t >> 3);
     const uint64_t mine = i < budget ? order_key(delta[__ldg(sel + i)]) : 0ull;
     int pos = 0;
     for (int base = 0; base < budget; base += kRankTile) {
@@ -752,6 +493,14 @@ __global__ void __launch_bounds__(128) k_topk_rank_split(const double* __restric
     pos += __shfl_xor_sync(0xffffffffu, pos, 2);
     pos += __shfl_xor_sync(0xffffffffu, pos, 4);
     if (i < budget && part == 0) rank[pos] = sel[i];
+}
+
+__global__ void __launch_bounds__(128) k_topk_rank_split(const double* __restrict__ delta,
+                                                         const int32_t* __restrict__ sel, int budget,
+                                                         int32_t* __restrict__ rank) {
+    griddep_wait();
+    griddep_launch();
+    rank_split_cta(delta, sel, budget, rank, blockIdx.x);
 }
 
 // ------------------------------------------------------------------ pack
@@ -827,16 +576,23 @@ __global__ void __launch_bounds__(256) k_pack(const uint8_t* __restrict__ rcodes
 // Pack straight from W: CTAs [0, budget) recompute the residual of selected block i with
 // the weight quantizer's arithmetic (base group, R = W - deq, NVFP4(R) with the same
 // tensor scale), bit-identical to packing the full residual; the full residual is never
-// stored. Warp q handles group column q, lane r the block rows r and r+32. The remaining
-// CTAs build the CSR and bitmap.
+// stored. Warp q handles group column q, lane r the block rows r and r+32. The next `ncsr`
+// CTAs build the CSR and bitmap; with rank != null the CTAs after them write rank (the
+// selection in Delta order, which nothing downstream of the pack reads) alongside.
 __global__ void __launch_bounds__(128) k_pack_w(const uint16_t* __restrict__ W, int N, int K,
                                                 const float* __restrict__ g_w, const int32_t* __restrict__ sel,
                                                 int budget, uint8_t* __restrict__ blk_codes,
                                                 uint8_t* __restrict__ blk_sf, int32_t* __restrict__ blk_kt,
-                                                int32_t* __restrict__ tile_ptr, uint32_t* __restrict__ bitmap) {
+                                                int32_t* __restrict__ tile_ptr, uint32_t* __restrict__ bitmap,
+                                                int ncsr, const double* __restrict__ delta,
+                                                int32_t* __restrict__ rank) {
     griddep_wait();
     griddep_launch();
     const int KB = K / 64;
+    if ((int)blockIdx.x >= budget + ncsr) {
+        rank_split_cta(delta, sel, budget, rank, (int)blockIdx.x - budget - ncsr);
+        return;
+    }
     if ((int)blockIdx.x >= budget) {
         pack_rows((blockIdx.x - budget) * blockDim.x + threadIdx.x, N / 64, KB, sel, budget, tile_ptr, bitmap);
         return;
@@ -914,41 +670,28 @@ cudaError_t launch_quant_delta(const uint16_t* W, const CUtensorMap& tw, int N, 
                       (const float*)partial, codes, sf, sf_swz, g, (uint8_t*)nullptr, (uint8_t*)nullptr, delta, err);
 }
 
-int topk_launches(int budget) { return budget <= 0 ? 0 : budget <= kSmallBudget ? 1 : 2; }
+int topk_launches(int budget) { return budget <= 0 ? 0 : 2; }
 
-cudaError_t launch_topk(const double* delta, int B, int budget, int32_t* rank, int32_t* sel, cudaStream_t s) {
+cudaError_t launch_topk_select(const double* delta, int B, int budget, int32_t* sel, cudaStream_t s) {
     if (budget <= 0) return cudaSuccess;
-    if (budget <= kSmallBudget) {
-        const size_t tail = (size_t)kSelThreads * 32 + (size_t)((B + 31) / 32) * 4;
-        const size_t keys_bytes = (size_t)((B + 1) & ~1) * 8;  // keeps the pairs 16-byte aligned
-        const bool smem_keys = keys_bytes + tail <= kSelSmemKeysMax;
-        const size_t smem = (smem_keys ? keys_bytes : 0) + tail;
-        static bool attr[2] = {false, false};
-        auto go = [&](auto kern, int which) -> cudaError_t {
-            if (!attr[which]) {
-                cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                     (int)kSelSmemKeysMax + 16 * 1024);
-                if (e != cudaSuccess) return e;
-                attr[which] = true;
-            }
-            return launch_pdl(kern, dim3(1), dim3(kSelThreads), smem, s, 1, delta, B, budget, rank, sel);
-        };
-        return smem_keys ? go(k_topk_small<true>, 0) : go(k_topk_small<false>, 1);
-    }
-    // larger budgets: radix select and compaction, then the split counting rank kernel
     const bool smem_keys = (size_t)B * 8 <= kSelSmemKeysMax;
     const size_t smem = smem_keys ? (size_t)B * 8 : 0;
-    static bool attr2[2] = {false, false};
-    auto go2 = [&](auto kern, int which) -> cudaError_t {
-        if (!attr2[which]) {
+    static bool attr[2] = {false, false};
+    auto go = [&](auto kern, int which) -> cudaError_t {
+        if (!attr[which]) {
             cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                  (int)kSelSmemKeysMax + 16 * 1024);
             if (e != cudaSuccess) return e;
-            attr2[which] = true;
+            attr[which] = true;
         }
         return launch_pdl(kern, dim3(1), dim3(kSelThreads), smem, s, 1, delta, B, budget, sel);
     };
-    cudaError_t e = smem_keys ? go2(k_topk_large<true>, 0) : go2(k_topk_large<false>, 1);
+    return smem_keys ? go(k_topk_large<true>, 0) : go(k_topk_large<false>, 1);
+}
+
+cudaError_t launch_topk(const double* delta, int B, int budget, int32_t* rank, int32_t* sel, cudaStream_t s) {
+    if (budget <= 0) return cudaSuccess;
+    cudaError_t e = launch_topk_select(delta, B, budget, sel, s);
     if (e != cudaSuccess) return e;
     return launch_pdl(k_topk_rank_split, dim3((budget + 15) / 16), dim3(128), 0, s, 1, delta, (const int32_t*)sel,
                       budget, rank);
@@ -965,11 +708,12 @@ cudaError_t launch_pack(const uint8_t* rcodes, const uint8_t* rsf, int N, int K,
 
 cudaError_t launch_pack_w(const uint16_t* W, int N, int K, const float* g_w, const int32_t* sel, int budget,
                           uint8_t* blk_codes, uint8_t* blk_sf, int32_t* blk_kt, int32_t* tile_ptr, uint32_t* bitmap,
-                          cudaStream_t s) {
+                          const double* delta, int32_t* rank, cudaStream_t s) {
     const int NBr = N / 64;
-    const int grid = budget + (NBr + 127) / 128;
-    return launch_pdl(k_pack_w, dim3(grid), dim3(128), 0, s, 1, W, N, K, g_w, sel, budget, blk_codes, blk_sf, blk_kt,
-                      tile_ptr, bitmap);
+    const int ncsr = (NBr + 127) / 128;
+    const int nrank = rank && budget > 0 ? (budget + 15) / 16 : 0;
+    return launch_pdl(k_pack_w, dim3(budget + ncsr + nrank), dim3(128), 0, s, 1, W, N, K, g_w, sel, budget, blk_codes,
+                      blk_sf, blk_kt, tile_ptr, bitmap, ncsr, delta, nrank ? rank : (int32_t*)nullptr);
 }
 
 }  // namespace mq
