@@ -240,6 +240,7 @@ __device__ __forceinline__ int block_exclusive_sum(int v, int* scratch, int& tot
 
 constexpr int kSelThreads = 1024;
 constexpr size_t kSelSmemKeysMax = 160 * 1024;
+constexpr int kSelBitWords = (int)(kSelSmemKeysMax / 8 / 32);  // bitmap words of the keys that fit
 
 constexpr int kDigitBits = 11;
 
@@ -277,12 +278,13 @@ __global__ void __launch_bounds__(kSelThreads) k_topk_large(const double* __rest
                                                             int32_t* __restrict__ sel) {
     extern __shared__ __align__(16) uint64_t dyn[];
     uint64_t* keys = dyn;  // [B] when kSmemKeys
-    __shared__ unsigned hist[1 << kDigitBits];
+    __shared__ unsigned hist[2][1 << kDigitBits];  // pass p counts into hist[p % 2]
+    __shared__ uint32_t s_gtw[kSelBitWords], s_eqw[kSelBitWords];
     __shared__ uint32_t s_and[64], s_or[64];
     __shared__ uint64_t s_prefix;
     __shared__ int s_pos, s_need, s_cand;
     __shared__ int s_gt[32], s_eq[32], s_base[32], s_eqb[32];
-    __shared__ int scratch[32];
+    __shared__ int scratch[32], scratch2[32];
     griddep_wait();  // Delta comes from the previous kernel
     griddep_launch();
     constexpr int U = 8;
@@ -320,6 +322,7 @@ __global__ void __launch_bounds__(kSelThreads) k_topk_large(const double* __rest
             s_or[2 * warp + 1] = ol;
         }
     }
+    for (int b = tid; b < (1 << kDigitBits); b += kSelThreads) hist[0][b] = 0;
     __syncthreads();
     if (warp == 0) {
         const uint32_t ah = __reduce_and_sync(0xffffffffu, s_and[2 * lane]);
@@ -337,13 +340,15 @@ __global__ void __launch_bounds__(kSelThreads) k_topk_large(const double* __rest
         }
     }
     __syncthreads();
-    while (s_pos > 0 && s_cand > s_need) {
+    for (int pass = 0; s_pos > 0 && s_cand > s_need; ++pass) {
         const int pos = s_pos, w = pos < kDigitBits ? pos : kDigitBits, shift = pos - w;
         const uint64_t prefix = s_prefix, hi = pos >= 64 ? 0ull : (~0ull << pos);
         const int need = s_need;
         const int nb = 1 << w;
-        for (int b = tid; b < nb; b += kSelThreads) hist[b] = 0;
-        __syncthreads();
+        unsigned* h = hist[pass & 1];
+        // the other buffer (read by the previous pass's scan, which every thread has left)
+        // is cleared for the next pass
+        for (int b = tid; b < (1 << kDigitBits); b += kSelThreads) hist[(pass + 1) & 1][b] = 0;
         for (int i0 = tid - lane; i0 < B; i0 += U * kSelThreads) {  // warp-uniform
             uint64_t k[U];
 #pragma unroll
@@ -356,12 +361,12 @@ __global__ void __launch_bounds__(kSelThreads) k_topk_large(const double* __rest
                 const int i = i0 + lane + u * kSelThreads;
                 unsigned digit = 1u << kDigitBits;  // not counted
                 if (i < B && (k[u] & hi) == prefix) digit = (unsigned)(k[u] >> shift) & (nb - 1);
-                if (digit < (1u << kDigitBits)) atomicAdd(&hist[digit], 1u);
+                if (digit < (1u << kDigitBits)) atomicAdd(&h[digit], 1u);
             }
         }
         __syncthreads();
         const int b0 = nb - 1 - 2 * tid;
-        const unsigned c0 = b0 >= 0 ? hist[b0] : 0u, c1 = b0 - 1 >= 0 ? hist[b0 - 1] : 0u;
+        const unsigned c0 = b0 >= 0 ? h[b0] : 0u, c1 = b0 - 1 >= 0 ? h[b0 - 1] : 0u;
         const int above = block_excl_sum_1bar<kSelThreads>((int)(c0 + c1), scratch);
         if (b0 >= 0 && above < need && above + (int)(c0 + c1) >= need) {
             const bool first = above + (int)c0 >= need;
@@ -376,6 +381,38 @@ __global__ void __launch_bounds__(kSelThreads) k_topk_large(const double* __rest
     const int pos = s_pos, need = s_need;
     const bool whole = s_cand == s_need;
     const uint64_t prefix = s_prefix, hi = pos >= 64 ? 0ull : (~0ull << pos);
+    if (kSmemKeys) {
+        // the keys above the bucket and in it as bitmaps (warp ballots over 32-key words),
+        // then thread t turns word t into sel entries at the count of selected keys before it
+        const int nw = (B + 31) >> 5;
+        for (int wd = warp; wd < nw; wd += 32) {
+            const int i = wd * 32 + lane;
+            const bool valid = i < B;
+            const uint64_t t = valid ? (keys[i] & hi) : 0ull;
+            const unsigned g = __ballot_sync(0xffffffffu, valid && t > prefix);
+            const unsigned e = __ballot_sync(0xffffffffu, valid && t == prefix);
+            if (lane == 0) {
+                s_gtw[wd] = g;
+                s_eqw[wd] = e;
+            }
+        }
+        __syncthreads();
+        const uint32_t g = tid < nw ? s_gtw[tid] : 0u, e = tid < nw ? s_eqw[tid] : 0u;
+        uint32_t take = g;
+        if (whole) {
+            take |= e;
+        } else {  // one tied value: its lowest-index `need` keys
+            int left = need - block_excl_sum_1bar<kSelThreads>(__popc(e), scratch2);
+            for (uint32_t ee = e; left > 0 && ee; --left) {
+                const uint32_t low = ee & (0u - ee);
+                take |= low;
+                ee ^= low;
+            }
+        }
+        int out = block_excl_sum_1bar<kSelThreads>(__popc(take), scratch);
+        for (uint32_t m = take; m; m &= m - 1) sel[out++] = tid * 32 + (__ffs(m) - 1);
+        return;
+    }
     const int CW = (B + 32 * 32 - 1) / (32 * 32) * 32;  // indices per warp, a multiple of 32
     const int w0 = min(B, warp * CW), w1 = min(B, w0 + CW);
     int gt = 0, eq = 0;
