@@ -38,11 +38,16 @@ __global__ void __launch_bounds__(512, 1) k_amax_partial(const uint16_t* __restr
     const uint4* v = reinterpret_cast<const uint4*>(W);
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
-    for (; i + 7 * stride < n8; i += 8 * stride) {
+    for (; i < n8; i += 8 * stride) {
         uint4 x[8];
-        // volatile: the eight loads are issued before any of them is used
+        // volatile: the eight loads are issued before any of them is used. In the last
+        // round an index past the end reads the last vector again (a repeated element does
+        // not change the maximum), so the remainder also goes out eight loads at a time.
 #pragma unroll
-        for (int u = 0; u < 8; ++u) x[u] = ld_stream16(v + i + u * stride);
+        for (int u = 0; u < 8; ++u) {
+            const int64_t j = i + u * stride;
+            x[u] = ld_stream16(v + (j < n8 ? j : n8 - 1));
+        }
         // every loaded word is an operand here, so all eight loads precede the first use
         asm volatile("" : "+r"(x[0].x), "+r"(x[0].y), "+r"(x[0].z), "+r"(x[0].w), "+r"(x[1].x), "+r"(x[1].y),
                      "+r"(x[1].z), "+r"(x[1].w), "+r"(x[2].x), "+r"(x[2].y), "+r"(x[2].z), "+r"(x[2].w),
@@ -57,13 +62,6 @@ __global__ void __launch_bounds__(512, 1) k_amax_partial(const uint16_t* __restr
             for (int j = 0; j < 4; ++j) m = fmaxf(m, fmaxf(fabsf(bf16_bits_to_f32(w[j] & 0xFFFFu)),
                                                            fabsf(bf16_bits_to_f32(w[j] >> 16))));
         }
-    }
-    for (; i < n8; i += stride) {
-        const uint4 x = __ldg(v + i);
-        const uint32_t w[4] = {x.x, x.y, x.z, x.w};
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-            m = fmaxf(m, fmaxf(fabsf(bf16_bits_to_f32(w[j] & 0xFFFFu)), fabsf(bf16_bits_to_f32(w[j] >> 16))));
     }
     __shared__ float red[16];
     m = warp_max(m);
