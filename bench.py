@@ -394,6 +394,48 @@ def gemm_sweep(peaks: dict, reps: int = 20) -> list:
     return out
 
 
+# the kernels of each call whose DRAM traffic a capture sums (in launch order per call)
+TRAFFIC_KERNELS = {"quantize_weight_delta": ("k_amax_partial", "k_quant_delta")}
+
+
+def write_traffic(csv_path: str, call: str = "quantize_weight_delta") -> dict:
+    """Turn an ncu CSV (--csv --print-units base, metrics dram__bytes_read.sum and
+    dram__bytes_write.sum, kernels of `call` only, caches not flushed) into
+    profiles/traffic.json: DRAM bytes per call, averaged over the complete calls captured,
+    keyed to the current source hash."""
+    import csv
+    with open(csv_path) as f:
+        lines = [ln for ln in f if not ln.startswith("==")]
+    launches = {}
+    for r in csv.DictReader(lines):
+        if r.get("Metric Name") not in ("dram__bytes_read.sum", "dram__bytes_write.sum"):
+            continue
+        e = launches.setdefault(int(r["ID"]), {"kernel": r["Kernel Name"], "bytes": 0.0})
+        e["bytes"] += float(r["Metric Value"].replace(",", ""))
+    first, last = TRAFFIC_KERNELS[call]
+    per_call, cur = [], None
+    for i in sorted(launches):
+        k = launches[i]
+        if first in k["kernel"]:
+            cur = k["bytes"]
+        elif last in k["kernel"] and cur is not None:
+            per_call.append(cur + k["bytes"])
+            cur = None
+    if not per_call:
+        raise SystemExit(f"no complete {call} call in {csv_path}")
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    d = {}
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+    d[call] = {"bytes_per_call": int(round(sum(per_call) / len(per_call))), "calls": len(per_call),
+               "kernels": list(TRAFFIC_KERNELS[call]), "source_hash": source_hash()}
+    with open(p, "w") as f:
+        json.dump(d, f, indent=1)
+        f.write("\n")
+    return d[call]
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -405,8 +447,13 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-sweep", action="store_true", help="skip the GEMM-vs-M sweep")
+    ap.add_argument("--traffic-from", metavar="CSV",
+                    help="write profiles/traffic.json from an ncu DRAM-bytes capture and exit (no GPU)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
+    if args.traffic_from:
+        print(json.dumps(write_traffic(args.traffic_from)))
+        return
 
     if args.impl == "reference":
         run_reference(args)
