@@ -398,11 +398,11 @@ def gemm_sweep(peaks: dict, reps: int = 20) -> list:
 TRAFFIC_KERNELS = {"quantize_weight_delta": ("k_amax_partial", "k_quant_delta")}
 
 
-def write_traffic(csv_path: str, call: str = "quantize_weight_delta") -> dict:
+def write_traffic(csv_path: str, call: str = "quantize_weight_delta", skip: int = 0) -> dict:
     """Turn an ncu CSV (--csv --print-units base, metrics dram__bytes_read.sum and
     dram__bytes_write.sum, kernels of `call` only, caches not flushed) into
-    profiles/traffic.json: DRAM bytes per call, averaged over the complete calls captured,
-    keyed to the current source hash."""
+    profiles/traffic.json: DRAM bytes per call, averaged over the complete calls captured
+    after the first `skip`, keyed to the current source hash."""
     import csv
     with open(csv_path) as f:
         lines = [ln for ln in f if not ln.startswith("==")]
@@ -421,8 +421,9 @@ def write_traffic(csv_path: str, call: str = "quantize_weight_delta") -> dict:
         elif last in k["kernel"] and cur is not None:
             per_call.append(cur + k["bytes"])
             cur = None
+    per_call = per_call[skip:]
     if not per_call:
-        raise SystemExit(f"no complete {call} call in {csv_path}")
+        raise SystemExit(f"no complete {call} call in {csv_path} after the first {skip}")
     p = os.path.join(ROOT, "profiles", "traffic.json")
     d = {}
     if os.path.exists(p):
@@ -449,10 +450,12 @@ def main():
     ap.add_argument("--no-sweep", action="store_true", help="skip the GEMM-vs-M sweep")
     ap.add_argument("--traffic-from", metavar="CSV",
                     help="write profiles/traffic.json from an ncu DRAM-bytes capture and exit (no GPU)")
+    ap.add_argument("--traffic-skip", type=int, default=0, metavar="N",
+                    help="with --traffic-from: leave out the first N captured calls (warm-up)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     if args.traffic_from:
-        print(json.dumps(write_traffic(args.traffic_from)))
+        print(json.dumps(write_traffic(args.traffic_from, skip=args.traffic_skip)))
         return
 
     if args.impl == "reference":
@@ -544,11 +547,25 @@ def main():
         pgraphs.append(pg)
         evs.append(e)
 
+    # the timed steps: a graph of R consecutive steps (input sets 0..R-1) replayed back to
+    # back, as a layer runs inside a model's captured forward, and the single-step graphs
+    # for the remainder; step k always uses input set k % R
+    gall = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gall):
+        for i in range(R):
+            step(i)
+
+    def run_steps(n):
+        for _ in range(n // R):
+            gall.replay()
+        for k in range(n - n % R, n):
+            graphs[k % R].replay()
+
     sampler = ClockSampler(local)
     sampler.start()
     time.sleep(0.3)
-    for w in range(args.warmup):
-        graphs[w % R].replay()
+    warmup_done = max(args.warmup, R)  # every graph replayed once before the timed region
+    run_steps(warmup_done)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
@@ -557,8 +574,7 @@ def main():
     ev0 = torch.cuda.Event(enable_timing=True)
     ev1 = torch.cuda.Event(enable_timing=True)
     ev0.record(stream)
-    for k in range(args.steps):
-        graphs[k % R].replay()
+    run_steps(args.steps)
     ev1.record(stream)
     torch.cuda.synchronize()
     t_wall1 = time.time()
@@ -673,12 +689,13 @@ def main():
     if rank != 0:
         return
     line = {"metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "warmup": warmup_done, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "nvfp4 (e2m1 x e2m1, e4m3 scales, fp32 accumulate; fp32/fp64 prep)",
             "data": "synthetic",
             "config": {"workload": args.workload, "M": M, "N": N, "K": K, "T": T, "budget_frac": 0.10,
                        "budget_blocks": budget, "parallelism": f"replicas x{world}",
-                       "l2": f"{R} rotating input sets (~{R * 57} MB touched) > 2x L2; no flush"},
+                       "l2": f"{R} rotating input sets (~{R * 57} MB touched) > 2x L2; no flush",
+                       "graphs": f"{R} steps per graph replay (one per input set)"},
             "roofline": roofline, "gemm": gemm, "gemm_vs_M": sweep, "kernels": kern, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": int(launches_per_step * args.steps), "clocks": clocks}
     print(json.dumps(line), flush=True)
