@@ -135,6 +135,29 @@ __device__ __forceinline__ bool mbar_wait_err(uint64_t* bar, uint32_t parity, in
 }
 
 // 2-D tiled TMA load with 16-bit elements (x in elements).
+// L2 cache policies for cache_hint operands: evict_last keeps lines ahead of normal data
+// (for a tensor the next kernel reads again), evict_first lets them go first.
+__device__ __forceinline__ uint64_t l2_policy_evict_last() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+
+// tma_load_2d_u16 with an L2 cache policy.
+__device__ __forceinline__ void tma_load_2d_u16_hint(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y,
+                                                     uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1, {%2, %3}], "
+        "[%4], %5;" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar)), "l"(policy)
+        : "memory");
+}
+
 __device__ __forceinline__ void tma_load_2d_u16(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y) {
     asm volatile(
         "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::

@@ -17,6 +17,15 @@ __device__ __forceinline__ uint4 ld_stream16(const uint4* p) {
     return r;
 }
 
+// ld_stream16 with an L2 cache policy.
+__device__ __forceinline__ uint4 ld_stream16_hint(const uint4* p, uint64_t policy) {
+    uint4 r;
+    asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.u32 {%0, %1, %2, %3}, [%4], %5;"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+                 : "l"(p), "l"(policy));
+    return r;
+}
+
 __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
@@ -36,6 +45,8 @@ __global__ void __launch_bounds__(512, 1) k_amax_partial(const uint16_t* __restr
     griddep_launch();
     float m = 0.0f;
     const uint4* v = reinterpret_cast<const uint4*>(W);
+    // W is read again right after by the quantize+Delta pass: keep it in L2 until then
+    const uint64_t keep = l2_policy_evict_last();
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
     for (; i < n8; i += 8 * stride) {
@@ -46,7 +57,7 @@ __global__ void __launch_bounds__(512, 1) k_amax_partial(const uint16_t* __restr
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
             const int64_t j = i + u * stride;
-            x[u] = ld_stream16(v + (j < n8 ? j : n8 - 1));
+            x[u] = ld_stream16_hint(v + (j < n8 ? j : n8 - 1), keep);
         }
         // every loaded word is an operand here, so all eight loads precede the first use
         asm volatile("" : "+r"(x[0].x), "+r"(x[0].y), "+r"(x[0].z), "+r"(x[0].w), "+r"(x[1].x), "+r"(x[1].y),

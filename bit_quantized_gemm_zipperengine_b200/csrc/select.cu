@@ -166,12 +166,14 @@ __global__ void __launch_bounds__(kQDThreads, 3) k_quant_delta(const __grid_cons
         tma_prefetch_desc(&tmap_w);
     }
     __syncthreads();
+    // this pass is the last full read of W (the weight maxima pass kept it in L2 for it)
+    const uint64_t done = l2_policy_evict_first();
     auto issue = [&](int i) {  // strip number i of this CTA into stage i % kQDStages
         const int b = blockIdx.x + i * gridDim.x;
         if (b < nstrips) {
             const int s = i % kQDStages;
             mbar_arrive_expect_tx(&full[s], kQDTile);
-            tma_load_2d_u16(sm + s * kQDTile, &tmap_w, &full[s], (b % KB) * 64, (b / KB) * kQDRows);
+            tma_load_2d_u16_hint(sm + s * kQDTile, &tmap_w, &full[s], (b % KB) * 64, (b / KB) * kQDRows, done);
         }
     };
     // W is an input of the call (never written by the preceding kernels): start loading
