@@ -217,10 +217,9 @@ def test_repeat_calls_deterministic(dev):
 
 
 def test_topk_blocks_alone_and_large_budgets(dev):
-    """A4 alone on many blocks and budgets (the one-CTA select-and-sort path up to its
-    budget limit, the radix select with the split rank kernel above it, keys in shared or
-    global memory, a threshold inside a bucket of one tied value, every block selected),
-    with ties, against the oracle's sort."""
+    """A4 alone on many blocks and budgets (the one-CTA radix selection and the split rank
+    kernel; keys in shared or global memory, a threshold inside a bucket of one tied value,
+    every block selected), with ties, against the oracle's sort."""
     from bit_quantized_gemm_zipperengine_b200 import mosaic
     rng = np.random.default_rng(12)
     cases = [(32, (0, 1, 3, 32), False), (4096, (409, 767, 768, 769, 1024, 1025), False),
