@@ -394,6 +394,24 @@ def gemm_sweep(peaks: dict, reps: int = 20) -> list:
     return out
 
 
+# ------------------------------------------------------------------ replicas
+def max_over_ranks(ms: float, world: int, device) -> float:
+    """The slowest rank's time (every rank calls this, in the same order on every rank)."""
+    if world <= 1:
+        return ms
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([ms], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replica_gbs(bytes_per_step: float, world: int, ms_per_step: float) -> float:
+    """Whole-job GB/s: every replica processes its own step of bytes_per_step in the
+    slowest rank's ms_per_step."""
+    return bytes_per_step * world / (ms_per_step * 1e-3) / 1e9
+
+
 # the kernels of each call whose DRAM traffic a capture sums (in launch order per call)
 TRAFFIC_KERNELS = {"quantize_weight_delta": ("k_amax_partial", "k_quant_delta")}
 
@@ -580,11 +598,7 @@ def main():
     t_wall1 = time.time()
     if world > 1:
         dist.barrier()
-    ms_total = ev0.elapsed_time(ev1)
-    if world > 1:
-        t = torch.tensor([ms_total], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_total = float(t.item())
+    ms_total = max_over_ranks(ev0.elapsed_time(ev1), world, dev)
     time.sleep(0.3)
     sampler.stop()
     clocks = sampler.summary(t_wall0, t_wall1)
@@ -595,7 +609,7 @@ def main():
     ms_step = ms_total / args.steps
     per_call = step_bytes(M, N, K, T, budget)
     bytes_step = sum(per_call.values())
-    value = bytes_step * world / (ms_step * 1e-3) / 1e9
+    value = replica_gbs(bytes_step, world, ms_step)
 
     # per-call device time: each call replayed back to back over the R rotating input sets
     # (CUDA events around graphs of R launches; programmatic dependent launch hides the
@@ -658,12 +672,8 @@ def main():
             mosaic.mq_run_layer(Wh, Xh, Ch, Yh, M, N, K, T, budget, 0, True, hb)
         a1.record(stream)
         torch.cuda.synchronize()
-        ms_e = a0.elapsed_time(a1) / ke
-        if world > 1:
-            t = torch.tensor([ms_e], device=dev, dtype=torch.float64)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ms_e = float(t.item())
-        e2e = {"value": bytes_step * world / (ms_e * 1e-3) / 1e9, "unit": "GB/s", "ms_per_step": ms_e,
+        ms_e = max_over_ranks(a0.elapsed_time(a1) / ke, world, dev)
+        e2e = {"value": replica_gbs(bytes_step, world, ms_e), "unit": "GB/s", "ms_per_step": ms_e,
                "h2d_bytes_per_step": 2 * N * K + 2 * M * K + 2 * T * K, "d2h_bytes_per_step": 2 * M * N,
                "steps": ke}
 
