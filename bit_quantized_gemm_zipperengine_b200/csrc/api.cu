@@ -278,9 +278,10 @@ static mq_status quantize_act_early(const mq_bf16* X, int M, int K, mq_nvfp4_mat
     return launched(launch_quant_act(X, M, K, xq->codes, xq->sf, xq->sf_swz, xq->gscale, true, as_stream(stream)), 1);
 }
 
-// prefetch: the caller guarantees wq was complete before the kernel preceding the GEMM in
-// the stream started (the whole-path call's order), so the decode kernel may load it
-// before waiting for that kernel.
+// prefetch: the caller guarantees wq and xq were complete before the GEMM could start (the
+// whole-path call's order: the pack before it lets it start only after its own wait, and
+// that wait already implies the activation quantizer and the quantize+Delta pass
+// completed), so the decode kernel may load them before waiting for the pack.
 static mq_status gemm_impl(const mq_nvfp4_mat* xq, const mq_nvfp4_mat* wq, const mq_residual_packed* r, mq_bf16* Y,
                            int M, int N, int K, unsigned flags, void* ws, size_t ws_bytes, bool prefetch,
                            mq_stream stream) {
@@ -425,8 +426,9 @@ mq_status mq_run_layer(const mq_bf16* W, const mq_bf16* X, const mq_bf16* Xcal, 
     // activation quantizer read only inputs of this call: they let their dependent start
     // at once, do their work and wait at their end (so their completion still implies
     // their predecessor's). The others let their dependent start right after their wait.
-    // When the GEMM starts, the quantize+Delta kernel has completed, and the GEMM requests
-    // W before waiting for its predecessor (prefetch). The activation quantizer runs as its
+    // When the GEMM starts, the quantize+Delta kernel and the activation quantizer have
+    // completed, and the GEMM requests W and X before waiting for its predecessor
+    // (prefetch). The activation quantizer runs as its
     // own kernel: on B200 at decode sizes that is faster than quantizing inside the GEMM
     // (mq_gemm_act), whose per-token maxima must first be exchanged between the K splits.
     mq_status st;

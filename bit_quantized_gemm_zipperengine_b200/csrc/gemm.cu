@@ -19,9 +19,10 @@
 // CTA of the tile (a tile counter).
 // The kernel is launched with programmatic dependent launch: its prologue overlaps the
 // preceding kernel. It waits for that kernel before its loads, unless the caller
-// guarantees that W was complete before that kernel started (GemmParams::prefetch, set by
-// the whole-path call, where the activation quantizer precedes the GEMM): then the first
-// stages' W is requested before the wait.
+// guarantees that W and X were complete before this kernel could start
+// (GemmParams::prefetch, set by the whole-path call: the pack before the GEMM lets it
+// start only after its own wait, which already implies that both quantizers completed):
+// then the first stages' W and X are requested before the wait.
 #include <cuda_bf16.h>
 
 #include "common.cuh"
@@ -261,18 +262,18 @@ __global__ void __launch_bounds__(192, 1)
             }
         };
         const int first = min(C::kStages, n_iters);
-        // W normally comes from an earlier kernel of the stream, so it is loaded after the
-        // wait for the preceding kernel; a caller that guarantees it was complete before
-        // that kernel started (p.prefetch) lets the first stages' W load at once. X (the
-        // activation quantizer's output) always waits.
+        // W and X normally come from earlier kernels of the stream, so they are loaded
+        // after the wait for the preceding kernel; a caller that guarantees both were
+        // complete before this kernel could start (p.prefetch) lets the first stages load
+        // at once, so their base MMAs need not wait for the residual's producer.
         if (!p.prefetch) griddep_wait();
         if (elect_one())
-            for (int it = 0; it < first; ++it) issue_w(it);
+            for (int it = 0; it < first; ++it) {
+                issue_w(it);
+                issue_x(it);
+            }
         __syncwarp();
         if (p.prefetch) griddep_wait();
-        if (elect_one())
-            for (int it = 0; it < first; ++it) issue_x(it);
-        __syncwarp();
         // the residual lookups (dependent index loads) run while W and X are in flight;
         // the base MMAs of a stage do not wait for its residual blocks
         if (p.has_resid && n_iters > 0) {

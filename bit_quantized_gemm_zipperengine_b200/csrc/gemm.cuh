@@ -25,8 +25,8 @@ struct GemmParams {
     int mode;                // 0 fused, 1 base only, 2 residual only
     int has_resid;
     int cluster;             // split-K reduced through the cluster's shared memory
-    int prefetch;            // W was complete before the preceding kernel started, so the
-                             // decode kernel may load it before waiting for that kernel
+    int prefetch;            // W and X were complete before this kernel could start, so the
+                             // decode kernel may load them before waiting for its predecessor
     const uint16_t* x_bf16;  // decode kernel: bf16 X [M][K] quantized inside the kernel
                              // (x_sf and g_x unused), or null
     float* gx_out;           // with x_bf16: per-token scales written here if not null
