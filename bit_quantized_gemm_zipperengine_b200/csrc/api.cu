@@ -21,7 +21,9 @@ cudaError_t launch_delta(const CUtensorMap& tw, int N, int K, const float* H, co
                          int* err, cudaStream_t s);
 cudaError_t launch_quant_delta(const uint16_t* W, const CUtensorMap& tw, int N, int K, const float* H,
                                uint8_t* codes, uint8_t* sf, uint8_t* sf_swz, float* g, uint8_t* rcodes, uint8_t* rsf,
-                               double* delta, float* partial, int* err, cudaStream_t s);
+                               double* delta, float* partial, int* err, cudaStream_t s, const uint16_t* X, int M,
+                               uint8_t* xcodes, uint8_t* xsf, uint8_t* xsf_swz, float* g_x);
+bool quant_delta_takes_act(int K);
 cudaError_t launch_topk(const double* delta, int B, int budget, int32_t* rank, int32_t* sel, cudaStream_t s);
 int topk_launches(int budget);
 cudaError_t launch_pack(const uint8_t* rcodes, const uint8_t* rsf, int N, int K, const int32_t* sel, int budget,
@@ -188,9 +190,11 @@ mq_status mq_delta_score_topk(const mq_bf16* W, const float* H, const mq_nvfp4_m
     return launched(launch_topk(delta, B, budget, rank, sel, s), topk_launches(budget));
 }
 
-mq_status mq_quantize_weight_delta(const mq_bf16* W, int N, int K, const float* H, mq_nvfp4_mat* base,
-                                   mq_nvfp4_mat* resid_full, double* delta, void* ws, size_t ws_bytes,
-                                   mq_stream stream) {
+// X/xq (may be null): the whole-path call's activation rows, quantized by the same kernel
+// after its strips (validated by the caller as mq_quantize_act does).
+static mq_status quantize_weight_delta_impl(const mq_bf16* W, int N, int K, const float* H, mq_nvfp4_mat* base,
+                                            mq_nvfp4_mat* resid_full, double* delta, void* ws, size_t ws_bytes,
+                                            const mq_bf16* X, int M, mq_nvfp4_mat* xq, mq_stream stream) {
     if (!W || !H || !delta || !base || !nvfp4_shape_ok(N, K) || N % 64) return MQ_ERR_INVALID_ARG;
     if (!base->codes || !base->sf_swz || !base->gscale) return MQ_ERR_INVALID_ARG;
     if (base->rows != N || base->cols != K) return MQ_ERR_INVALID_ARG;
@@ -206,8 +210,16 @@ mq_status mq_quantize_weight_delta(const mq_bf16* W, int N, int K, const float* 
     if (!err || !make_tmap_bf16_blocks(&tw, W, (uint64_t)K, (uint64_t)N)) return MQ_ERR_CUDA;
     cudaError_t e = launch_quant_delta(W, tw, N, K, H, base->codes, base->sf, base->sf_swz, base->gscale,
                                        resid_full ? resid_full->codes : nullptr, resid_full ? resid_full->sf : nullptr,
-                                       delta, static_cast<float*>(ws), err, as_stream(stream));
+                                       delta, static_cast<float*>(ws), err, as_stream(stream), X, M,
+                                       xq ? xq->codes : nullptr, xq ? xq->sf : nullptr, xq ? xq->sf_swz : nullptr,
+                                       xq ? xq->gscale : nullptr);
     return launched(e, 2);
+}
+
+mq_status mq_quantize_weight_delta(const mq_bf16* W, int N, int K, const float* H, mq_nvfp4_mat* base,
+                                   mq_nvfp4_mat* resid_full, double* delta, void* ws, size_t ws_bytes,
+                                   mq_stream stream) {
+    return quantize_weight_delta_impl(W, N, K, H, base, resid_full, delta, ws, ws_bytes, nullptr, 0, nullptr, stream);
 }
 
 mq_status mq_topk_blocks(const double* delta, int nblk, int budget, int32_t* rank, int32_t* sel, mq_stream stream) {
@@ -433,10 +445,19 @@ mq_status mq_run_layer(const mq_bf16* W, const mq_bf16* X, const mq_bf16* Xcal, 
     // (mq_gemm_act), whose per-token maxima must first be exchanged between the K splits.
     mq_status st;
     if ((st = mq_hessian_diag(xc, T, K, buf->H, stream)) != MQ_OK) return st;
-    if ((st = mq_quantize_weight_delta(w, N, K, buf->H, &buf->base, nullptr, buf->delta, buf->ws_quant,
-                                       buf->ws_quant_bytes, stream)) != MQ_OK)
+    // A6 rides on the quantize+Delta kernel when its CTAs can hold a row (K <= 4096): its
+    // CTAs with the fewest strips quantize the activation rows at the end; otherwise the
+    // activation quantizer runs as its own kernel in early mode
+    mq_nvfp4_mat* xq = &buf->xq;
+    if (!x || !xq->codes || !xq->sf_swz || !xq->gscale || xq->rows != M || xq->cols != K || !aligned(x, 16) ||
+        !aligned(xq->codes, 8) || !aligned(xq->sf_swz, 4))
+        return MQ_ERR_INVALID_ARG;
+    const bool act_in_qd = quant_delta_takes_act(K);
+    if ((st = quantize_weight_delta_impl(w, N, K, buf->H, &buf->base, nullptr, buf->delta, buf->ws_quant,
+                                         buf->ws_quant_bytes, act_in_qd ? x : nullptr, M, act_in_qd ? xq : nullptr,
+                                         stream)) != MQ_OK)
         return st;
-    if ((st = quantize_act_early(x, M, K, &buf->xq, stream)) != MQ_OK) return st;
+    if (!act_in_qd && (st = quantize_act_early(x, M, K, xq, stream)) != MQ_OK) return st;
     // A4 as two parts: the selection kernel writes sel, and rank (which the GEMM does not
     // read) is written by extra CTAs of the pack kernel, beside the packing
     {

@@ -26,12 +26,6 @@ __device__ __forceinline__ uint4 ld_stream16_hint(const uint4* p, uint64_t polic
     return r;
 }
 
-__device__ __forceinline__ float warp_max(float v) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-    return v;
-}
-
 // Per-CTA maxima of |W| over a grid-stride range of 8-element vectors (kAmaxBlocks
 // CTAs of 512 threads, 8 independent 16-byte loads in flight per thread: 64 KB per SM,
 // about what HBM needs in flight to run at full rate).
@@ -86,15 +80,6 @@ __global__ void __launch_bounds__(512, 1) k_amax_partial(const uint16_t* __restr
     griddep_wait();
 }
 
-// Gathers the scale bytes of 4 consecutive groups (lanes l..l+3, l % 4 == 0) into one
-// 32-bit word for lane l.
-__device__ __forceinline__ uint32_t gather4(uint32_t b) {
-    const uint32_t b1 = __shfl_down_sync(0xffffffffu, b, 1);
-    const uint32_t b2 = __shfl_down_sync(0xffffffffu, b, 2);
-    const uint32_t b3 = __shfl_down_sync(0xffffffffu, b, 3);
-    return b | (b1 << 8) | (b2 << 16) | (b3 << 24);
-}
-
 // A1: base NVFP4(W, g) and residual NVFP4(W - deq Q(W), g) for every group.
 // One thread per group; the group count is a multiple of 32 (K % 64 == 0 and
 // N % 64 == 0), so whole warps stay together for the 4-group scale gather. The groups of
@@ -141,65 +126,6 @@ __global__ void __launch_bounds__(256) k_quant_weight(const uint16_t* __restrict
     }
 }
 
-// A6: one CTA per (padded) token row, every group held in registers (kGPT groups per
-// thread, groups tid + j * blockDim), so the row is read once. Rows >= M only clear
-// their tiled scales.
-template <int kGPT>
-__device__ __forceinline__ void quant_act_row(const uint16_t* __restrict__ X, int M, int K,
-                                              uint8_t* __restrict__ codes, uint8_t* __restrict__ sf,
-                                              uint8_t* __restrict__ sf_swz, float* __restrict__ g_x) {
-    const int m = blockIdx.x;
-    const int G = K / 16;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    if (m >= M) {
-        for (int q = threadIdx.x * 4; q < G; q += blockDim.x * 4)
-            *reinterpret_cast<uint32_t*>(sf_swz + sf_swz_offset(m, q, K)) = 0u;
-        return;
-    }
-    const uint16_t* row = X + (int64_t)m * K;
-    float a[kGPT][16];
-    float amax = 0.0f;
-#pragma unroll
-    for (int j = 0; j < kGPT; ++j) {
-        const int q = threadIdx.x + j * blockDim.x;
-        if (q < G) {
-            load16_bf16(row + q * 16, a[j]);
-#pragma unroll
-            for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(a[j][i]));
-        }
-    }
-    __shared__ float red[32];
-    __shared__ float s_g;
-    amax = warp_max(amax);
-    if (lane == 0) red[warp] = amax;
-    __syncthreads();
-    if (warp == 0) {
-        float t = lane < (int)(blockDim.x >> 5) ? red[lane] : 0.0f;
-        t = warp_max(t);
-        if (lane == 0) {
-            s_g = (t == 0.0f) ? 1.0f : __fdiv_rn(t, 2688.0f);
-            g_x[m] = s_g;
-        }
-    }
-    __syncthreads();
-    const float g = s_g, g6 = __fmul_rn(6.0f, g);
-#pragma unroll
-    for (int j = 0; j < kGPT; ++j) {
-        const int q = threadIdx.x + j * blockDim.x;
-        const bool live = q < G;
-        uint32_t sfb = 0;
-        if (live) {
-            float deq[16];
-            uint32_t lo, hi;
-            sfb = nvfp4_group(a[j], g, g6, lo, hi, deq);
-            reinterpret_cast<uint2*>(codes + (int64_t)m * (K / 2))[q] = make_uint2(lo, hi);
-            if (sf) sf[(int64_t)m * G + q] = (uint8_t)sfb;
-        }
-        const uint32_t word = gather4(sfb);
-        if (live && (lane & 3) == 0) *reinterpret_cast<uint32_t*>(sf_swz + sf_swz_offset(m, q, K)) = word;
-    }
-}
-
 // early == 0: wait for the preceding kernel, let the dependent start, quantize.
 // early != 0: let the dependent start, quantize, then wait for the preceding kernel before
 // exiting (so this kernel's completion still implies its predecessor's). For a caller
@@ -210,7 +136,7 @@ __global__ void __launch_bounds__(1024)
                 uint8_t* __restrict__ sf, uint8_t* __restrict__ sf_swz, float* __restrict__ g_x, int early) {
     if (!early) griddep_wait();
     griddep_launch();
-    quant_act_row<kGPT>(X, M, K, codes, sf, sf_swz, g_x);
+    quant_act_row<kGPT>(X, M, K, codes, sf, sf_swz, g_x, blockIdx.x);
     if (early) griddep_wait();
 }
 

@@ -145,17 +145,30 @@ __device__ __forceinline__ void quant_delta_strip(const uint8_t* tile, uint8_t* 
     }
 }
 
+// Activation rows the whole-path call hands to the quantize+Delta kernel (act.rows == 0:
+// none). The CTAs with the fewest strips take them after their strips, one row per CTA
+// at a time, so the rows fill the pass's tail instead of following it. K <= 16 x threads.
+struct ActRows {
+    const uint16_t* X;
+    int M, rows;  // rows: M padded to a multiple of 128 (rows >= M clear their scales)
+    uint8_t* codes;
+    uint8_t* sf;
+    uint8_t* sf_swz;
+    float* g_x;
+};
+
 // kWriteCodes = false: Delta only, tensor scale read from g_in. kWriteCodes = true: base
 // codes and scales, Delta, and (kWriteResid) the full residual, in one pass over W; the
 // tensor scale comes from the |W| maximum partials. Persistent: CTA c handles strips c,
-// c + gridDim.x, ... in (strip row, kt) order, kt fastest.
+// c + gridDim.x, ... in (strip row, kt) order, kt fastest; then activation rows (act).
 template <bool kWriteCodes, bool kWriteResid>
 __global__ void __launch_bounds__(kQDThreads, 3) k_quant_delta(const __grid_constant__ CUtensorMap tmap_w, int N, int K,
                                                             const float* __restrict__ H, const float* __restrict__ g_in,
                                                             uint8_t* __restrict__ codes, uint8_t* __restrict__ sf,
                                                             uint8_t* __restrict__ sf_swz, float* __restrict__ g_out,
                                                             uint8_t* __restrict__ rcodes, uint8_t* __restrict__ rsf,
-                                                            double* __restrict__ delta, int* __restrict__ err) {
+                                                            double* __restrict__ delta, int* __restrict__ err,
+                                                            const ActRows act) {
     extern __shared__ uint8_t qd_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(qd_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* full = reinterpret_cast<uint64_t*>(sm + kQDOffBar);
@@ -199,6 +212,11 @@ __global__ void __launch_bounds__(kQDThreads, 3) k_quant_delta(const __grid_cons
         __syncthreads();  // stage s and the strip's staging are free again
         // every copy issued here is waited for by a later iteration of this loop
         if (threadIdx.x == 0 && ok) issue(i + kQDStages);
+    }
+    // the activation rows, the last CTAs (fewest strips) first; X is an input of the call
+    for (int m = gridDim.x - 1 - blockIdx.x; m < act.rows; m += gridDim.x) {
+        quant_act_row<1>(act.X, act.M, K, act.codes, act.sf, act.sf_swz, act.g_x, m);
+        __syncthreads();  // the row's shared scratch is free again
     }
 }
 
@@ -691,22 +709,29 @@ static int qd_strips(int N, int K) { return ((N / 64 + 1) / 2) * (K / 64); }
 
 cudaError_t launch_delta(const CUtensorMap& tw, int N, int K, const float* H, const float* g, double* delta,
                          int* err, cudaStream_t s) {
+    const ActRows none = {nullptr, 0, 0, nullptr, nullptr, nullptr, nullptr};
     return launch_pdl(k_quant_delta<false, false>, dim3(quant_delta_grid(qd_strips(N, K))), dim3(kQDThreads),
                       kQDSmem, s, 1, tw, N, K, H, g, (uint8_t*)nullptr, (uint8_t*)nullptr, (uint8_t*)nullptr,
-                      (float*)nullptr, (uint8_t*)nullptr, (uint8_t*)nullptr, delta, err);
+                      (float*)nullptr, (uint8_t*)nullptr, (uint8_t*)nullptr, delta, err, none);
 }
+
+bool quant_delta_takes_act(int K) { return K / 16 <= kQDThreads; }
 
 cudaError_t launch_quant_delta(const uint16_t* W, const CUtensorMap& tw, int N, int K, const float* H,
                                uint8_t* codes, uint8_t* sf, uint8_t* sf_swz, float* g, uint8_t* rcodes, uint8_t* rsf,
-                               double* delta, float* partial, int* err, cudaStream_t s) {
+                               double* delta, float* partial, int* err, cudaStream_t s, const uint16_t* X, int M,
+                               uint8_t* xcodes, uint8_t* xsf, uint8_t* xsf_swz, float* g_x) {
+    if (X && !quant_delta_takes_act(K)) return cudaErrorInvalidValue;
     cudaError_t e = launch_amax(W, (int64_t)N * K, partial, s);
     if (e != cudaSuccess) return e;
     const dim3 grid(quant_delta_grid(qd_strips(N, K)));
+    const ActRows act = {X, X ? M : 0, X ? (M + 127) / 128 * 128 : 0, xcodes, xsf, xsf_swz, g_x};
     if (rcodes)
         return launch_pdl(k_quant_delta<true, true>, grid, dim3(kQDThreads), kQDSmem, s, 1, tw, N, K, H,
-                          (const float*)partial, codes, sf, sf_swz, g, rcodes, rsf, delta, err);
+                          (const float*)partial, codes, sf, sf_swz, g, rcodes, rsf, delta, err, act);
     return launch_pdl(k_quant_delta<true, false>, grid, dim3(kQDThreads), kQDSmem, s, 1, tw, N, K, H,
-                      (const float*)partial, codes, sf, sf_swz, g, (uint8_t*)nullptr, (uint8_t*)nullptr, delta, err);
+                      (const float*)partial, codes, sf, sf_swz, g, (uint8_t*)nullptr, (uint8_t*)nullptr, delta, err,
+                      act);
 }
 
 int topk_launches(int budget) { return budget <= 0 ? 0 : 2; }

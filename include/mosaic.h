@@ -274,8 +274,9 @@ typedef struct {
 /*
  * The whole path for one layer: A2 H from the T calibration tokens, A1+A3 quantize W and
  * score every block (mq_quantize_weight_delta, residual not stored), A6 quantize X
- * (mq_quantize_act; it depends on X alone and runs ahead of the selection so that it
- * overlaps the Delta pass), A4 top-`budget` selection, A5 pack the selected residual from
+ * (mq_quantize_act's results; for K <= 4096 the quantize+Delta kernel's least loaded CTAs
+ * quantize the rows after their strips, otherwise its own kernel runs ahead of the
+ * selection), A4 top-`budget` selection, A5 pack the selected residual from
  * W (mq_pack_residual_weight), A7+A8 fused GEMM into Y. Results are those of the
  * individual calls. The call's first kernel waits for the kernel preceding the call in
  * the stream before the others may start, so no input is read before that kernel ends. With host == 0, W, X, Xcal and Y are device
