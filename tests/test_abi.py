@@ -66,3 +66,13 @@ def test_host_validation_rejects_bad_arguments(L):
     wm1 = mosaic.NVFP4Mat(1024, 4096, fake, None, fake, fake)
     assert L.mq_gemm(ctypes.byref(xm1), ctypes.byref(wm1), None, fake, 16, 1024, 4096, 0, None, 0, None) == 3
     assert L.mq_status_string(3) == b"workspace missing or too small"
+    # A2 takes 1..1024 calibration tokens and a 16-byte aligned Xcal
+    assert L.mq_hessian_diag(fake, 1025, 4096, fake, None) == 2
+    assert L.mq_hessian_diag(ctypes.c_void_p(0x10002), 512, 4096, fake, None) == 1
+    assert L.mq_hessian_diag(fake, 0, 4096, fake, None) == 1
+    # A6 holds a row in one CTA: K up to 65536
+    big = mosaic.NVFP4Mat(16, 65536 + 64, fake, None, fake, fake)
+    assert L.mq_quantize_act(fake, 16, 65536 + 64, ctypes.byref(big), None) == 2
+    # top-K: budget outside [0, nblk]
+    assert L.mq_topk_blocks(fake, 4096, 4097, fake, fake, None) == 1
+    assert L.mq_topk_blocks(fake, 4096, -1, fake, fake, None) == 1
