@@ -416,7 +416,7 @@ def replica_gbs(bytes_per_step: float, world: int, ms_per_step: float) -> float:
 TRAFFIC_KERNELS = {"quantize_weight_delta": ("k_amax_partial", "k_quant_delta")}
 
 
-def write_traffic(csv_path: str, call: str = "quantize_weight_delta", skip: int = 0) -> dict:
+def write_traffic(csv_path: str, call: str = "quantize_weight_delta", skip: int = 0, out_path: str | None = None) -> dict:
     """Turn an ncu CSV (--csv --print-units base, metrics dram__bytes_read.sum and
     dram__bytes_write.sum, kernels of `call` only, caches not flushed) into
     profiles/traffic.json: DRAM bytes per call, averaged over the complete calls captured
@@ -442,7 +442,7 @@ def write_traffic(csv_path: str, call: str = "quantize_weight_delta", skip: int 
     per_call = per_call[skip:]
     if not per_call:
         raise SystemExit(f"no complete {call} call in {csv_path} after the first {skip}")
-    p = os.path.join(ROOT, "profiles", "traffic.json")
+    p = out_path or os.path.join(ROOT, "profiles", "traffic.json")
     d = {}
     if os.path.exists(p):
         with open(p) as f:
