@@ -342,6 +342,8 @@ class Layer:
         return b
 
     def forward(self, X: torch.Tensor, flags: int = 0, stream=None) -> torch.Tensor:
+        """A6 + A7/A8 on bf16 X [M][K] (device). Returns the layer's output buffer for this M
+        and flags: the next call with the same M and flags writes into the same tensor."""
         M = X.shape[0]
         xq, Y, ws = self.act_buffers(M, flags)
         mq_quantize_act(X, xq, stream)
