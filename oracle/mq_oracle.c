@@ -28,8 +28,8 @@
  * 16-element blocks and an E2M1 mantissa ("Problem" section of that page).
  *
  * Arithmetic: fp32 IEEE operations exactly as written (compile with
- * -ffp-contract=off, no fast-math; the one fused multiply-add is an explicit fmaf),
- * fp64 where stated. Rounding is RNE throughout.
+ * -ffp-contract=off, no fast-math, no fused multiply-add), fp64 where stated.
+ * Rounding is RNE throughout.
  *
  * Parity pins (tests/test_oracle_*.py): grid round trips and tie tables against a
  * brute-force nearest-value search, torch's float8 conversion, closed-form error
@@ -238,12 +238,6 @@ void orc_hessian_diag(const uint16_t* Xcal, int T, int K, float* H) {
 }
 
 /* Pairwise tree over 64 values: v[i] += v[i+32] (i<32), then +16, +8, +4, +2, +1. */
-static float tree64f(float* v) {
-    for (int h = 32; h >= 1; h >>= 1)
-        for (int i = 0; i < h; ++i) v[i] = v[i] + v[i + h];
-    return v[0];
-}
-
 static double tree64(double* v) {
     for (int h = 32; h >= 1; h >>= 1)
         for (int i = 0; i < h; ++i) v[i] = v[i] + v[i + h];
@@ -251,12 +245,15 @@ static double tree64(double* v) {
 }
 
 /*
- * Delta-score (A3) for every 64x64 block b = nt*(K/64) + kt:
+ * Delta-score (A3) for every 64x64 block b = nt*(K/64) + kt: the block's reduction of
+ * the H-weighted squared error when its residual is kept (summary, "Methodology",
+ * section 2):
  *   e   = R = fp32(W - deq Q(W))            (base quantization error)
  *   e'  = fp32(R - deq R)                   (error left after the residual)
- *   tau = fp32( e*e - fp32(e'*e') )         (one fused multiply-add, fp32)
- *   c_k = tree64 over the block's 64 rows of tau, in fp32
- *   p_k = fp64(H_k) * fp64(c_k)
+ *   tau = fp64(e)*fp64(e) - fp64(e')*fp64(e')
+ *         (both squares are exact in fp64, so the subtraction is the one rounding)
+ *   c_k = tree64 over the block's 64 rows of tau, in fp64
+ *   p_k = fp64(H_k) * c_k
  *   Delta_b = tree64 over the block's 64 columns of p_k, in fp64
  */
 void orc_delta_score(const uint16_t* W, int N, int K, const float* H, const uint8_t* base_codes,
@@ -271,18 +268,18 @@ void orc_delta_score(const uint16_t* W, int N, int K, const float* H, const uint
 #pragma omp parallel for schedule(static)
     for (int b = 0; b < NBr * KB; ++b) {
         int nt = b / KB, kt = b % KB;
-        double p[64];
-        float col[64];
+        double p[64], col[64];
         for (int c = 0; c < 64; ++c) {
             int k = kt * 64 + c;
             for (int r = 0; r < 64; ++r) {
                 int64_t i = (int64_t)(nt * 64 + r) * K + k;
                 float e = bf16_to_f32(W[i]) - dq[i];
                 float e2 = e - dr[i];
-                float e2sq = e2 * e2;
-                col[r] = fmaf(e, e, -e2sq);
+                double sq = (double)e * (double)e;      /* exact */
+                double sq2 = (double)e2 * (double)e2;   /* exact */
+                col[r] = sq - sq2;
             }
-            p[c] = (double)H[k] * (double)tree64f(col);
+            p[c] = (double)H[k] * tree64(col);
         }
         delta[b] = tree64(p);
     }

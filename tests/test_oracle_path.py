@@ -102,18 +102,20 @@ def test_delta_nonnegative_and_distortion_identity(orc, tiny):
     H, delta, wq = tiny["H"], tiny["delta"], tiny["wq"]
     e, e2 = _errors(tiny["W"], wq)
     E0 = _distortion(H, e, e2, np.zeros((N, K), bool))
-    # tau and the row tree are fp32 (relative rounding 2^-24 per operation), so the
-    # identities below hold to ~1e-7 of the magnitudes involved
-    assert np.all(delta >= -1e-8 * E0)
+    # the squares are exact and every sum is fp64 (relative rounding 2^-53 per add), so
+    # the identities below hold to ~1e-13 of the magnitudes involved; an fp32 tau or an
+    # fp32 row tree (2^-24 per operation) misses these bounds by five orders of magnitude
+    assert np.all(delta >= -1e-13 * E0)
     # E(S) = E(empty) - sum_{b in S} Delta_b for arbitrary S
     rng = np.random.default_rng(0)
     flat = delta.reshape(-1)
     for size in (1, 3, 7, flat.size):
         S = rng.choice(flat.size, size=size, replace=False)
         ES = _distortion(H, e, e2, _elem_mask(S, N, K))
-        assert abs((E0 - ES) - flat[S].sum()) <= 1e-7 * E0
-    # each block's Delta, written out element by element in fp64 (order and precision
-    # differ: bound by 1e-6 of the block's sum of H (e^2 + e'^2))
+        assert abs((E0 - ES) - flat[S].sum()) <= 1e-12 * E0
+    # each block's Delta, written out element by element in fp64 (only the summation
+    # order differs: bound by 1e-12 of the block's sum of H (e^2 + e'^2))
+    worst = 0.0
     for b in range(flat.size):
         nt, kt = divmod(b, K // 64)
         sl = (slice(nt * 64, nt * 64 + 64), slice(kt * 64, kt * 64 + 64))
@@ -121,7 +123,8 @@ def test_delta_nonnegative_and_distortion_identity(orc, tiny):
         e64, e264 = e[sl].astype(np.float64), e2[sl].astype(np.float64)
         ref = np.sum(h * (e64 ** 2 - e264 ** 2))
         scale = np.sum(h * (e64 ** 2 + e264 ** 2))
-        assert abs(ref - flat[b]) <= 1e-6 * scale + 1e-300
+        worst = max(worst, abs(ref - flat[b]) / (scale + 1e-300))
+    assert worst <= 1e-12, worst
 
 
 def test_outlier_blocks_score_highest(orc, tiny):
