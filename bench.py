@@ -1,20 +1,31 @@
 #!/usr/bin/env python
 """Benchmark of the MosaicQuant / ZipperEngine path on B200.
 
-One step = one pass of the whole path over one batch of synthetic inputs, the
-sequence `mq_run_layer` runs, captured in a CUDA graph: H from the calibration tokens,
-quantize W (base + full residual) and score every block in one pass, top-K, pack the
-residual, quantize X, fused NVFP4 GEMM. Default workload: LLaMA3-8B q_proj at decode batch 16 (M=16, N=K=4096, 512
-calibration tokens, 10% block budget = 409 blocks).
+The metric is the fused NVFP4 base + sparse-residual GEMM's throughput (TFLOPS, GB/s and
+fraction of the FP4 / HBM roofline) against the token count M.
 
-value  = algorithmic bytes of the step (what each call must read and write once)
-         / device time per step, GB/s, summed over ranks (weak scaling, one replica
-         per GPU; the path has no exchange step).
-e2e    = same metric through mq_run_layer with pinned HOST buffers: the H2D copies of
-         W, X, Xcal and the D2H copy of Y are inside the timed region.
-Timing: CUDA events on the launching stream around K graph replays, barrier +
-synchronize on both sides, max over ranks. Six input sets rotate so that the touched
-footprint (~340 MB) is far above L2 (126 MB): every step starts L2-cold.
+One step = one call of the fused GEMM (mq_gemm, A7 + A8) on the LLaMA3-8B q_proj decode
+layer (M=16 tokens, N=K=4096, 10% block budget = 409 residual blocks), with its
+quantized weight, packed residual and quantized activations resident in HBM.
+
+value  = the call's algorithmic bytes (W codes and scales, residual blocks and index,
+         X codes and scales, bf16 Y) / device time per call, GB/s, summed over ranks
+         (weak scaling, one replica per GPU; the path has no exchange step).
+         Consecutive steps rotate over copies of the operands whose total exceeds 2x the
+         L2, so every call reads its bytes from HBM.
+e2e    = the same bytes per step through mq_run_layer with pinned HOST buffers and a
+         prepared layer: the H2D copy of the step's bf16 X, the activation quantizer, the
+         GEMM and the D2H copy of Y are all in the timed region.
+whole_path = one mq_run_layer step (A1..A8: H, quantize + Delta, top-K, pack, quantize X,
+         GEMM) and each of its calls timed alone, for the same layer.
+sweep  = the fused GEMM on every workload's layers and token counts (and the 70B MLP's
+         budget sweep), beside its dense-only time (residual overhead), the unfused
+         ablation, and for M <= 128 the in-kernel activation quantization.
+fp4_peak = the measured dense FP4 tensor rate (tcgen05 mxf4nvf4 MMA loop, operands
+         resident on chip), the denominator of the prefill fractions beside 4x the
+         measured bf16 cuBLAS rate.
+Timing: CUDA events on the launching stream, barrier + synchronize on both sides, max
+over ranks.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 """
@@ -38,6 +49,7 @@ if ROOT not in sys.path:
 METRIC = "fused NVFP4 base+residual GEMM TFLOPS, GB/s and % of FP4/HBM roofline vs M"
 DEFAULT_WORKLOAD = "llama3_8b_qproj_decode"
 FP4_PER_BF16 = 4.0  # nominal dense FP4 / bf16 tensor throughput ratio (9 / 2.25 PFLOP/s)
+L2_BYTES = 126e6
 
 
 # ------------------------------------------------------------------ work accounting
@@ -155,123 +167,170 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ oracle CPU baseline
-def oracle_band(wl, M: int, rows: int):
-    import synth
-    L = synth.layer(wl, M=M)
-    band = L["W"][:rows]
-    budget = synth.budget_blocks(rows, L["K"], 0.10)
-    return band, L["X"], L["Xcal"], budget
+def gemm_bytes(M: int, N: int, K: int, nblk: int) -> int:
+    """Algorithmic bytes of one fused GEMM call (step_bytes()["gemm"])."""
+    return step_bytes(M, N, K, 512, nblk)["gemm"]
 
 
-def cpu_baseline(wl_name: str, M: int, min_seconds: float = 10.0, max_runs: int = 50):
-    """The oracle (as it stands) on a row band of the workload until >= min_seconds of CPU
-    work; GB/s of the band's algorithmic bytes."""
+def oracle_gemm_sample(wl_name: str, target_s: float):
+    """A bounded sample of the headline workload for the CPU oracle: its fp64 GEMM
+    reference on a band of weight rows (every token), with the band sized so that one call
+    takes about target_s seconds. Returns (run, bytes of the band's GEMM, description)."""
+    import numpy as np
+
     import oracle
     import synth
     wl = synth.WORKLOADS[wl_name]
-    K, T = wl.matrices[0].K, wl.T
-    rows = min(wl.matrices[0].N, 1024)
-    band, X, Xcal, budget = oracle_band(wl, M, rows)
-    oracle.run_path(band, X, Xcal, budget)  # build + page in
+    M, N, K = wl.Ms[0], wl.matrices[0].N, wl.matrices[0].K
+    L = synth.layer(wl_name, M=M)
+    budget = synth.budget_blocks(N, K, 0.10)
+    ref = oracle.run_path(L["W"], L["X"], L["Xcal"], budget, rows=np.arange(1, dtype=np.int32))
+    xq, wq, sel = ref["xq"], ref["wq"], ref["sel"]
+
+    def band(rows):
+        # the first `rows` weight rows (a multiple of 64) and their selected blocks
+        KB = K // 64
+        s = sel[sel < (rows // 64) * KB]
+        w = {k: (v[:rows] if isinstance(v, np.ndarray) and v.ndim == 2 else v) for k, v in wq.items()}
+        return w, s, rows
+
+    def run(b):
+        w, s, rows = b
+        oracle.gemm_rows(xq, w, s, M, rows, K)
+
+    rows = 64
+    t0 = time.perf_counter()
+    run(band(rows))
+    per_row = (time.perf_counter() - t0) / rows
+    rows = int(max(64, min(N, target_s / max(per_row, 1e-9))) // 64 * 64)
+    b = band(rows)
+    nblk = len(b[1])
+    return (lambda: run(b)), gemm_bytes(M, rows, K, nblk), \
+        f"fp64 GEMM reference on a {rows}-row band of W ({rows}x{K}, all {M} tokens, {nblk} residual blocks)"
+
+
+def cpu_baseline(wl_name: str, min_seconds: float = 10.0, max_runs: int = 200):
+    """The oracle (as it stands) on a band of the headline GEMM until >= min_seconds of CPU
+    work; GB/s of the band's algorithmic bytes."""
+    run, nbytes, desc = oracle_gemm_sample(wl_name, 0.5)
+    run()  # page in
     t0 = time.perf_counter()
     runs = 0
     while True:
-        oracle.run_path(band, X, Xcal, budget)
+        run()
         runs += 1
         el = time.perf_counter() - t0
         if el >= min_seconds or runs >= max_runs:
             break
     per = el / runs
-    b = sum(step_bytes(M, rows, K, T, budget).values())
-    return {"value": b / per / 1e9, "unit": "GB/s", "cores": os.cpu_count(), "kind": "oracle",
-            "sample": f"whole path on a {rows}-row band of W ({rows}x{K}, M={M}, T={T}, {budget} blocks), "
-                      f"{runs} runs, {per:.3f} s/run"}
+    return {"value": nbytes / per / 1e9, "unit": "GB/s", "cores": os.cpu_count(), "kind": "oracle",
+            "sample": f"{desc}, {runs} runs, {per:.3f} s/run"}
 
 
 def run_reference(args):
-    """CPU oracle arm: rank 0 times the oracle's whole path on a bounded band sample."""
+    """CPU oracle arm: rank 0 times the oracle's GEMM reference on a band of the headline
+    workload, one band per step, sized so the whole run ends within about two minutes."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    import oracle
     import synth
     wl = synth.WORKLOADS[args.workload]
-    M, K, T = wl.Ms[0], wl.matrices[0].K, wl.T
-    rows = min(wl.matrices[0].N, 512)
-    band, X, Xcal, budget = oracle_band(wl, M, rows)
+    M, N, K = wl.Ms[0], wl.matrices[0].N, wl.matrices[0].K
+    per_step = min(0.5, 120.0 / max(1, args.steps + args.warmup))
+    run, nbytes, desc = oracle_gemm_sample(args.workload, per_step)
     for _ in range(args.warmup):
-        oracle.run_path(band, X, Xcal, budget)
+        run()
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        oracle.run_path(band, X, Xcal, budget)
+        run()
     el = time.perf_counter() - t0
-    b = sum(step_bytes(M, rows, K, T, budget).values())
-    value = b * args.steps / el / 1e9
-    sample = f"whole path on a {rows}-row band of W ({rows}x{K}, M={M}, T={T}, {budget} blocks) per step"
+    value = nbytes * args.steps / el / 1e9
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32/f64 (CPU oracle)",
-            "data": "synthetic", "config": {"workload": args.workload, "M": M, "N": wl.matrices[0].N, "K": K,
-                                            "T": T, "budget_frac": 0.10},
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64 (CPU oracle)",
+            "data": "synthetic",
+            "config": {"workload": args.workload + " fused GEMM", "M": M, "N": N, "K": K, "budget_frac": 0.10},
             "cpu_baseline": {"value": value, "unit": "GB/s", "cores": os.cpu_count(), "kind": "oracle",
-                             "sample": sample},
+                             "sample": desc + " per step"},
             "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
 
-# ------------------------------------------------------------------ GPU arm
-def isolated_profile(sets, calls, M, N, K, budget, reps, stream):
-    """Average device time of each call alone: a graph of len(sets) launches over the
-    rotating input sets, replayed until `reps` launches were timed."""
+# ------------------------------------------------------------------ GPU helpers
+def graph_time_us(issue, n_calls: int, reps: int, stream=None) -> float:
+    """Device time per call: `issue()` captured once as a CUDA graph of n_calls launches,
+    replayed `reps` times between CUDA events (after one untimed replay)."""
+    import torch
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        issue()
+    g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        g.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    del g
+    return e0.elapsed_time(e1) * 1e3 / (reps * n_calls)
+
+
+def operand_copies(layer, xq, Y, ws, per_call: float, min_copies: int = 2):
+    """Copies of the GEMM's operands (quantized weight, packed residual, quantized X, Y,
+    workspace) whose total exceeds 2.5x the L2, so that back-to-back calls over them
+    read every byte from HBM."""
+    import torch
+    R = max(min_copies, int(math.ceil(2.5 * L2_BYTES / per_call)))
+
+    def cl(d):
+        return {k: (v.clone() if isinstance(v, torch.Tensor) else v) for k, v in d.items() if k != "blob"}
+    return [(cl(layer.base), cl(layer.packed), cl(xq), torch.empty_like(Y), None if ws is None else ws.clone())
+            for _ in range(R)]
+
+
+def fp4_peak(sampler, ctas: int = 148, iters: int = 40000) -> dict:
+    """The FP4 MMA-loop probe on every SM: TFLOP/s from CUDA events, with the SM clock
+    sampled meanwhile (repeated for about a second)."""
     import torch
     from bit_quantized_gemm_zipperengine_b200 import mosaic
-
-    def issue(c, s):
-        layer = s["layer"]
-        xq, Yb, ws = layer.act_buffers(M)
-        if c == "quantize_weight_delta":
-            mosaic.mq_quantize_weight_delta(s["W"], layer.H, layer.base, None, layer.delta, layer.qws)
-        elif c == "hessian_diag":
-            mosaic.mq_hessian_diag(s["Xcal"], layer.H)
-        elif c == "topk_blocks":
-            mosaic.mq_topk_blocks(layer.delta, budget, layer.rank, layer.sel)
-        elif c == "pack_residual":
-            mosaic.mq_pack_residual_weight(s["W"], layer.base, layer.sel, budget, layer.packed)
-        elif c == "quantize_act":
-            mosaic.mq_quantize_act(s["X"], xq)
-        else:
-            mosaic.mq_gemm(xq, layer.base, layer.packed, Yb, M, N, K, 0, ws)
-
-    out = {}
-    inner = 4  # passes over the sets per graph, so graph launch gaps are amortised
-    for c in calls:
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
-            for _ in range(inner):
-                for s in sets:
-                    issue(c, s)
-        g.replay()
+    mosaic.mq_fp4_mma_loop(ctas, 1000)
+    torch.cuda.synchronize()
+    best, runs = None, 0
+    t0 = time.time()
+    while time.time() - t0 < 1.0 or runs < 3:
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        fl = mosaic.mq_fp4_mma_loop(ctas, iters)
+        e1.record()
         torch.cuda.synchronize()
-        n = max(1, reps // (inner * len(sets)))
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        for _ in range(n):
-            g.replay()
-        b.record(stream)
-        torch.cuda.synchronize()
-        out[c] = a.elapsed_time(b) / (n * inner * len(sets)) * reps
-    return out
+        tf = fl / (e0.elapsed_time(e1) * 1e-3) / 1e12
+        best = tf if best is None else max(best, tf)
+        runs += 1
+    t1 = time.time()
+    assert mosaic.mq_get_error() == 0
+    return {"tflops": round(best, 1), "ctas": ctas, "iters_per_cta": iters, "runs": runs,
+            "shape": "tcgen05.mma kind::mxf4nvf4 M=128 N=256 K=64, operands resident on chip",
+            "clocks": sampler.summary(t0, t1) if sampler else None}
 
 
-# ------------------------------------------------------------------ GEMM vs M
-SWEEP = (("qwen3_32b", "q", (1, 16, 128, 1024, 8192)), ("qwen3_32b", "up", (16, 1024, 8192)),
-         ("llama3_8b_mlp_prefill", "up", (2048,)))
+# ------------------------------------------------------------------ GEMM sweep over every workload
+SWEEP = (("tiny", "w", (16,), (0.10,)),
+         ("llama3_8b_qproj_decode", "q_proj", (16,), (0.10,)),
+         ("llama3_8b_mlp_prefill", "up", (2048,), (0.10,)),      # gate has the same shape
+         ("llama3_8b_mlp_prefill", "down", (2048,), (0.10,)),
+         ("qwen3_32b", "q", (1, 16, 128, 1024, 8192), (0.10,)),
+         ("qwen3_32b", "up", (1, 16, 128, 1024, 8192), (0.10,)),
+         ("qwen3_32b", "down", (1, 16, 128, 1024, 8192), (0.10,)),
+         ("llama3_70b_mlp", "up", (4096,), (0.0, 0.05, 0.10, 0.20)),
+         ("llama3_70b_mlp", "down", (4096,), (0.0, 0.05, 0.10, 0.20)))
 
 
-def gemm_sweep(peaks: dict, reps: int = 20) -> list:
-    """The fused GEMM alone (and dense-only) across token counts: device time per call from
-    CUDA events around graphs of back-to-back calls over enough rotating copies of the
-    quantized weight, residual and activations that every call reads them from HBM."""
+def gemm_sweep(peaks: dict, fp4_measured: float | None, reps: int = 20) -> tuple[list, list]:
+    """The fused GEMM alone, dense-only and residual-only on every workload's layers and
+    token counts: device time per call from CUDA events around graphs of back-to-back
+    calls over copies of the operands that exceed 2.5x the L2. Also the Delta-score +
+    top-K pass of the 70B MLP layers at every budget. Returns (gemm rows, delta rows)."""
     import numpy as np
     import torch
 
@@ -279,119 +338,101 @@ def gemm_sweep(peaks: dict, reps: int = 20) -> list:
     from bit_quantized_gemm_zipperengine_b200 import mosaic
 
     dev = torch.device("cuda", torch.cuda.current_device())
-    fp4_sus = peaks["bf16_tflops_sustained"] * FP4_PER_BF16
     fp4_burst = peaks["bf16_tflops"] * FP4_PER_BF16
-    out = []
-    for wl, mat, Ms in SWEEP:
+    rows, drows = [], []
+    for wl, mat, Ms, fracs in SWEEP:
         L = synth.layer(wl, matrix=mat, M=max(Ms))
         N, K = L["N"], L["K"]
-        budget = synth.budget_blocks(N, K, 0.10)
-        layer = mosaic.Layer(N, K, budget, dev, with_sf=False)
         W = torch.from_numpy(L["W"].view(np.int16)).view(torch.bfloat16).to(dev)
         C = torch.from_numpy(L["Xcal"].view(np.int16)).view(torch.bfloat16).to(dev)
         Xall = torch.from_numpy(L["X"].view(np.int16)).view(torch.bfloat16).to(dev)
-        layer.prepare_path(W, C)
-        del W, C
-        for M in Ms:
-            X = Xall[:M].contiguous()
-            xq, Y, ws = layer.act_buffers(M)
-            mosaic.mq_quantize_act(X, xq)
-            per_call = N * K * 0.5625 + budget * 2304 + M * K * 0.5625 + 4 * M + 2 * M * N
-            R = max(2, int(np.ceil(3 * 126e6 / per_call)))
-            copies = []
-            for _ in range(R):
-                b = {k: (v.clone() if isinstance(v, torch.Tensor) else v) for k, v in layer.base.items()}
-                p = {k: (v.clone() if isinstance(v, torch.Tensor) else v) for k, v in layer.packed.items()}
-                a = {k: (v.clone() if isinstance(v, torch.Tensor) else v) for k, v in xq.items()}
-                copies.append((b, p, a, torch.empty_like(Y), None if ws is None else ws.clone()))
-            res = {}
-            for flags, lab in ((0, "fused"), (mosaic.MQ_GEMM_BASE_ONLY, "base"),
-                               (mosaic.MQ_GEMM_RESIDUAL_ONLY, "resid")):
-                g = torch.cuda.CUDAGraph()
-                with torch.cuda.graph(g):
-                    for b, p, a, y, w in copies:
-                        mosaic.mq_gemm(a, b, p, y, M, N, K, flags, w)
-                g.replay()
-                torch.cuda.synchronize()
-                n = max(1, reps * 4 // R)
-                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                e0.record()
-                for _ in range(n):
-                    g.replay()
-                e1.record()
-                torch.cuda.synchronize()
-                res[lab] = e0.elapsed_time(e1) * 1e3 / (n * R)
-            # the decode kernel quantizing the bf16 activations itself (mq_gemm_act)
-            if M <= 128:
-                ga = torch.cuda.CUDAGraph()
-                with torch.cuda.graph(ga):
-                    for b, p, a, y, w in copies:
-                        mosaic.mq_gemm_act(X, b, p, y, M, N, K, 0, w)
-                ga.replay()
-                torch.cuda.synchronize()
-                n = max(1, reps * 4 // R)
-                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                e0.record()
-                for _ in range(n):
-                    ga.replay()
-                e1.record()
-                torch.cuda.synchronize()
-                res["act_fused"] = e0.elapsed_time(e1) * 1e3 / (n * R)
-                del ga
-                # the same with the separate activation quantizer in front
-                gs = torch.cuda.CUDAGraph()
-                with torch.cuda.graph(gs):
-                    for b, p, a, y, w in copies:
-                        mosaic.mq_quantize_act(X, a)
-                        mosaic.mq_gemm(a, b, p, y, M, N, K, 0, w)
-                gs.replay()
-                torch.cuda.synchronize()
-                e0.record()
-                for _ in range(n):
-                    gs.replay()
-                e1.record()
-                torch.cuda.synchronize()
-                res["act_separate"] = e0.elapsed_time(e1) * 1e3 / (n * R)
-                del gs
-            # the unfused design the pages argue against: dense GEMM, a separate residual-block
-            # GEMM (it reads X again), then an elementwise merge of the two outputs (a torch
-            # add here: this ablation is not part of the path)
-            g = torch.cuda.CUDAGraph()
-            ys = [torch.empty_like(Y) for _ in range(2)]
-            with torch.cuda.graph(g):
-                for _ in range(R):
-                    ys[0].add_(ys[1])
-            g.replay()
+        del L
+        for frac in fracs:
+            budget = synth.budget_blocks(N, K, frac)
+            layer = mosaic.Layer(N, K, budget, dev, with_sf=False)
+            layer.prepare_path(W, C)
             torch.cuda.synchronize()
-            n = max(1, reps * 4 // R)
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record()
-            for _ in range(n):
-                g.replay()
-            e1.record()
-            torch.cuda.synchronize()
-            res["merge"] = e0.elapsed_time(e1) * 1e3 / (n * R)
-            del copies, ys
-            fl = 2.0 * M * N * K + 2.0 * M * 4096 * budget
-            us = res["fused"]
-            tf = fl / (us * 1e-6) / 1e12
-            gbs = per_call / (us * 1e-6) / 1e9
-            out.append({"workload": wl, "matrix": mat, "M": M, "N": N, "K": K, "budget_blocks": budget,
-                        "kernel": "prefill" if (M > 128 and N % 256 == 0) else "decode", "us": round(us, 3),
-                        "us_dense_only": round(res["base"], 3),
-                        "residual_overhead": round(us / res["base"] - 1.0, 4),
-                        "us_residual_only": round(res["resid"], 3),
-                        "us_unfused": round(res["base"] + res["resid"] + res["merge"], 3),
-                        "us_quantize_act_then_gemm": round(res["act_separate"], 3) if "act_separate" in res else None,
-                        "us_gemm_act": round(res["act_fused"], 3) if "act_fused" in res else None,
-                        "tflops_executed": round(tf, 1), "gbs": round(gbs, 1),
-                        "frac_fp4_sustained": round(tf / fp4_sus, 4), "frac_fp4_burst": round(tf / fp4_burst, 4),
-                        "frac_hbm": round(gbs / peaks["hbm_gbs"], 4),
-                        "bound": "hbm" if M <= 316 else "tensor", "rotating_copies": R})
-        del layer, Xall
+            if wl == "llama3_70b_mlp":
+                # the Delta-score + top-K pass (A1 + A3 in one pass over W, then A4), two
+                # copies of W (> 2x L2)
+                Ws = [W, W.clone()]
+                us_qd = graph_time_us(lambda: [mosaic.mq_quantize_weight_delta(w, layer.H, layer.base, None,
+                                                                                layer.delta, layer.qws) for w in Ws],
+                                      len(Ws), 5)
+                us_tk = graph_time_us(lambda: mosaic.mq_topk_blocks(layer.delta, budget, layer.rank, layer.sel), 1,
+                                      20) if budget else 0.0
+                qd_bytes = step_bytes(16, N, K, 512, budget)["quantize_weight_delta"]
+                drows.append({"workload": wl, "matrix": mat, "N": N, "K": K, "blocks": (N // 64) * (K // 64),
+                              "budget_blocks": budget, "us_quantize_delta": round(us_qd, 2),
+                              "gbs_quantize_delta": round(qd_bytes / (us_qd * 1e-6) / 1e9, 1),
+                              "frac_hbm_quantize_delta": round(qd_bytes / (us_qd * 1e-6) / 1e9 / peaks["hbm_gbs"], 4),
+                              "us_topk": round(us_tk, 2)})
+                del Ws
+                layer.prepare_path(W, C)  # restore this budget's selection after the timing
+            for M in Ms:
+                X = Xall[:M].contiguous()
+                xq, Y, ws = layer.act_buffers(M)
+                mosaic.mq_quantize_act(X, xq)
+                per_call = gemm_bytes(M, N, K, budget)
+                copies = operand_copies(layer, xq, Y, ws, per_call)
+                R = len(copies)
+                n = max(2, reps * 4 // R)
+                res = {}
+                for flags, lab in ((0, "fused"), (mosaic.MQ_GEMM_BASE_ONLY, "base"),
+                                   (mosaic.MQ_GEMM_RESIDUAL_ONLY, "resid")):
+                    if lab != "fused" and budget == 0:
+                        continue
+
+                    def issue(flags=flags):
+                        for b, p, a, y, w in copies:
+                            mosaic.mq_gemm(a, b, p, y, M, N, K, flags, w)
+                    res[lab] = graph_time_us(issue, R, n)
+                if M <= 128 and budget:
+                    def issue_act():
+                        for b, p, a, y, w in copies:
+                            mosaic.mq_gemm_act(X, b, p, y, M, N, K, 0, w)
+                    res["act_fused"] = graph_time_us(issue_act, R, n)
+
+                    def issue_sep():
+                        for b, p, a, y, w in copies:
+                            mosaic.mq_quantize_act(X, a)
+                            mosaic.mq_gemm(a, b, p, y, M, N, K, 0, w)
+                    res["act_separate"] = graph_time_us(issue_sep, R, n)
+                if budget:
+                    # the unfused design the pages argue against: dense GEMM, a separate
+                    # residual-block GEMM (it reads X again), then an elementwise merge of
+                    # the two outputs (a torch add: this ablation is not part of the path)
+                    ys = [torch.empty_like(Y) for _ in range(2)]
+                    res["merge"] = graph_time_us(lambda: [ys[0].add_(ys[1]) for _ in range(R)], R, n)
+                    del ys
+                del copies
+                us = res["fused"]
+                fl_exec, fl_dense = gemm_flops(M, N, K, budget)
+                tf = fl_exec / (us * 1e-6) / 1e12
+                gbs = per_call / (us * 1e-6) / 1e9
+                prefill = M > 128 and N % 256 == 0
+                rows.append({
+                    "workload": wl, "matrix": mat, "M": M, "N": N, "K": K, "budget_frac": frac,
+                    "budget_blocks": budget, "kernel": "prefill" if prefill else "decode (stream-K)",
+                    "us": round(us, 3), "tflops_executed": round(tf, 1),
+                    "tflops_dense_equiv": round(fl_dense / (us * 1e-6) / 1e12, 1), "gbs": round(gbs, 1),
+                    "frac_hbm": round(gbs / peaks["hbm_gbs"], 4), "frac_fp4_burst": round(tf / fp4_burst, 4),
+                    "frac_fp4_measured": round(tf / fp4_measured, 4) if fp4_measured else None,
+                    "bound": "hbm" if M <= 316 else "tensor",
+                    "us_dense_only": round(res["base"], 3) if "base" in res else None,
+                    "residual_overhead": round(us / res["base"] - 1.0, 4) if "base" in res else None,
+                    "us_residual_only": round(res["resid"], 3) if "resid" in res else None,
+                    "us_unfused": round(res["base"] + res["resid"] + res["merge"], 3) if "merge" in res else None,
+                    "us_quantize_act_then_gemm": round(res["act_separate"], 3) if "act_separate" in res else None,
+                    "us_gemm_act": round(res["act_fused"], 3) if "act_fused" in res else None,
+                    "rotating_copies": R})
+                print(json.dumps(rows[-1]), file=sys.stderr, flush=True)
+            del layer
+            torch.cuda.empty_cache()
+        del W, C, Xall
         torch.cuda.empty_cache()
     assert mosaic.mq_get_error() == 0
-    return out
+    return rows, drows
 
 
 # ------------------------------------------------------------------ replicas
@@ -413,7 +454,7 @@ def replica_gbs(bytes_per_step: float, world: int, ms_per_step: float) -> float:
 
 
 # the kernels of each call whose DRAM traffic a capture sums (in launch order per call)
-TRAFFIC_KERNELS = {"quantize_weight_delta": ("k_amax_partial", "k_quant_delta")}
+TRAFFIC_KERNELS = {"quantize_weight_delta": ("k_amax_partial", "k_quant_delta"), "gemm": ("k_gemm_streamk",)}
 
 
 def write_traffic(csv_path: str, call: str = "quantize_weight_delta", skip: int = 0, out_path: str | None = None) -> dict:
@@ -430,15 +471,18 @@ def write_traffic(csv_path: str, call: str = "quantize_weight_delta", skip: int 
             continue
         e = launches.setdefault(int(r["ID"]), {"kernel": r["Kernel Name"], "bytes": 0.0})
         e["bytes"] += float(r["Metric Value"].replace(",", ""))
-    first, last = TRAFFIC_KERNELS[call]
-    per_call, cur = [], None
+    names = TRAFFIC_KERNELS[call]  # the call's kernels in launch order
+    per_call, cur, nxt = [], 0.0, 0
     for i in sorted(launches):
         k = launches[i]
-        if first in k["kernel"]:
-            cur = k["bytes"]
-        elif last in k["kernel"] and cur is not None:
-            per_call.append(cur + k["bytes"])
-            cur = None
+        if names[0] in k["kernel"]:
+            cur, nxt = 0.0, 0
+        if nxt < len(names) and names[nxt] in k["kernel"]:
+            cur += k["bytes"]
+            nxt += 1
+            if nxt == len(names):
+                per_call.append(cur)
+                cur, nxt = 0.0, len(names)
     per_call = per_call[skip:]
     if not per_call:
         raise SystemExit(f"no complete {call} call in {csv_path} after the first {skip}")
@@ -455,25 +499,94 @@ def write_traffic(csv_path: str, call: str = "quantize_weight_delta", skip: int 
     return d[call]
 
 
+def whole_path(dev, wl_name: str, sets_n: int, steps: int, stream) -> dict:
+    """One mq_run_layer step (A1..A8) on the headline layer, timed as replays of a graph of
+    `sets_n` steps over rotating input sets (> 2x L2), and each of its calls alone."""
+    import numpy as np
+    import torch
+
+    import synth
+    from bit_quantized_gemm_zipperengine_b200 import mosaic
+    wl = synth.WORKLOADS[wl_name]
+    mat = wl.matrices[0]
+    N, K, M, T = mat.N, mat.K, wl.Ms[0], wl.T
+    budget = synth.budget_blocks(N, K, 0.10)
+    L = synth.layer(wl, M=M)
+    W0 = torch.from_numpy(L["W"].view(np.int16)).view(torch.bfloat16).to(dev)
+    X0 = torch.from_numpy(L["X"].view(np.int16)).view(torch.bfloat16).to(dev)
+    C0 = torch.from_numpy(L["Xcal"].view(np.int16)).view(torch.bfloat16).to(dev)
+    sets = []
+    for _ in range(sets_n):
+        layer = mosaic.Layer(N, K, budget, dev, with_sf=False)
+        sets.append({"layer": layer, "W": W0.clone(), "X": X0.clone(), "Xcal": C0.clone(),
+                     "Y": layer.act_buffers(M)[1], "buf": layer.buffers(M, T)})
+
+    def step(s):
+        mosaic.mq_run_layer(s["W"], s["X"], s["Xcal"], s["Y"], M, N, K, T, budget, 0, False, s["buf"])
+    c0 = mosaic.mq_launch_count()
+    step(sets[0])
+    launches = mosaic.mq_launch_count() - c0
+    for s in sets:
+        step(s)
+    torch.cuda.synchronize()
+    assert mosaic.mq_get_error() == 0
+    us_step = graph_time_us(lambda: [step(s) for s in sets], sets_n, max(3, steps // sets_n), stream)
+    per_call = step_bytes(M, N, K, T, budget)
+
+    def issue(c, s):
+        layer = s["layer"]
+        xq, Yb, ws = layer.act_buffers(M)
+        if c == "quantize_weight_delta":
+            mosaic.mq_quantize_weight_delta(s["W"], layer.H, layer.base, None, layer.delta, layer.qws)
+        elif c == "hessian_diag":
+            mosaic.mq_hessian_diag(s["Xcal"], layer.H)
+        elif c == "topk_blocks":
+            mosaic.mq_topk_blocks(layer.delta, budget, layer.rank, layer.sel)
+        elif c == "pack_residual":
+            mosaic.mq_pack_residual_weight(s["W"], layer.base, layer.sel, budget, layer.packed)
+        elif c == "quantize_act":
+            mosaic.mq_quantize_act(s["X"], xq)
+        else:
+            mosaic.mq_gemm(xq, layer.base, layer.packed, Yb, M, N, K, 0, ws)
+    hbm = load_peaks()["hbm_gbs"]
+    kern = {}
+    for c in ("hessian_diag", "quantize_weight_delta", "quantize_act", "topk_blocks", "pack_residual", "gemm"):
+        us = graph_time_us(lambda: [issue(c, s) for _ in range(4) for s in sets], 4 * sets_n, 20, stream)
+        gbs = per_call[c] / (us * 1e-6) / 1e9
+        kern[c] = {"us": round(us, 3), "alg_bytes": per_call[c], "gbs": round(gbs, 1), "frac_hbm": round(gbs / hbm, 4),
+                   "traffic": dram_traffic(c)}
+    bytes_step = sum(per_call.values())
+    out = {"workload": wl_name, "us_per_step": round(us_step, 3), "alg_bytes": bytes_step,
+           "gbs": round(bytes_step / (us_step * 1e-6) / 1e9, 1), "launches_per_step": int(launches),
+           "timing": f"graph of {sets_n} mq_run_layer steps over rotating input sets, replayed",
+           "calls": kern}
+    for s in sets:
+        s.clear()
+    return out
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10000)
+    ap.add_argument("--steps", type=int, default=3000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
-    ap.add_argument("--sets", type=int, default=6, help="rotating input sets (L2 defeat)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--no-sweep", action="store_true", help="skip the GEMM-vs-M sweep")
+    ap.add_argument("--no-sweep", action="store_true", help="skip the GEMM sweep over every workload")
+    ap.add_argument("--no-path", action="store_true", help="skip the whole-path step")
+    ap.add_argument("--no-fp4-peak", action="store_true", help="skip the FP4 MMA-loop probe")
     ap.add_argument("--traffic-from", metavar="CSV",
                     help="write profiles/traffic.json from an ncu DRAM-bytes capture and exit (no GPU)")
+    ap.add_argument("--traffic-call", default="gemm", choices=sorted(TRAFFIC_KERNELS),
+                    help="with --traffic-from: the call whose kernels the capture holds")
     ap.add_argument("--traffic-skip", type=int, default=0, metavar="N",
                     help="with --traffic-from: leave out the first N captured calls (warm-up)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     if args.traffic_from:
-        print(json.dumps(write_traffic(args.traffic_from, skip=args.traffic_skip)))
+        print(json.dumps(write_traffic(args.traffic_from, call=args.traffic_call, skip=args.traffic_skip)))
         return
 
     if args.impl == "reference":
@@ -498,7 +611,10 @@ def main():
     torch.cuda.set_device(dev)
     if not os.path.exists(mosaic.LIB_PATH):
         libbuild.build()
+    stream = torch.cuda.current_stream(dev)
+    peaks = load_peaks()
 
+    # ---- the headline layer, prepared once (A1..A5), its activations quantized (A6)
     wl = synth.WORKLOADS[args.workload]
     mat = wl.matrices[0]
     N, K, M, T = mat.N, mat.K, wl.Ms[0], wl.T
@@ -507,207 +623,158 @@ def main():
     W0 = torch.from_numpy(L["W"].view(np.int16)).view(torch.bfloat16)
     X0 = torch.from_numpy(L["X"].view(np.int16)).view(torch.bfloat16)
     C0 = torch.from_numpy(L["Xcal"].view(np.int16)).view(torch.bfloat16)
-
-    R = max(1, args.sets)
-    sets = []
-    for i in range(R):
-        layer = mosaic.Layer(N, K, budget, dev, with_sf=False)
-        Wd, Xd, Cd = W0.to(dev), X0.to(dev), C0.to(dev)
-        Y = layer.act_buffers(M)[1]
-        sets.append({"layer": layer, "W": Wd, "X": Xd, "Xcal": Cd, "Y": Y, "buf": layer.buffers(M, T)})
-    stream = torch.cuda.current_stream(dev)
-
-    def step(i):
-        s = sets[i % R]
-        mosaic.mq_run_layer(s["W"], s["X"], s["Xcal"], s["Y"], M, N, K, T, budget, 0, False, s["buf"])
-
-    # eager warm-up (sets kernel attributes, pages everything in); count launches per step
-    c0 = mosaic.mq_launch_count()
-    step(0)
-    launches_per_step = mosaic.mq_launch_count() - c0
-    for i in range(R):
-        step(i)
+    layer = mosaic.Layer(N, K, budget, dev, with_sf=False)
+    layer.prepare_path(W0.to(dev), C0.to(dev))
+    xq, Y, ws = layer.act_buffers(M)
+    mosaic.mq_quantize_act(X0.to(dev), xq)
     torch.cuda.synchronize()
     assert mosaic.mq_get_error() == 0
+    per_call = gemm_bytes(M, N, K, budget)
+    copies = operand_copies(layer, xq, Y, ws, per_call)
+    R = len(copies)
 
-    # per input set: the timed step graph is one mq_run_layer call (the whole path as a
-    # user issues it; consecutive kernels overlap through programmatic dependent launch),
-    # and a profiling graph issues the same steps as separate public calls with event
-    # nodes between them (which serialise them) for the in-step per-call times
-    calls = ["hessian_diag", "quantize_weight_delta", "quantize_act", "topk_blocks", "pack_residual", "gemm"]
+    def call(k):
+        b, p, a, y, w = copies[k % R]
+        mosaic.mq_gemm(a, b, p, y, M, N, K, 0, w)
 
-    def issue_step(s, events=None, cs=None):
-        layer = s["layer"]
-        xq, Yb, ws = layer.act_buffers(M)
-        ops = [lambda: mosaic.mq_hessian_diag(s["Xcal"], layer.H),
-               lambda: mosaic.mq_quantize_weight_delta(s["W"], layer.H, layer.base, None, layer.delta, layer.qws),
-               lambda: mosaic.mq_quantize_act(s["X"], xq),
-               lambda: mosaic.mq_topk_blocks(layer.delta, budget, layer.rank, layer.sel),
-               lambda: mosaic.mq_pack_residual_weight(s["W"], layer.base, layer.sel, budget, layer.packed),
-               lambda: mosaic.mq_gemm(xq, layer.base, layer.packed, Yb, M, N, K, 0, ws)]
-        for j, op in enumerate(ops):
-            if events is not None:
-                events[j].record(cs)
-            op()
-        if events is not None:
-            events[len(ops)].record(cs)
-
-    graphs, pgraphs, evs = [], [], []
-    for i in range(R):
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
-            step(i)
-        graphs.append(g)
-        e = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(len(calls) + 1)]
-        pg = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(pg):
-            issue_step(sets[i], e, torch.cuda.current_stream())
-        pgraphs.append(pg)
-        evs.append(e)
-
-    # the timed steps: a graph of R consecutive steps (input sets 0..R-1) replayed back to
-    # back, as a layer runs inside a model's captured forward, and the single-step graphs
-    # for the remainder; step k always uses input set k % R
+    c0 = mosaic.mq_launch_count()
+    for k in range(R):
+        call(k)
+    launches_per_step = (mosaic.mq_launch_count() - c0) / R
+    torch.cuda.synchronize()
+    # the timed steps: a graph of R consecutive calls (copies 0..R-1) replayed back to back,
+    # and single-call graphs for a remainder; step k always uses copy k % R
     gall = torch.cuda.CUDAGraph()
     with torch.cuda.graph(gall):
-        for i in range(R):
-            step(i)
+        for k in range(R):
+            call(k)
+    singles = []
+    for k in range(R):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            call(k)
+        singles.append(g)
 
     def run_steps(n):
         for _ in range(n // R):
             gall.replay()
         for k in range(n - n % R, n):
-            graphs[k % R].replay()
+            singles[k % R].replay()
 
     sampler = ClockSampler(local)
     sampler.start()
     time.sleep(0.3)
-    warmup_done = max(args.warmup, R)  # every graph replayed once before the timed region
+    warmup_done = max(args.warmup, R)  # every graph replayed before the timed region
     run_steps(warmup_done)
+    for g in singles:
+        g.replay()
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     t_wall0 = time.time()
-    ev0 = torch.cuda.Event(enable_timing=True)
-    ev1 = torch.cuda.Event(enable_timing=True)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     ev0.record(stream)
     run_steps(args.steps)
     ev1.record(stream)
     torch.cuda.synchronize()
     t_wall1 = time.time()
+    # the same steps for one more second, so the SM clock has samples under this load
+    # even when the timed region is shorter than the sampling interval
+    while time.time() - t_wall1 < 1.0:
+        run_steps(R * 50)
+        torch.cuda.synchronize()
+    t_wall2 = time.time()
     if world > 1:
         dist.barrier()
     ms_total = max_over_ranks(ev0.elapsed_time(ev1), world, dev)
-    time.sleep(0.3)
-    sampler.stop()
-    clocks = sampler.summary(t_wall0, t_wall1)
     err = mosaic.mq_get_error()
     if err != 0:
         raise RuntimeError(f"device error word {err}")
-
     ms_step = ms_total / args.steps
-    per_call = step_bytes(M, N, K, T, budget)
-    bytes_step = sum(per_call.values())
-    value = replica_gbs(bytes_step, world, ms_step)
-
-    # per-call device time: each call replayed back to back over the R rotating input sets
-    # (CUDA events around graphs of R launches; programmatic dependent launch hides the
-    # launch latency between them, so this is the kernel's own duration). The same calls
-    # timed inside the step graph (event nodes between calls, which serialise them and
-    # add the launch gap to every call) are reported beside it as in_step_us.
-    prof_reps = min(args.steps, 300)
-    profile_mode = f"isolated (each call replayed back to back, {R} rotating sets)"
-    acc = isolated_profile(sets, calls, M, N, K, budget, prof_reps, stream)
-    in_step = {c: 0.0 for c in calls}
-    try:
-        for r in range(prof_reps):
-            i = r % R
-            pgraphs[i].replay()
-            torch.cuda.synchronize()
-            e = evs[i]
-            for j, c in enumerate(calls):
-                in_step[c] += e[j].elapsed_time(e[j + 1])
-    except RuntimeError:
-        in_step = None
-    peaks = load_peaks()
-    kern = {}
-    for c in calls:
-        us = acc[c] / prof_reps * 1e3
-        gbs = per_call[c] / (us * 1e-6) / 1e9
-        kern[c] = {"us": round(us, 3), "alg_bytes": per_call[c], "gbs": round(gbs, 1),
-                   "frac_hbm": round(gbs / peaks["hbm_gbs"], 4), "traffic": dram_traffic(c),
-                   "in_step_us": None if in_step is None else round(in_step[c] / prof_reps * 1e3, 3)}
-    dom = max(calls, key=lambda c: kern[c]["us"])
-    roofline = {"bound": "hbm", "kernel": dom, "timing": profile_mode, "achieved": kern[dom]["gbs"], "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": kern[dom]["frac_hbm"], "traffic": kern[dom]["traffic"],
-                "peak_source": f"{peaks['source']} (copy bandwidth)"}
+    us = ms_step * 1e3
+    value = replica_gbs(per_call, world, ms_step)
+    clocks = sampler.summary(t_wall0, t_wall2)
+    if clocks:
+        clocks["window"] = "timed region + 1 s of the same steps"
     fl_exec, fl_dense = gemm_flops(M, N, K, budget)
-    g_us = kern["gemm"]["us"]
-    fp4_peak = peaks["bf16_tflops_sustained"] * FP4_PER_BF16
-    gemm = {"us": g_us, "gbs": kern["gemm"]["gbs"], "frac_hbm": kern["gemm"]["frac_hbm"],
-            "tflops_executed": round(fl_exec / (g_us * 1e-6) / 1e12, 2),
-            "tflops_dense_equiv": round(fl_dense / (g_us * 1e-6) / 1e12, 2),
-            "frac_fp4": round(fl_exec / (g_us * 1e-6) / 1e12 / fp4_peak, 5),
-            "fp4_peak_tflops": fp4_peak, "bound": "hbm" if M <= 316 else "tensor"}
+    gbs_rank = per_call / (us * 1e-6) / 1e9
+    fp4_burst = peaks["bf16_tflops"] * FP4_PER_BF16
+    tf = fl_exec / (us * 1e-6) / 1e12
+    gemm = {"us": round(us, 3), "alg_bytes": per_call, "gbs": round(gbs_rank, 1),
+            "frac_hbm": round(gbs_rank / peaks["hbm_gbs"], 4), "tflops_executed": round(tf, 2),
+            "tflops_dense_equiv": round(fl_dense / (us * 1e-6) / 1e12, 2),
+            "frac_fp4_burst": round(tf / fp4_burst, 5), "rotating_copies": R,
+            "kernel": "k_gemm_streamk<16> (decode, stream-K)"}
+    roofline = {"bound": "hbm", "kernel": "gemm (k_gemm_streamk<16>)",
+                "timing": f"CUDA events around {args.steps} back-to-back calls over {R} operand copies",
+                "achieved": round(gbs_rank, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": round(gbs_rank / peaks["hbm_gbs"], 4), "traffic": dram_traffic("gemm"),
+                "peak_source": f"{peaks['source']} (copy bandwidth)"}
+    for g in singles:
+        del g
+    del gall, singles
 
-    # end to end: whole path through mq_run_layer with pinned host buffers
+    # ---- end to end: inference on the prepared layer through mq_run_layer with pinned
+    # host buffers (H2D of X, activation quantizer, GEMM, D2H of Y in every step)
     e2e = None
     if not args.no_e2e:
-        s = sets[0]
-        hb = s["layer"].buffers(M, T, staging=True)
-        Wh, Xh, Ch = W0.pin_memory(), X0.pin_memory(), C0.pin_memory()
+        hb = layer.buffers(M, T, staging=True)
+        Xh = X0.pin_memory()
         Yh = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
         for _ in range(3):
-            mosaic.mq_run_layer(Wh, Xh, Ch, Yh, M, N, K, T, budget, 0, True, hb)
+            mosaic.mq_run_layer(None, Xh, None, Yh, M, N, K, T, budget, mosaic.MQ_LAYER_PREPARED, True, hb)
         torch.cuda.synchronize()
-        ke = max(3, min(args.steps, 50))
+        ke = max(20, min(args.steps, 2000))
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize()
-        a0 = torch.cuda.Event(enable_timing=True)
-        a1 = torch.cuda.Event(enable_timing=True)
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a0.record(stream)
         for _ in range(ke):
-            mosaic.mq_run_layer(Wh, Xh, Ch, Yh, M, N, K, T, budget, 0, True, hb)
+            mosaic.mq_run_layer(None, Xh, None, Yh, M, N, K, T, budget, mosaic.MQ_LAYER_PREPARED, True, hb)
         a1.record(stream)
         torch.cuda.synchronize()
         ms_e = max_over_ranks(a0.elapsed_time(a1) / ke, world, dev)
-        e2e = {"value": replica_gbs(bytes_step, world, ms_e), "unit": "GB/s", "ms_per_step": ms_e,
-               "h2d_bytes_per_step": 2 * N * K + 2 * M * K + 2 * T * K, "d2h_bytes_per_step": 2 * M * N,
-               "steps": ke}
+        e2e = {"value": round(replica_gbs(per_call, world, ms_e), 2), "unit": "GB/s", "ms_per_step": ms_e,
+               "h2d_bytes_per_step": 2 * M * K, "d2h_bytes_per_step": 2 * M * N, "steps": ke,
+               "call": "mq_run_layer(host=1, MQ_LAYER_PREPARED): H2D X, quantize X, GEMM, D2H Y"}
+    del copies, layer
+    torch.cuda.empty_cache()
 
+    path = None
+    if world == 1 and not args.no_path:
+        path = whole_path(dev, args.workload, 6, 600, stream)
+    peak = None
+    if world == 1 and not args.no_fp4_peak:
+        peak = fp4_peak(sampler)
+    sampler.stop()
+    sweep = drows = None
+    if world == 1 and not args.no_sweep:
+        torch.cuda.empty_cache()
+        sweep, drows = gemm_sweep(peaks, peak["tflops"] if peak else None)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(args.workload, M)
-
-    sweep = None
-    if world == 1 and not args.no_sweep:
-        for st in sets:
-            st.clear()
-        sets.clear()
-        graphs.clear()
-        pgraphs.clear()
-        torch.cuda.empty_cache()
-        sweep = gemm_sweep(load_peaks())
+        cpu = cpu_baseline(args.workload)
+    if peak:
+        gemm["frac_fp4_measured"] = round(tf / peak["tflops"], 5)
 
     if world > 1:
-        graphs.clear()
-        pgraphs.clear()
         dist.barrier()
         dist.destroy_process_group()
     if rank != 0:
         return
     line = {"metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
             "warmup": warmup_done, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "nvfp4 (e2m1 x e2m1, e4m3 scales, fp32 accumulate; fp32/fp64 prep)",
+            "vs_baseline": None, "dtype": "nvfp4 (e2m1 x e2m1, e4m3 scales, fp32 accumulate)",
             "data": "synthetic",
-            "config": {"workload": args.workload, "M": M, "N": N, "K": K, "T": T, "budget_frac": 0.10,
+            "config": {"workload": f"{args.workload} fused GEMM", "M": M, "N": N, "K": K, "budget_frac": 0.10,
                        "budget_blocks": budget, "parallelism": f"replicas x{world}",
-                       "l2": f"{R} rotating input sets (~{R * 57} MB touched) > 2x L2; no flush",
-                       "graphs": f"{R} steps per graph replay (one per input set)"},
-            "roofline": roofline, "gemm": gemm, "gemm_vs_M": sweep, "kernels": kern, "cpu_baseline": cpu, "e2e": e2e,
-            "gpu_launches": int(launches_per_step * args.steps), "clocks": clocks}
+                       "l2": f"{R} rotating operand copies ({R * per_call / 1e6:.0f} MB) > 2x L2; no flush",
+                       "graphs": f"{R} calls per graph replay (one per copy)"},
+            "roofline": roofline, "gemm": gemm, "fp4_peak": peak, "gemm_sweep": sweep, "delta_topk": drows,
+            "whole_path": path, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": int(round(launches_per_step * args.steps)), "clocks": clocks}
     print(json.dumps(line), flush=True)
 
 

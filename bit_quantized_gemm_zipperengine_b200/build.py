@@ -28,7 +28,8 @@ def sources():
 
 
 def deps():
-    return sources() + sorted(glob.glob(os.path.join(CSRC, "*.cuh"))) + [os.path.join(INCLUDE, "mosaic.h"), __file__]
+    return (sources() + sorted(glob.glob(os.path.join(CSRC, "*.cuh"))) + sorted(glob.glob(os.path.join(INCLUDE, "*.h")))
+            + [__file__])
 
 
 def stale() -> bool:

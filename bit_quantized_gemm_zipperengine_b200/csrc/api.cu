@@ -1,5 +1,6 @@
 // Host side of libmosaic: argument validation, TMA descriptors and kernel dispatch
 // behind the C ABI declared in mosaic.h.
+#include <algorithm>
 #include <atomic>
 #include <cstdio>
 #include <cstring>
@@ -119,6 +120,11 @@ size_t mq_sf_swz_bytes(int rows, int cols) {
     return (size_t)((rows + 127) / 128) * 128 * (size_t)(cols / 16);
 }
 
+size_t mq_weight_bytes(int N, int K) {
+    if (N <= 0 || K <= 0 || N % 64 || K % 64) return 0;
+    return (size_t)N * (size_t)(K / 2) + mq_sf_swz_bytes(N, K) + 16;
+}
+
 int mq_budget_blocks(int N, int K, double frac) {
     if (N <= 0 || K <= 0 || N % 64 || K % 64 || !(frac >= 0.0 && frac <= 1.0)) return -1;
     const double nb = (double)(N / 64) * (double)(K / 64);
@@ -143,7 +149,9 @@ size_t mq_gemm_workspace_bytes(int M, int N, int K, unsigned flags) {
     bool prefill = M > 128 && N % 256 == 0;
     if (flags & MQ_GEMM_DECODE) prefill = false;
     if (flags & MQ_GEMM_PREFILL) prefill = true;
-    return prefill ? 0 : decode_workspace_bytes(M, N, K);
+    if (prefill) return 0;
+    // mq_gemm's decode kernel (stream-K) and mq_gemm_act's (split-K): the larger of the two
+    return std::max(plan_streamk(M, N, K).ws, decode_workspace_bytes(M, N, K));
 }
 
 mq_status mq_quantize_weight(const mq_bf16* W, int N, int K, mq_nvfp4_mat* base, mq_nvfp4_mat* resid_full,
@@ -290,13 +298,21 @@ static mq_status quantize_act_early(const mq_bf16* X, int M, int K, mq_nvfp4_mat
     return launched(launch_quant_act(X, M, K, xq->codes, xq->sf, xq->sf_swz, xq->gscale, true, as_stream(stream)), 1);
 }
 
+}  // extern "C"
+
+namespace mq {
+
+// The fused GEMM behind mq_gemm and mq_gemm_noalloc: argument checks, kernel choice (the
+// flags, else prefill for M > 128 with N % 256 == 0), parameters, launch.
 // prefetch: the caller guarantees wq and xq were complete before the GEMM could start (the
 // whole-path call's order: the pack before it lets it start only after its own wait, and
 // that wait already implies the activation quantizer and the quantize+Delta pass
 // completed), so the decode kernel may load them before waiting for the pack.
-static mq_status gemm_impl(const mq_nvfp4_mat* xq, const mq_nvfp4_mat* wq, const mq_residual_packed* r, mq_bf16* Y,
-                           int M, int N, int K, unsigned flags, void* ws, size_t ws_bytes, bool prefetch,
-                           mq_stream stream) {
+// clear_counters: zero the workspace's tile counters on the stream before the kernel (a
+// scratch that other calls share and that may hold anything).
+mq_status gemm_dispatch(const mq_nvfp4_mat* xq, const mq_nvfp4_mat* wq, const mq_residual_packed* r, mq_bf16* Y,
+                        int M, int N, int K, unsigned flags, void* ws, size_t ws_bytes, bool prefetch,
+                        bool clear_counters, mq_stream stream) {
     if (!xq || !wq || !Y || M <= 0 || N <= 0 || K <= 0 || N % 64 || K % 64) return MQ_ERR_INVALID_ARG;
     if (N % 128 || K % 256) return MQ_ERR_UNSUPPORTED_SHAPE;
     if (!xq->codes || !xq->sf_swz || !xq->gscale || !wq->codes || !wq->sf_swz || !wq->gscale)
@@ -337,29 +353,38 @@ static mq_status gemm_impl(const mq_nvfp4_mat* xq, const mq_nvfp4_mat* wq, const
     p.K = K;
     p.mode = (flags & MQ_GEMM_BASE_ONLY) ? 1 : (flags & MQ_GEMM_RESIDUAL_ONLY) ? 2 : 0;
     p.prefetch = prefetch ? 1 : 0;
+    p.w_ready = (flags & MQ_GEMM_WEIGHTS_READY) ? 1 : 0;
     CUtensorMap tw, tx;
     if (prefill) {
         if (!make_tmap_bytes(&tw, wq->codes, (uint64_t)K / 2, (uint64_t)N, 128, 256)) return MQ_ERR_CUDA;
         if (!make_tmap_bytes(&tx, xq->codes, (uint64_t)K / 2, (uint64_t)M, 128, 128)) return MQ_ERR_CUDA;
         return launched(launch_gemm_prefill(tw, tx, p, as_stream(stream)), 1);
     }
-    DecodePlan d = plan_decode(M, N, K);
-    const size_t need = decode_workspace_bytes(M, N, K);
+    const StreamKPlan d = plan_streamk(M, N, K);
+    // the kernel splits the units with 32-bit arithmetic (units x grid < 2^32)
+    if ((int64_t)d.units * d.grid >= (int64_t(1) << 32)) return MQ_ERR_UNSUPPORTED_SHAPE;
+    const size_t need = d.ws;
     if (need > 0 && (!ws || ws_bytes < need || !aligned(ws, 16))) return MQ_ERR_WORKSPACE;
     if (!make_tmap_bytes(&tw, wq->codes, (uint64_t)K / 2, (uint64_t)N, 128, 128)) return MQ_ERR_CUDA;
     if (!make_tmap_bytes(&tx, xq->codes, (uint64_t)K / 2, (uint64_t)M, 128, (uint32_t)d.BN)) return MQ_ERR_CUDA;
     if (need > 0) {
-        size_t part = (size_t)d.splits * d.tiles_m * d.BN * N * sizeof(float);  // workspace path only
-        part = (part + 255) & ~size_t(255);
         p.partial = static_cast<float*>(ws);
-        p.counters = reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + part);
+        p.counters = reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + d.slots_bytes);
+        if (clear_counters &&
+            cudaMemsetAsync(p.counters, 0, (size_t)d.tiles_m * d.tiles_n * sizeof(int), as_stream(stream)) !=
+                cudaSuccess)
+            return MQ_ERR_CUDA;
     }
-    return launched(launch_gemm_decode(tw, tx, p, d, as_stream(stream)), 1);
+    return launched(launch_gemm_streamk(tw, tx, p, d, as_stream(stream)), 1);
 }
+
+}  // namespace mq
+
+extern "C" {
 
 mq_status mq_gemm(const mq_nvfp4_mat* xq, const mq_nvfp4_mat* wq, const mq_residual_packed* r, mq_bf16* Y, int M,
                   int N, int K, unsigned flags, void* ws, size_t ws_bytes, mq_stream stream) {
-    return gemm_impl(xq, wq, r, Y, M, N, K, flags, ws, ws_bytes, false, stream);
+    return gemm_dispatch(xq, wq, r, Y, M, N, K, flags, ws, ws_bytes, false, false, stream);
 }
 
 // Decode kernel with the activation quantization inside it (X bf16).
@@ -418,6 +443,31 @@ mq_status mq_gemm_act(const mq_bf16* X, const mq_nvfp4_mat* wq, const mq_residua
 
 mq_status mq_run_layer(const mq_bf16* W, const mq_bf16* X, const mq_bf16* Xcal, mq_bf16* Y, int M, int N, int K,
                        int T, int budget, unsigned flags, int host, mq_layer_buffers* buf, mq_stream stream) {
+    const bool prepared = (flags & MQ_LAYER_PREPARED) != 0;
+    flags &= ~(unsigned)MQ_LAYER_PREPARED;
+    if (prepared) {
+        // inference on a prepared layer: A6 + A7 + A8 (X in, Y out)
+        if (!X || !Y || !buf || M <= 0 || N <= 0 || K <= 0) return MQ_ERR_INVALID_ARG;
+        if (buf->packed.nblk != budget) return MQ_ERR_INVALID_ARG;
+        cudaStream_t s = as_stream(stream);
+        const mq_bf16* x = X;
+        mq_bf16* y = Y;
+        if (host) {
+            if (!buf->X_dev || !buf->Y_dev) return MQ_ERR_INVALID_ARG;
+            if (cudaMemcpyAsync(buf->X_dev, X, (size_t)M * K * 2, cudaMemcpyHostToDevice, s) != cudaSuccess)
+                return MQ_ERR_CUDA;
+            x = buf->X_dev;
+            y = buf->Y_dev;
+        }
+        mq_status st;
+        if ((st = mq_quantize_act(x, M, K, &buf->xq, stream)) != MQ_OK) return st;
+        if ((st = gemm_dispatch(&buf->xq, &buf->base, &buf->packed, y, M, N, K, flags, buf->ws_gemm,
+                                buf->ws_gemm_bytes, false, false, stream)) != MQ_OK)
+            return st;
+        if (host && cudaMemcpyAsync(Y, buf->Y_dev, (size_t)M * N * 2, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+            return MQ_ERR_CUDA;
+        return MQ_OK;
+    }
     if (!W || !X || !Xcal || !Y || !buf || M <= 0 || N <= 0 || K <= 0 || T <= 0) return MQ_ERR_INVALID_ARG;
     cudaStream_t s = as_stream(stream);
     const mq_bf16 *w = W, *x = X, *xc = Xcal;
@@ -470,8 +520,8 @@ mq_status mq_run_layer(const mq_bf16* W, const mq_bf16* X, const mq_bf16* Xcal, 
     if ((st = pack_residual_weight_impl(w, &buf->base, buf->sel, budget, &buf->packed, buf->delta, buf->rank,
                                         stream)) != MQ_OK)
         return st;
-    if ((st = gemm_impl(&buf->xq, &buf->base, &buf->packed, y, M, N, K, flags, buf->ws_gemm, buf->ws_gemm_bytes, true,
-                        stream)) != MQ_OK)
+    if ((st = gemm_dispatch(&buf->xq, &buf->base, &buf->packed, y, M, N, K, flags, buf->ws_gemm, buf->ws_gemm_bytes,
+                            true, false, stream)) != MQ_OK)
         return st;
     if (host && cudaMemcpyAsync(Y, buf->Y_dev, (size_t)M * N * 2, cudaMemcpyDeviceToHost, s) != cudaSuccess)
         return MQ_ERR_CUDA;

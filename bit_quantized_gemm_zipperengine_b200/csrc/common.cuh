@@ -5,6 +5,7 @@
 // (tensor-memory allocation, block-scaled MMA, scale-factor copies, loads).
 #pragma once
 
+#include <atomic>
 #include <cstdint>
 #include <utility>
 #include <cuda.h>
@@ -274,6 +275,21 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
     for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Host: run `set` (kernel attribute calls, which belong to the current device) once per
+// device. `done` is the caller's per-device record. Two threads arriving together both
+// run `set`, which only repeats idempotent calls.
+template <typename F>
+inline cudaError_t once_per_device(std::atomic<bool> (&done)[64], F&& set) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (done[dev].load(std::memory_order_acquire)) return cudaSuccess;
+    e = set();
+    if (e == cudaSuccess) done[dev].store(true, std::memory_order_release);
+    return e;
 }
 
 // Host: launch `kern` with programmatic stream serialization (and a (1, cluster_y, 1)

@@ -23,6 +23,9 @@
 // (GemmParams::prefetch, set by the whole-path call: the pack before the GEMM lets it
 // start only after its own wait, which already implies that both quantizers completed):
 // then the first stages' W and X are requested before the wait.
+#include <algorithm>
+#include <atomic>
+
 #include <cuda_bf16.h>
 
 #include "common.cuh"
@@ -602,6 +605,422 @@ __global__ void __launch_bounds__(192, 1)
     }
 }
 
+// Element i of a small per-stage register array (unrolled select, no local memory).
+template <int N>
+__device__ __forceinline__ int pick(const int (&a)[N], int i) {
+    int v = a[0];
+#pragma unroll
+    for (int j = 1; j < N; ++j)
+        if (i == j) v = a[j];
+    return v;
+}
+template <int N>
+__device__ __forceinline__ void put(int (&a)[N], int i, int v) {
+#pragma unroll
+    for (int j = 0; j < N; ++j)
+        if (i == j) a[j] = v;
+}
+
+// ------------------------------------------------------------------ stream-K decode kernel
+// Small M, HBM-bound: every byte of W must stream through the SMs at the full rate of
+// the memory. The work is a list of units, (output tile, 256-K stage) pairs, tile-major;
+// a grid of one persistent CTA per SM takes equal contiguous ranges of it, so every SM
+// streams the same number of W bytes whatever the tile count. A range cuts a tile into
+// segments; each segment accumulates in its own tensor-memory buffer (two, alternating,
+// so the next segment's MMAs overlap this one's epilogue). A tile held whole by one CTA
+// is scaled and stored at once; the segments of a split tile leave fp32 partials in
+// per-CTA workspace slots, and the CTA that finishes the tile's last segment (a tile
+// counter) adds them in segment order, so the result does not depend on timing.
+// Shared memory: a deep ring of stages (W 128 x 256 K, X BN x 256 K, their scale chunks),
+// 8 stages for BN = 16 (128 KB of W in flight per SM), and a ring of 16 residual-block
+// slots (2048 B codes + 512 B scales each) that a stage's blocks take in order and its
+// release frees. A residual block is one M = 128 MMA over its 64 rows and the 2 KB next
+// to them in the ring (the other half of the 128-row operand), whose scales are zero.
+template <int BN>
+struct SKCfg {
+    static constexpr int kStages = BN <= 16 ? 8 : BN <= 32 ? 7 : BN <= 64 ? 6 : 5;
+    static constexpr int kOffW = 0;                     // 128 rows x 128 B, swizzled
+    static constexpr int kOffX = 16384;                 // BN rows x 128 B, swizzled
+    static constexpr int kOffSFW = kOffX + BN * 128;    // 4 x 512 B
+    static constexpr int kOffSFX = kOffSFW + 2048;      // 4 x 512 B
+    static constexpr int kStageBytes = kOffSFX + 2048;
+    static constexpr int kRSlots = 16;
+    static constexpr int kRSlotBytes = 2560;            // 2048 B codes + 512 B scales
+    static constexpr int kOffRing = kStages * kStageBytes;
+    // 2 KB after the ring: the last slot's lower-half MMA reads 2 KB past its codes
+    static constexpr int kCtrlOff = kOffRing + kRSlots * kRSlotBytes + 2048;
+    static constexpr int kMaxSegs = 160;                 // segments of one tile (<= CTAs)
+    static constexpr int kCtrlBytes = 512 + 4 * kMaxSegs;
+    static constexpr int kSmemBytes = kCtrlOff + kCtrlBytes + 1024;
+    static constexpr int kThreads = 256;
+    static constexpr uint32_t kTmemCols = 512;
+    static constexpr uint32_t kDStride = BN <= 64 ? 64 : 128;        // accumulator buffers
+    static constexpr uint32_t kSfCol0 = 2 * kDStride;                  // stage s: 32 columns
+    static constexpr uint32_t kRSfCol0 = kSfCol0 + kStages * 32;       // ring slot i: 4 columns
+    static_assert(kStageBytes % 1024 == 0, "stage alignment");
+    static_assert(kSmemBytes <= 232448, "shared memory budget");
+    static_assert(kRSfCol0 + kRSlots * 4 <= kTmemCols, "tensor memory budget");
+};
+
+// CTA holding unit u when `units` are split into `grid` equal contiguous ranges, and the
+// first unit of CTA c (units * grid < 2^32, checked on the host: 32-bit arithmetic).
+__device__ __forceinline__ uint32_t sk_owner(uint32_t u, uint32_t units, uint32_t grid) {
+    return ((u + 1) * grid - 1) / units;
+}
+__device__ __forceinline__ uint32_t sk_start(uint32_t c, uint32_t units, uint32_t grid) { return c * units / grid; }
+
+// Atomic add with acquire-release semantics at GPU scope: the CTA's partial stores that a
+// barrier ordered before it are released with it, and the partials other CTAs released
+// before their own increments are acquired.
+__device__ __forceinline__ int atom_add_acq_rel_gpu(int* ptr, int v) {
+    int old;
+    asm volatile("atom.add.acq_rel.gpu.s32 %0, [%1], %2;" : "=r"(old) : "l"(ptr), "r"(v) : "memory");
+    return old;
+}
+
+// Does block row pair (n_tile) carry a selected residual block in stages [ks_a, ks_b)?
+__device__ __forceinline__ bool resid_in_range(const GemmParams& p, int n_tile, int ks_a, int ks_b) {
+    if (!p.has_resid) return false;
+    const int KB = p.K / 64, KW = (KB + 31) / 32;
+    for (int h = 0; h < 2; ++h) {
+        const uint32_t* row = p.bitmap + (int64_t)(n_tile * 2 + h) * KW;
+        for (int kt = ks_a * 4; kt < ks_b * 4; kt += 4)
+            if ((__ldg(row + (kt >> 5)) >> (kt & 31)) & 15u) return true;
+    }
+    return false;
+}
+
+template <int BN>
+__global__ void __launch_bounds__(256, 1)
+    k_gemm_streamk(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
+                   const GemmParams p) {
+    using C = SKCfg<BN>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kCtrlOff);  // W, X and scales landed
+    uint64_t* rfull = full + C::kStages;                                // residual blocks landed
+    uint64_t* empty = rfull + C::kStages;                               // stage and its ring slots consumed
+    uint64_t* accf = empty + C::kStages;                                // [2] accumulator complete
+    uint64_t* acce = accf + 2;                                          // [2] accumulator read out
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(acce + 2);
+    uint32_t* rmask = tmem_holder + 1;  // [kStages]: bit 2 * kk + h
+    int* s_last = reinterpret_cast<int*>(rmask + C::kStages);
+    int* s_slot = s_last + 1;  // [kMaxSegs]: workspace slot of each segment of the tile being added
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int KS = p.K / 256, KS64 = p.K / 64;
+    const uint32_t U = (uint32_t)p.units, G = gridDim.x;
+    const uint32_t u0 = sk_start(blockIdx.x, U, G), u1 = sk_start(blockIdx.x + 1, U, G);
+    const int nu = (int)(u1 - u0);
+    const bool dense = p.mode != 2;
+    const bool resid = p.has_resid && p.mode != 1;
+
+    if (warp == 0 && lane == 0) {
+        for (int s = 0; s < C::kStages; ++s) {
+            mbar_init(&full[s], 2);  // the W producer's and the X producer's arrivals
+            mbar_init(&rfull[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&accf[b], 1);
+            mbar_init(&acce[b], 4);
+        }
+        mbar_fence_init();
+        tma_prefetch_desc(&tmap_w);
+        tma_prefetch_desc(&tmap_x);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_holder, C::kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+    const uint32_t sbase = smem_u32(smem);
+
+    // Three producer warps keep the copies of a unit off one another's path: the W stream
+    // (the bytes that bound the kernel) never waits for an index lookup or a residual copy.
+    if (warp == 0) {
+        // ---------------------------------------------------- W producer
+        // W may be requested before the wait for the preceding kernel when no running kernel
+        // can still write it (the caller's weights-ready guarantee, or the whole-path order)
+        if (!(p.prefetch || p.w_ready)) griddep_wait();
+        int issued = 0;
+        int t = (int)(u0 / (uint32_t)KS), ks = (int)(u0 % (uint32_t)KS);
+        for (int i = 0; i < nu; ++i, ks = ks + 1 == KS ? 0 : ks + 1, t += ks == 0) {
+            const int s = i % C::kStages;
+            if (i >= C::kStages && !mbar_wait_warp(&empty[s], (uint32_t)(((i / C::kStages) - 1) & 1))) break;
+            if (elect_one()) {
+                uint8_t* st = smem + s * C::kStageBytes;
+                const int n_tile = t / p.tiles_m;
+                mbar_arrive_expect_tx(&full[s], dense ? 16384 + 2048 : 0);
+                if (dense) {
+                    tma_load_2d(st + C::kOffW, &tmap_w, &full[s], ks * 128, n_tile * 128);
+                    bulk_load(st + C::kOffSFW, p.w_sf + ((int64_t)n_tile * KS64 + ks * 4) * 512, 2048, &full[s]);
+                }
+            }
+            __syncwarp();
+            issued = i + 1;
+        }
+        // Do not leave while copies into this CTA's shared memory are in flight.
+        for (int v = issued > C::kStages ? issued - C::kStages : 0; v < issued; ++v)
+            mbar_wait_warp(&full[v % C::kStages], (uint32_t)((v / C::kStages) & 1));
+    } else if (warp == 2) {
+        // ---------------------------------------------------- X producer
+        if (!p.prefetch) griddep_wait();
+        griddep_launch();
+        int issued = 0;
+        int t = (int)(u0 / (uint32_t)KS), ks = (int)(u0 % (uint32_t)KS);
+        for (int i = 0; i < nu; ++i, ks = ks + 1 == KS ? 0 : ks + 1, t += ks == 0) {
+            const int s = i % C::kStages;
+            if (i >= C::kStages && !mbar_wait_warp(&empty[s], (uint32_t)(((i / C::kStages) - 1) & 1))) break;
+            if (elect_one()) {
+                uint8_t* st = smem + s * C::kStageBytes;
+                const int m_tile = t % p.tiles_m;
+                mbar_arrive_expect_tx(&full[s], BN * 128 + 2048);
+                tma_load_2d(st + C::kOffX, &tmap_x, &full[s], ks * 128, m_tile * BN);
+                bulk_load(st + C::kOffSFX, p.x_sf + ((int64_t)(m_tile * BN / 128) * KS64 + ks * 4) * 512, 2048,
+                          &full[s]);
+            }
+            __syncwarp();
+            issued = i + 1;
+        }
+        for (int v = issued > C::kStages ? issued - C::kStages : 0; v < issued; ++v)
+            mbar_wait_warp(&full[v % C::kStages], (uint32_t)((v / C::kStages) & 1));
+    } else if (warp == 3) {
+        // ---------------------------------------------------- residual producer
+        if (!(p.prefetch || p.w_ready)) griddep_wait();
+        int nres = 0;               // units whose residual copies are issued
+        int rc = 0, rdone = 0;      // residual blocks issued / known consumed
+        int ends[C::kStages] = {};  // rc after the latest unit held by each stage
+        RowCursor cur0, cur1;
+        int cur_t = -1;
+        bool ok = true;
+        int t = (int)(u0 / (uint32_t)KS), ks = (int)(u0 % (uint32_t)KS);
+        for (int i = 0; i < nu && ok; ++i, ks = ks + 1 == KS ? 0 : ks + 1, t += ks == 0) {
+            const int s = i % C::kStages;
+            // residual blocks of the unit: both 64-row block rows of the tile, 4 block columns
+            uint32_t m = 0;
+            int idx0[4] = {0, 0, 0, 0}, idx1[4] = {0, 0, 0, 0};
+            if (resid) {
+                const int n_tile = t / p.tiles_m;
+                if (t != cur_t) {
+                    cur0 = row_cursor(p, n_tile * 2 + 0, ks * 4);
+                    cur1 = row_cursor(p, n_tile * 2 + 1, ks * 4);
+                    cur_t = t;
+                }
+                const uint32_t m0b = row_step(cur0, ks * 4, idx0);
+                const uint32_t m1b = row_step(cur1, ks * 4, idx1);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    m |= (((m0b >> kk) & 1u) << (2 * kk)) | (((m1b >> kk) & 1u) << (2 * kk + 1));
+            }
+            if (i >= C::kStages) {  // the stage's mask and barrier phase are free again
+                if (!mbar_wait_warp(&empty[s], (uint32_t)(((i / C::kStages) - 1) & 1))) { ok = false; break; }
+                rdone = max(rdone, pick(ends, s));
+            }
+            const int n = __popc(m);
+            // ring slots [rc, rc + n) must be free: wait for younger units until they are
+            for (int v = i - C::kStages + 1; rc + n - C::kRSlots > rdone && v < i && ok; ++v) {
+                if (v < 0) continue;
+                ok = mbar_wait_warp(&empty[v % C::kStages], (uint32_t)((v / C::kStages) & 1));
+                rdone = max(rdone, pick(ends, v % C::kStages));
+            }
+            if (!ok) break;
+            if (elect_one()) {
+                rmask[s] = m;
+                mbar_arrive_expect_tx(&rfull[s], n * C::kRSlotBytes);
+                int r = rc;
+                for (uint32_t mm = m; mm; mm &= mm - 1, ++r) {
+                    const int j = __ffs(mm) - 1, kk = j >> 1, h = j & 1;
+                    int bi = 0;
+#pragma unroll
+                    for (int a = 0; a < 4; ++a)
+                        if (a == kk) bi = h ? idx1[a] : idx0[a];
+                    const uint32_t slot = sbase + C::kOffRing + (r % C::kRSlots) * C::kRSlotBytes;
+                    bulk_load_s(slot, p.blk_codes + (int64_t)bi * 2048, 2048, &rfull[s]);
+                    bulk_load_s(slot + 2048, p.blk_sf + (int64_t)bi * 512, 512, &rfull[s]);
+                }
+            }
+            __syncwarp();
+            ++nres;
+            rc += n;
+            put(ends, s, rc);
+        }
+        for (int v = nres > C::kStages ? nres - C::kStages : 0; v < nres; ++v)
+            mbar_wait_warp(&rfull[v % C::kStages], (uint32_t)((v / C::kStages) & 1));
+    } else if (warp == 1) {
+        // ---------------------------------------------------- MMA issuer
+        constexpr uint32_t idesc = idesc_mxf4nvf4(128, BN);
+        int rc = 0, seg = 0;
+        uint32_t acc = 0;
+        bool ok = true;
+        int ks = (int)(u0 % (uint32_t)KS);
+        for (int i = 0; i < nu && ok; ++i, ks = ks + 1 == KS ? 0 : ks + 1) {
+            const int s = i % C::kStages;
+            const uint32_t par = (uint32_t)((i / C::kStages) & 1);
+            const uint32_t d = tmem + (uint32_t)(seg & 1) * C::kDStride;
+            if (i == 0 || ks == 0) {  // a segment starts: its accumulator buffer must be free
+                if (!mbar_wait_warp(&acce[seg & 1], (uint32_t)(((seg >> 1) & 1) ^ 1))) break;
+                tc_fence_after();
+                acc = 0;
+            }
+            if (!mbar_wait_warp(&full[s], par)) break;
+            tc_fence_after();
+            const uint32_t st = sbase + s * C::kStageBytes;
+            const uint32_t sfc = tmem + C::kSfCol0 + s * 32;
+            if (elect_one()) {
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+                    if (dense) tc_cp_sf_chunk(sfc + 4 * kk, smem_desc(st + C::kOffSFW + kk * 512, 0, 128, 0));
+                    tc_cp_sf_chunk(sfc + 16 + 4 * kk, smem_desc(st + C::kOffSFX + kk * 512, 0, 128, 0));
+                }
+                if (dense) {
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_mxf4nvf4(d, smem_desc(st + C::kOffW + 32 * kk, 16, 1024, 2),
+                                     smem_desc(st + C::kOffX + 32 * kk, 16, 1024, 2), idesc, sfc + 4 * kk,
+                                     sfc + 16 + 4 * kk, (acc | kk) != 0);
+                    acc = 1;
+                }
+            }
+            __syncwarp();
+            acc = __shfl_sync(0xffffffffu, acc, 0);
+            if (!mbar_wait_warp(&rfull[s], par)) break;
+            tc_fence_after();
+            const uint32_t m = resid ? rmask[s] : 0u;
+            if (elect_one()) {
+                int r = rc;
+                for (uint32_t mm = m; mm; mm &= mm - 1, ++r) {
+                    const int j = __ffs(mm) - 1, kk = j >> 1, h = j & 1;
+                    const int slot_i = r % C::kRSlots;
+                    const uint32_t slot = sbase + C::kOffRing + slot_i * C::kRSlotBytes;
+                    const uint32_t rsf = tmem + C::kRSfCol0 + 4 * slot_i;
+                    tc_cp_sf_chunk(rsf, smem_desc(slot + 2048, 0, 128, 0));
+                    // the block's 64 rows are half h of a 128-row operand; the other half
+                    // (2 KB of the ring next to it) has zero scales
+                    mma_mxf4nvf4(d, smem_desc(slot - 2048 * h, 128, 256, 0),
+                                 smem_desc(st + C::kOffX + 32 * kk, 16, 1024, 2), idesc, rsf, sfc + 16 + 4 * kk,
+                                 acc);
+                    acc = 1;
+                }
+                tc_commit(&empty[s]);
+            }
+            __syncwarp();
+            acc = __shfl_sync(0xffffffffu, acc, 0);
+            rc += __popc(m);
+            if (i == nu - 1 || ks == KS - 1) {  // the segment ends
+                if (elect_one()) tc_commit(&accf[seg & 1]);
+                __syncwarp();
+                ++seg;
+            }
+        }
+    } else {
+        // ---------------------------------------------------- epilogue (warps 4..7)
+        const int q = warp & 3, row = 32 * q + lane;
+        griddep_wait();  // g_x, Y and the workspace follow the previous kernel
+        const float gw = __ldg(p.g_w);
+        const int tq = threadIdx.x - 128;
+        const uint32_t t_first = u0 / (uint32_t)KS, t_last = (u1 - 1) / (uint32_t)KS;
+        int seg = 0;
+        for (uint32_t t = t_first; t <= t_last; ++t, ++seg) {
+            const int n_tile = (int)t / p.tiles_m, m_tile = (int)t % p.tiles_m;
+            const uint32_t ta = t * (uint32_t)KS, tb = ta + (uint32_t)KS;  // the tile's units
+            const uint32_t sa = max(ta, u0), sb = min(tb, u1);              // this segment's units
+            const bool waited = mbar_wait_warp(&accf[seg & 1], (uint32_t)((seg >> 1) & 1));
+            tc_fence_after();
+            const bool have = waited && (dense || resid_in_range(p, n_tile, (int)(sa - ta), (int)(sb - ta)));
+            float acc[BN];
+#pragma unroll
+            for (int c0 = 0; c0 < BN; c0 += 16) {
+                if (have) {
+                    tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(seg & 1) * C::kDStride + c0, acc + c0);
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) acc[c0 + j] = 0.0f;
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acce[seg & 1]);  // the buffer is free for segment seg + 2
+            if (!waited) break;
+            const int m0 = m_tile * BN;
+            const int n = n_tile * 128 + row;
+            const int c_lo = (int)sk_owner(ta, U, G), c_hi = (int)sk_owner(tb - 1, U, G);
+            if (c_lo == c_hi) {
+                // the whole tile is this CTA's: scale and store
+#pragma unroll
+                for (int j = 0; j < BN; ++j) {
+                    const int mm = m0 + j;
+                    if (mm < p.M) {
+                        const float sc = __fmul_rn(__ldg(p.g_x + mm), gw);
+                        const __nv_bfloat16 y = __float2bfloat16_rn(__fmul_rn(acc[j], sc));
+                        p.Y[(int64_t)mm * p.N + n] = *reinterpret_cast<const uint16_t*>(&y);
+                    }
+                }
+                continue;
+            }
+            // a split tile: partial into this CTA's slot (first tile of its range: slot 2c,
+            // last: 2c + 1), then the tile's last finisher adds every segment in order
+            float* mine = p.partial + (size_t)(2 * blockIdx.x + (t == t_first ? 0 : 1)) * (BN * 128);
+#pragma unroll
+            for (int j = 0; j < BN; ++j) __stcg(mine + j * 128 + row, acc[j]);
+            asm volatile("bar.sync 1, 128;" ::: "memory");  // every partial store before the release
+            int* ctr = p.counters + t;
+            if (tq == 0) *s_last = (atom_add_acq_rel_gpu(ctr, 1) == c_hi - c_lo);
+            asm volatile("bar.sync 1, 128;" ::: "memory");  // the acquire before every load below
+            if (!*s_last) continue;
+            const int nseg = c_hi - c_lo + 1;
+            for (int g = tq; g < nseg; g += 128) {
+                const uint32_t c = (uint32_t)(c_lo + g);
+                s_slot[g] = 2 * (int)c + (sk_start(c, U, G) / (uint32_t)KS == t ? 0 : 1);
+            }
+            asm volatile("bar.sync 1, 128;" ::: "memory");
+            // 16 tokens at a time; the partials of up to 4 segments requested together, then
+            // added in segment order
+#pragma unroll 1
+            for (int j0 = 0; j0 < BN && m0 + j0 < p.M; j0 += 16) {
+                float sum[16];
+#pragma unroll 1
+                for (int g0 = 0; g0 < nseg; g0 += 4) {
+                    float v[4][16];
+#pragma unroll
+                    for (int gg = 0; gg < 4; ++gg) {
+                        if (g0 + gg < nseg) {
+                            const float* src = p.partial + (size_t)s_slot[g0 + gg] * (BN * 128) + j0 * 128 + row;
+#pragma unroll
+                            for (int jj = 0; jj < 16; ++jj) v[gg][jj] = __ldcg(src + jj * 128);
+                        }
+                    }
+#pragma unroll
+                    for (int gg = 0; gg < 4; ++gg) {
+                        if (g0 + gg < nseg) {
+#pragma unroll
+                            for (int jj = 0; jj < 16; ++jj) sum[jj] = g0 + gg ? __fadd_rn(sum[jj], v[gg][jj]) : v[gg][jj];
+                        }
+                    }
+                }
+#pragma unroll
+                for (int jj = 0; jj < 16; ++jj) {
+                    const int mm = m0 + j0 + jj;
+                    if (mm < p.M) {
+                        const float sc = __fmul_rn(__ldg(p.g_x + mm), gw);
+                        const __nv_bfloat16 y = __float2bfloat16_rn(__fmul_rn(sum[jj], sc));
+                        p.Y[(int64_t)mm * p.N + n] = *reinterpret_cast<const uint16_t*>(&y);
+                    }
+                }
+            }
+            if (tq == 0) *ctr = 0;
+        }
+    }
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::kTmemCols);
+    }
+}
+
 // ------------------------------------------------------------------ prefill kernel
 // Large M: the tokens are the MMA's M side (128 per tile, A = X) and the weight its N
 // side (256 rows per tile, B = W), K = 256 per pipeline stage. CTAs are persistent and
@@ -650,22 +1069,6 @@ __device__ __forceinline__ uint32_t prefill_tile_slices(const GemmParams& p, int
     for (int h = 0; h < 4; ++h)
         if (__ldg(p.tile_ptr + n_tile * 4 + h + 1) > __ldg(p.tile_ptr + n_tile * 4 + h)) m |= 1u << h;
     return m;
-}
-
-// Element i of a small per-stage register array (unrolled select, no local memory).
-template <int N>
-__device__ __forceinline__ int pick(const int (&a)[N], int i) {
-    int v = a[0];
-#pragma unroll
-    for (int j = 1; j < N; ++j)
-        if (i == j) v = a[j];
-    return v;
-}
-template <int N>
-__device__ __forceinline__ void put(int (&a)[N], int i, int v) {
-#pragma unroll
-    for (int j = 0; j < N; ++j)
-        if (i == j) a[j] = v;
 }
 
 __global__ void __launch_bounds__(320, 1)
@@ -930,13 +1333,11 @@ template <int BN>
 static cudaError_t launch_decode_bn(const CUtensorMap& tw, const CUtensorMap& tx, const GemmParams& p,
                                    const DecodePlan& d, cudaStream_t s) {
     using C = DecodeCfg<BN>;
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(k_gemm_decode<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             C::kSmemBytes);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
+    static std::atomic<bool> attr_set[64];
+    cudaError_t e = once_per_device(attr_set, [] {
+        return cudaFuncSetAttribute(k_gemm_decode<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    });
+    if (e != cudaSuccess) return e;
     dim3 grid(d.tiles_n, d.splits, d.tiles_m);
     return launch_pdl(k_gemm_decode<BN>, grid, dim3(C::kThreads), C::kSmemBytes, s, d.cluster ? d.splits : 1, tw, tx,
                       p);
@@ -955,19 +1356,72 @@ cudaError_t launch_gemm_decode(const CUtensorMap& tw, const CUtensorMap& tx, Gem
     }
 }
 
+static int device_sms() {
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) !=
+                                                   cudaSuccess || sms <= 0) {
+        cudaGetLastError();
+        return 148;
+    }
+    return sms;
+}
+
+StreamKPlan plan_streamk(int M, int N, int K) {
+    StreamKPlan d;
+    d.BN = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : 128;
+    d.tiles_m = (M + d.BN - 1) / d.BN;
+    d.tiles_n = N / 128;
+    const int KS = K / 256;
+    const int64_t tiles = (int64_t)d.tiles_m * d.tiles_n;
+    const int64_t units = tiles * KS;
+    d.units = (int)units;
+    d.grid = (int)std::min<int64_t>(units, device_sms());
+    // a tile is split when its first and last units belong to different CTAs
+    bool split = false;
+    auto owner = [&](int64_t u) { return ((u + 1) * d.grid - 1) / units; };
+    for (int64_t t = 0; t < tiles && !split; ++t) split = owner(t * KS) != owner((t + 1) * KS - 1);
+    d.slots_bytes = split ? (((size_t)2 * d.grid * d.BN * 128 * sizeof(float) + 255) & ~size_t(255)) : 0;
+    d.ws = split ? d.slots_bytes + (size_t)tiles * sizeof(int) : 0;
+    return d;
+}
+
+template <int BN>
+static cudaError_t launch_streamk_bn(const CUtensorMap& tw, const CUtensorMap& tx, const GemmParams& p,
+                                     const StreamKPlan& d, cudaStream_t s) {
+    using C = SKCfg<BN>;
+    static std::atomic<bool> attr_set[64];
+    cudaError_t e = once_per_device(attr_set, [] {
+        return cudaFuncSetAttribute(k_gemm_streamk<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    });
+    if (e != cudaSuccess) return e;
+    return launch_pdl(k_gemm_streamk<BN>, dim3(d.grid), dim3(C::kThreads), C::kSmemBytes, s, 1, tw, tx, p);
+}
+
+cudaError_t launch_gemm_streamk(const CUtensorMap& tw, const CUtensorMap& tx, GemmParams p, const StreamKPlan& d,
+                                cudaStream_t s) {
+    p.units = d.units;
+    p.tiles_m = d.tiles_m;
+    p.tiles_n = d.tiles_n;
+    switch (d.BN) {
+        case 16: return launch_streamk_bn<16>(tw, tx, p, d, s);
+        case 32: return launch_streamk_bn<32>(tw, tx, p, d, s);
+        case 64: return launch_streamk_bn<64>(tw, tx, p, d, s);
+        default: return launch_streamk_bn<128>(tw, tx, p, d, s);
+    }
+}
+
 // Device address of the error word (for kernels of other translation units).
 cudaError_t error_word(int** ptr) { return cudaGetSymbolAddress(reinterpret_cast<void**>(ptr), g_error); }
 
 cudaError_t launch_gemm_prefill(const CUtensorMap& tw, const CUtensorMap& tx, const GemmParams& p, cudaStream_t s) {
-    static bool attr_set[64] = {};
+    static std::atomic<bool> attr_set[64];
+    cudaError_t e = once_per_device(attr_set, [] {
+        return cudaFuncSetAttribute(k_gemm_prefill, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    PrefillCfg::kSmemBytes);
+    });
+    if (e != cudaSuccess) return e;
     int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(k_gemm_prefill, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             PrefillCfg::kSmemBytes);
-        if (e != cudaSuccess) return e;
-        attr_set[dev] = true;
-    }
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
     int sms = 148;
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int ntiles = ((p.M + 127) / 128) * (p.N / 256);

@@ -6,6 +6,8 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include "mosaic.h"
+
 namespace mq {
 
 struct GemmParams {
@@ -27,10 +29,28 @@ struct GemmParams {
     int cluster;             // split-K reduced through the cluster's shared memory
     int prefetch;            // W and X were complete before this kernel could start, so the
                              // decode kernel may load them before waiting for its predecessor
+    int w_ready;             // W, its scales and the packed residual were complete before this
+                             // kernel could start (X may not be): W may be loaded before the wait
     const uint16_t* x_bf16;  // decode kernel: bf16 X [M][K] quantized inside the kernel
                              // (x_sf and g_x unused), or null
     float* gx_out;           // with x_bf16: per-token scales written here if not null
+    // stream-K decode kernel: `units` = tiles x (K / 256) work units, CTA c takes units
+    // [c * units / grid, (c + 1) * units / grid); tile t = n_tile * tiles_m + m_tile
+    int units, tiles_m, tiles_n;
 };
+
+// Stream-K decode kernel plan: token tile BN (the MMA's N side), tiles_n x tiles_m
+// output tiles of 128 weight rows x BN tokens, `grid` persistent CTAs sharing the
+// tiles x (K / 256) units equally; `ws` workspace bytes (0 when no tile is split).
+struct StreamKPlan {
+    int BN, tiles_m, tiles_n, units, grid;
+    size_t ws;
+    size_t slots_bytes;  // partial slots before the tile counters
+};
+
+StreamKPlan plan_streamk(int M, int N, int K);
+cudaError_t launch_gemm_streamk(const CUtensorMap& tw, const CUtensorMap& tx, GemmParams p, const StreamKPlan& d,
+                                cudaStream_t s);
 
 // Decode kernel tiling: token tile BN, grid tiles_n x splits x tiles_m, `iters`
 // K stages (256 elements each) per split.
@@ -45,6 +65,11 @@ cudaError_t launch_gemm_decode(const CUtensorMap& tw, const CUtensorMap& tx, Gem
                                cudaStream_t s);
 cudaError_t launch_gemm_prefill(const CUtensorMap& tw, const CUtensorMap& tx, const GemmParams& p, cudaStream_t s);
 cudaError_t read_clear_error(int* value);
+
+// The fused GEMM's host side (api.cu), shared by mq_gemm and mq_gemm_noalloc.
+mq_status gemm_dispatch(const mq_nvfp4_mat* xq, const mq_nvfp4_mat* wq, const mq_residual_packed* r, mq_bf16* Y,
+                        int M, int N, int K, unsigned flags, void* ws, size_t ws_bytes, bool prefetch,
+                        bool clear_counters, mq_stream stream);
 cudaError_t error_word(int** ptr);
 
 }  // namespace mq

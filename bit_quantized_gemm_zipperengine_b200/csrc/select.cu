@@ -19,8 +19,8 @@ namespace mq {
 // pairs, and at the end lanes 2c and 2c+1 hold column c of the group. e and e' are
 // recomputed from W and the tensor scale with the weight quantizer's arithmetic, so they
 // are bit-identical to the stored codes.
-// tau = fma(e, e, -fp32(e'^2)) (fp32); the column sums are widened to fp64 for
-// p_k = H_k c_k and the 64-column tree.
+// tau = fp64(e)^2 - fp64(e')^2 (both squares exact in fp64, one rounding), the row tree,
+// p_k = H_k c_k and the 64-column tree all in fp64.
 // Codes and scales are gathered in shared memory and written as whole 32-byte sectors:
 // a strip's 128 rows x 32 bytes of codes, and its 512-byte chunk of the GEMM's tiled scale
 // layout (one 128-row tile x 4 groups) at once.
@@ -63,7 +63,7 @@ __device__ __forceinline__ void quant_delta_strip(const uint8_t* tile, uint8_t* 
     const int KB = K / 64;
     const float g6 = __fmul_rn(6.0f, g);
     double* pcol = reinterpret_cast<double*>(st + kQDOffP) + blk * 64;
-    float v[16];
+    double v[16];
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
         const int rl = blk * 64 + lane + 32 * h;  // strip row
@@ -84,16 +84,13 @@ __device__ __forceinline__ void quant_delta_strip(const uint8_t* tile, uint8_t* 
             *reinterpret_cast<uint2*>(st + kQDOffRC + rl * 32 + q * 8) = make_uint2(rlo, rhi);
             st[kQDOffRSl + rl * 4 + q] = (uint8_t)rsb;
         }
-        // tau = fma(e, e, -fp32(e'^2)) with e = R, e' = R - deqR; the squares of e' are
-        // taken in pairs
+        // tau = fp64(e)^2 - fp64(e')^2 with e = R, e' = R - deqR: e'^2 is exact in fp64, so
+        // the fused multiply-add rounds only the difference, as e*e - e'*e' does
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const float e0 = R[2 * j], e1 = R[2 * j + 1];
-            const float f0 = __fsub_rn(e0, rdeq[2 * j]), f1 = __fsub_rn(e1, rdeq[2 * j + 1]);
-            const float2 sq = mul2(make_float2(f0, f1), make_float2(f0, f1));
-            const float t0 = __fmaf_rn(e0, e0, -sq.x), t1 = __fmaf_rn(e1, e1, -sq.y);
-            v[2 * j] = h ? __fadd_rn(v[2 * j], t0) : t0;
-            v[2 * j + 1] = h ? __fadd_rn(v[2 * j + 1], t1) : t1;
+        for (int j = 0; j < 16; ++j) {
+            const double e = (double)R[j], f = (double)__fsub_rn(R[j], rdeq[j]);
+            const double t = __fma_rn(e, e, -__dmul_rn(f, f));
+            v[j] = h ? __dadd_rn(v[j], t) : t;
         }
     }
     // butterfly: masks 16, 8, 4, 2 keep n = 8, 4, 2, 1 columns; then mask 1 adds pairs
@@ -102,14 +99,14 @@ __device__ __forceinline__ void quant_delta_strip(const uint8_t* tile, uint8_t* 
         const bool upper = (lane & m) != 0;
 #pragma unroll
         for (int j = 0; j < n; ++j) {
-            const float send = upper ? v[j] : v[j + n];
-            const float keep = upper ? v[j + n] : v[j];
-            v[j] = __fadd_rn(keep, __shfl_xor_sync(0xffffffffu, send, m));
+            const double send = upper ? v[j] : v[j + n];
+            const double keep = upper ? v[j + n] : v[j];
+            v[j] = __dadd_rn(keep, __shfl_xor_sync(0xffffffffu, send, m));
         }
     }
-    const float colsum = __fadd_rn(v[0], __shfl_xor_sync(0xffffffffu, v[0], 1));
+    const double colsum = __dadd_rn(v[0], __shfl_xor_sync(0xffffffffu, v[0], 1));
     const int c = (lane >> 1) & 15;
-    if ((lane & 1) == 0) pcol[q * 16 + c] = __dmul_rn((double)__ldg(H + kt * 64 + q * 16 + c), (double)colsum);
+    if ((lane & 1) == 0) pcol[q * 16 + c] = __dmul_rn((double)__ldg(H + kt * 64 + q * 16 + c), colsum);
     __syncthreads();
     const int nt = 2 * si + blk;
     if (q == 0 && nt < nblk_rows) {  // warps 0 and 4: the 64-column tree of their block
@@ -688,15 +685,21 @@ __global__ void __launch_bounds__(128) k_pack_w(const uint16_t* __restrict__ W, 
 
 // ------------------------------------------------------------------ launchers
 static int quant_delta_grid(int nstrips) {
-    static int per_sm = 0;
-    if (!per_sm) {
+    static std::atomic<bool> attr_set[64];
+    static std::atomic<int> per_sm_cache{0};
+    once_per_device(attr_set, [] {
         cudaFuncSetAttribute(k_quant_delta<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kQDSmem);
         cudaFuncSetAttribute(k_quant_delta<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kQDSmem);
-        cudaFuncSetAttribute(k_quant_delta<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kQDSmem);
+        return cudaFuncSetAttribute(k_quant_delta<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)kQDSmem);
+    });
+    int per_sm = per_sm_cache.load(std::memory_order_relaxed);
+    if (!per_sm) {
         if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_quant_delta<true, true>, kQDThreads, kQDSmem) !=
                 cudaSuccess ||
             per_sm < 1)
             per_sm = 2;
+        per_sm_cache.store(per_sm, std::memory_order_relaxed);
     }
     int sms = 148;
     int dev = 0;
@@ -740,17 +743,17 @@ cudaError_t launch_topk_select(const double* delta, int B, int budget, int32_t* 
     if (budget <= 0) return cudaSuccess;
     const bool smem_keys = (size_t)B * 8 <= kSelSmemKeysMax;
     const size_t smem = smem_keys ? (size_t)B * 8 : 0;
-    static bool attr[2] = {false, false};
-    auto go = [&](auto kern, int which) -> cudaError_t {
-        if (!attr[which]) {
-            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 (int)kSelSmemKeysMax + 16 * 1024);
-            if (e != cudaSuccess) return e;
-            attr[which] = true;
-        }
-        return launch_pdl(kern, dim3(1), dim3(kSelThreads), smem, s, 1, delta, B, budget, sel);
-    };
-    return smem_keys ? go(k_topk_large<true>, 0) : go(k_topk_large<false>, 1);
+    static std::atomic<bool> attr_set[64];
+    cudaError_t e = once_per_device(attr_set, [] {
+        const cudaError_t e1 = cudaFuncSetAttribute(k_topk_large<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                    (int)kSelSmemKeysMax + 16 * 1024);
+        if (e1 != cudaSuccess) return e1;
+        return cudaFuncSetAttribute(k_topk_large<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)kSelSmemKeysMax + 16 * 1024);
+    });
+    if (e != cudaSuccess) return e;
+    if (smem_keys) return launch_pdl(k_topk_large<true>, dim3(1), dim3(kSelThreads), smem, s, 1, delta, B, budget, sel);
+    return launch_pdl(k_topk_large<false>, dim3(1), dim3(kSelThreads), smem, s, 1, delta, B, budget, sel);
 }
 
 cudaError_t launch_topk(const double* delta, int B, int budget, int32_t* rank, int32_t* sel, cudaStream_t s) {

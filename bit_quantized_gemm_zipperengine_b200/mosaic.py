@@ -21,13 +21,15 @@ MQ_GEMM_DECODE = 1
 MQ_GEMM_PREFILL = 2
 MQ_GEMM_BASE_ONLY = 4
 MQ_GEMM_RESIDUAL_ONLY = 8
+MQ_LAYER_PREPARED = 16
+MQ_GEMM_WEIGHTS_READY = 32
 
 EXPORTED = (
     "mq_sf_swz_bytes", "mq_budget_blocks", "mq_quantize_weight_workspace_bytes", "mq_delta_topk_workspace_bytes",
     "mq_gemm_workspace_bytes", "mq_quantize_weight", "mq_hessian_diag", "mq_delta_score_topk", "mq_pack_residual",
     "mq_quantize_act", "mq_gemm", "mq_run_layer", "mq_get_error", "mq_status_string", "mq_launch_count",
     "mq_gemm_noalloc", "mq_gemm_noalloc_scratch_limit", "mq_quantize_weight_delta", "mq_topk_blocks",
-    "mq_pack_residual_weight", "mq_gemm_act",
+    "mq_pack_residual_weight", "mq_gemm_act", "mq_weight_bytes", "mq_fp4_mma_loop", "mq_fp4_mma_loop_flops",
 )
 
 
@@ -66,6 +68,12 @@ def lib():
     P = ctypes.POINTER
     L.mq_sf_swz_bytes.argtypes = [i32, i32]
     L.mq_sf_swz_bytes.restype = sz
+    L.mq_weight_bytes.argtypes = [i32, i32]
+    L.mq_weight_bytes.restype = sz
+    L.mq_fp4_mma_loop.argtypes = [i32, i32, vp]
+    L.mq_fp4_mma_loop.restype = i32
+    L.mq_fp4_mma_loop_flops.argtypes = [i32, i32]
+    L.mq_fp4_mma_loop_flops.restype = ctypes.c_double
     L.mq_budget_blocks.argtypes = [i32, i32, ctypes.c_double]
     L.mq_budget_blocks.restype = i32
     L.mq_quantize_weight_workspace_bytes.argtypes = [i32, i32]
@@ -142,11 +150,21 @@ def packed_struct(p: dict | None) -> ResidualPacked | None:
 
 # ------------------------------------------------------------------ allocation helpers
 def alloc_weight(N: int, K: int, device, with_sf: bool = True) -> tuple[dict, dict]:
+    """Base (GEMM-ready NVFP4 weight) and full-residual buffers of an N x K weight.
+
+    The base's codes, tiled scales and tensor scale are views of ONE allocation of
+    mq_weight_bytes(N, K) bytes at the offsets include/mosaic.h states; its optional
+    linear scales and the residual are separate tensors."""
     L = lib()
-    base = {"rows": N, "cols": K, "codes": _u8(N, K // 2, device=device),
+    nbytes = L.mq_weight_bytes(N, K)
+    if nbytes == 0:
+        raise MosaicError(f"bad weight shape {N} x {K}")
+    blob = _u8(nbytes, device=device)
+    nc, ns = N * (K // 2), L.mq_sf_swz_bytes(N, K)
+    base = {"rows": N, "cols": K, "codes": blob[:nc].view(N, K // 2),
             "sf": _u8(N, K // 16, device=device) if with_sf else None,
-            "sf_swz": _u8(L.mq_sf_swz_bytes(N, K), device=device),
-            "gscale": torch.empty(1, dtype=torch.float32, device=device)}
+            "sf_swz": blob[nc:nc + ns],
+            "gscale": blob[nc + ns:nc + ns + 4].view(torch.float32), "blob": blob}
     resid = {"rows": N, "cols": K, "codes": _u8(N, K // 2, device=device), "sf": _u8(N, K // 16, device=device),
              "sf_swz": None, "gscale": None}
     return base, resid
@@ -232,6 +250,8 @@ def mq_run_layer(W, X, Xcal, Y, M: int, N: int, K: int, T: int, budget: int, fla
                  buf: LayerBuffers, stream=None):
     """Whole path in one call. With host=True, W/X/Xcal/Y are pinned CPU tensors."""
     def p(t):
+        if t is None:
+            return None
         if host:
             if t.is_cuda:
                 raise MosaicError("host=True expects CPU tensors")
@@ -257,6 +277,12 @@ def mq_gemm_noalloc(xq: dict, wq: dict, packed: dict | None, Y: torch.Tensor, M:
     ps = packed_struct(packed)
     _check(lib().mq_gemm_noalloc(ctypes.byref(mat(xq)), ctypes.byref(mat(wq)), None if ps is None else ctypes.byref(ps),
                                  _ptr(Y), M, N, K, flags, _stream(stream)), "mq_gemm_noalloc")
+
+
+def mq_fp4_mma_loop(ctas: int, iters: int, stream=None) -> float:
+    """Launch the FP4 MMA-loop probe (include/mosaic_probe.h); returns its flop count."""
+    _check(lib().mq_fp4_mma_loop(ctas, iters, _stream(stream)), "mq_fp4_mma_loop")
+    return float(lib().mq_fp4_mma_loop_flops(ctas, iters))
 
 
 def mq_get_error(stream=None) -> int:

@@ -12,8 +12,10 @@
  * E4M3 scale per 16 consecutive K elements, and an fp32 tensor scale g (one per weight
  * matrix, one per token for activations). g = amax / 2688 (1 if amax = 0). Per group:
  * s = amax_group / (6 g); sf = E4M3_rne_satfinite(s); d = dec(sf) * g; r = 1 / d;
- * code_i = E2M1_rne_satfinite(a_i * r) (a signed zero when d = 0). All fp32 IEEE
- * operations, no fused multiply-add; codes and scales are bit-exact with the CPU oracle.
+ * code_i = E2M1_rne_satfinite(a_i * r) (a signed zero when d = 0). Each step is one fp32
+ * IEEE operation with round-to-nearest-even, none contracted into a fused multiply-add;
+ * codes and scales are bit-exact with the CPU oracle. The Delta-score is computed in
+ * fp64 (see mq_delta_score_topk).
  *
  * Conventions for every call:
  *  - All pointers are DEVICE pointers unless stated otherwise; the caller allocates and
@@ -54,7 +56,9 @@ enum {
     MQ_GEMM_DECODE = 1,        /* small-M kernel: W as the MMA's M side, split-K */
     MQ_GEMM_PREFILL = 2,       /* large-M kernel: X as the MMA's M side; needs N % 256 == 0 */
     MQ_GEMM_BASE_ONLY = 4,     /* skip the residual blocks (dense-only reference) */
-    MQ_GEMM_RESIDUAL_ONLY = 8  /* only the residual blocks (linearity check) */
+    MQ_GEMM_RESIDUAL_ONLY = 8, /* only the residual blocks (linearity check) */
+    MQ_LAYER_PREPARED = 16,    /* mq_run_layer only: the weight is already prepared (see there) */
+    MQ_GEMM_WEIGHTS_READY = 32 /* the weight is complete before this call (see mq_gemm) */
 };
 
 /*
@@ -110,6 +114,17 @@ typedef struct {
 /* Bytes of an sf_swz buffer for a rows x cols matrix: ceil(rows/128)*128*(cols/16). */
 size_t mq_sf_swz_bytes(int rows, int cols);
 
+/*
+ * Bytes of one GEMM-ready NVFP4 weight (the base Q(W) that mq_gemm reads), for a caller
+ * that allocates it as one buffer: codes (N*K/2 bytes) at offset 0, sf_swz
+ * (mq_sf_swz_bytes(N, K) bytes) at offset N*K/2, and the fp32 tensor scale at offset
+ * N*K/2 + mq_sf_swz_bytes(N, K), padded to 16 bytes. Every offset is a multiple of 16
+ * for a 16-byte aligned buffer, as the calls require. The optional linear scales
+ * (sf, N*K/16 bytes), the full residual of mq_quantize_weight and the packed residual
+ * are separate buffers. 0 on a bad shape (N, K <= 0 or not multiples of 64).
+ */
+size_t mq_weight_bytes(int N, int K);
+
 /* floor(frac * (N/64) * (K/64)); -1 on a bad shape or frac outside [0, 1]. */
 int mq_budget_blocks(int N, int K, double frac);
 
@@ -119,9 +134,12 @@ size_t mq_quantize_weight_workspace_bytes(int N, int K);
 /* Workspace of mq_delta_score_topk for `budget` selected blocks. */
 size_t mq_delta_topk_workspace_bytes(int N, int K, int budget);
 
-/* Workspace of mq_gemm: split-K fp32 partials plus per-tile counters. The counter
- * region must be zero before the first call on a workspace; every call leaves it zero
- * again when it completes. Calls sharing a workspace must not overlap on the GPU. */
+/* Workspace of mq_gemm and mq_gemm_act: fp32 partials of the output tiles whose K range
+ * is split between CTAs, plus per-tile counters (0 when the large-M kernel runs or no
+ * tile is split). The size depends on the current device's SM count. The counter region
+ * must be zero before the first call on a workspace; every call leaves it zero again
+ * when it completes (a call that ended in MQ_ERR_TIMEOUT may not: zero it again). Calls
+ * sharing a workspace must not overlap on the GPU. */
 size_t mq_gemm_workspace_bytes(int M, int N, int K, unsigned flags);
 
 /* ---- the path ----------------------------------------------------------------- */
@@ -151,10 +169,13 @@ mq_status mq_hessian_diag(const mq_bf16* Xcal, int T, int K, float* H, mq_stream
  * A3 + A4. Delta-score and top-K block selection (summary, "Methodology", section 2:
  * marginal reduction of the output distortion per block, residual error weighted by
  * the diagonal Hessian). For block b = (nt, kt):
- *   Delta_b = T64_k( fp64(H_k) * T64_r( fp64(e)^2 - fp64(e')^2 ) ),
+ *   Delta_b = T64_k( fp64(H_k) * T64_r( fp64(e)*fp64(e) - fp64(e')*fp64(e') ) ),
  *   e = fp32(W - deq Q(W)), e' = fp32(e - deq R),
  * where T64 is the pairwise tree v[i] += v[i+32], +16, +8, +4, +2, +1 over the block's
- * 64 rows (inner) and 64 columns (outer). The kernel recomputes e and e' from W and the
+ * 64 rows (inner) and 64 columns (outer), every add and multiply in fp64 with
+ * round-to-nearest-even. Both squares are exact in fp64, so each element's term is
+ * rounded once (the kernel takes it as one fp64 fused multiply-add, e*e - (e'*e'),
+ * which gives the same bits). The kernel recomputes e and e' from W and the
  * tensor scale base->gscale, bit-identical to mq_quantize_weight's codes; base->codes and
  * resid_full are not read (they may be NULL).
  * Then blocks are ordered by (Delta descending, b ascending): rank[0..budget) = the
@@ -221,10 +242,18 @@ mq_status mq_quantize_act(const mq_bf16* X, int M, int K, mq_nvfp4_mat* xq, mq_s
  *   acc[m,n] = sum_k xh[m,k] * ( wh[n,k] + [block (n/64, k/64) selected] rh[n,k] ),
  * with xh, wh, rh the scaled E2M1 values (val * dec(sf)). Base and residual blocks
  * accumulate into one fp32 tensor-memory accumulator (tcgen05 kind::mxf4nvf4 MMAs, one
- * extra MMA per selected block); the decode kernel then adds its split-K partials in a
- * fixed order. r == NULL (or r->nblk == 0) is the dense base alone.
+ * extra MMA per selected block). The decode kernel (small M) gives every SM an equal
+ * share of the (tile, 256-K) work units; a tile whose K range is split between CTAs is
+ * summed from their fp32 partials in a fixed order, so repeated calls give the same bits.
+ * r == NULL (or r->nblk == 0) is the dense base alone.
  * xq: codes, sf_swz, gscale [M]. wq: codes, sf_swz, gscale [1]. Y: bf16 [M][N].
  * flags: MQ_GEMM_* (one of AUTO/DECODE/PREFILL, optionally BASE_ONLY or RESIDUAL_ONLY).
+ * MQ_GEMM_WEIGHTS_READY: the caller guarantees that no kernel that may still be running
+ * when this call's kernel starts writes wq or r (as for a layer's weights at inference,
+ * prepared once); the decode kernel then requests its first W stages before it waits for
+ * the preceding kernel in the stream, so they overlap that kernel's tail. X, g_x, Y and
+ * the workspace are still touched only after that wait. Without the flag every input is
+ * read after the wait.
  * ws: mq_gemm_workspace_bytes(M, N, K, flags) bytes (see there); may be NULL if that
  * size is 0.
  */
@@ -239,8 +268,9 @@ mq_status mq_gemm(const mq_nvfp4_mat* xq, const mq_nvfp4_mat* wq, const mq_resid
  * straight into the MMA's operand layout; the per-token scale g_x[m] = amax(X[m,:])/2688
  * (1 if 0) comes from maxima exchanged between the K splits of a tile through the
  * thread-block cluster's shared memory (or, for more than 8 splits, each CTA reads the
- * whole row). Codes, scales and Y are those of mq_quantize_act followed by mq_gemm with
- * the decode kernel (bit-identical). gx_out: [M] fp32, receives g_x, or NULL. Other
+ * whole row). The codes and scales are those of mq_quantize_act (bit-identical); this
+ * kernel splits K at fixed points of its own, so Y equals mq_gemm's within the GEMM's
+ * tolerance, not bit for bit. gx_out: [M] fp32, receives g_x, or NULL. Other
  * arguments, flags and workspace as in mq_gemm; MQ_GEMM_PREFILL returns
  * MQ_ERR_UNSUPPORTED_SHAPE (the large-M kernel takes a quantized X).
  */
@@ -279,10 +309,15 @@ typedef struct {
  * selection), A4 top-`budget` selection, A5 pack the selected residual from
  * W (mq_pack_residual_weight), A7+A8 fused GEMM into Y. Results are those of the
  * individual calls. The call's first kernel waits for the kernel preceding the call in
- * the stream before the others may start, so no input is read before that kernel ends. With host == 0, W, X, Xcal and Y are device
- * pointers. With host != 0 they are HOST pointers (page-locked for the copies to be
- * asynchronous): the inputs are copied into buf->W_dev, X_dev, Xcal_dev and the result
- * from buf->Y_dev back to Y, all on `stream`. Errors as the individual calls.
+ * the stream before the others may start, so no input is read before that kernel ends.
+ * With host == 0, W, X, Xcal and Y are device pointers. With host != 0 they are HOST
+ * pointers (page-locked for the copies to be asynchronous): the inputs are copied into
+ * buf->W_dev, X_dev, Xcal_dev and the result from buf->Y_dev back to Y, all on `stream`.
+ * flags: the GEMM flags, plus MQ_LAYER_PREPARED for inference on a layer whose weight a
+ * previous call prepared: buf->base and buf->packed already hold the quantized weight and
+ * the packed residual of `budget` blocks, A1..A5 are skipped, W and Xcal are not read
+ * (they may be NULL) and only X (and Y) cross the host link. Errors as the individual
+ * calls.
  */
 mq_status mq_run_layer(const mq_bf16* W, const mq_bf16* X, const mq_bf16* Xcal, mq_bf16* Y, int M, int N, int K,
                        int T, int budget, unsigned flags, int host, mq_layer_buffers* buf, mq_stream stream);
@@ -292,11 +327,14 @@ mq_status mq_run_layer(const mq_bf16* W, const mq_bf16* X, const mq_bf16* Xcal, 
  * (for example code embedded in a framework that owns all device memory and offers no
  * workspace hook, or paths where an allocation is not allowed). The paper has no
  * counterpart to this call; it exists for such integrations.
- * Same arguments, checks and results as mq_gemm, minus ws/ws_bytes. The split-K scratch
- * is a static array inside the library, mq_gemm_noalloc_scratch_limit() bytes (8 MiB)
- * on every GPU that loads the library, held until the process exits. A problem whose
- * mq_gemm_workspace_bytes() exceeds that limit is rejected with MQ_ERR_WORKSPACE (use
- * mq_gemm with a workspace instead). The first call on each device looks up the
+ * Same arguments, checks, kernel choice (the flags, else by shape) and results as
+ * mq_gemm, minus ws/ws_bytes. The decode kernel's scratch (fp32 partials of the tiles
+ * that CTAs share, and the tile counters) is a static array inside the library,
+ * mq_gemm_noalloc_scratch_limit() bytes (16 MiB) on every GPU that loads the library,
+ * held until the process exits; the large-M kernel needs none. A problem whose
+ * mq_gemm_workspace_bytes() exceeds that limit (decode shapes with more than 64 tokens)
+ * is rejected with MQ_ERR_WORKSPACE before anything is launched (use mq_gemm with a
+ * workspace instead). The first call on each device looks up the
  * array's device address (set-up, once per device, with that device current); make
  * that first call before any stream capture. Each call clears the scratch's tile
  * counters on `stream` before its kernel. All calls share the one array, which keeps
