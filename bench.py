@@ -257,9 +257,11 @@ def run_reference(args):
 
 
 # ------------------------------------------------------------------ GPU helpers
-def graph_time_us(issue, n_calls: int, reps: int, stream=None) -> float:
+def graph_time_us(issue, n_calls: int, reps: int, stream=None, target_ms: float = 40.0) -> float:
     """Device time per call: `issue()` captured once as a CUDA graph of n_calls launches,
-    replayed `reps` times between CUDA events (after one untimed replay)."""
+    replayed between CUDA events after one untimed replay. The replay count is `reps`, or
+    fewer when one replay is long, so that each measurement takes about target_ms (at
+    least one replay)."""
     import torch
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g):
@@ -267,6 +269,12 @@ def graph_time_us(issue, n_calls: int, reps: int, stream=None) -> float:
     g.replay()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    g.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    one_ms = max(e0.elapsed_time(e1), 1e-3)
+    reps = max(1, min(reps, int(target_ms / one_ms)))
     e0.record(stream)
     for _ in range(reps):
         g.replay()
@@ -276,7 +284,29 @@ def graph_time_us(issue, n_calls: int, reps: int, stream=None) -> float:
     return e0.elapsed_time(e1) * 1e3 / (reps * n_calls)
 
 
-def operand_copies(layer, xq, Y, ws, per_call: float, min_copies: int = 2):
+def small_split(M: int, N: int, K: int, sms: int = 148) -> int:
+    """The library's choice of the small-problem decode kernel (its cluster split S), or 0
+    for the stream-K kernel (the rule of plan_small in the library's GEMM host code)."""
+    tiles, KS = N // 128, K // 256
+    if M > 32 or 2 * tiles > sms:
+        return 0
+    S = min(8, sms // tiles, KS)
+    return 0 if (KS + S - 1) // S > 8 else S
+
+
+def gemm_kernel(M: int, N: int, K: int, sms: int = 148) -> tuple[str, str]:
+    """(kernel, description) that mq_gemm runs with flags 0 (the library's rule: the
+    CTA-pair prefill kernel for M > 128 with N % 256 == 0, else a decode kernel)."""
+    if M > 128 and N % 256 == 0:
+        return "k_gemm_prefill2", "prefill (CTA pairs)"
+    bn = 16 if M <= 16 else 32 if M <= 32 else 64 if M <= 64 else 128
+    S = small_split(M, N, K, sms)
+    if S:
+        return f"k_gemm_small<{bn}>", f"decode, {S}-CTA cluster split"
+    return f"k_gemm_streamk<{bn}>", "decode, stream-K"
+
+
+def operand_copies(layer, xq, Y, ws, per_call: float, min_copies: int = 1):
     """Copies of the GEMM's operands (quantized weight, packed residual, quantized X, Y,
     workspace) whose total exceeds 2.5x the L2, so that back-to-back calls over them
     read every byte from HBM."""
@@ -359,8 +389,10 @@ def gemm_sweep(peaks: dict, fp4_measured: float | None, reps: int = 20) -> tuple
                 us_qd = graph_time_us(lambda: [mosaic.mq_quantize_weight_delta(w, layer.H, layer.base, None,
                                                                                 layer.delta, layer.qws) for w in Ws],
                                       len(Ws), 5)
-                us_tk = graph_time_us(lambda: mosaic.mq_topk_blocks(layer.delta, budget, layer.rank, layer.sel), 1,
-                                      20) if budget else 0.0
+                # ten back-to-back calls per graph replay (a replay boundary costs
+                # microseconds, as much as a call)
+                us_tk = graph_time_us(lambda: [mosaic.mq_topk_blocks(layer.delta, budget, layer.rank, layer.sel)
+                                               for _ in range(10)], 10, 20) if budget else 0.0
                 qd_bytes = step_bytes(16, N, K, 512, budget)["quantize_weight_delta"]
                 drows.append({"workload": wl, "matrix": mat, "N": N, "K": K, "blocks": (N // 64) * (K // 64),
                               "budget_blocks": budget, "us_quantize_delta": round(us_qd, 2),
@@ -410,10 +442,10 @@ def gemm_sweep(peaks: dict, fp4_measured: float | None, reps: int = 20) -> tuple
                 fl_exec, fl_dense = gemm_flops(M, N, K, budget)
                 tf = fl_exec / (us * 1e-6) / 1e12
                 gbs = per_call / (us * 1e-6) / 1e9
-                prefill = M > 128 and N % 256 == 0
+                kname = "%s (%s)" % gemm_kernel(M, N, K)
                 rows.append({
                     "workload": wl, "matrix": mat, "M": M, "N": N, "K": K, "budget_frac": frac,
-                    "budget_blocks": budget, "kernel": "prefill" if prefill else "decode (stream-K)",
+                    "budget_blocks": budget, "kernel": kname,
                     "us": round(us, 3), "tflops_executed": round(tf, 1),
                     "tflops_dense_equiv": round(fl_dense / (us * 1e-6) / 1e12, 1), "gbs": round(gbs, 1),
                     "frac_hbm": round(gbs / peaks["hbm_gbs"], 4), "frac_fp4_burst": round(tf / fp4_burst, 4),
@@ -454,7 +486,7 @@ def replica_gbs(bytes_per_step: float, world: int, ms_per_step: float) -> float:
 
 
 # the kernels of each call whose DRAM traffic a capture sums (in launch order per call)
-TRAFFIC_KERNELS = {"quantize_weight_delta": ("k_amax_partial", "k_quant_delta"), "gemm": ("k_gemm_streamk",)}
+TRAFFIC_KERNELS = {"quantize_weight_delta": ("k_amax_partial", "k_quant_delta"), "gemm": ("k_gemm_small",)}
 
 
 def write_traffic(csv_path: str, call: str = "quantize_weight_delta", skip: int = 0, out_path: str | None = None) -> dict:
@@ -705,12 +737,22 @@ def main():
             "frac_hbm": round(gbs_rank / peaks["hbm_gbs"], 4), "tflops_executed": round(tf, 2),
             "tflops_dense_equiv": round(fl_dense / (us * 1e-6) / 1e12, 2),
             "frac_fp4_burst": round(tf / fp4_burst, 5), "rotating_copies": R,
-            "kernel": "k_gemm_streamk<16> (decode, stream-K)"}
-    roofline = {"bound": "hbm", "kernel": "gemm (k_gemm_streamk<16>)",
+            "kernel": "%s (%s)" % gemm_kernel(M, N, K)}
+    roofline = {"bound": "hbm", "kernel": f"gemm ({gemm_kernel(M, N, K)[0]})",
                 "timing": f"CUDA events around {args.steps} back-to-back calls over {R} operand copies",
                 "achieved": round(gbs_rank, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": round(gbs_rank / peaks["hbm_gbs"], 4), "traffic": dram_traffic("gemm"),
                 "peak_source": f"{peaks['source']} (copy bandwidth)"}
+    # the same calls with MQ_GEMM_WEIGHTS_READY (a layer's weights at inference: the next
+    # call's W is requested before it waits for the current one)
+    def issue_wr():
+        for k in range(R):
+            b, p, a, y, w = copies[k]
+            mosaic.mq_gemm(a, b, p, y, M, N, K, mosaic.MQ_GEMM_WEIGHTS_READY, w)
+    us_wr = graph_time_us(issue_wr, R, max(1, args.steps // R), stream)
+    gemm["us_weights_ready"] = round(us_wr, 3)
+    gemm["gbs_weights_ready"] = round(per_call / (us_wr * 1e-6) / 1e9, 1)
+    gemm["frac_hbm_weights_ready"] = round(per_call / (us_wr * 1e-6) / 1e9 / peaks["hbm_gbs"], 4)
     for g in singles:
         del g
     del gall, singles

@@ -7,6 +7,7 @@
 
 #include "common.cuh"
 #include "gemm.cuh"
+#include "mosaic_test.h"
 
 namespace mq {
 
@@ -34,12 +35,21 @@ cudaError_t launch_pack_w(const uint16_t* W, int N, int K, const float* g_w, con
                           uint8_t* blk_codes, uint8_t* blk_sf, int32_t* blk_kt, int32_t* tile_ptr, uint32_t* bitmap,
                           const double* delta, int32_t* rank, cudaStream_t s);
 cudaError_t launch_topk_select(const double* delta, int B, int budget, int32_t* sel, cudaStream_t s);
+cudaError_t launch_smooth_scales(const uint16_t* Xcal, int T, const uint16_t* W, int N, int K, float* s,
+                                 cudaStream_t st);
+cudaError_t launch_smooth_apply(const uint16_t* A, int rows, int K, const float* s, int invert, uint16_t* out,
+                                cudaStream_t st);
 
 }  // namespace mq
 
 using namespace mq;
 
 static std::atomic<uint64_t> g_launches{0};
+
+// Test hook (mq_test_arm_wait_fault): the next decode GEMM launch skips one unit's W copies
+// in CTA 0 and gives up each wait after g_fault_ns.
+static std::atomic<int> g_fault_unit{-1};
+static std::atomic<unsigned long long> g_fault_ns{0};
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -69,6 +79,21 @@ static bool make_tmap_bytes(CUtensorMap* map, const void* base, uint64_t row_byt
     cuuint32_t es[2] = {1, 1};
     CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, es,
                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// u32 matrix [rows][row_u32] (row-major, no swizzle) in boxes of box_u32 x box_rows.
+static bool make_tmap_u32(CUtensorMap* map, const void* base, uint64_t row_u32, uint64_t rows, uint32_t box_u32,
+                          uint32_t box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {row_u32, rows};
+    cuuint64_t strides[1] = {row_u32 * 4};
+    cuuint32_t box[2] = {box_u32, box_rows};
+    cuuint32_t es[2] = {1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<void*>(base), dims, strides, box, es,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
@@ -150,8 +175,10 @@ size_t mq_gemm_workspace_bytes(int M, int N, int K, unsigned flags) {
     if (flags & MQ_GEMM_DECODE) prefill = false;
     if (flags & MQ_GEMM_PREFILL) prefill = true;
     if (prefill) return 0;
-    // mq_gemm's decode kernel (stream-K) and mq_gemm_act's (split-K): the larger of the two
-    return std::max(plan_streamk(M, N, K).ws, decode_workspace_bytes(M, N, K));
+    // mq_gemm's decode kernels (the small-problem one needs none, stream-K its partials)
+    // and mq_gemm_act's (split-K): the larger of the two
+    const size_t gemm_ws = plan_small(M, N, K) ? 0 : plan_streamk(M, N, K).ws;
+    return std::max(gemm_ws, decode_workspace_bytes(M, N, K));
 }
 
 mq_status mq_quantize_weight(const mq_bf16* W, int N, int K, mq_nvfp4_mat* base, mq_nvfp4_mat* resid_full,
@@ -347,6 +374,7 @@ mq_status gemm_dispatch(const mq_nvfp4_mat* xq, const mq_nvfp4_mat* wq, const mq
         p.bitmap = r->bitmap;
     }
     p.has_resid = has_r ? 1 : 0;
+    p.nblk = has_r ? r->nblk : 0;
     p.Y = Y;
     p.M = M;
     p.N = N;
@@ -356,9 +384,34 @@ mq_status gemm_dispatch(const mq_nvfp4_mat* xq, const mq_nvfp4_mat* wq, const mq
     p.w_ready = (flags & MQ_GEMM_WEIGHTS_READY) ? 1 : 0;
     CUtensorMap tw, tx;
     if (prefill) {
-        if (!make_tmap_bytes(&tw, wq->codes, (uint64_t)K / 2, (uint64_t)N, 128, 256)) return MQ_ERR_CUDA;
+        // CTA pairs: each CTA stages 128 tokens and 128 of the tile's 256 weight rows
+        CUtensorMap twsf, txsf, trc, trsf;
+        const uint64_t KS64 = (uint64_t)K / 64;
+        if (!make_tmap_bytes(&tw, wq->codes, (uint64_t)K / 2, (uint64_t)N, 128, 128)) return MQ_ERR_CUDA;
         if (!make_tmap_bytes(&tx, xq->codes, (uint64_t)K / 2, (uint64_t)M, 128, 128)) return MQ_ERR_CUDA;
-        return launched(launch_gemm_prefill(tw, tx, p, as_stream(stream)), 1);
+        if (!make_tmap_u32(&twsf, wq->sf_swz, 128, (uint64_t)((N + 127) / 128) * KS64, 128, 4)) return MQ_ERR_CUDA;
+        if (!make_tmap_u32(&txsf, xq->sf_swz, 128, (uint64_t)((M + 127) / 128) * KS64, 128, 4)) return MQ_ERR_CUDA;
+        // without a residual these two maps are never used: any valid buffer will do
+        const void* rc = has_r ? (const void*)r->blk_codes : (const void*)xq->sf_swz;
+        const void* rs = has_r ? (const void*)r->blk_sf : (const void*)xq->sf_swz;
+        const uint64_t nb = has_r ? (uint64_t)r->nblk : 1;
+        if (!make_tmap_u32(&trc, rc, 256, has_r ? 2 * nb : 1, 256, 1)) return MQ_ERR_CUDA;
+        if (!make_tmap_u32(&trsf, rs, 128, nb, 128, 1)) return MQ_ERR_CUDA;
+        return launched(launch_gemm_prefill2(tw, tx, twsf, txsf, trc, trsf, p, as_stream(stream)), 1);
+    }
+    p.wait_ns = 2000000000ull;
+    p.skip_unit = -1;
+    const int fault_unit = g_fault_unit.exchange(-1);
+    if (fault_unit >= 0) {
+        p.skip_unit = fault_unit;
+        p.wait_ns = g_fault_ns.load();
+    }
+    if (const int S = plan_small(M, N, K)) {
+        // small problems: each tile split among the CTAs of one cluster, no workspace
+        if (!make_tmap_bytes(&tw, wq->codes, (uint64_t)K / 2, (uint64_t)N, 128, 128)) return MQ_ERR_CUDA;
+        if (!make_tmap_bytes(&tx, xq->codes, (uint64_t)K / 2, (uint64_t)M, 128, M <= 16 ? 16 : 32))
+            return MQ_ERR_CUDA;
+        return launched(launch_gemm_small(tw, tx, p, S, as_stream(stream)), 1);
     }
     const StreamKPlan d = plan_streamk(M, N, K);
     // the kernel splits the units with 32-bit arithmetic (units x grid < 2^32)
@@ -413,6 +466,7 @@ static mq_status gemm_act_impl(const mq_bf16* X, const mq_nvfp4_mat* wq, const m
         p.bitmap = r->bitmap;
     }
     p.has_resid = has_r ? 1 : 0;
+    p.nblk = has_r ? r->nblk : 0;
     p.Y = Y;
     p.M = M;
     p.N = N;
@@ -528,6 +582,19 @@ mq_status mq_run_layer(const mq_bf16* W, const mq_bf16* X, const mq_bf16* Xcal, 
     return MQ_OK;
 }
 
+mq_status mq_smooth_scales(const mq_bf16* Xcal, int T, const mq_bf16* W, int N, int K, float* s, mq_stream stream) {
+    if (!Xcal || !W || !s || T <= 0 || N <= 0 || K <= 0 || K % 64) return MQ_ERR_INVALID_ARG;
+    if (!aligned(Xcal, 16) || !aligned(W, 16)) return MQ_ERR_INVALID_ARG;
+    return launched(launch_smooth_scales(Xcal, T, W, N, K, s, as_stream(stream)), 1);
+}
+
+mq_status mq_smooth_apply(const mq_bf16* A, int rows, int K, const float* s, int invert, mq_bf16* out,
+                          mq_stream stream) {
+    if (!A || !s || !out || rows <= 0 || K <= 0 || K % 64) return MQ_ERR_INVALID_ARG;
+    if (!aligned(A, 16) || !aligned(out, 16)) return MQ_ERR_INVALID_ARG;
+    return launched(launch_smooth_apply(A, rows, K, s, invert ? 1 : 0, out, as_stream(stream)), 1);
+}
+
 mq_status mq_get_error(mq_stream stream) {
     if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return MQ_ERR_CUDA;
     int v = 0;
@@ -548,5 +615,12 @@ const char* mq_status_string(mq_status s) {
 }
 
 uint64_t mq_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+mq_status mq_test_arm_wait_fault(int unit, double wait_ms) {
+    if (unit < 0 || !(wait_ms >= 0.01 && wait_ms <= 2000.0)) return MQ_ERR_INVALID_ARG;
+    g_fault_ns.store((unsigned long long)(wait_ms * 1e6));
+    g_fault_unit.store(unit);
+    return MQ_OK;
+}
 
 }  // extern "C"

@@ -58,6 +58,17 @@ __device__ __forceinline__ uint32_t mapa_u32(uint32_t local_saddr, uint32_t rank
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(local_saddr), "r"(rank));
     return ra;
 }
+// 32- and 64-bit loads from the same shared-memory offset in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t ld_dsmem_u32(const void* local, uint32_t rank) {
+    uint32_t v;
+    asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(mapa_u32(smem_u32(local), rank)) : "memory");
+    return v;
+}
+__device__ __forceinline__ uint64_t ld_dsmem_u64(const void* local, uint32_t rank) {
+    uint64_t v;
+    asm volatile("ld.shared::cluster.u64 %0, [%1];" : "=l"(v) : "r"(mapa_u32(smem_u32(local), rank)) : "memory");
+    return v;
+}
 // fp32 store into (possibly another CTA's) shared memory of the cluster.
 __device__ __forceinline__ void st_dsmem_f32(uint32_t cluster_saddr, float v) {
     asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(cluster_saddr), "f"(v) : "memory");
@@ -277,6 +288,112 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
     for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// tcgen05.ld of 16 consecutive 32-bit columns of the warp's 32 lanes, not waited for: the
+// registers hold the data only after tmem_ld_wait16 on them.
+__device__ __forceinline__ void tmem_ld16_issue(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+}
+// Waits for all of this thread's outstanding tcgen05.ld. The registers are operands of the
+// wait, so no use of them is scheduled ahead of it (a second wait returns at once).
+__device__ __forceinline__ void tmem_ld_wait16(uint32_t (&r)[16]) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                   "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]),
+                   "+r"(r[15])
+                 :
+                 : "memory");
+}
+// NC chunks of 16 columns from taddr (chunk c at column 16 c) into v[16 c ..], all loads in
+// flight together and one wait; a chunk whose bit in `mask` is clear reads as zeros
+// (mask must be the same in the whole warp).
+template <int NC>
+__device__ __forceinline__ void tmem_ld_chunks(uint32_t taddr, uint32_t mask, float* v) {
+    uint32_t r[NC][16];
+#pragma unroll
+    for (int c = 0; c < NC; ++c) {
+        if ((mask >> c) & 1u) {
+            tmem_ld16_issue(taddr + 16 * c, r[c]);
+        } else {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) r[c][j] = 0u;
+        }
+    }
+#pragma unroll
+    for (int c = 0; c < NC; ++c) tmem_ld_wait16(r[c]);
+#pragma unroll
+    for (int c = 0; c < NC; ++c)
+#pragma unroll
+        for (int j = 0; j < 16; ++j) v[16 * c + j] = __uint_as_float(r[c][j]);
+}
+
+// ---------------------------------------------------------------- tcgen05, CTA pairs (cta_group::2)
+// A pair of CTAs (a cluster of 2) shares one MMA: the even CTA issues it, A's rows are split
+// between the two CTAs' shared memory (128 each), B's rows too (N/2 each), and D's rows
+// land in each CTA's own tensor memory. Allocation and release are done by one warp of
+// each CTA, with the same warp index in both.
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t* dst_smem, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
+                 "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+// D (+)= (A * sfA) x (B * sfB)^T for the pair (issued by the even CTA).
+__device__ __forceinline__ void mma_mxf4nvf4_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                                  uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %6, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.scale_vec::4X [%0], %1, %2, %3, [%4], [%5], p;\n\t}" ::"r"(
+            d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(sfa_tmem), "r"(sfb_tmem), "r"(accumulate)
+        : "memory");
+}
+
+// A 512-byte scale chunk from each CTA's shared memory (same offset) into the same four
+// tensor-memory columns of each CTA (issued by the even CTA).
+__device__ __forceinline__ void tc_cp_sf_chunk_pair(uint32_t taddr, uint64_t src_desc) {
+    asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(src_desc) : "memory");
+}
+
+// Arrive on the mbarrier at the same offset in every CTA of `cta_mask` once the pair's
+// tcgen05 operations issued by this thread have completed.
+__device__ __forceinline__ void tc_commit_pair_mc(uint64_t* bar, uint16_t cta_mask) {
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+            smem_u32(bar)),
+        "h"(cta_mask)
+        : "memory");
+}
+
+// Arrive on an mbarrier of this CTA once the pair's tcgen05 operations issued by this
+// thread have completed.
+__device__ __forceinline__ void tc_commit_pair(uint64_t* bar) {
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+
+// 2-D tiled TMA load into this CTA's shared memory that signals an mbarrier of either CTA
+// of the pair (`bar_cluster`: a shared::cluster address, e.g. the even CTA's barrier).
+__device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* map, uint32_t bar_cluster, int x,
+                                                 int y) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, "
+        "%3}], [%4];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar_cluster)
+        : "memory");
+}
+
 // Host: run `set` (kernel attribute calls, which belong to the current device) once per
 // device. `done` is the caller's per-device record. Two threads arriving together both
 // run `set`, which only repeats idempotent calls.
@@ -290,6 +407,27 @@ inline cudaError_t once_per_device(std::atomic<bool> (&done)[64], F&& set) {
     e = set();
     if (e == cudaSuccess) done[dev].store(true, std::memory_order_release);
     return e;
+}
+
+// Host: launch `kern` with programmatic stream serialization in clusters of `dims`.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl_cluster(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                                      dim3 dims, Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attrs[2];
+    attrs[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attrs[0].val.programmaticStreamSerializationAllowed = 1;
+    attrs[1].id = cudaLaunchAttributeClusterDimension;
+    attrs[1].val.clusterDim.x = dims.x;
+    attrs[1].val.clusterDim.y = dims.y;
+    attrs[1].val.clusterDim.z = dims.z;
+    cfg.attrs = attrs;
+    cfg.numAttrs = 2;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
 }
 
 // Host: launch `kern` with programmatic stream serialization (and a (1, cluster_y, 1)

@@ -1,28 +1,19 @@
 // ZipperEngine fused GEMM on sm_100a (MosaicQuant summary, "Methodology" section 3;
 // arXiv 2606.15652 abstract: sparse block computation fused into the dense 4-bit GEMM
-// through an overlapped pipeline).
+// through an overlapped pipeline). Base and residual blocks accumulate into one fp32
+// tensor-memory accumulator (tcgen05 kind::mxf4nvf4, one extra MMA per selected block).
 //
-// Decode kernel (small M): the weight is the MMA's M side (128 weight rows per tile),
-// tokens are its N side (BN = 16..128), so a tile streams 128 x K of W exactly once.
-// Warp roles: warp 0 issues TMA / bulk copies, warp 1 owns tensor memory and issues
-// tcgen05 MMAs from one thread, warps 2-5 run the epilogue. Per K stage (256 K
-// elements) the producer loads the W and X tiles (128-byte swizzle), their 4 scale
-// chunks, and every selected residual block of the tile's two 64-row block rows.
-// The MMA thread issues 4 base MMAs (K = 64 each) and one more MMA per selected
-// residual block into the SAME fp32 accumulator: the residual block's rows fill one
-// half of a 128-row operand whose other half carries zero scales.
-// Split-K: the K splits of a tile run as one thread-block cluster; each CTA leaves its
-// fp32 partial in its own shared memory and, after a cluster barrier, reduces a slice of
-// the tile's rows by reading its peers' partials (distributed shared memory) in split
-// order, then scales by g_x[m] * g_w and stores bf16. Above 8 splits (narrow layers) the
-// partials go through a global workspace instead, added in the same order by the last
-// CTA of the tile (a tile counter).
-// The kernel is launched with programmatic dependent launch: its prologue overlaps the
-// preceding kernel. It waits for that kernel before its loads, unless the caller
-// guarantees that W and X were complete before this kernel could start
-// (GemmParams::prefetch, set by the whole-path call: the pack before the GEMM lets it
-// start only after its own wait, which already implies that both quantizers completed):
-// then the first stages' W and X are requested before the wait.
+// Three kernels:
+//  - k_gemm_streamk (small M, HBM-bound): the weight is the MMA's M side (128 weight rows
+//    per tile), the tokens its N side; persistent CTAs take equal ranges of (tile,
+//    256-K stage) units; W, X and residual blocks come from three producer warps.
+//  - k_gemm_prefill2 (large M, tensor-bound): 256 tokens x 256 weight rows per pair of
+//    CTAs sharing each MMA (cta_group::2).
+//  - k_gemm_decode (small M with the activation quantization inside the kernel,
+//    mq_gemm_act): a fixed K split per tile, reduced through a thread-block cluster.
+// Every kernel is launched with programmatic dependent launch: its prologue overlaps the
+// preceding kernel, and it waits for that kernel before touching anything it may write
+// (W may be requested earlier when the caller states that it is complete).
 #include <algorithm>
 #include <atomic>
 
@@ -77,6 +68,35 @@ __device__ __forceinline__ bool elect_one() {
 // a loop run by a single lane of an otherwise waiting warp issues far more slowly.
 __device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity) {
     const bool ok = mbar_wait(bar, parity);
+    return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+}
+
+// AND of `v` over the 128 epilogue threads (named barrier 1): every thread leaves with the
+// same verdict, so the epilogue warps never split on a wait that ran out for one of them.
+__device__ __forceinline__ bool epi_all(bool v) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.and.pred q, 1, 128, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)(v ? 1 : 0))
+        : "memory");
+    return r != 0;
+}
+
+// mbar_wait_warp with the wall-clock limit given (ns).
+__device__ __forceinline__ bool mbar_wait_warp_ns(uint64_t* bar, uint32_t parity, unsigned long long limit) {
+    bool ok = mbar_try_wait(bar, parity);
+    if (!ok) {
+        const unsigned long long t0 = globaltimer();
+        while (!(ok = mbar_try_wait(bar, parity)))
+            if (globaltimer() - t0 > limit) {
+                atomicCAS(&g_error, 0, (int)MQ_ERR_TIMEOUT);
+                break;
+            }
+    }
     return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
 }
 
@@ -259,6 +279,7 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
                 for (int a = 0; a < 4; ++a)
                     if (a == kk) idx = h ? idx1[a] : idx0[a];
+                idx = min(max(idx, 0), p.nblk - 1);  // a well-formed index is already in range
                 bulk_load(st + C::kOffRC + kk * 4096 + h * 2048, p.blk_codes + (int64_t)idx * 2048, 2048,
                           &rfull[s]);
                 bulk_load(st + C::kOffRSF + j * 512, p.blk_sf + (int64_t)idx * 512, 512, &rfull[s]);
@@ -750,7 +771,10 @@ __global__ void __launch_bounds__(256, 1)
         int t = (int)(u0 / (uint32_t)KS), ks = (int)(u0 % (uint32_t)KS);
         for (int i = 0; i < nu; ++i, ks = ks + 1 == KS ? 0 : ks + 1, t += ks == 0) {
             const int s = i % C::kStages;
-            if (i >= C::kStages && !mbar_wait_warp(&empty[s], (uint32_t)(((i / C::kStages) - 1) & 1))) break;
+            if (i >= C::kStages && !mbar_wait_warp_ns(&empty[s], (uint32_t)(((i / C::kStages) - 1) & 1), p.wait_ns)) break;
+            // test hook (mq_test_arm_wait_fault): this unit's W is never requested, so the
+            // MMA issuer's wait for it runs out with nothing in flight
+            if (blockIdx.x == 0 && i == p.skip_unit) continue;
             if (elect_one()) {
                 uint8_t* st = smem + s * C::kStageBytes;
                 const int n_tile = t / p.tiles_m;
@@ -765,7 +789,7 @@ __global__ void __launch_bounds__(256, 1)
         }
         // Do not leave while copies into this CTA's shared memory are in flight.
         for (int v = issued > C::kStages ? issued - C::kStages : 0; v < issued; ++v)
-            mbar_wait_warp(&full[v % C::kStages], (uint32_t)((v / C::kStages) & 1));
+            mbar_wait_warp_ns(&full[v % C::kStages], (uint32_t)((v / C::kStages) & 1), p.wait_ns);
     } else if (warp == 2) {
         // ---------------------------------------------------- X producer
         if (!p.prefetch) griddep_wait();
@@ -774,7 +798,7 @@ __global__ void __launch_bounds__(256, 1)
         int t = (int)(u0 / (uint32_t)KS), ks = (int)(u0 % (uint32_t)KS);
         for (int i = 0; i < nu; ++i, ks = ks + 1 == KS ? 0 : ks + 1, t += ks == 0) {
             const int s = i % C::kStages;
-            if (i >= C::kStages && !mbar_wait_warp(&empty[s], (uint32_t)(((i / C::kStages) - 1) & 1))) break;
+            if (i >= C::kStages && !mbar_wait_warp_ns(&empty[s], (uint32_t)(((i / C::kStages) - 1) & 1), p.wait_ns)) break;
             if (elect_one()) {
                 uint8_t* st = smem + s * C::kStageBytes;
                 const int m_tile = t % p.tiles_m;
@@ -787,10 +811,12 @@ __global__ void __launch_bounds__(256, 1)
             issued = i + 1;
         }
         for (int v = issued > C::kStages ? issued - C::kStages : 0; v < issued; ++v)
-            mbar_wait_warp(&full[v % C::kStages], (uint32_t)((v / C::kStages) & 1));
+            mbar_wait_warp_ns(&full[v % C::kStages], (uint32_t)((v / C::kStages) & 1), p.wait_ns);
     } else if (warp == 3) {
         // ---------------------------------------------------- residual producer
-        if (!(p.prefetch || p.w_ready)) griddep_wait();
+        // The packed residual may come from the preceding kernel (the whole-path call's
+        // pack): only the caller's weights-ready guarantee lets it be read before the wait.
+        if (!p.w_ready) griddep_wait();
         int nres = 0;               // units whose residual copies are issued
         int rc = 0, rdone = 0;      // residual blocks issued / known consumed
         int ends[C::kStages] = {};  // rc after the latest unit held by each stage
@@ -817,14 +843,14 @@ __global__ void __launch_bounds__(256, 1)
                     m |= (((m0b >> kk) & 1u) << (2 * kk)) | (((m1b >> kk) & 1u) << (2 * kk + 1));
             }
             if (i >= C::kStages) {  // the stage's mask and barrier phase are free again
-                if (!mbar_wait_warp(&empty[s], (uint32_t)(((i / C::kStages) - 1) & 1))) { ok = false; break; }
+                if (!mbar_wait_warp_ns(&empty[s], (uint32_t)(((i / C::kStages) - 1) & 1), p.wait_ns)) { ok = false; break; }
                 rdone = max(rdone, pick(ends, s));
             }
             const int n = __popc(m);
             // ring slots [rc, rc + n) must be free: wait for younger units until they are
             for (int v = i - C::kStages + 1; rc + n - C::kRSlots > rdone && v < i && ok; ++v) {
                 if (v < 0) continue;
-                ok = mbar_wait_warp(&empty[v % C::kStages], (uint32_t)((v / C::kStages) & 1));
+                ok = mbar_wait_warp_ns(&empty[v % C::kStages], (uint32_t)((v / C::kStages) & 1), p.wait_ns);
                 rdone = max(rdone, pick(ends, v % C::kStages));
             }
             if (!ok) break;
@@ -838,6 +864,7 @@ __global__ void __launch_bounds__(256, 1)
 #pragma unroll
                     for (int a = 0; a < 4; ++a)
                         if (a == kk) bi = h ? idx1[a] : idx0[a];
+                    bi = min(max(bi, 0), p.nblk - 1);  // a well-formed index is already in range
                     const uint32_t slot = sbase + C::kOffRing + (r % C::kRSlots) * C::kRSlotBytes;
                     bulk_load_s(slot, p.blk_codes + (int64_t)bi * 2048, 2048, &rfull[s]);
                     bulk_load_s(slot + 2048, p.blk_sf + (int64_t)bi * 512, 512, &rfull[s]);
@@ -849,7 +876,7 @@ __global__ void __launch_bounds__(256, 1)
             put(ends, s, rc);
         }
         for (int v = nres > C::kStages ? nres - C::kStages : 0; v < nres; ++v)
-            mbar_wait_warp(&rfull[v % C::kStages], (uint32_t)((v / C::kStages) & 1));
+            mbar_wait_warp_ns(&rfull[v % C::kStages], (uint32_t)((v / C::kStages) & 1), p.wait_ns);
     } else if (warp == 1) {
         // ---------------------------------------------------- MMA issuer
         constexpr uint32_t idesc = idesc_mxf4nvf4(128, BN);
@@ -862,11 +889,11 @@ __global__ void __launch_bounds__(256, 1)
             const uint32_t par = (uint32_t)((i / C::kStages) & 1);
             const uint32_t d = tmem + (uint32_t)(seg & 1) * C::kDStride;
             if (i == 0 || ks == 0) {  // a segment starts: its accumulator buffer must be free
-                if (!mbar_wait_warp(&acce[seg & 1], (uint32_t)(((seg >> 1) & 1) ^ 1))) break;
+                if (!mbar_wait_warp_ns(&acce[seg & 1], (uint32_t)(((seg >> 1) & 1) ^ 1), p.wait_ns)) break;
                 tc_fence_after();
                 acc = 0;
             }
-            if (!mbar_wait_warp(&full[s], par)) break;
+            if (!mbar_wait_warp_ns(&full[s], par, p.wait_ns)) break;
             tc_fence_after();
             const uint32_t st = sbase + s * C::kStageBytes;
             const uint32_t sfc = tmem + C::kSfCol0 + s * 32;
@@ -887,7 +914,7 @@ __global__ void __launch_bounds__(256, 1)
             }
             __syncwarp();
             acc = __shfl_sync(0xffffffffu, acc, 0);
-            if (!mbar_wait_warp(&rfull[s], par)) break;
+            if (!mbar_wait_warp_ns(&rfull[s], par, p.wait_ns)) break;
             tc_fence_after();
             const uint32_t m = resid ? rmask[s] : 0u;
             if (elect_one()) {
@@ -928,19 +955,12 @@ __global__ void __launch_bounds__(256, 1)
             const int n_tile = (int)t / p.tiles_m, m_tile = (int)t % p.tiles_m;
             const uint32_t ta = t * (uint32_t)KS, tb = ta + (uint32_t)KS;  // the tile's units
             const uint32_t sa = max(ta, u0), sb = min(tb, u1);              // this segment's units
-            const bool waited = mbar_wait_warp(&accf[seg & 1], (uint32_t)((seg >> 1) & 1));
+            const bool waited = epi_all(mbar_wait_warp_ns(&accf[seg & 1], (uint32_t)((seg >> 1) & 1), p.wait_ns));
             tc_fence_after();
             const bool have = waited && (dense || resid_in_range(p, n_tile, (int)(sa - ta), (int)(sb - ta)));
             float acc[BN];
-#pragma unroll
-            for (int c0 = 0; c0 < BN; c0 += 16) {
-                if (have) {
-                    tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(seg & 1) * C::kDStride + c0, acc + c0);
-                } else {
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) acc[c0 + j] = 0.0f;
-                }
-            }
+            tmem_ld_chunks<BN / 16>(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(seg & 1) * C::kDStride,
+                                    have ? 0xFFu : 0u, acc);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&acce[seg & 1]);  // the buffer is free for segment seg + 2
@@ -1021,44 +1041,6 @@ __global__ void __launch_bounds__(256, 1)
     }
 }
 
-// ------------------------------------------------------------------ prefill kernel
-// Large M: the tokens are the MMA's M side (128 per tile, A = X) and the weight its N
-// side (256 rows per tile, B = W), K = 256 per pipeline stage. CTAs are persistent and
-// walk the tiles m-fastest, so CTAs running at the same time share W tiles through L2.
-// A selected residual block (64 weight rows x 64 K) is one N = 64 MMA written into its
-// 64-column slice of the same fp32 accumulator: exactly the block's work. The residual
-// blocks of a stage land in a ring of shared-memory slots on the stage's own barrier,
-// and the stage's release frees them with it.
-// Warps: 0 producer (TMA / bulk copies), 1 MMA issuer, 2-9 epilogue (two warps per
-// 32-lane quarter of tensor memory, 128 accumulator columns each). Producer and MMA
-// warps run their loops converged and let one elected lane issue. The epilogue copies
-// the accumulator to registers and releases it before scaling and storing, so the next
-// tile's MMAs overlap the stores.
-struct PrefillCfg {
-    static constexpr int kStages = 3;
-    static constexpr int kOffX = 0;                    // 128 rows x 128 B, swizzled
-    static constexpr int kOffW = 16384;                // 256 rows x 128 B, swizzled
-    static constexpr int kOffSFX = kOffW + 32768;      // 4 x 512 B
-    static constexpr int kOffSFW = kOffSFX + 2048;     // 2 row tiles x 4 x 512 B
-    static constexpr int kStageBytes = kOffSFW + 4096; // 55296
-    static constexpr int kBaseTx = kStageBytes;        // bytes a stage's base operands bring
-    static constexpr int kRSlots = 16;                 // residual ring: 2048 B codes + 512 B scales
-    static constexpr int kRSlotBytes = 2560;
-    static constexpr int kOffRing = kStages * kStageBytes;
-    static constexpr int kCtrlOff = kOffRing + kRSlots * kRSlotBytes;
-    static constexpr int kCtrlBytes = 512;
-    static constexpr int kSmemBytes = kCtrlOff + kCtrlBytes + 1024;
-    static constexpr int kThreads = 320;
-    static constexpr uint32_t kTmemCols = 512;
-    static constexpr int kSfCol0 = 256;                // after the 256-column accumulator
-    static constexpr int kSfStageCols = 48;            // X: 4 x 4, W: 4 x 8
-    static constexpr int kRSfCol0 = kSfCol0 + kStages * kSfStageCols;
-    static_assert(kStageBytes % 1024 == 0, "stage alignment");
-    static_assert(kSmemBytes <= 232448, "shared memory budget");
-    static_assert(kRSfCol0 + kRSlots * 4 <= 512, "tensor memory budget");
-    static_assert(kRSlots >= 16, "a stage may carry 16 residual blocks");
-};
-
 // Which 64-column slices of a tile's accumulator receive an MMA (bit h: weight rows
 // 64h..64h+63)? All of them unless only the residual is computed, in which case a slice
 // is written only if its block row has selected blocks.
@@ -1071,32 +1053,71 @@ __device__ __forceinline__ uint32_t prefill_tile_slices(const GemmParams& p, int
     return m;
 }
 
-__global__ void __launch_bounds__(320, 1)
-    k_gemm_prefill(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
-                   const GemmParams p) {
-    using C = PrefillCfg;
+// ------------------------------------------------------------------ small decode kernel
+// Decode problems too small to keep every SM streaming for long (LLaMA3-8B q_proj at 16
+// tokens: 10.5 MB) are bound by fixed latencies: the wait for the preceding kernel, the
+// first data's latency, the reduce-sum. This variant splits each 128-row tile's K range
+// evenly among the S CTAs of one thread-block cluster (S <= 8, tiles x S <= SMs) and adds
+// the S fp32 partials through the cluster's shared memory, in split order. A CTA is small
+// enough for two to share an SM (3-4 stages, an 8-slot residual ring, 256 tensor-memory
+// columns), so the next call's CTAs are already resident while this call finishes and,
+// when the caller states that the weight is ready (MQ_GEMM_WEIGHTS_READY), stream their W
+// meanwhile. Warp 0 issues every copy (W, X, residual blocks), warp 1 the MMAs, warps 2-5
+// the epilogue.
+template <int BN>
+struct SmallCfg {
+    static constexpr int kStages = BN <= 16 ? 4 : 3;
+    static constexpr int kOffW = 0;                     // 128 rows x 128 B, swizzled
+    static constexpr int kOffX = 16384;                 // BN rows x 128 B, swizzled
+    static constexpr int kOffSFW = kOffX + BN * 128;    // 4 x 512 B
+    static constexpr int kOffSFX = kOffSFW + 2048;      // 4 x 512 B
+    static constexpr int kStageBytes = kOffSFX + 2048;
+    static constexpr int kRSlots = 8;
+    static constexpr int kRSlotBytes = 2560;
+    static constexpr int kOffRing = kStages * kStageBytes;
+    static constexpr int kCtrlOff = kOffRing + kRSlots * kRSlotBytes + 2048;  // 2 KB after the ring
+    static constexpr int kCtrlBytes = 256;
+    static constexpr int kSmemBytes = kCtrlOff + kCtrlBytes + 1024;
+    static constexpr int kThreads = 192;
+    static constexpr uint32_t kTmemCols = 256;
+    static constexpr uint32_t kSfCol0 = 32;                          // after D (BN <= 32 columns)
+    static constexpr uint32_t kRSfCol0 = kSfCol0 + kStages * 32;
+    static_assert(kStageBytes % 1024 == 0, "stage alignment");
+    static_assert(kSmemBytes <= 113 * 1024, "two CTAs per SM");
+    static_assert(kRSfCol0 + kRSlots * 4 <= kTmemCols, "tensor memory budget");
+    static_assert(kStages * kStageBytes >= BN * 128 * 4, "the partial fits in the stage area");
+};
+
+template <int BN>
+__global__ void __launch_bounds__(192, 2)
+    k_gemm_small(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
+                 const GemmParams p) {
+    using C = SmallCfg<BN>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kCtrlOff);  // base operands + residual blocks landed
-    uint64_t* empty = full + C::kStages;                                // stage (and its ring slots) consumed
-    uint64_t* accf = empty + C::kStages;
-    uint64_t* acce = accf + 1;
-    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(acce + 1);
-    uint32_t* rmask = tmem_holder + 1;  // [kStages]: bit 4*kk + h
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kCtrlOff);  // W, X and scales landed
+    uint64_t* rfull = full + C::kStages;                                // residual blocks landed
+    uint64_t* empty = rfull + C::kStages;                               // stage and its ring slots consumed
+    uint64_t* accf = empty + C::kStages;                                // accumulator complete
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(accf + 1);
+    uint32_t* rmask = tmem_holder + 1;  // [kStages]: bit 2 * kk + h
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int S = p.splits;
+    const int tile = blockIdx.x / S, split = blockIdx.x % S;  // split = rank in the (S, 1, 1) cluster
+    const int n_tile = tile / p.tiles_m, m_tile = tile % p.tiles_m;
     const int KS = p.K / 256, KS64 = p.K / 64;
-    const int tiles_m = (p.M + 127) / 128, tiles_n = p.N / 256;
-    const int ntiles = tiles_m * tiles_n;
+    const int ks0 = split * KS / S, nu = (split + 1) * KS / S - ks0;
+    const bool dense = p.mode != 2;
     const bool resid = p.has_resid && p.mode != 1;
 
     if (warp == 0 && lane == 0) {
         for (int s = 0; s < C::kStages; ++s) {
             mbar_init(&full[s], 1);
+            mbar_init(&rfull[s], 1);
             mbar_init(&empty[s], 1);
         }
         mbar_init(accf, 1);
-        mbar_init(acce, 8);
         mbar_fence_init();
         tma_prefetch_desc(&tmap_w);
         tma_prefetch_desc(&tmap_x);
@@ -1112,13 +1133,354 @@ __global__ void __launch_bounds__(320, 1)
     const uint32_t sbase = smem_u32(smem);
 
     if (warp == 0) {
-        // ---------------------------------------------------- producer
+        // ---------------------------------------------------- producer: W, X, residual blocks
+        auto issue_w = [&](int i) {
+            // test hook (mq_test_arm_wait_fault): this unit's W is never requested, so the
+            // MMA issuer's wait for it runs out with nothing in flight
+            if (blockIdx.x == 0 && i == p.skip_unit) return;
+            const int s = i % C::kStages, ks = ks0 + i;
+            uint8_t* st = smem + s * C::kStageBytes;
+            mbar_arrive_expect_tx(&full[s], (dense ? 16384 + 2048 : 0) + BN * 128 + 2048);
+            if (dense) {
+                tma_load_2d(st + C::kOffW, &tmap_w, &full[s], ks * 128, n_tile * 128);
+                bulk_load(st + C::kOffSFW, p.w_sf + ((int64_t)n_tile * KS64 + ks * 4) * 512, 2048, &full[s]);
+            }
+        };
+        auto issue_x = [&](int i) {
+            const int s = i % C::kStages, ks = ks0 + i;
+            uint8_t* st = smem + s * C::kStageBytes;
+            tma_load_2d(st + C::kOffX, &tmap_x, &full[s], ks * 128, m_tile * BN);
+            bulk_load(st + C::kOffSFX, p.x_sf + ((int64_t)(m_tile * BN / 128) * KS64 + ks * 4) * 512, 2048,
+                      &full[s]);
+        };
+        const int first = nu < C::kStages ? nu : C::kStages;
+        const bool w_early = p.prefetch || p.w_ready;
+        if (w_early && elect_one())
+            for (int i = 0; i < first; ++i) issue_w(i);
+        __syncwarp();
+        if (!p.w_ready) griddep_wait();  // the packed residual may come from the preceding kernel
+        RowCursor cur0, cur1;
+        if (resid) {
+            cur0 = row_cursor(p, n_tile * 2 + 0, ks0 * 4);
+            cur1 = row_cursor(p, n_tile * 2 + 1, ks0 * 4);
+        }
+        int rc = 0, rdone = 0, nres = 0, nbase = 0;
+        int ends[C::kStages] = {};
+        bool waited = !p.w_ready, ok = true;
+        for (int i = 0; i < nu && ok; ++i) {
+            const int s = i % C::kStages;
+            if (i >= C::kStages) {
+                if (!mbar_wait_warp_ns(&empty[s], (uint32_t)(((i / C::kStages) - 1) & 1), p.wait_ns)) break;
+                rdone = max(rdone, pick(ends, s));
+            }
+            // W (unless requested before the wait) and X: X only after the wait
+            if (i >= first || !w_early) {
+                if (!waited && !p.prefetch) { griddep_wait(); waited = true; }
+                if (elect_one()) issue_w(i);
+                __syncwarp();
+            }
+            if (!waited && !p.prefetch) { griddep_wait(); waited = true; }
+            if (elect_one()) issue_x(i);
+            __syncwarp();
+            nbase = i + 1;
+            uint32_t m = 0;
+            int idx0[4] = {0, 0, 0, 0}, idx1[4] = {0, 0, 0, 0};
+            if (resid) {
+                const uint32_t m0b = row_step(cur0, (ks0 + i) * 4, idx0);
+                const uint32_t m1b = row_step(cur1, (ks0 + i) * 4, idx1);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    m |= (((m0b >> kk) & 1u) << (2 * kk)) | (((m1b >> kk) & 1u) << (2 * kk + 1));
+            }
+            const int n = __popc(m);
+            for (int v = i - C::kStages + 1; rc + n - C::kRSlots > rdone && v < i && ok; ++v) {
+                if (v < 0) continue;
+                ok = mbar_wait_warp_ns(&empty[v % C::kStages], (uint32_t)((v / C::kStages) & 1), p.wait_ns);
+                rdone = max(rdone, pick(ends, v % C::kStages));
+            }
+            if (!ok) break;
+            if (elect_one()) {
+                rmask[s] = m;
+                mbar_arrive_expect_tx(&rfull[s], n * C::kRSlotBytes);
+                int r = rc;
+                for (uint32_t mm = m; mm; mm &= mm - 1, ++r) {
+                    const int j = __ffs(mm) - 1, kk = j >> 1, h = j & 1;
+                    int bi = 0;
+#pragma unroll
+                    for (int a = 0; a < 4; ++a)
+                        if (a == kk) bi = h ? idx1[a] : idx0[a];
+                    bi = min(max(bi, 0), p.nblk - 1);  // a well-formed index is already in range
+                    const uint32_t slot = sbase + C::kOffRing + (r % C::kRSlots) * C::kRSlotBytes;
+                    bulk_load_s(slot, p.blk_codes + (int64_t)bi * 2048, 2048, &rfull[s]);
+                    bulk_load_s(slot + 2048, p.blk_sf + (int64_t)bi * 512, 512, &rfull[s]);
+                }
+            }
+            __syncwarp();
+            nres = i + 1;
+            rc += n;
+            put(ends, s, rc);
+        }
+        if (!waited && !p.prefetch) griddep_wait();
+        griddep_launch();
+        // Do not leave while copies into this CTA's shared memory are in flight.
+        const int nw = w_early ? (nbase > first ? nbase : first) : nbase;
+        for (int v = nw > C::kStages ? nw - C::kStages : 0; v < nw; ++v)
+            mbar_wait_warp_ns(&full[v % C::kStages], (uint32_t)((v / C::kStages) & 1), p.wait_ns);
+        for (int v = nres > C::kStages ? nres - C::kStages : 0; v < nres; ++v)
+            mbar_wait_warp_ns(&rfull[v % C::kStages], (uint32_t)((v / C::kStages) & 1), p.wait_ns);
+    } else if (warp == 1) {
+        // ---------------------------------------------------- MMA issuer
+        constexpr uint32_t idesc = idesc_mxf4nvf4(128, BN);
+        int rc = 0;
+        uint32_t acc = 0;
+        for (int i = 0; i < nu; ++i) {
+            const int s = i % C::kStages;
+            const uint32_t par = (uint32_t)((i / C::kStages) & 1);
+            if (!mbar_wait_warp_ns(&full[s], par, p.wait_ns)) break;
+            tc_fence_after();
+            const uint32_t st = sbase + s * C::kStageBytes;
+            const uint32_t sfc = tmem + C::kSfCol0 + s * 32;
+            if (elect_one()) {
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+                    if (dense) tc_cp_sf_chunk(sfc + 4 * kk, smem_desc(st + C::kOffSFW + kk * 512, 0, 128, 0));
+                    tc_cp_sf_chunk(sfc + 16 + 4 * kk, smem_desc(st + C::kOffSFX + kk * 512, 0, 128, 0));
+                }
+                if (dense) {
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_mxf4nvf4(tmem, smem_desc(st + C::kOffW + 32 * kk, 16, 1024, 2),
+                                     smem_desc(st + C::kOffX + 32 * kk, 16, 1024, 2), idesc, sfc + 4 * kk,
+                                     sfc + 16 + 4 * kk, (acc | kk) != 0);
+                    acc = 1;
+                }
+            }
+            __syncwarp();
+            acc = __shfl_sync(0xffffffffu, acc, 0);
+            if (!mbar_wait_warp_ns(&rfull[s], par, p.wait_ns)) break;
+            tc_fence_after();
+            const uint32_t m = resid ? rmask[s] : 0u;
+            if (elect_one()) {
+                int r = rc;
+                for (uint32_t mm = m; mm; mm &= mm - 1, ++r) {
+                    const int j = __ffs(mm) - 1, kk = j >> 1, h = j & 1;
+                    const int slot_i = r % C::kRSlots;
+                    const uint32_t slot = sbase + C::kOffRing + slot_i * C::kRSlotBytes;
+                    const uint32_t rsf = tmem + C::kRSfCol0 + 4 * slot_i;
+                    tc_cp_sf_chunk(rsf, smem_desc(slot + 2048, 0, 128, 0));
+                    mma_mxf4nvf4(tmem, smem_desc(slot - 2048 * h, 128, 256, 0),
+                                 smem_desc(st + C::kOffX + 32 * kk, 16, 1024, 2), idesc, rsf, sfc + 16 + 4 * kk, acc);
+                    acc = 1;
+                }
+                tc_commit(&empty[s]);
+            }
+            __syncwarp();
+            acc = __shfl_sync(0xffffffffu, acc, 0);
+            rc += __popc(m);
+        }
+        if (elect_one()) tc_commit(accf);
+        __syncwarp();
+    }
+    // ---------------------------------------------------- epilogue (warps 2..5)
+    // the accumulator of this CTA's K range; with S > 1 it goes to shared memory (the stage
+    // area: every MMA has completed) and the cluster adds the S partials in split order
+    float* part = reinterpret_cast<float*>(smem);  // [BN][128]
+    const int q = warp & 3, row = 32 * q + lane;
+    bool ok = true;
+    if (warp >= 2) {
+        griddep_wait();  // g_x and Y follow the preceding kernel
+        ok = epi_all(mbar_wait_warp_ns(accf, 0, p.wait_ns));
+        tc_fence_after();
+        const bool have = ok && (dense || resid_in_range(p, n_tile, ks0, ks0 + nu));
+        float acc[BN];
+        tmem_ld_chunks<BN / 16>(tmem + ((uint32_t)(32 * q) << 16), have ? 0xFFu : 0u, acc);
+        tc_fence_before();
+        const float gw = __ldg(p.g_w);
+        const int m0 = m_tile * BN, n = n_tile * 128 + row;
+        if (S == 1) {
+#pragma unroll
+            for (int j = 0; j < BN; ++j) {
+                const int mm = m0 + j;
+                if (ok && mm < p.M) {
+                    const float sc = __fmul_rn(__ldg(p.g_x + mm), gw);
+                    const __nv_bfloat16 y = __float2bfloat16_rn(__fmul_rn(acc[j], sc));
+                    p.Y[(int64_t)mm * p.N + n] = *reinterpret_cast<const uint16_t*>(&y);
+                }
+            }
+        } else {
+#pragma unroll
+            for (int j = 0; j < BN; ++j) part[j * 128 + row] = acc[j];
+        }
+    }
+    if (S > 1) {
+        // every CTA of the cluster holds its partial; CTA r adds rows [r*128/S, (r+1)*128/S)
+        __syncwarp();
+        cluster_sync();
+        if (warp >= 2) {
+            const int r0 = split * 128 / S, r1 = (split + 1) * 128 / S, rows = r1 - r0;
+            const float gw = __ldg(p.g_w);
+            const int m0 = m_tile * BN;
+            const int total = rows * BN;
+            for (int e = threadIdx.x - 64; e < total; e += 128) {
+                const int j = e / rows, nl = r0 + e % rows;
+                float v[8];
+#pragma unroll
+                for (int s2 = 0; s2 < 8; ++s2)
+                    if (s2 < S) v[s2] = ld_dsmem_f32(part + j * 128 + nl, (uint32_t)s2);
+                float sum = v[0];
+#pragma unroll
+                for (int s2 = 1; s2 < 8; ++s2)
+                    if (s2 < S) sum = __fadd_rn(sum, v[s2]);
+                const int mm = m0 + j;
+                if (ok && mm < p.M) {
+                    const float sc = __fmul_rn(__ldg(p.g_x + mm), gw);
+                    const __nv_bfloat16 y = __float2bfloat16_rn(__fmul_rn(sum, sc));
+                    p.Y[(int64_t)mm * p.N + n_tile * 128 + nl] = *reinterpret_cast<const uint16_t*>(&y);
+                }
+            }
+        }
+        __syncwarp();
+        cluster_sync();  // peers may still be reading this CTA's partial until here
+    }
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::kTmemCols);
+    }
+}
+
+// ------------------------------------------------------------------ prefill kernel, CTA pairs
+// Large M with the tensor cores of two SMs on one 256 x 256 tile (tokens x weight rows):
+// a cluster of two CTAs shares every MMA (tcgen05 cta_group::2, issued by the even CTA).
+// Each CTA stages its own 128 tokens of X, its own half (128 rows) of the 256 weight rows
+// and the scales, so an SM brings in 32 KB of operands per 256-K stage where a CTA that
+// computed a 128 x 256 tile alone would bring in 48 KB: the per-SM ingest that bounds the
+// single-CTA kernel drops by a third. Both CTAs' copies complete on the even CTA's stage
+// barrier; the MMA's completion is signalled to both CTAs' barriers at once. A selected
+// residual block is one M = 256, N = 64 MMA into its 64-column slice of the accumulator,
+// its 64 weight rows split 32 + 32 between the pair. Each CTA's epilogue drains its own
+// 128 accumulator rows. In the even CTA a scale warp copies each stage's scale chunks into
+// tensor memory and signals a barrier, so the MMA-issuing thread issues MMAs only (a stage
+// has 12 scale copies for 4 MMAs: issued from one thread they took about as long as the
+// MMAs run).
+struct Prefill2Cfg {
+    static constexpr int kStages = 4;
+    static constexpr int kOffX = 0;                      // 128 rows x 128 B, swizzled
+    static constexpr int kOffW = 16384;                  // 128 rows x 128 B, swizzled
+    static constexpr int kOffSFX = 32768;                // 4 x 512 B
+    static constexpr int kOffSFW = kOffSFX + 2048;       // 2 row tiles x 4 x 512 B
+    static constexpr int kStageBytes = kOffSFW + 4096;   // 38912
+    static constexpr int kRSlots = 16;
+    static constexpr int kRSlotBytes = 1536;             // 1024 B (32 rows) of codes + 512 B scales
+    static constexpr int kOffRing = kStages * kStageBytes;
+    static constexpr int kCtrlOff = kOffRing + kRSlots * kRSlotBytes;
+    static constexpr int kCtrlBytes = 512;
+    static constexpr int kSmemBytes = kCtrlOff + kCtrlBytes + 1024;
+    static constexpr int kThreads = 320;  // 0 producer, 1 MMA (even CTA), 2-9 epilogue
+    static constexpr uint32_t kTmemCols = 512;
+    static constexpr int kSfCol0 = 256;                  // after the 256-column accumulator
+    static constexpr int kSfStageCols = 48;              // X: 4 x 4, W: 4 x 8
+    static constexpr int kRSfCol0 = kSfCol0 + kStages * kSfStageCols;
+    static_assert(kStageBytes % 1024 == 0, "stage alignment");
+    static_assert(kSmemBytes <= 232448, "shared memory budget");
+    static_assert(kRSfCol0 + kRSlots * 4 <= 512, "tensor memory budget");
+};
+
+// AND of `v` over the 256 epilogue threads of the pair kernel (named barrier 1).
+__device__ __forceinline__ bool epi_all256(bool v) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.and.pred q, 1, 256, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)(v ? 1 : 0))
+        : "memory");
+    return r != 0;
+}
+
+// try_wait on a barrier whose completing arrivals come from both CTAs of the pair.
+__device__ __forceinline__ bool mbar_wait_warp_cluster(uint64_t* bar, uint32_t parity) {
+    bool ok = mbar_try_wait_cluster(bar, parity);
+    if (!ok) {
+        const unsigned long long t0 = globaltimer();
+        while (!(ok = mbar_try_wait_cluster(bar, parity)))
+            if (globaltimer() - t0 > kWaitLimitNs) {
+                atomicCAS(&g_error, 0, (int)MQ_ERR_TIMEOUT);
+                break;
+            }
+    }
+    return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+}
+
+__global__ void __launch_bounds__(Prefill2Cfg::kThreads, 1)
+    k_gemm_prefill2(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
+                    const __grid_constant__ CUtensorMap tmap_wsf, const __grid_constant__ CUtensorMap tmap_xsf,
+                    const __grid_constant__ CUtensorMap tmap_rc, const __grid_constant__ CUtensorMap tmap_rsf,
+                    const GemmParams p) {
+    using C = Prefill2Cfg;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kCtrlOff);  // (even CTA) both CTAs' copies landed
+    uint64_t* empty = full + C::kStages;                                // stage and its ring slots consumed
+    uint64_t* accf = empty + C::kStages;                                // accumulator complete
+    uint64_t* acce = accf + 1;                                          // (even CTA) both epilogues read it
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(acce + 1);
+    uint32_t* rmask = tmem_holder + 1;  // [kStages] (even CTA): bit 4 * kk + h
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    const bool leader = rank == 0;
+    const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+    const int KS = p.K / 256, KS64 = p.K / 64;
+    const int tiles_m = (p.M + 255) / 256, tiles_n = p.N / 256;
+    const int ntiles = tiles_m * tiles_n;
+    const bool dense = p.mode != 2;
+    const bool resid = p.has_resid && p.mode != 1;
+
+    if (warp == 0 && lane == 0) {
+        for (int s = 0; s < C::kStages; ++s) {
+            // The even CTA's producer arrives with the bytes of both CTAs. A stage carrying
+            // copies from both CTAs cannot complete before the odd CTA issued it; with only
+            // the residual computed, a stage may carry none, so the odd CTA's producer also
+            // arrives: either way its view of its empty barrier never falls two phases behind.
+            mbar_init(&full[s], p.mode == 2 ? 2 : 1);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(accf, 1);
+        mbar_init(acce, 16);  // 8 epilogue warps of each CTA
+        mbar_fence_init();
+        tma_prefetch_desc(&tmap_w);
+        tma_prefetch_desc(&tmap_x);
+        tma_prefetch_desc(&tmap_wsf);
+        tma_prefetch_desc(&tmap_xsf);
+        if (resid) {
+            tma_prefetch_desc(&tmap_rc);
+            tma_prefetch_desc(&tmap_rsf);
+        }
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(tmem_holder, C::kTmemCols);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before();
+    // both CTAs' barriers initialised and tensor memory allocated before either goes on
+    __syncwarp();
+    cluster_sync();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+    const uint32_t sbase = smem_u32(smem);
+
+    if (warp == 0) {
+        // ---------------------------------------------------- producer (both CTAs)
         griddep_wait();
+        griddep_launch();
         int sc = 0, rc = 0;  // stages and residual blocks issued so far
-        int rdone = 0;       // residual blocks known consumed (ring slots below it are free)
-        int ends[C::kStages] = {};  // rc after the latest stage held by each stage buffer
+        int rdone = 0;       // residual blocks known consumed
+        int ends[C::kStages] = {};
         bool ok = true;
-        for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+        for (int t = pair; t < ntiles && ok; t += npairs) {
             const int m_tile = t % tiles_m, n_tile = t / tiles_m;
             RowCursor cur[4];
             if (resid)
@@ -1140,35 +1502,33 @@ __global__ void __launch_bounds__(320, 1)
                         for (int kk = 0; kk < 4; ++kk) m |= ((mb >> kk) & 1u) << (4 * kk + h);
                     }
                 const int n = __popc(m);
-                // ring slots [rc, rc + n) must be free: wait for younger stages until they are
+                // ring slots of blocks released with earlier stages
                 for (int u = sc - C::kStages + 1; rc + n - C::kRSlots > rdone && u < sc && ok; ++u) {
                     if (u < 0) continue;
                     ok = mbar_wait_warp(&empty[u % C::kStages], (u / C::kStages) & 1);
                     rdone = max(rdone, pick(ends, u % C::kStages));
                 }
                 if (!ok) break;
-                const uint32_t st = sbase + s * C::kStageBytes;
                 if (elect_one()) {
-                    rmask[s] = m;
-                    // only the residual computed: no dense W tile, and no X tile for a stage
-                    // without residual blocks (its barrier completes on the plain arrive)
-                    const bool dense = p.mode != 2, xneed = dense || n > 0;
-                    mbar_arrive_expect_tx(&full[s], (dense ? C::kBaseTx : xneed ? 16384 + 2048 : 0) +
-                                                        n * C::kRSlotBytes);
+                    const bool xneed = dense || n > 0;
+                    const uint32_t bar = mapa_u32(smem_u32(&full[s]), 0);
+                    uint8_t* st = smem + s * C::kStageBytes;
+                    if (leader) {
+                        rmask[s] = m;
+                        mbar_arrive_expect_tx(&full[s], 2u * ((dense ? 16384 + 4096 : 0) + (xneed ? 16384 + 2048 : 0) +
+                                                              n * C::kRSlotBytes));
+                    }
                     if (xneed) {
-                        tma_load_2d(smem + s * C::kStageBytes + C::kOffX, &tmap_x, &full[s], ks * 128,
-                                    m_tile * 128);
-                        bulk_load_s(st + C::kOffSFX, p.x_sf + ((int64_t)m_tile * KS64 + ks * 4) * 512, 2048,
-                                    &full[s]);
+                        tma_load_2d_pair(st + C::kOffX, &tmap_x, bar, ks * 128, m_tile * 256 + 128 * (int)rank);
+                        tma_load_2d_pair(st + C::kOffSFX, &tmap_xsf, bar, 0, (m_tile * 2 + (int)rank) * KS64 + ks * 4);
                     }
                     if (dense) {
-                        tma_load_2d(smem + s * C::kStageBytes + C::kOffW, &tmap_w, &full[s], ks * 128, n_tile * 256);
-                        bulk_load_s(st + C::kOffSFW, p.w_sf + ((int64_t)(n_tile * 2) * KS64 + ks * 4) * 512, 2048,
-                                    &full[s]);
-                        bulk_load_s(st + C::kOffSFW + 2048,
-                                    p.w_sf + ((int64_t)(n_tile * 2 + 1) * KS64 + ks * 4) * 512, 2048, &full[s]);
+                        tma_load_2d_pair(st + C::kOffW, &tmap_w, bar, ks * 128, n_tile * 256 + 128 * (int)rank);
+                        tma_load_2d_pair(st + C::kOffSFW, &tmap_wsf, bar, 0, (n_tile * 2) * KS64 + ks * 4);
+                        tma_load_2d_pair(st + C::kOffSFW + 2048, &tmap_wsf, bar, 0, (n_tile * 2 + 1) * KS64 + ks * 4);
                     }
-                    // residual blocks of the stage in (kk, h) order, into consecutive ring slots
+                    // residual blocks in (kk, h) order into consecutive ring slots: this
+                    // CTA's 32 rows of each block, and the block's whole scale chunk
                     int r = rc;
                     for (uint32_t mm = m; mm; mm &= mm - 1, ++r) {
                         const int j = __ffs(mm) - 1, kk = j >> 2, h = j & 3;
@@ -1178,128 +1538,153 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
                             for (int b = 0; b < 4; ++b)
                                 if (a == h && b == kk) bi = idx[a][b];
-                        const uint32_t slot = sbase + C::kOffRing + (r % C::kRSlots) * C::kRSlotBytes;
-                        bulk_load_s(slot, p.blk_codes + (int64_t)bi * 2048, 2048, &full[s]);
-                        bulk_load_s(slot + 2048, p.blk_sf + (int64_t)bi * 512, 512, &full[s]);
+                        bi = min(max(bi, 0), p.nblk - 1);  // a well-formed index is already in range
+                        uint8_t* slot = smem + C::kOffRing + (r % C::kRSlots) * C::kRSlotBytes;
+                        tma_load_2d_pair(slot, &tmap_rc, bar, 0, 2 * bi + (int)rank);
+                        tma_load_2d_pair(slot + 1024, &tmap_rsf, bar, 0, bi);
                     }
+                    if (!leader && p.mode == 2) mbar_arrive_remote(bar);  // this CTA's copies are issued
                 }
                 __syncwarp();
                 rc += n;
                 put(ends, s, rc);
             }
         }
-        // Do not leave while copies into this CTA's shared memory are in flight.
-        for (int u = max(0, sc - C::kStages); u < sc; ++u) mbar_wait_warp(&full[u % C::kStages], (u / C::kStages) & 1);
+        // Do not leave while copies are in flight: the even CTA's barrier counts both CTAs'
+        // bytes (the odd CTA waits for the even one at the closing cluster barrier).
+        if (leader)
+            for (int u = max(0, sc - C::kStages); u < sc; ++u)
+                mbar_wait_warp_cluster(&full[u % C::kStages], (u / C::kStages) & 1);
     } else if (warp == 1) {
-        // ---------------------------------------------------- MMA issuer
-        constexpr uint32_t idesc_d = idesc_mxf4nvf4(128, 256);
-        constexpr uint32_t idesc_r = idesc_mxf4nvf4(128, 64);
-        int sc = 0, rc = 0, tc = 0;
-        bool ok = true;
-        for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++tc) {
-            if (!mbar_wait_warp(acce, (tc & 1) ^ 1)) break;  // the epilogue has read the previous tile
-            tc_fence_after();
-            uint32_t acc4 = 0;  // bit h: the tile's slice h already holds a partial sum
-            for (int ks = 0; ks < KS; ++ks, ++sc) {
-                const int s = sc % C::kStages;
-                if (!mbar_wait_warp(&full[s], (sc / C::kStages) & 1)) { ok = false; break; }
+        // ---------------------------------------------------- MMA issuer (even CTA)
+        if (leader) {
+            constexpr uint32_t idesc_d = idesc_mxf4nvf4(256, 256);
+            constexpr uint32_t idesc_r = idesc_mxf4nvf4(256, 64);
+            // stage 0's descriptors; a stage or K step moves the start address field only
+            const uint64_t xd0 = smem_desc(sbase + C::kOffX, 16, 1024, 2);
+            const uint64_t wd0 = smem_desc(sbase + C::kOffW, 16, 1024, 2);
+            const uint64_t rd0 = smem_desc(sbase + C::kOffRing, 128, 256, 0);
+            const uint64_t sd0 = smem_desc(sbase, 0, 128, 0);
+            int sc = 0, rc = 0, tc = 0;
+            bool ok = true;
+            for (int t = pair; t < ntiles && ok; t += npairs, ++tc) {
+                if (!mbar_wait_warp_cluster(acce, (tc & 1) ^ 1)) break;  // both epilogues read the previous tile
                 tc_fence_after();
-                const uint32_t st = sbase + s * C::kStageBytes;
-                const uint32_t sfc = tmem + C::kSfCol0 + s * C::kSfStageCols;
-                const uint32_t m = resid ? rmask[s] : 0u;
-                if (elect_one()) {
-                    if (p.mode != 2 || m) {
+                uint32_t acc4 = 0;  // bit h: slice h already holds a partial sum
+                for (int ks = 0; ks < KS; ++ks, ++sc) {
+                    const int s = sc % C::kStages;
+                    const uint32_t par = (sc / C::kStages) & 1;
+                    if (!mbar_wait_warp_cluster(&full[s], par)) { ok = false; break; }  // rmask[s] is written
+                    const uint32_t m = resid ? rmask[s] : 0u;
+                    tc_fence_after();
+                    const uint64_t so = (uint64_t)((s * C::kStageBytes) >> 4);
+                    const uint32_t sfc = tmem + C::kSfCol0 + s * C::kSfStageCols;
+                    if (elect_one()) {
+                        // the stage's scales into tensor memory, issued ahead of the MMAs that
+                        // read them from the same thread (the pipe runs them in order); a
+                        // stage's columns, and a ring slot's, are rewritten only after the
+                        // MMAs that read them completed (the stage was released first)
+                        const uint64_t st = sd0 + so;
+                        if (dense || m) {
 #pragma unroll
-                        for (int kk = 0; kk < 4; ++kk)
-                            tc_cp_sf_chunk(sfc + 4 * kk, smem_desc(st + C::kOffSFX + kk * 512, 0, 128, 0));
-                    }
-                    if (p.mode != 2) {
-#pragma unroll
-                        for (int kk = 0; kk < 4; ++kk) {
-                            tc_cp_sf_chunk(sfc + 16 + 8 * kk, smem_desc(st + C::kOffSFW + kk * 512, 0, 128, 0));
-                            tc_cp_sf_chunk(sfc + 16 + 8 * kk + 4,
-                                           smem_desc(st + C::kOffSFW + 2048 + kk * 512, 0, 128, 0));
+                            for (int kk = 0; kk < 4; ++kk)
+                                tc_cp_sf_chunk_pair(sfc + 4 * kk, st + ((C::kOffSFX + kk * 512) >> 4));
                         }
+                        if (dense) {
 #pragma unroll
-                        for (int kk = 0; kk < 4; ++kk)
-                            mma_mxf4nvf4(tmem, smem_desc(st + C::kOffX + 32 * kk, 16, 1024, 2),
-                                         smem_desc(st + C::kOffW + 32 * kk, 16, 1024, 2), idesc_d, sfc + 4 * kk,
-                                         sfc + 16 + 8 * kk, (acc4 | kk) != 0);
-                        acc4 = 0xFu;
+                            for (int kk = 0; kk < 4; ++kk) {
+                                tc_cp_sf_chunk_pair(sfc + 16 + 8 * kk, st + ((C::kOffSFW + kk * 512) >> 4));
+                                tc_cp_sf_chunk_pair(sfc + 16 + 8 * kk + 4, st + ((C::kOffSFW + 2048 + kk * 512) >> 4));
+                            }
+                        }
+                        {
+                            int r = rc;
+                            for (uint32_t mm = m; mm; mm &= mm - 1, ++r) {
+                                const int slot_i = r % C::kRSlots;
+                                tc_cp_sf_chunk_pair(tmem + C::kRSfCol0 + 4 * slot_i,
+                                                    sd0 + (uint64_t)((C::kOffRing + slot_i * C::kRSlotBytes + 1024) >> 4));
+                            }
+                        }
+                        if (dense) {
+#pragma unroll
+                            for (int kk = 0; kk < 4; ++kk)
+                                mma_mxf4nvf4_pair(tmem, xd0 + so + 2 * kk, wd0 + so + 2 * kk, idesc_d, sfc + 4 * kk,
+                                                  sfc + 16 + 8 * kk, (acc4 | kk) != 0);
+                            acc4 = 0xFu;
+                        }
+                        int r = rc;
+                        for (uint32_t mm = m; mm; mm &= mm - 1, ++r) {
+                            const int j = __ffs(mm) - 1, kk = j >> 2, h = j & 3;
+                            const int slot_i = r % C::kRSlots;
+                            mma_mxf4nvf4_pair(tmem + 64 * h, xd0 + so + 2 * kk,
+                                              rd0 + (uint64_t)((slot_i * C::kRSlotBytes) >> 4), idesc_r, sfc + 4 * kk,
+                                              tmem + C::kRSfCol0 + 4 * slot_i + 2 * (h & 1), (acc4 >> h) & 1u);
+                            acc4 |= 1u << h;
+                        }
+                        // both CTAs' stage (and ring slots) are free once these MMAs complete
+                        tc_commit_pair_mc(&empty[s], 0x3);
                     }
-                    // residual blocks in (kk, h) order: block (kk, h) adds into accumulator slice h
-                    int r = rc;
-                    for (uint32_t mm = m; mm; mm &= mm - 1, ++r) {
-                        const int j = __ffs(mm) - 1, kk = j >> 2, h = j & 3;
-                        const int slot_i = r % C::kRSlots;
-                        const uint32_t slot = sbase + C::kOffRing + slot_i * C::kRSlotBytes;
-                        const uint32_t rsf = tmem + C::kRSfCol0 + 4 * slot_i;
-                        tc_cp_sf_chunk(rsf, smem_desc(slot + 2048, 0, 128, 0));
-                        mma_mxf4nvf4(tmem + 64 * h, smem_desc(st + C::kOffX + 32 * kk, 16, 1024, 2),
-                                     smem_desc(slot, 128, 256, 0), idesc_r, sfc + 4 * kk, rsf + 2 * (h & 1),
-                                     (acc4 >> h) & 1u);
-                        acc4 |= 1u << h;
-                    }
-                    // releases the stage and its ring slots once every MMA above has completed
-                    tc_commit(&empty[s]);
+                    __syncwarp();
+                    acc4 = __shfl_sync(0xffffffffu, acc4, 0);
+                    rc += __popc(m);
                 }
+                if (ok && elect_one()) tc_commit_pair_mc(accf, 0x3);
                 __syncwarp();
-                acc4 = __shfl_sync(0xffffffffu, acc4, 0);
-                rc += __popc(m);
             }
-            if (elect_one()) tc_commit(accf);
-            __syncwarp();
         }
     } else {
-        // ---------------------------------------------------- epilogue (warps 2..9)
+        // ---------------------------------------------------- epilogue (warps 2..9, both CTAs)
         const int q = warp & 3, half = (warp - 2) >> 2;
         griddep_wait();  // g_x and Y follow the previous kernel
         const float gw = __ldg(p.g_w);
+        const uint32_t acce_even = mapa_u32(smem_u32(acce), 0);
         int tc = 0;
-        for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++tc) {
+        for (int t = pair; t < ntiles; t += npairs, ++tc) {
             const int m_tile = t % tiles_m, n_tile = t / tiles_m;
-            const bool waited = mbar_wait_warp(accf, tc & 1);
+            // this thread's row and its scale, loaded before the accumulator is waited for
+            const int mm = m_tile * 256 + 128 * (int)rank + 32 * q + lane;
+            const float sc = mm < p.M ? __fmul_rn(__ldg(p.g_x + mm), gw) : 0.0f;
+            const bool waited = epi_all256(mbar_wait_warp(accf, tc & 1));
             tc_fence_after();
             const uint32_t slices = waited ? prefill_tile_slices(p, n_tile) : 0u;
-            float acc[128];
+            // this thread's row: 128 columns, read 64 at a time (one 64-column slice, its four
+            // loads in flight together) and kept as scaled bf16 pairs, so the accumulator is
+            // released before the stores
+            uint32_t packed[64];
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                // columns 128*half + 16c .. +15 lie in slice 2*half + c/4
-                if ((slices >> (2 * half + (c >> 2))) & 1u) {
-                    tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + 128 * half + 16 * c, acc + 16 * c);
-                } else {
+            for (int b = 0; b < 2; ++b) {
+                float v[64];
+                tmem_ld_chunks<4>(tmem + ((uint32_t)(32 * q) << 16) + 128 * half + 64 * b,
+                                  (slices >> (2 * half + b)) & 1u ? 0xFu : 0u, v);
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) acc[16 * c + j] = 0.0f;
+                for (int u = 0; u < 32; ++u) {
+                    const __nv_bfloat16 lo = __float2bfloat16_rn(__fmul_rn(v[2 * u], sc));
+                    const __nv_bfloat16 hi = __float2bfloat16_rn(__fmul_rn(v[2 * u + 1], sc));
+                    packed[32 * b + u] = (uint32_t)(*reinterpret_cast<const uint16_t*>(&lo)) |
+                                         ((uint32_t)(*reinterpret_cast<const uint16_t*>(&hi)) << 16);
                 }
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(acce);  // accumulator free for the next tile
-            const int mm = m_tile * 128 + 32 * q + lane;
-            if (waited && mm < p.M) {
-                const float sc = __fmul_rn(__ldg(p.g_x + mm), gw);
+            if (lane == 0) mbar_arrive_remote(acce_even);  // this CTA's rows are read
+            if (!waited) break;
+            if (mm < p.M) {
                 uint16_t* yrow = p.Y + (int64_t)mm * p.N + n_tile * 256 + 128 * half;
 #pragma unroll
-                for (int c = 0; c < 16; ++c) {
-                    uint32_t w[4];
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const __nv_bfloat16 lo = __float2bfloat16_rn(__fmul_rn(acc[8 * c + 2 * u], sc));
-                        const __nv_bfloat16 hi = __float2bfloat16_rn(__fmul_rn(acc[8 * c + 2 * u + 1], sc));
-                        w[u] = (uint32_t)(*reinterpret_cast<const uint16_t*>(&lo)) |
-                               ((uint32_t)(*reinterpret_cast<const uint16_t*>(&hi)) << 16);
-                    }
-                    *reinterpret_cast<uint4*>(yrow + 8 * c) = make_uint4(w[0], w[1], w[2], w[3]);
-                }
+                for (int c = 0; c < 16; ++c)
+                    *reinterpret_cast<uint4*>(yrow + 8 * c) =
+                        make_uint4(packed[4 * c], packed[4 * c + 1], packed[4 * c + 2], packed[4 * c + 3]);
             }
-            if (!waited) break;
         }
     }
-    griddep_launch();
-    __syncthreads();
+    // the pair's MMAs read both CTAs' shared memory and write both tensor memories: neither
+    // CTA releases its tensor memory or exits before both are done
+    tc_fence_before();
+    __syncwarp();
+    cluster_sync();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem, C::kTmemCols);
+        tmem_dealloc_pair(tmem, C::kTmemCols);
     }
 }
 
@@ -1413,21 +1798,52 @@ cudaError_t launch_gemm_streamk(const CUtensorMap& tw, const CUtensorMap& tx, Ge
 // Device address of the error word (for kernels of other translation units).
 cudaError_t error_word(int** ptr) { return cudaGetSymbolAddress(reinterpret_cast<void**>(ptr), g_error); }
 
-cudaError_t launch_gemm_prefill(const CUtensorMap& tw, const CUtensorMap& tx, const GemmParams& p, cudaStream_t s) {
+int plan_small(int M, int N, int K) {
+    if (M > 32) return 0;
+    const int tiles = N / 128, KS = K / 256, sms = device_sms();
+    if (2 * tiles > sms) return 0;  // enough tiles to keep every SM streaming: stream-K
+    int S = sms / tiles;
+    if (S > 8) S = 8;
+    if (S > KS) S = KS;
+    if ((KS + S - 1) / S > 8) return 0;  // long K ranges stream better through the deep ring
+    return S;
+}
+
+template <int BN>
+static cudaError_t launch_small_bn(const CUtensorMap& tw, const CUtensorMap& tx, const GemmParams& p, int S,
+                                   cudaStream_t s) {
+    using C = SmallCfg<BN>;
     static std::atomic<bool> attr_set[64];
     cudaError_t e = once_per_device(attr_set, [] {
-        return cudaFuncSetAttribute(k_gemm_prefill, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    PrefillCfg::kSmemBytes);
+        return cudaFuncSetAttribute(k_gemm_small<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     });
     if (e != cudaSuccess) return e;
-    int dev = 0;
-    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
-    int sms = 148;
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const int ntiles = ((p.M + 127) / 128) * (p.N / 256);
-    const int grid = ntiles < sms ? ntiles : sms;
-    return launch_pdl(k_gemm_prefill, dim3(grid), dim3(PrefillCfg::kThreads), PrefillCfg::kSmemBytes, s, 1, tw, tx,
-                      p);
+    const int tiles = p.N / 128;
+    return launch_pdl_cluster(k_gemm_small<BN>, dim3(tiles * S), dim3(C::kThreads), C::kSmemBytes, s, dim3(S, 1, 1),
+                              tw, tx, p);
+}
+
+cudaError_t launch_gemm_small(const CUtensorMap& tw, const CUtensorMap& tx, GemmParams p, int S, cudaStream_t s) {
+    p.splits = S;
+    p.tiles_m = 1;
+    p.tiles_n = p.N / 128;
+    return p.M <= 16 ? launch_small_bn<16>(tw, tx, p, S, s) : launch_small_bn<32>(tw, tx, p, S, s);
+}
+
+cudaError_t launch_gemm_prefill2(const CUtensorMap& tw, const CUtensorMap& tx, const CUtensorMap& twsf,
+                                 const CUtensorMap& txsf, const CUtensorMap& trc, const CUtensorMap& trsf,
+                                 const GemmParams& p, cudaStream_t s) {
+    static std::atomic<bool> attr_set[64];
+    cudaError_t e = once_per_device(attr_set, [] {
+        return cudaFuncSetAttribute(k_gemm_prefill2, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    Prefill2Cfg::kSmemBytes);
+    });
+    if (e != cudaSuccess) return e;
+    const int pairs_max = device_sms() / 2;
+    const int ntiles = ((p.M + 255) / 256) * (p.N / 256);
+    const int pairs = ntiles < pairs_max ? ntiles : pairs_max;
+    return launch_pdl_cluster(k_gemm_prefill2, dim3(2 * pairs), dim3(Prefill2Cfg::kThreads), Prefill2Cfg::kSmemBytes,
+                              s, dim3(2, 1, 1), tw, tx, twsf, txsf, trc, trsf, p);
 }
 
 cudaError_t read_clear_error(int* value) {

@@ -26,6 +26,7 @@ struct GemmParams {
     int splits, iters_per_split;
     int mode;                // 0 fused, 1 base only, 2 residual only
     int has_resid;
+    int nblk;                // packed residual blocks (when has_resid)
     int cluster;             // split-K reduced through the cluster's shared memory
     int prefetch;            // W and X were complete before this kernel could start, so the
                              // decode kernel may load them before waiting for its predecessor
@@ -37,6 +38,8 @@ struct GemmParams {
     // stream-K decode kernel: `units` = tiles x (K / 256) work units, CTA c takes units
     // [c * units / grid, (c + 1) * units / grid); tile t = n_tile * tiles_m + m_tile
     int units, tiles_m, tiles_n;
+    unsigned long long wait_ns;  // stream-K kernel: wall-clock limit of every pipeline wait
+    int skip_unit;               // test hook: CTA 0 does not request this unit's W (-1: none)
 };
 
 // Stream-K decode kernel plan: token tile BN (the MMA's N side), tiles_n x tiles_m
@@ -49,6 +52,10 @@ struct StreamKPlan {
 };
 
 StreamKPlan plan_streamk(int M, int N, int K);
+// Small decode problems (M <= 32, at most half as many 128-row tiles as SMs, short K
+// ranges): the cluster split S (>= 1) of each tile's K range, or 0 for the stream-K kernel.
+int plan_small(int M, int N, int K);
+cudaError_t launch_gemm_small(const CUtensorMap& tw, const CUtensorMap& tx, GemmParams p, int S, cudaStream_t s);
 cudaError_t launch_gemm_streamk(const CUtensorMap& tw, const CUtensorMap& tx, GemmParams p, const StreamKPlan& d,
                                 cudaStream_t s);
 
@@ -63,7 +70,12 @@ DecodePlan plan_decode(int M, int N, int K);
 size_t decode_workspace_bytes(int M, int N, int K);
 cudaError_t launch_gemm_decode(const CUtensorMap& tw, const CUtensorMap& tx, GemmParams p, const DecodePlan& d,
                                cudaStream_t s);
-cudaError_t launch_gemm_prefill(const CUtensorMap& tw, const CUtensorMap& tx, const GemmParams& p, cudaStream_t s);
+// Large-M kernel on CTA pairs: W and X code maps with 128-row boxes, u32 maps over the
+// tiled scales (128 x 4 boxes: four 512-byte chunks) and over the packed residual (codes
+// as rows of 1 KB, scales as rows of 512 B).
+cudaError_t launch_gemm_prefill2(const CUtensorMap& tw, const CUtensorMap& tx, const CUtensorMap& twsf,
+                                 const CUtensorMap& txsf, const CUtensorMap& trc, const CUtensorMap& trsf,
+                                 const GemmParams& p, cudaStream_t s);
 cudaError_t read_clear_error(int* value);
 
 // The fused GEMM's host side (api.cu), shared by mq_gemm and mq_gemm_noalloc.

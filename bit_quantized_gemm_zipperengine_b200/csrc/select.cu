@@ -504,19 +504,237 @@ __global__ void __launch_bounds__(kSelThreads) k_topk_large(const double* __rest
     }
 }
 
+// Top-K selection for more keys than one CTA's shared memory holds: a cluster of C CTAs
+// (one cluster, grid == cluster), CTA c holding the keys of blocks [c chunk, (c+1) chunk)
+// in its shared memory (chunk a multiple of 32). The steps are those of k_topk_large with
+// its shared-memory keys, and every decision is taken identically in every CTA from the
+// same cluster-wide counts:
+//  - the common leading bits from each CTA's AND / OR of its keys, read through DSMEM;
+//  - in each radix pass, every CTA counts its keys into its own histogram, then each thread
+//    adds its two bins over the C histograms (DSMEM loads) before the block scan. The
+//    histograms rotate over three buffers: the one a pass clears was last read by the other
+//    CTAs two passes earlier, and every CTA has crossed the previous pass's cluster barrier
+//    since;
+//  - compaction: each CTA's counts above the bucket and in it are exchanged once, giving its
+//    offset in sel and the tied keys that the lower CTAs take; a last cluster barrier keeps
+//    every CTA resident until the others have read its counts.
+constexpr int kTkMaxCluster = 8;
+constexpr int kTkCtaKeys = 20480;  // keys one CTA holds (160 KB)
+
+__global__ void __launch_bounds__(kSelThreads) k_topk_cluster(const double* __restrict__ delta, int B, int budget,
+                                                              int chunk, int32_t* __restrict__ sel) {
+    extern __shared__ __align__(16) uint64_t dyn[];
+    uint64_t* keys = dyn;  // [chunk]
+    __shared__ unsigned hist[3][1 << kDigitBits];
+    __shared__ uint32_t s_gtw[kTkCtaKeys / 32], s_eqw[kTkCtaKeys / 32];
+    __shared__ uint32_t s_and[64], s_or[64];
+    __shared__ uint64_t s_ao[2];   // this CTA's AND and OR of its keys (read by the cluster)
+    __shared__ int s_cnt[2];       // this CTA's keys above the bucket and in it (read by the cluster)
+    __shared__ int s_out0, s_eqb;  // this CTA's first sel entry; tied keys taken by lower CTAs
+    __shared__ uint64_t s_prefix;
+    __shared__ int s_pos, s_need, s_cand;
+    __shared__ int scratch[32], scratch2[32];
+    griddep_wait();  // Delta comes from the previous kernel
+    griddep_launch();
+    constexpr int U = 8;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int C = (int)gridDim.x, c = (int)cluster_ctarank();
+    const int base = c * chunk, n = max(0, min(chunk, B - base));
+
+    uint64_t a = ~0ull, o = 0ull;
+    for (int i0 = tid; i0 < n; i0 += U * kSelThreads) {
+        double d[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int i = i0 + u * kSelThreads;
+            d[u] = i < n ? delta[base + i] : 0.0;
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int i = i0 + u * kSelThreads;
+            if (i < n) {
+                const uint64_t k = order_key(d[u]);
+                keys[i] = k;
+                a &= k;
+                o |= k;
+            }
+        }
+    }
+    {
+        const uint32_t ah = __reduce_and_sync(0xffffffffu, (uint32_t)(a >> 32));
+        const uint32_t al = __reduce_and_sync(0xffffffffu, (uint32_t)a);
+        const uint32_t oh = __reduce_or_sync(0xffffffffu, (uint32_t)(o >> 32));
+        const uint32_t ol = __reduce_or_sync(0xffffffffu, (uint32_t)o);
+        if (lane == 0) {
+            s_and[2 * warp] = ah;
+            s_and[2 * warp + 1] = al;
+            s_or[2 * warp] = oh;
+            s_or[2 * warp + 1] = ol;
+        }
+    }
+    for (int b = tid; b < (1 << kDigitBits); b += kSelThreads) hist[0][b] = 0;
+    __syncthreads();
+    if (warp == 0) {
+        const uint32_t ah = __reduce_and_sync(0xffffffffu, s_and[2 * lane]);
+        const uint32_t al = __reduce_and_sync(0xffffffffu, s_and[2 * lane + 1]);
+        const uint32_t oh = __reduce_or_sync(0xffffffffu, s_or[2 * lane]);
+        const uint32_t ol = __reduce_or_sync(0xffffffffu, s_or[2 * lane + 1]);
+        if (lane == 0) {
+            s_ao[0] = ((uint64_t)ah << 32) | al;
+            s_ao[1] = ((uint64_t)oh << 32) | ol;
+        }
+    }
+    cluster_sync();  // every CTA's AND / OR and cleared first histogram
+    if (warp == 0) {
+        const uint64_t ar = lane < C ? ld_dsmem_u64(&s_ao[0], lane) : ~0ull;
+        const uint64_t orr = lane < C ? ld_dsmem_u64(&s_ao[1], lane) : 0ull;
+        const uint32_t ah = __reduce_and_sync(0xffffffffu, (uint32_t)(ar >> 32));
+        const uint32_t al = __reduce_and_sync(0xffffffffu, (uint32_t)ar);
+        const uint32_t oh = __reduce_or_sync(0xffffffffu, (uint32_t)(orr >> 32));
+        const uint32_t ol = __reduce_or_sync(0xffffffffu, (uint32_t)orr);
+        a = ((uint64_t)ah << 32) | al;
+        o = ((uint64_t)oh << 32) | ol;
+        if (lane == 0) {
+            const int cp = (a ^ o) ? __clzll((long long)(a ^ o)) : 64;
+            s_pos = 64 - cp;
+            s_prefix = cp ? (a & (~0ull << (64 - cp))) : 0ull;
+            s_need = budget;
+            s_cand = B;
+        }
+    }
+    __syncthreads();
+    for (int pass = 0; s_pos > 0 && s_cand > s_need; ++pass) {  // identical in every CTA
+        const int pos = s_pos, w = pos < kDigitBits ? pos : kDigitBits, shift = pos - w;
+        const uint64_t prefix = s_prefix, hi = pos >= 64 ? 0ull : (~0ull << pos);
+        const int need = s_need;
+        const int nb = 1 << w;
+        unsigned* h = hist[pass % 3];
+        for (int b = tid; b < (1 << kDigitBits); b += kSelThreads) hist[(pass + 1) % 3][b] = 0;
+        for (int i0 = tid - lane; i0 < n; i0 += U * kSelThreads) {  // warp-uniform
+            uint64_t k[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int i = i0 + lane + u * kSelThreads;
+                k[u] = i < n ? keys[i] : 0ull;
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int i = i0 + lane + u * kSelThreads;
+                if (i < n && (k[u] & hi) == prefix) atomicAdd(&h[(unsigned)(k[u] >> shift) & (nb - 1)], 1u);
+            }
+        }
+        cluster_sync();  // every CTA's histogram of this pass is complete
+        const int b0 = nb - 1 - 2 * tid;
+        unsigned c0 = 0u, c1 = 0u;
+        if (b0 >= 0) {
+            for (int r = 0; r < C; ++r) {
+                c0 += ld_dsmem_u32(&h[b0], r);
+                if (b0 >= 1) c1 += ld_dsmem_u32(&h[b0 - 1], r);
+            }
+        }
+        const int above = block_excl_sum_1bar<kSelThreads>((int)(c0 + c1), scratch);
+        if (b0 >= 0 && above < need && above + (int)(c0 + c1) >= need) {
+            const bool first = above + (int)c0 >= need;
+            const int digit = first ? b0 : b0 - 1;
+            s_need = need - (first ? above : above + (int)c0);
+            s_cand = (int)(first ? c0 : c1);
+            s_prefix = prefix | ((uint64_t)digit << shift);
+            s_pos = shift;
+        }
+        __syncthreads();
+    }
+    const int pos = s_pos, need = s_need;
+    const bool whole = s_cand == s_need;
+    const uint64_t prefix = s_prefix, hi = pos >= 64 ? 0ull : (~0ull << pos);
+    // this CTA's keys above the bucket and in it, as bitmaps of 32-key words
+    const int nw = (n + 31) >> 5;
+    for (int wd = warp; wd < nw; wd += 32) {
+        const int i = wd * 32 + lane;
+        const bool valid = i < n;
+        const uint64_t t = valid ? (keys[i] & hi) : 0ull;
+        const unsigned g = __ballot_sync(0xffffffffu, valid && t > prefix);
+        const unsigned e = __ballot_sync(0xffffffffu, valid && t == prefix);
+        if (lane == 0) {
+            s_gtw[wd] = g;
+            s_eqw[wd] = e;
+        }
+    }
+    __syncthreads();
+    const uint32_t g = tid < nw ? s_gtw[tid] : 0u, e = tid < nw ? s_eqw[tid] : 0u;
+    int n_gt = 0, n_eq = 0;
+    block_exclusive_sum<kSelThreads>(__popc(g), scratch, n_gt);
+    const int eq_local = block_exclusive_sum<kSelThreads>(__popc(e), scratch2, n_eq);
+    if (tid == 0) {
+        s_cnt[0] = n_gt;
+        s_cnt[1] = n_eq;
+    }
+    cluster_sync();  // every CTA's counts
+    if (warp == 0) {
+        const int gr = lane < C ? (int)ld_dsmem_u32(&s_cnt[0], lane) : 0;
+        const int er = lane < C ? (int)ld_dsmem_u32(&s_cnt[1], lane) : 0;
+        int ie = er;
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, ie, d);
+            if (lane >= d) ie += y;
+        }
+        const int eqb = ie - er;  // tied keys in the lower CTAs
+        const int take = whole ? er : max(0, min(er, need - eqb));
+        int it = gr + take;
+        const int t0 = it;
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, it, d);
+            if (lane >= d) it += y;
+        }
+        if (lane == c) {
+            s_out0 = it - t0;
+            s_eqb = eqb;
+        }
+    }
+    cluster_sync();  // no CTA leaves while another still reads its counts
+    uint32_t take = g;
+    if (whole) {
+        take |= e;
+    } else {  // one tied value: its lowest-index `need` keys over the whole cluster
+        int left = need - s_eqb - eq_local;
+        for (uint32_t ee = e; left > 0 && ee; --left) {
+            const uint32_t low = ee & (0u - ee);
+            take |= low;
+            ee ^= low;
+        }
+    }
+    int out = s_out0 + block_excl_sum_1bar<kSelThreads>(__popc(take), scratch);
+    for (uint32_t m = take; m; m &= m - 1) sel[out++] = base + tid * 32 + (__ffs(m) - 1);
+}
+
 // rank: position of selected block i = #{j : key_j > key_i} + #{j < i : key_j == key_i}
-// over the selected set (sel ascending, so a lower list index is a lower block index). A
-// CTA of 128 threads owns the 16 selected blocks 16 c .. 16 c + 15, eight threads each; it
-// stages the selected keys in tiles of 2048 and each of the eight threads counts every
-// eighth key of a tile.
+// over the selected set (sel ascending, so a lower list index is a lower block index),
+// that is #{j < i : key_j >= key_i} + #{j > i : key_j > key_i}. A CTA of 4 warps owns the
+// 32 selected blocks 32 c .. 32 c + 31, eight per warp, whose keys every lane keeps in
+// registers; it stages the selected keys in tiles of 2048, and lane l compares every 32nd
+// key of a tile with its warp's eight (one shared-memory load per eight comparisons). A
+// tile wholly before (after) the CTA's blocks needs only the >= (>) test.
 constexpr int kRankTile = 2048;
+constexpr int kRankPerWarp = 8;
+constexpr int kRankPerCta = 4 * kRankPerWarp;  // 128 threads
 __device__ __forceinline__ void rank_split_cta(const double* __restrict__ delta, const int32_t* __restrict__ sel,
                                                int budget, int32_t* __restrict__ rank, int c) {
     __shared__ uint64_t tk[kRankTile];
-    const int t = threadIdx.x, part = t & 7;
-    const int i = c * 16 + (t >> 3);
-    const uint64_t mine = i < budget ? order_key(delta[__ldg(sel + i)]) : 0ull;
-    int pos = 0;
+    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+    const int c0 = c * kRankPerCta, c1 = min(budget, c0 + kRankPerCta);
+    const int i0 = c0 + warp * kRankPerWarp;
+    uint64_t mine[kRankPerWarp];
+    int cnt[kRankPerWarp];
+    {
+        const int i = i0 + (lane & (kRankPerWarp - 1));
+        const uint64_t k = i < budget ? order_key(delta[__ldg(sel + i)]) : 0ull;
+#pragma unroll
+        for (int e = 0; e < kRankPerWarp; ++e) {
+            mine[e] = __shfl_sync(0xffffffffu, k, e);
+            cnt[e] = 0;
+        }
+    }
     for (int base = 0; base < budget; base += kRankTile) {
         const int n = min(kRankTile, budget - base);
         __syncthreads();  // the previous tile is no longer read
@@ -535,18 +753,34 @@ __device__ __forceinline__ void rank_split_cta(const double* __restrict__ delta,
                 if (j0 + 128 * u < n) tk[j0 + 128 * u] = order_key(d[u]);
         }
         __syncthreads();
-        if (i < budget) {
-            const int lim = i - base;  // tile entries below lim precede i among equal keys
-            for (int j = part; j < n; j += 8) {
+        if (base + n <= c0) {  // every staged block precedes the CTA's
+            for (int j = lane; j < n; j += 32) {
                 const uint64_t kj = tk[j];
-                pos += (kj > mine) | ((kj == mine) & (j < lim));
+#pragma unroll
+                for (int e = 0; e < kRankPerWarp; ++e) cnt[e] += kj >= mine[e];
+            }
+        } else if (base >= c1) {  // every staged block follows them
+            for (int j = lane; j < n; j += 32) {
+                const uint64_t kj = tk[j];
+#pragma unroll
+                for (int e = 0; e < kRankPerWarp; ++e) cnt[e] += kj > mine[e];
+            }
+        } else {
+            for (int j = lane; j < n; j += 32) {
+                const uint64_t kj = tk[j];
+                const int g = base + j;
+#pragma unroll
+                for (int e = 0; e < kRankPerWarp; ++e) cnt[e] += g < i0 + e ? kj >= mine[e] : kj > mine[e];
             }
         }
     }
-    pos += __shfl_xor_sync(0xffffffffu, pos, 1);
-    pos += __shfl_xor_sync(0xffffffffu, pos, 2);
-    pos += __shfl_xor_sync(0xffffffffu, pos, 4);
-    if (i < budget && part == 0) rank[pos] = sel[i];
+    int pos = 0;
+#pragma unroll
+    for (int e = 0; e < kRankPerWarp; ++e) {
+        const int v = (int)__reduce_add_sync(0xffffffffu, (unsigned)cnt[e]);
+        if (lane == e) pos = v;
+    }
+    if (lane < kRankPerWarp && i0 + lane < budget) rank[pos] = __ldg(sel + i0 + lane);
 }
 
 __global__ void __launch_bounds__(128) k_topk_rank_split(const double* __restrict__ delta,
@@ -737,6 +971,14 @@ cudaError_t launch_quant_delta(const uint16_t* W, const CUtensorMap& tw, int N, 
                       act);
 }
 
+// The cluster selection takes more keys than one CTA holds, up to kTkMaxCluster CTAs' worth;
+// beyond that the one-CTA kernel reads its keys from global memory in every pass.
+int topk_cluster_ctas(int B) {
+    if ((size_t)B * 8 <= kSelSmemKeysMax || B > kTkMaxCluster * kTkCtaKeys) return 0;
+    return kTkMaxCluster;
+}
+int topk_cluster_chunk(int B, int C) { return ((B + C - 1) / C + 31) / 32 * 32; }
+
 int topk_launches(int budget) { return budget <= 0 ? 0 : 2; }
 
 cudaError_t launch_topk_select(const double* delta, int B, int budget, int32_t* sel, cudaStream_t s) {
@@ -753,6 +995,18 @@ cudaError_t launch_topk_select(const double* delta, int B, int budget, int32_t* 
     });
     if (e != cudaSuccess) return e;
     if (smem_keys) return launch_pdl(k_topk_large<true>, dim3(1), dim3(kSelThreads), smem, s, 1, delta, B, budget, sel);
+    const int C = topk_cluster_ctas(B);
+    if (C) {
+        static std::atomic<bool> attr_c[64];
+        e = once_per_device(attr_c, [] {
+            return cudaFuncSetAttribute(k_topk_cluster, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        kTkCtaKeys * (int)sizeof(uint64_t));
+        });
+        if (e != cudaSuccess) return e;
+        const int chunk = topk_cluster_chunk(B, C);
+        return launch_pdl_cluster(k_topk_cluster, dim3(C), dim3(kSelThreads), (size_t)chunk * sizeof(uint64_t), s,
+                                  dim3(C, 1, 1), delta, B, budget, chunk, sel);
+    }
     return launch_pdl(k_topk_large<false>, dim3(1), dim3(kSelThreads), smem, s, 1, delta, B, budget, sel);
 }
 
@@ -760,8 +1014,8 @@ cudaError_t launch_topk(const double* delta, int B, int budget, int32_t* rank, i
     if (budget <= 0) return cudaSuccess;
     cudaError_t e = launch_topk_select(delta, B, budget, sel, s);
     if (e != cudaSuccess) return e;
-    return launch_pdl(k_topk_rank_split, dim3((budget + 15) / 16), dim3(128), 0, s, 1, delta, (const int32_t*)sel,
-                      budget, rank);
+    return launch_pdl(k_topk_rank_split, dim3((budget + kRankPerCta - 1) / kRankPerCta), dim3(128), 0, s, 1, delta,
+                      (const int32_t*)sel, budget, rank);
 }
 
 cudaError_t launch_pack(const uint8_t* rcodes, const uint8_t* rsf, int N, int K, const int32_t* sel, int budget,
@@ -778,7 +1032,7 @@ cudaError_t launch_pack_w(const uint16_t* W, int N, int K, const float* g_w, con
                           const double* delta, int32_t* rank, cudaStream_t s) {
     const int NBr = N / 64;
     const int ncsr = (NBr + 127) / 128;
-    const int nrank = rank && budget > 0 ? (budget + 15) / 16 : 0;
+    const int nrank = rank && budget > 0 ? (budget + kRankPerCta - 1) / kRankPerCta : 0;
     return launch_pdl(k_pack_w, dim3(budget + ncsr + nrank), dim3(128), 0, s, 1, W, N, K, g_w, sel, budget, blk_codes,
                       blk_sf, blk_kt, tile_ptr, bitmap, ncsr, delta, nrank ? rank : (int32_t*)nullptr);
 }

@@ -30,6 +30,7 @@ EXPORTED = (
     "mq_quantize_act", "mq_gemm", "mq_run_layer", "mq_get_error", "mq_status_string", "mq_launch_count",
     "mq_gemm_noalloc", "mq_gemm_noalloc_scratch_limit", "mq_quantize_weight_delta", "mq_topk_blocks",
     "mq_pack_residual_weight", "mq_gemm_act", "mq_weight_bytes", "mq_fp4_mma_loop", "mq_fp4_mma_loop_flops",
+    "mq_test_arm_wait_fault", "mq_smooth_scales", "mq_smooth_apply",
 )
 
 
@@ -74,6 +75,12 @@ def lib():
     L.mq_fp4_mma_loop.restype = i32
     L.mq_fp4_mma_loop_flops.argtypes = [i32, i32]
     L.mq_fp4_mma_loop_flops.restype = ctypes.c_double
+    L.mq_test_arm_wait_fault.argtypes = [i32, ctypes.c_double]
+    L.mq_test_arm_wait_fault.restype = i32
+    L.mq_smooth_scales.argtypes = [vp, i32, vp, i32, i32, vp, vp]
+    L.mq_smooth_scales.restype = i32
+    L.mq_smooth_apply.argtypes = [vp, i32, i32, vp, i32, vp, vp]
+    L.mq_smooth_apply.restype = i32
     L.mq_budget_blocks.argtypes = [i32, i32, ctypes.c_double]
     L.mq_budget_blocks.restype = i32
     L.mq_quantize_weight_workspace_bytes.argtypes = [i32, i32]
@@ -189,6 +196,18 @@ def alloc_packed(N: int, K: int, budget: int, device) -> dict:
 
 
 # ------------------------------------------------------------------ the path (C names)
+def mq_smooth_scales(Xcal: torch.Tensor, W: torch.Tensor, s: torch.Tensor, stream=None):
+    T, K = Xcal.shape
+    N = W.shape[0]
+    _check(lib().mq_smooth_scales(_ptr(Xcal), T, _ptr(W), N, K, _ptr(s), _stream(stream)), "mq_smooth_scales")
+
+
+def mq_smooth_apply(A: torch.Tensor, s: torch.Tensor, invert: bool, out: torch.Tensor, stream=None):
+    rows, K = A.shape
+    _check(lib().mq_smooth_apply(_ptr(A), rows, K, _ptr(s), 1 if invert else 0, _ptr(out), _stream(stream)),
+           "mq_smooth_apply")
+
+
 def mq_quantize_weight(W: torch.Tensor, base: dict, resid: dict, ws: torch.Tensor, stream=None):
     N, K = W.shape
     _check(lib().mq_quantize_weight(_ptr(W), N, K, ctypes.byref(mat(base)), ctypes.byref(mat(resid)), _ptr(ws),

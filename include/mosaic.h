@@ -145,6 +145,25 @@ size_t mq_gemm_workspace_bytes(int M, int N, int K, unsigned flags);
 /* ---- the path ----------------------------------------------------------------- */
 
 /*
+ * A0. Equivalent transform ahead of quantization (MosaicQuant summary, "Methodology",
+ * section 1: activation outliers are migrated into the weights by an equivalent
+ * transform such as SmoothQuant; the pages name it without defining it). SmoothQuant's
+ * per-input-channel rule with migration strength 1/2:
+ *   s_k = fp32( sqrt( fp32( max_t |Xcal[t][k]| / max_n |W[n][k]| ) ) )  (1 if either is 0),
+ * each operation IEEE with round-to-nearest-even. Xcal: bf16 [T][K], W: bf16 [N][K], both
+ * 16-byte aligned; s: fp32 [K]. K % 64 == 0.
+ */
+mq_status mq_smooth_scales(const mq_bf16* Xcal, int T, const mq_bf16* W, int N, int K, float* s, mq_stream stream);
+
+/*
+ * Applies the transform: out = bf16_rn(A[r][k] * s_k) for a weight (invert = 0) or
+ * bf16_rn(A[r][k] / s_k) for activations (invert != 0), so that X W^T = X' W'^T up to the
+ * two bf16 roundings. A, out: bf16 [rows][K], 16-byte aligned (out may equal A).
+ */
+mq_status mq_smooth_apply(const mq_bf16* A, int rows, int K, const float* s, int invert, mq_bf16* out,
+                          mq_stream stream);
+
+/*
  * A1. Weight quantization (MosaicQuant summary, "Methodology", section 1).
  * W: bf16 [N][K]. Writes base = NVFP4(W, g_w) and resid_full = NVFP4(W - deq Q(W), g_w)
  * for EVERY element (the residual uses the base's tensor scale g_w; selection happens

@@ -63,9 +63,11 @@ def lib():
     L.orc_pack_residual.argtypes = [vp, vp, i32, i32, vp, i32, vp, vp, vp, vp, vp]
     L.orc_sf_tile.argtypes = [vp, i32, i32, vp]
     L.orc_gemm_rows.argtypes = [vp, vp, vp, vp, vp, f32, vp, vp, vp, i32, i32, i32, i32, vp, i32, vp, vp]
+    L.orc_smooth_scales.argtypes = [vp, i32, vp, i32, i32, vp]
+    L.orc_smooth_apply.argtypes = [vp, i32, i32, vp, i32, vp]
     for name in ("orc_nvfp4_quantize", "orc_nvfp4_dequantize", "orc_quantize_weight", "orc_quantize_act",
                  "orc_hessian_diag", "orc_delta_score", "orc_topk", "orc_pack_residual", "orc_sf_tile",
-                 "orc_gemm_rows"):
+                 "orc_gemm_rows", "orc_smooth_scales", "orc_smooth_apply"):
         getattr(L, name).restype = None
     _lib = L
     return L
@@ -221,6 +223,25 @@ def gemm_rows(xq: dict, wq: dict, sel, M: int, N: int, K: int, mode: int = 0, ro
                         _p(_c(wq["r_codes"], np.uint8)), _p(_c(wq["r_sf"], np.uint8)), _p(mask), M, N, K, mode,
                         _p(rows), rows.size, _p(y), _p(ya))
     return y, ya
+
+
+def smooth_scales(Xcal: np.ndarray, W: np.ndarray) -> np.ndarray:
+    """Equivalent transform (SmoothQuant, alpha = 1/2): s_k = sqrt(max|Xcal_k| / max|W_k|)."""
+    Xcal, W = _c(Xcal, np.uint16), _c(W, np.uint16)
+    T, K = Xcal.shape
+    N = W.shape[0]
+    s = np.zeros(K, np.float32)
+    lib().orc_smooth_scales(_p(Xcal), T, _p(W), N, K, _p(s))
+    return s
+
+
+def smooth_apply(A: np.ndarray, s: np.ndarray, invert: bool) -> np.ndarray:
+    """bf16(A * s_k) (weights) or bf16(A / s_k) (activations), as bf16 bits."""
+    A = _c(A, np.uint16)
+    rows, K = A.shape
+    out = np.zeros_like(A)
+    lib().orc_smooth_apply(_p(A), rows, K, _p(_c(s, np.float32)), 1 if invert else 0, _p(out))
+    return out
 
 
 def run_path(W: np.ndarray, X: np.ndarray, Xcal: np.ndarray, budget: int, rows=None) -> dict:

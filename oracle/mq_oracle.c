@@ -423,3 +423,42 @@ void orc_gemm_rows(const uint8_t* x_codes, const uint8_t* x_sf, const float* g_x
     }
     free(xh);
 }
+
+/*
+ * Equivalent transform ahead of quantization (MosaicQuant summary, "Methodology",
+ * section 1: activation outliers are first migrated into the weights by an equivalent
+ * transform such as SmoothQuant). The pages name the transform but do not define it;
+ * this is SmoothQuant's per-input-channel rule with migration strength alpha = 1/2:
+ *   ax_k = max_t |Xcal[t][k]|,  aw_k = max_n |W[n][k]|,
+ *   s_k  = fp32( sqrt( fp32(ax_k / aw_k) ) )   (1 if ax_k or aw_k is 0),
+ * so that X W^T = (X diag(s)^-1) (W diag(s))^T, and both sides then peak at
+ * sqrt(ax_k * aw_k) in channel k. Division and square root are IEEE, rounded once each.
+ */
+void orc_smooth_scales(const uint16_t* Xcal, int T, const uint16_t* W, int N, int K, float* s) {
+    for (int k = 0; k < K; ++k) {
+        float ax = 0.0f, aw = 0.0f;
+        for (int t = 0; t < T; ++t) ax = fmaxf(ax, fabsf(bf16_to_f32(Xcal[(int64_t)t * K + k])));
+        for (int n = 0; n < N; ++n) aw = fmaxf(aw, fabsf(bf16_to_f32(W[(int64_t)n * K + k])));
+        s[k] = (ax == 0.0f || aw == 0.0f) ? 1.0f : sqrtf(ax / aw);
+    }
+}
+
+/* Round an fp32 value to bf16 (nearest, ties to even; the inputs here are finite). */
+static uint16_t f32_to_bf16_rne(float f) {
+    uint32_t u;
+    memcpy(&u, &f, 4);
+    uint32_t lsb = (u >> 16) & 1u;
+    u += 0x7FFFu + lsb;
+    return (uint16_t)(u >> 16);
+}
+
+/* Apply the transform to rows x K bf16 values: out = bf16(a * s_k) for the weight
+ * (invert = 0), out = bf16(a / s_k) for activations (invert = 1), one IEEE operation and
+ * one rounding to bf16 each. */
+void orc_smooth_apply(const uint16_t* A, int rows, int K, const float* s, int invert, uint16_t* out) {
+    for (int64_t r = 0; r < rows; ++r)
+        for (int k = 0; k < K; ++k) {
+            float a = bf16_to_f32(A[r * K + k]);
+            out[r * K + k] = f32_to_bf16_rne(invert ? a / s[k] : a * s[k]);
+        }
+}

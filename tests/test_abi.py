@@ -45,10 +45,13 @@ def test_size_helpers(L):
     assert L.mq_budget_blocks(28672, 8192, 0.05) == 2867
     assert L.mq_budget_blocks(256, 512, 1.5) == -1
     assert L.mq_quantize_weight_workspace_bytes(4096, 4096) >= 4 * 148 * 8
-    # decode GEMM at M=16, N=K=4096 (no GPU here: 148 SMs assumed): 32 weight tiles x 16
-    # K stages over 148 CTAs, so tiles are split; two fp32 partial slots of 128 x 16 per
-    # CTA, then one counter per tile
-    assert L.mq_gemm_workspace_bytes(16, 4096, 4096, 0) == 2 * 148 * 16 * 128 * 4 + 32 * 4
+    # decode GEMM at M=16, N=K=4096 (no GPU here: 148 SMs assumed): 32 weight tiles, each
+    # split among the 4 CTAs of a cluster and added through its shared memory: nothing
+    assert L.mq_gemm_workspace_bytes(16, 4096, 4096, 0) == 0
+    # 150 weight tiles (more than half the SMs): the stream-K kernel, 2400 units over 148
+    # CTAs, tiles split between CTAs: two fp32 partial slots of 128 x 16 per CTA, then one
+    # counter per tile
+    assert L.mq_gemm_workspace_bytes(16, 150 * 128, 4096, 0) == 2 * 148 * 16 * 128 * 4 + 150 * 4
     # a tile held whole by every CTA needs nothing: 148 tiles of one K stage each
     assert L.mq_gemm_workspace_bytes(16, 148 * 128, 256, 0) == 0
     # the large-M kernel needs no workspace
@@ -93,9 +96,10 @@ def test_host_validation_rejects_bad_arguments(L):
     wm2 = wt(4096, 4096)
     assert L.mq_gemm(ctypes.byref(xm), ctypes.byref(wm2), None, Y, 16, 4096, 4096,
                      mosaic.MQ_GEMM_BASE_ONLY | mosaic.MQ_GEMM_RESIDUAL_ONLY, None, 0, None) == 1
-    # a split-K problem on the workspace path needs its workspace
-    wm1 = wt(1024, 4096)
-    assert L.mq_gemm(ctypes.byref(xm), ctypes.byref(wm1), None, Y, 16, 1024, 4096, 0, None, 0, None) == 3
+    # a decode problem whose tiles are split between CTAs (the stream-K kernel at 150
+    # tiles) needs its workspace
+    wm1, Y1 = wt(19200, 4096), buf(16 * 19200 * 2)
+    assert L.mq_gemm(ctypes.byref(xm), ctypes.byref(wm1), None, Y1, 16, 19200, 4096, 0, None, 0, None) == 3
     assert L.mq_status_string(3) == b"workspace missing or too small"
     # A2 takes 1..1024 calibration tokens and a 16-byte aligned Xcal
     xcal, H = buf(1025 * 4096 * 2), buf(4096 * 4)
@@ -134,3 +138,10 @@ def test_binding_sizes_the_weight_from_weight_bytes(L):
         assert base["sf_swz"].data_ptr() == b0 + N * K // 2
         assert base["gscale"].data_ptr() == b0 + N * K // 2 + L.mq_sf_swz_bytes(N, K)
         assert all((t.data_ptr() - b0) % 16 == 0 for t in parts)
+
+
+def test_wait_fault_hook_refuses_out_of_range(L):
+    # the hook only arms the next decode GEMM launch; out-of-range arguments are refused
+    assert L.mq_test_arm_wait_fault(-1, 1.0) == 1
+    assert L.mq_test_arm_wait_fault(0, 0.0) == 1
+    assert L.mq_test_arm_wait_fault(0, 5000.0) == 1

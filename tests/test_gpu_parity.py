@@ -150,6 +150,41 @@ def test_gemm_prefill_modes(dev):
     check_gemm(outs["resid"].float().cpu().numpy().astype(np.float64), yr, yra, "prefill residual only")
 
 
+@pytest.mark.parametrize("mode", ["fused", "BASE_ONLY", "RESIDUAL_ONLY"])
+def test_gemm_prefill_pairs_many_tiles(mode, dev):
+    """The large-M kernel on CTA pairs with several tiles per pair and more K stages than
+    pipeline stages (128 tiles of 256 x 256 over at most 74 pairs, 8 stages of K each):
+    the stage and accumulator barriers cycle through many phases, including stages that
+    carry no copies for one CTA of the pair (residual-only stages without a selected
+    block). Sampled token rows against the oracle, and a repeat bit for bit."""
+    from bit_quantized_gemm_zipperengine_b200 import mosaic
+    N, K, M = 4096, 2048, 2048
+    L = {"N": N, "K": K, "M": M, "T": 128,
+         "W": synth.weight(N, K, 721, 724, 0.02, int(0.005 * N * K), (N // 64) * (K // 64) // 20, 20.0),
+         "X": synth.act(M, K, 722, 724, 20, 30.0), "Xcal": synth.act(128, K, 723, 724, 20, 30.0)}
+    budget = synth.budget_blocks(N, K, 0.10)
+    flags = mosaic.MQ_GEMM_PREFILL | (0 if mode == "fused" else getattr(mosaic, "MQ_GEMM_" + mode))
+    layer = mosaic.Layer(N, K, budget, dev)
+    layer.prepare(to_dev(L["W"], dev), to_dev(L["Xcal"], dev))
+    X = to_dev(L["X"], dev)
+    outs = []
+    for _ in range(2):
+        layer.act_buffers(M, flags)[1].fill_(float("nan"))
+        outs.append(layer.forward(X, flags).clone())
+    torch.cuda.synchronize()
+    assert mosaic.mq_get_error() == 0
+    assert torch.equal(outs[0].view(torch.int16), outs[1].view(torch.int16))
+    rows = np.array(sorted(set(list(range(0, M, 97)) + [127, 128, 255, 256, M - 1])), dtype=np.int32)
+    wq = oracle.quantize_weight(L["W"])
+    H = oracle.hessian_diag(L["Xcal"])
+    _, sel = oracle.topk(oracle.delta_score(L["W"], H, wq), budget)
+    assert np.array_equal(layer.sel[:budget].cpu().numpy(), sel)
+    xo = oracle.quantize_act(L["X"])
+    y, ya = oracle.gemm_rows(xo, wq, sel, M, N, K, {"fused": 0, "BASE_ONLY": 1, "RESIDUAL_ONLY": 2}[mode], rows)
+    got = outs[0][torch.from_numpy(rows).long().to(dev)].float().cpu().numpy().astype(np.float64)
+    check_gemm(got, y, ya, f"pairs {mode}")
+
+
 @pytest.mark.parametrize("M", [16, 100, 128])
 def test_gemm_narrow_layer_workspace_split_k(M, dev):
     """A 1024 x 4096 layer: 8 weight tiles, so K is split 16 ways and the partials are
@@ -246,6 +281,36 @@ def test_topk_blocks_alone_and_large_budgets(dev):
             r_ref, s_ref = oracle.topk(d, k)
             assert np.array_equal(rank[:k].cpu().numpy(), r_ref), (B, k)
             assert np.array_equal(sel[:k].cpu().numpy(), s_ref), (B, k)
+
+
+def test_topk_cluster_sizes_and_ties_across_ctas(dev):
+    """Key counts that take the cluster selection (more keys than one CTA holds, spread over
+    eight CTAs): just above one CTA's capacity (a ragged last CTA), LLaMA3-70B MLP's 57344
+    blocks, the largest count the cluster holds and one key more (the one-CTA kernel with
+    keys in global memory); one value tied across every CTA with the threshold inside it,
+    and all keys equal; budgets 1 .. B. Against the oracle's sort."""
+    from bit_quantized_gemm_zipperengine_b200 import mosaic
+    rng = np.random.default_rng(77)
+    for B in (20481, 57344, 163840, 163841):
+        for mode in ("spread", "tied", "equal"):
+            d = rng.standard_normal(B) * np.exp2(rng.integers(-20, 5, B))
+            if mode == "tied":
+                d[rng.choice(B, B // 3, replace=False)] = 0.5
+            elif mode == "equal":
+                d[:] = 1.25
+            dd = torch.from_numpy(d).to(dev)
+            # rank counts over the selected set (budget squared comparisons): the full
+            # budget range on the smaller key counts only
+            ks = (1, 7, B // 20, B // 3, B - 1, B) if B <= 60000 else (1, 7, B // 20, B // 3)
+            for k in ks:
+                rank = torch.empty(k, dtype=torch.int32, device=dev)
+                sel = torch.empty(k, dtype=torch.int32, device=dev)
+                mosaic.mq_topk_blocks(dd, k, rank, sel)
+                torch.cuda.synchronize()
+                assert mosaic.mq_get_error() == 0
+                r_ref, s_ref = oracle.topk(d, k)
+                assert np.array_equal(sel.cpu().numpy(), s_ref), (B, mode, k)
+                assert np.array_equal(rank.cpu().numpy(), r_ref), (B, mode, k)
 
 
 @pytest.mark.parametrize("host", [False, True])

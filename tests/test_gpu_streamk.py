@@ -1,10 +1,12 @@
-"""The decode GEMM's work split (GPU): persistent CTAs take equal contiguous ranges of
-(tile, 256-K stage) units, so tiles are cut into segments that different CTAs finish and
-one of them adds in order. The cases cover a tile held whole and a tile cut into 16
-one-unit segments, every token tile (16/32/64/128 tokens, and several of them), every
-64x64 block selected (the residual ring full on every stage), and the base-only and
-residual-only modes (segments without any residual block). Each runs twice on the same
-workspace: the tile counters must come back to zero and the output repeat bit for bit."""
+"""The decode GEMM's two kernels and their work splits (GPU). Small problems: each 128-row
+tile's K range split evenly among the CTAs of a cluster, the partials added through the
+cluster's shared memory. Larger ones (stream-K): persistent CTAs take equal contiguous
+ranges of (tile, 256-K stage) units, so tiles are cut into segments that different CTAs
+finish and one of them adds in order. The cases cover both kernels with every token tile
+(16/32/64/128 tokens, and several of them), every 64x64 block selected (the residual
+ring full on every stage), and the base-only and residual-only modes (segments without
+any residual block). Each runs twice on the same workspace: the tile counters must come
+back to zero and the output repeat bit for bit."""
 import numpy as np
 import pytest
 import torch
@@ -25,14 +27,22 @@ def dev():
 
 CASES = [
     # N, K, M, budget fraction, flags
-    (128, 256, 1, 0.50, "AUTO"),          # one unit: one CTA, one tile
-    (512, 4096, 16, 0.10, "AUTO"),        # 64 units on 64 CTAs: every tile in 16 one-unit segments
+    # the small-problem kernel (M <= 32, at most 74 tiles, short K ranges): each tile split
+    # among the CTAs of a cluster
+    (128, 256, 1, 0.50, "AUTO"),          # one tile, one K stage: one CTA
+    (512, 4096, 16, 0.10, "AUTO"),        # 4 tiles x 8 splits
     (4096, 4096, 16, 1.00, "AUTO"),       # every block selected: 8 residual blocks per stage
+    (4096, 4096, 16, 0.10, "RESIDUAL_ONLY"),
+    (4096, 4096, 16, 0.10, "BASE_ONLY"),
+    (5120, 5120, 32, 0.10, "AUTO"),       # 40 tiles x 3 splits of 6-7 stages, 32-token tile
+    # the stream-K kernel
+    (19200, 4096, 16, 0.10, "AUTO"),      # 150 tiles: 2400 units on 148 CTAs, tiles split
+    (19200, 4096, 16, 1.00, "AUTO"),      # every block selected
+    (4096, 14336, 16, 0.10, "RESIDUAL_ONLY"),  # long K: segments without residual blocks
+    (4096, 14336, 16, 0.10, "BASE_ONLY"),
     (25600, 512, 33, 0.10, "AUTO"),       # 400 units, 2-3 per CTA, 64-token tile
     (1024, 8192, 100, 0.20, "AUTO"),      # 128-token tile
     (512, 1024, 300, 0.10, "DECODE"),     # three 128-token tiles
-    (4096, 4096, 16, 0.10, "RESIDUAL_ONLY"),
-    (4096, 4096, 16, 0.10, "BASE_ONLY"),
 ]
 
 

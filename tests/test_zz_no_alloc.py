@@ -28,19 +28,20 @@ def dev():
     return torch.device("cuda:0")
 
 
-def _narrow_layer(M):
-    """A 1024 x 4096 layer: 8 weight tiles, so the decode GEMM splits K 16 ways and its
-    partials go through scratch memory (the case this entry point exists for)."""
-    N, K = 1024, 4096
+def _narrow_layer(M, N=1024):
+    """A layer whose decode GEMM (the stream-K kernel at these token counts) splits tiles
+    between CTAs, so its partials go through scratch memory (the case this entry point
+    exists for): N = 1024 (8 tiles) at 64 tokens, N = 19200 (150 tiles) at 16."""
+    K = 4096
     return {"N": N, "K": K, "M": M, "T": 128,
-            "W": synth.weight(N, K, 901, 904, 0.02, int(0.005 * N * K), 51, 20.0),
+            "W": synth.weight(N, K, 901, 904, 0.02, int(0.005 * N * K), (N // 64) * (K // 64) // 20, 20.0),
             "X": synth.act(M, K, 902, 904, 40, 30.0), "Xcal": synth.act(128, K, 903, 904, 40, 30.0)}
 
 
-@pytest.mark.parametrize("M", [16, 64])
-def test_noalloc_matches_workspace_gemm_twice(M, dev):
+@pytest.mark.parametrize("M,N", [(16, 19200), (64, 1024)])
+def test_noalloc_matches_workspace_gemm_twice(M, N, dev):
     from bit_quantized_gemm_zipperengine_b200 import mosaic
-    L = _narrow_layer(M)
+    L = _narrow_layer(M, N)
     N, K = L["N"], L["K"]
     name = f"narrow M={M}"
     assert mosaic.lib().mq_gemm_workspace_bytes(M, N, K, 0) > 0  # the scratch is really used
@@ -93,7 +94,7 @@ def test_noalloc_refuses_problems_beyond_the_static_scratch(dev):
     assert limit == 16 << 20
     # the first shape fits the static scratch; the second needs more than it holds and
     # must be refused before any launch
-    assert 0 < Lb.mq_gemm_workspace_bytes(16, 1024, 16384, 0) <= limit
+    assert 0 < Lb.mq_gemm_workspace_bytes(64, 1024, 16384, 0) <= limit
     M, N, K = 128, 1024, 16384
     assert Lb.mq_gemm_workspace_bytes(M, N, K, 0) > limit
     # real, correctly sized buffers: were the refusal to regress, the kernel would read
