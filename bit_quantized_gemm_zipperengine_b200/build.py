@@ -11,6 +11,9 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libmosaic.so")
+# the same library with MQ_TIMELINE defined: the small decode GEMM records per-CTA event
+# times (mq_timeline_read); used by timeline.py, never by the path
+LIB_TIMELINE = os.path.join(PKG, "libmosaic_timeline.so")
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -32,22 +35,24 @@ def deps():
             + [__file__])
 
 
-def stale() -> bool:
-    if not os.path.exists(LIB):
+def stale(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return any(os.path.getmtime(p) > t for p in deps())
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not (force or stale()):
-        return LIB
+def build(force: bool = False, verbose: bool = False, timeline: bool = False) -> str:
+    lib = LIB_TIMELINE if timeline else LIB
+    if not (force or stale(lib)):
+        return lib
     nvcc = os.environ.get("NVCC", "nvcc")
-    tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [nvcc, *NVCC_FLAGS, *(["-Xptxas", "-v"] if verbose else []), "-o", tmp, *sources()]
+    tmp = lib + f".tmp{os.getpid()}"
+    cmd = [nvcc, *NVCC_FLAGS, *(["-DMQ_TIMELINE"] if timeline else []), *(["-Xptxas", "-v"] if verbose else []),
+           "-o", tmp, *sources()]
     subprocess.check_call(cmd)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":

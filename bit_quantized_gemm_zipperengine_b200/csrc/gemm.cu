@@ -21,12 +21,30 @@
 
 #include "common.cuh"
 #include "gemm.cuh"
+#include "mosaic_probe.h"
 #include "quant.cuh"
 
 namespace mq {
 
 // Device error word (0 = fine, otherwise an mq_status); read and cleared by mq_get_error.
 __device__ int g_error = 0;
+
+#ifdef MQ_TIMELINE
+// Event times of the first CTAs of the latest small-problem decode launch (mq_timeline_read).
+__device__ unsigned long long g_timeline[MQ_TIMELINE_CTAS][MQ_TIMELINE_EVENTS];
+#endif
+// Records event `ev` of this CTA in a timeline build; nothing otherwise.
+__device__ __forceinline__ void tl_event(int ev) {
+#ifdef MQ_TIMELINE
+    if (blockIdx.x < MQ_TIMELINE_CTAS) {
+        unsigned long long t;
+        asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+        g_timeline[blockIdx.x][ev] = t;
+    }
+#else
+    (void)ev;
+#endif
+}
 
 // Wall-clock budget of a single pipeline wait before a kernel gives up (2 s).
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
@@ -1131,6 +1149,7 @@ __global__ void __launch_bounds__(192, 2)
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
     const uint32_t sbase = smem_u32(smem);
+    if (threadIdx.x == 0) tl_event(0);
 
     if (warp == 0) {
         // ---------------------------------------------------- producer: W, X, residual blocks
@@ -1155,10 +1174,15 @@ __global__ void __launch_bounds__(192, 2)
         };
         const int first = nu < C::kStages ? nu : C::kStages;
         const bool w_early = p.prefetch || p.w_ready;
-        if (w_early && elect_one())
+        if (w_early && elect_one()) {
             for (int i = 0; i < first; ++i) issue_w(i);
+            tl_event(1);
+        }
         __syncwarp();
-        if (!p.w_ready) griddep_wait();  // the packed residual may come from the preceding kernel
+        if (!p.w_ready) {
+            griddep_wait();  // the packed residual may come from the preceding kernel
+            if (lane == 0) tl_event(2);
+        }
         RowCursor cur0, cur1;
         if (resid) {
             cur0 = row_cursor(p, n_tile * 2 + 0, ks0 * 4);
@@ -1176,11 +1200,21 @@ __global__ void __launch_bounds__(192, 2)
             // W (unless requested before the wait) and X: X only after the wait
             if (i >= first || !w_early) {
                 if (!waited && !p.prefetch) { griddep_wait(); waited = true; }
-                if (elect_one()) issue_w(i);
+                if (elect_one()) {
+                    issue_w(i);
+                    if (i == 0) tl_event(1);
+                }
                 __syncwarp();
             }
-            if (!waited && !p.prefetch) { griddep_wait(); waited = true; }
-            if (elect_one()) issue_x(i);
+            if (!waited && !p.prefetch) {
+                griddep_wait();
+                waited = true;
+                if (lane == 0) tl_event(2);
+            }
+            if (elect_one()) {
+                issue_x(i);
+                if (i == 0) tl_event(3);
+            }
             __syncwarp();
             nbase = i + 1;
             uint32_t m = 0;
@@ -1237,6 +1271,7 @@ __global__ void __launch_bounds__(192, 2)
             const int s = i % C::kStages;
             const uint32_t par = (uint32_t)((i / C::kStages) & 1);
             if (!mbar_wait_warp_ns(&full[s], par, p.wait_ns)) break;
+            if (i == 0 && lane == 0) tl_event(4);
             tc_fence_after();
             const uint32_t st = sbase + s * C::kStageBytes;
             const uint32_t sfc = tmem + C::kSfCol0 + s * 32;
@@ -1278,7 +1313,10 @@ __global__ void __launch_bounds__(192, 2)
             acc = __shfl_sync(0xffffffffu, acc, 0);
             rc += __popc(m);
         }
-        if (elect_one()) tc_commit(accf);
+        if (elect_one()) {
+            tc_commit(accf);
+            tl_event(5);
+        }
         __syncwarp();
     }
     // ---------------------------------------------------- epilogue (warps 2..5)
@@ -1290,6 +1328,7 @@ __global__ void __launch_bounds__(192, 2)
     if (warp >= 2) {
         griddep_wait();  // g_x and Y follow the preceding kernel
         ok = epi_all(mbar_wait_warp_ns(accf, 0, p.wait_ns));
+        if (threadIdx.x == 64) tl_event(6);
         tc_fence_after();
         const bool have = ok && (dense || resid_in_range(p, n_tile, ks0, ks0 + nu));
         float acc[BN];
@@ -1316,6 +1355,7 @@ __global__ void __launch_bounds__(192, 2)
         // every CTA of the cluster holds its partial; CTA r adds rows [r*128/S, (r+1)*128/S)
         __syncwarp();
         cluster_sync();
+        if (threadIdx.x == 64) tl_event(7);
         if (warp >= 2) {
             const int r0 = split * 128 / S, r1 = (split + 1) * 128 / S, rows = r1 - r0;
             const float gw = __ldg(p.g_w);
@@ -1339,8 +1379,10 @@ __global__ void __launch_bounds__(192, 2)
                 }
             }
         }
+        if (threadIdx.x == 64) tl_event(8);
         __syncwarp();
         cluster_sync();  // peers may still be reading this CTA's partial until here
+        if (threadIdx.x == 64) tl_event(9);
     }
     __syncthreads();
     if (warp == 1) {
@@ -1795,6 +1837,22 @@ cudaError_t launch_gemm_streamk(const CUtensorMap& tw, const CUtensorMap& tx, Ge
     }
 }
 
+}  // namespace mq
+
+extern "C" mq_status mq_timeline_read(void* out, size_t bytes) {
+#ifdef MQ_TIMELINE
+    if (!out || bytes < sizeof(mq::g_timeline)) return MQ_ERR_INVALID_ARG;
+    if (cudaMemcpyFromSymbol(out, mq::g_timeline, sizeof(mq::g_timeline)) != cudaSuccess) return MQ_ERR_CUDA;
+    static const unsigned long long zero[MQ_TIMELINE_CTAS][MQ_TIMELINE_EVENTS] = {};
+    return cudaMemcpyToSymbol(mq::g_timeline, zero, sizeof(zero)) == cudaSuccess ? MQ_OK : MQ_ERR_CUDA;
+#else
+    (void)out;
+    (void)bytes;
+    return MQ_ERR_INVALID_ARG;
+#endif
+}
+
+namespace mq {
 // Device address of the error word (for kernels of other translation units).
 cudaError_t error_word(int** ptr) { return cudaGetSymbolAddress(reinterpret_cast<void**>(ptr), g_error); }
 

@@ -30,7 +30,7 @@ EXPORTED = (
     "mq_quantize_act", "mq_gemm", "mq_run_layer", "mq_get_error", "mq_status_string", "mq_launch_count",
     "mq_gemm_noalloc", "mq_gemm_noalloc_scratch_limit", "mq_quantize_weight_delta", "mq_topk_blocks",
     "mq_pack_residual_weight", "mq_gemm_act", "mq_weight_bytes", "mq_fp4_mma_loop", "mq_fp4_mma_loop_flops",
-    "mq_test_arm_wait_fault", "mq_smooth_scales", "mq_smooth_apply",
+    "mq_test_arm_wait_fault", "mq_smooth_scales", "mq_smooth_apply", "mq_timeline_read",
 )
 
 
@@ -75,6 +75,8 @@ def lib():
     L.mq_fp4_mma_loop.restype = i32
     L.mq_fp4_mma_loop_flops.argtypes = [i32, i32]
     L.mq_fp4_mma_loop_flops.restype = ctypes.c_double
+    L.mq_timeline_read.argtypes = [vp, ctypes.c_size_t]
+    L.mq_timeline_read.restype = i32
     L.mq_test_arm_wait_fault.argtypes = [i32, ctypes.c_double]
     L.mq_test_arm_wait_fault.restype = i32
     L.mq_smooth_scales.argtypes = [vp, i32, vp, i32, i32, vp, vp]

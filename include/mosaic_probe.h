@@ -30,6 +30,27 @@ mq_status mq_fp4_mma_loop(int ctas, int iters, mq_stream stream);
 /* 2 * 128 * 256 * 64 flops per MMA, times ctas * iters. */
 double mq_fp4_mma_loop_flops(int ctas, int iters);
 
+/*
+ * Event times of the small-problem decode GEMM (the cluster-split kernel), for a library
+ * built with MQ_TIMELINE defined (bit_quantized_gemm_zipperengine_b200/build.py builds it as
+ * libmosaic_timeline.so): every launch records %globaltimer (ns) at fixed points of its
+ * first MQ_TIMELINE_CTAS CTAs, over the previous launch's values. The table is
+ * uint64 [MQ_TIMELINE_CTAS][MQ_TIMELINE_EVENTS], 0 where an event did not happen:
+ *   0 CTA set up (barriers initialised, tensor memory allocated)
+ *   1 first W copies issued          2 the wait for the preceding kernel returned
+ *   3 first X copies issued          4 first stage landed (MMA issuer)
+ *   5 last MMAs issued               6 accumulator complete (epilogue)
+ *   7 partial in shared memory, first cluster barrier passed
+ *   8 this CTA's rows added and stored   9 last cluster barrier passed
+ * Copies the table into `out` (host memory of at least `bytes` >= its size) and clears
+ * it on the device. Synchronous with the device. Returns MQ_ERR_INVALID_ARG for a null
+ * or short `out`, and in a library built without MQ_TIMELINE; MQ_ERR_CUDA if a copy
+ * fails.
+ */
+#define MQ_TIMELINE_CTAS 160
+#define MQ_TIMELINE_EVENTS 16
+mq_status mq_timeline_read(void* out, size_t bytes);
+
 #ifdef __cplusplus
 }
 #endif

@@ -140,6 +140,13 @@ def test_binding_sizes_the_weight_from_weight_bytes(L):
         assert all((t.data_ptr() - b0) % 16 == 0 for t in parts)
 
 
+def test_timeline_read_needs_the_timeline_build(L):
+    # the event table exists only in the library built with MQ_TIMELINE
+    buf = (ctypes.c_uint64 * (160 * 16))()
+    assert L.mq_timeline_read(ctypes.byref(buf), ctypes.sizeof(buf)) == 1
+    assert L.mq_timeline_read(None, 0) == 1
+
+
 def test_wait_fault_hook_refuses_out_of_range(L):
     # the hook only arms the next decode GEMM launch; out-of-range arguments are refused
     assert L.mq_test_arm_wait_fault(-1, 1.0) == 1
