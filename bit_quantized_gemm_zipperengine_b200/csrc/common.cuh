@@ -69,6 +69,19 @@ __device__ __forceinline__ uint64_t ld_dsmem_u64(const void* local, uint32_t ran
     asm volatile("ld.shared::cluster.u64 %0, [%1];" : "=l"(v) : "r"(mapa_u32(smem_u32(local), rank)) : "memory");
     return v;
 }
+// Two adjacent 32-bit words (8-byte aligned) from CTA `rank` of the cluster.
+__device__ __forceinline__ uint2 ld_dsmem_u32x2(const void* local, uint32_t rank) {
+    uint2 v;
+    asm volatile("ld.shared::cluster.v2.u32 {%0, %1}, [%2];"
+                 : "=r"(v.x), "=r"(v.y)
+                 : "r"(mapa_u32(smem_u32(local), rank))
+                 : "memory");
+    return v;
+}
+// Atomic add (no return value) to a 32-bit word in the shared memory of a CTA of the cluster.
+__device__ __forceinline__ void red_add_dsmem_u32(uint32_t cluster_saddr, uint32_t v) {
+    asm volatile("red.shared::cluster.add.u32 [%0], %1;" ::"r"(cluster_saddr), "r"(v) : "memory");
+}
 // fp32 store into (possibly another CTA's) shared memory of the cluster.
 __device__ __forceinline__ void st_dsmem_f32(uint32_t cluster_saddr, float v) {
     asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(cluster_saddr), "f"(v) : "memory");

@@ -510,11 +510,12 @@ __global__ void __launch_bounds__(kSelThreads) k_topk_large(const double* __rest
 // its shared-memory keys, and every decision is taken identically in every CTA from the
 // same cluster-wide counts:
 //  - the common leading bits from each CTA's AND / OR of its keys, read through DSMEM;
-//  - in each radix pass, every CTA counts its keys into its own histogram, then each thread
-//    adds its two bins over the C histograms (DSMEM loads) before the block scan. The
-//    histograms rotate over three buffers: the one a pass clears was last read by the other
-//    CTAs two passes earlier, and every CTA has crossed the previous pass's cluster barrier
-//    since;
+//  - in each radix pass, every CTA counts its keys into its own histogram and adds its
+//    non-zero bins into the sum histogram of the bin pair's owner, CTA (b / 2) % C (remote
+//    atomic adds, which do not wait for a reply); after a cluster barrier each thread reads
+//    its two bins of the sum from their owner (one load) before the block scan. The sums
+//    rotate over three buffers: the one a pass clears was last read two passes earlier, and
+//    every CTA has crossed the previous pass's cluster barrier since;
 //  - compaction: each CTA's counts above the bucket and in it are exchanged once, giving its
 //    offset in sel and the tied keys that the lower CTAs take; a last cluster barrier keeps
 //    every CTA resident until the others have read its counts.
@@ -525,7 +526,8 @@ __global__ void __launch_bounds__(kSelThreads) k_topk_cluster(const double* __re
                                                               int chunk, int32_t* __restrict__ sel) {
     extern __shared__ __align__(16) uint64_t dyn[];
     uint64_t* keys = dyn;  // [chunk]
-    __shared__ unsigned hist[3][1 << kDigitBits];
+    __shared__ unsigned hist[1 << kDigitBits];        // this CTA's counts of the pass
+    __shared__ __align__(8) unsigned hsum[3][1 << kDigitBits];  // the cluster's counts of owned bins
     __shared__ uint32_t s_gtw[kTkCtaKeys / 32], s_eqw[kTkCtaKeys / 32];
     __shared__ uint32_t s_and[64], s_or[64];
     __shared__ uint64_t s_ao[2];   // this CTA's AND and OR of its keys (read by the cluster)
@@ -572,7 +574,7 @@ __global__ void __launch_bounds__(kSelThreads) k_topk_cluster(const double* __re
             s_or[2 * warp + 1] = ol;
         }
     }
-    for (int b = tid; b < (1 << kDigitBits); b += kSelThreads) hist[0][b] = 0;
+    for (int b = tid; b < (1 << kDigitBits); b += kSelThreads) hsum[0][b] = 0;
     __syncthreads();
     if (warp == 0) {
         const uint32_t ah = __reduce_and_sync(0xffffffffu, s_and[2 * lane]);
@@ -584,7 +586,7 @@ __global__ void __launch_bounds__(kSelThreads) k_topk_cluster(const double* __re
             s_ao[1] = ((uint64_t)oh << 32) | ol;
         }
     }
-    cluster_sync();  // every CTA's AND / OR and cleared first histogram
+    cluster_sync();  // every CTA's AND / OR, and the first sum histogram cleared
     if (warp == 0) {
         const uint64_t ar = lane < C ? ld_dsmem_u64(&s_ao[0], lane) : ~0ull;
         const uint64_t orr = lane < C ? ld_dsmem_u64(&s_ao[1], lane) : 0ull;
@@ -608,8 +610,13 @@ __global__ void __launch_bounds__(kSelThreads) k_topk_cluster(const double* __re
         const uint64_t prefix = s_prefix, hi = pos >= 64 ? 0ull : (~0ull << pos);
         const int need = s_need;
         const int nb = 1 << w;
-        unsigned* h = hist[pass % 3];
-        for (int b = tid; b < (1 << kDigitBits); b += kSelThreads) hist[(pass + 1) % 3][b] = 0;
+        unsigned* h = hist;
+        unsigned* hs = hsum[pass % 3];
+        for (int b = tid; b < (1 << kDigitBits); b += kSelThreads) {
+            h[b] = 0;
+            hsum[(pass + 1) % 3][b] = 0;
+        }
+        __syncthreads();
         for (int i0 = tid - lane; i0 < n; i0 += U * kSelThreads) {  // warp-uniform
             uint64_t k[U];
 #pragma unroll
@@ -623,14 +630,21 @@ __global__ void __launch_bounds__(kSelThreads) k_topk_cluster(const double* __re
                 if (i < n && (k[u] & hi) == prefix) atomicAdd(&h[(unsigned)(k[u] >> shift) & (nb - 1)], 1u);
             }
         }
-        cluster_sync();  // every CTA's histogram of this pass is complete
+        __syncthreads();  // this CTA's counts are complete
         const int b0 = nb - 1 - 2 * tid;
+        // bins b0 - 1 and b0 (b0 odd: nb is even) belong to CTA (b0 / 2) % C
+        const uint32_t owner = b0 >= 0 ? (uint32_t)((b0 >> 1) % C) : 0u;
+        if (b0 >= 1) {
+            const unsigned v0 = h[b0], v1 = h[b0 - 1];
+            if (v0) red_add_dsmem_u32(mapa_u32(smem_u32(&hs[b0]), owner), v0);
+            if (v1) red_add_dsmem_u32(mapa_u32(smem_u32(&hs[b0 - 1]), owner), v1);
+        }
+        cluster_sync();  // the cluster's counts of this pass are complete at their owners
         unsigned c0 = 0u, c1 = 0u;
-        if (b0 >= 0) {
-            for (int r = 0; r < C; ++r) {
-                c0 += ld_dsmem_u32(&h[b0], r);
-                if (b0 >= 1) c1 += ld_dsmem_u32(&h[b0 - 1], r);
-            }
+        if (b0 >= 1) {
+            const uint2 v = ld_dsmem_u32x2(&hs[b0 - 1], owner);
+            c0 = v.y;
+            c1 = v.x;
         }
         const int above = block_excl_sum_1bar<kSelThreads>((int)(c0 + c1), scratch);
         if (b0 >= 0 && above < need && above + (int)(c0 + c1) >= need) {
