@@ -58,6 +58,15 @@ __device__ __forceinline__ uint32_t mapa_u32(uint32_t local_saddr, uint32_t rank
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(local_saddr), "r"(rank));
     return ra;
 }
+// 16-byte load (16-byte aligned) from the same shared-memory offset in CTA `rank`.
+__device__ __forceinline__ float4 ld_dsmem_f32x4(const void* local, uint32_t rank) {
+    float4 v;
+    asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "r"(mapa_u32(smem_u32(local), rank))
+                 : "memory");
+    return v;
+}
 // 32- and 64-bit loads from the same shared-memory offset in CTA `rank` of the cluster.
 __device__ __forceinline__ uint32_t ld_dsmem_u32(const void* local, uint32_t rank) {
     uint32_t v;

@@ -1357,25 +1357,39 @@ __global__ void __launch_bounds__(192, 2)
         cluster_sync();
         if (threadIdx.x == 64) tl_event(7);
         if (warp >= 2) {
-            const int r0 = split * 128 / S, r1 = (split + 1) * 128 / S, rows = r1 - r0;
+            // rows [r0, r1) of every token, four rows (a 16-byte run of each CTA's partial)
+            // per work item: one 16-byte DSMEM load per split instead of four scalar ones
+            const int r0 = split * 128 / S, r1 = (split + 1) * 128 / S;
+            const int q0 = r0 >> 2, q1 = (r1 + 3) >> 2;  // the 4-row runs touching [r0, r1)
             const float gw = __ldg(p.g_w);
             const int m0 = m_tile * BN;
-            const int total = rows * BN;
+            const int total = (q1 - q0) * BN;
             for (int e = threadIdx.x - 64; e < total; e += 128) {
-                const int j = e / rows, nl = r0 + e % rows;
-                float v[8];
+                const int j = e / (q1 - q0), nq = 4 * (q0 + e % (q1 - q0));
+                float4 v[8];
 #pragma unroll
                 for (int s2 = 0; s2 < 8; ++s2)
-                    if (s2 < S) v[s2] = ld_dsmem_f32(part + j * 128 + nl, (uint32_t)s2);
-                float sum = v[0];
+                    if (s2 < S) v[s2] = ld_dsmem_f32x4(part + j * 128 + nq, (uint32_t)s2);
+                float4 sum = v[0];
 #pragma unroll
                 for (int s2 = 1; s2 < 8; ++s2)
-                    if (s2 < S) sum = __fadd_rn(sum, v[s2]);
+                    if (s2 < S) {
+                        sum.x = __fadd_rn(sum.x, v[s2].x);
+                        sum.y = __fadd_rn(sum.y, v[s2].y);
+                        sum.z = __fadd_rn(sum.z, v[s2].z);
+                        sum.w = __fadd_rn(sum.w, v[s2].w);
+                    }
                 const int mm = m0 + j;
                 if (ok && mm < p.M) {
                     const float sc = __fmul_rn(__ldg(p.g_x + mm), gw);
-                    const __nv_bfloat16 y = __float2bfloat16_rn(__fmul_rn(sum, sc));
-                    p.Y[(int64_t)mm * p.N + n_tile * 128 + nl] = *reinterpret_cast<const uint16_t*>(&y);
+                    const float r4[4] = {sum.x, sum.y, sum.z, sum.w};
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int nl = nq + u;
+                        if (nl < r0 || nl >= r1) continue;  // a run that straddles the range
+                        const __nv_bfloat16 y = __float2bfloat16_rn(__fmul_rn(r4[u], sc));
+                        p.Y[(int64_t)mm * p.N + n_tile * 128 + nl] = *reinterpret_cast<const uint16_t*>(&y);
+                    }
                 }
             }
         }
