@@ -1624,8 +1624,6 @@ __global__ void __launch_bounds__(Prefill2Cfg::kThreads, 1)
             int sc = 0, rc = 0, tc = 0;
             bool ok = true;
             for (int t = pair; t < ntiles && ok; t += npairs, ++tc) {
-                if (!mbar_wait_warp_cluster(acce, (tc & 1) ^ 1)) break;  // both epilogues read the previous tile
-                tc_fence_after();
                 uint32_t acc4 = 0;  // bit h: slice h already holds a partial sum
                 for (int ks = 0; ks < KS; ++ks, ++sc) {
                     const int s = sc % C::kStages;
@@ -1661,6 +1659,16 @@ __global__ void __launch_bounds__(Prefill2Cfg::kThreads, 1)
                                                     sd0 + (uint64_t)((C::kOffRing + slot_i * C::kRSlotBytes + 1024) >> 4));
                             }
                         }
+                    }
+                    if (ks == 0) {
+                        // A tile's first scale copies go into the pipe before the wait for
+                        // both epilogues to have read the previous tile's accumulator: they
+                        // write scale columns only, and run while the accumulator drains.
+                        __syncwarp();
+                        if (!mbar_wait_warp_cluster(acce, (tc & 1) ^ 1)) { ok = false; break; }
+                        tc_fence_after();
+                    }
+                    if (elect_one()) {
                         if (dense) {
 #pragma unroll
                             for (int kk = 0; kk < 4; ++kk)
@@ -1703,23 +1711,12 @@ __global__ void __launch_bounds__(Prefill2Cfg::kThreads, 1)
             const bool waited = epi_all256(mbar_wait_warp(accf, tc & 1));
             tc_fence_after();
             const uint32_t slices = waited ? prefill_tile_slices(p, n_tile) : 0u;
-            // this thread's row: 128 columns, read 64 at a time (one 64-column slice, its four
-            // loads in flight together) and kept as scaled bf16 pairs, so the accumulator is
-            // released before the stores
-            uint32_t packed[64];
-#pragma unroll
-            for (int b = 0; b < 2; ++b) {
-                float v[64];
-                tmem_ld_chunks<4>(tmem + ((uint32_t)(32 * q) << 16) + 128 * half + 64 * b,
-                                  (slices >> (2 * half + b)) & 1u ? 0xFu : 0u, v);
-#pragma unroll
-                for (int u = 0; u < 32; ++u) {
-                    const __nv_bfloat16 lo = __float2bfloat16_rn(__fmul_rn(v[2 * u], sc));
-                    const __nv_bfloat16 hi = __float2bfloat16_rn(__fmul_rn(v[2 * u + 1], sc));
-                    packed[32 * b + u] = (uint32_t)(*reinterpret_cast<const uint16_t*>(&lo)) |
-                                         ((uint32_t)(*reinterpret_cast<const uint16_t*>(&hi)) << 16);
-                }
-            }
+            // this thread's row: 128 columns (two 64-column slices), all eight loads in flight
+            // together; the accumulator is released before the scaling and the stores
+            float v[128];
+            tmem_ld_chunks<8>(tmem + ((uint32_t)(32 * q) << 16) + 128 * half,
+                              ((slices >> (2 * half)) & 1u ? 0x0Fu : 0u) | ((slices >> (2 * half + 1)) & 1u ? 0xF0u : 0u),
+                              v);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_remote(acce_even);  // this CTA's rows are read
@@ -1727,9 +1724,17 @@ __global__ void __launch_bounds__(Prefill2Cfg::kThreads, 1)
             if (mm < p.M) {
                 uint16_t* yrow = p.Y + (int64_t)mm * p.N + n_tile * 256 + 128 * half;
 #pragma unroll
-                for (int c = 0; c < 16; ++c)
-                    *reinterpret_cast<uint4*>(yrow + 8 * c) =
-                        make_uint4(packed[4 * c], packed[4 * c + 1], packed[4 * c + 2], packed[4 * c + 3]);
+                for (int c = 0; c < 16; ++c) {
+                    uint32_t w[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const __nv_bfloat16 lo = __float2bfloat16_rn(__fmul_rn(v[8 * c + 2 * u], sc));
+                        const __nv_bfloat16 hi = __float2bfloat16_rn(__fmul_rn(v[8 * c + 2 * u + 1], sc));
+                        w[u] = (uint32_t)(*reinterpret_cast<const uint16_t*>(&lo)) |
+                               ((uint32_t)(*reinterpret_cast<const uint16_t*>(&hi)) << 16);
+                    }
+                    *reinterpret_cast<uint4*>(yrow + 8 * c) = make_uint4(w[0], w[1], w[2], w[3]);
+                }
             }
         }
     }
