@@ -101,15 +101,16 @@ def source_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def dram_traffic(call: str):
-    """Bytes per call from a committed ncu capture, if it was taken on the current sources."""
+def dram_traffic(call: str, workload: str):
+    """Bytes per call from a committed ncu capture, if it was taken on the current sources
+    and on this workload."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
         d = json.load(f)
     e = d.get(call)
-    if not e or e.get("source_hash") != source_hash():
+    if not e or e.get("source_hash") != source_hash() or e.get("workload") != workload:
         return None
     return e.get("bytes_per_call")
 
@@ -489,7 +490,8 @@ def replica_gbs(bytes_per_step: float, world: int, ms_per_step: float) -> float:
 TRAFFIC_KERNELS = {"quantize_weight_delta": ("k_amax_partial", "k_quant_delta"), "gemm": ("k_gemm_small",)}
 
 
-def write_traffic(csv_path: str, call: str = "quantize_weight_delta", skip: int = 0, out_path: str | None = None) -> dict:
+def write_traffic(csv_path: str, call: str = "quantize_weight_delta", skip: int = 0, out_path: str | None = None,
+                  workload: str = DEFAULT_WORKLOAD) -> dict:
     """Turn an ncu CSV (--csv --print-units base, metrics dram__bytes_read.sum and
     dram__bytes_write.sum, kernels of `call` only, caches not flushed) into
     profiles/traffic.json: DRAM bytes per call, averaged over the complete calls captured
@@ -524,7 +526,7 @@ def write_traffic(csv_path: str, call: str = "quantize_weight_delta", skip: int 
         with open(p) as f:
             d = json.load(f)
     d[call] = {"bytes_per_call": int(round(sum(per_call) / len(per_call))), "calls": len(per_call),
-               "kernels": list(TRAFFIC_KERNELS[call]), "source_hash": source_hash()}
+               "kernels": list(TRAFFIC_KERNELS[call]), "workload": workload, "source_hash": source_hash()}
     with open(p, "w") as f:
         json.dump(d, f, indent=1)
         f.write("\n")
@@ -586,7 +588,7 @@ def whole_path(dev, wl_name: str, sets_n: int, steps: int, stream) -> dict:
         us = graph_time_us(lambda: [issue(c, s) for _ in range(4) for s in sets], 4 * sets_n, 20, stream)
         gbs = per_call[c] / (us * 1e-6) / 1e9
         kern[c] = {"us": round(us, 3), "alg_bytes": per_call[c], "gbs": round(gbs, 1), "frac_hbm": round(gbs / hbm, 4),
-                   "traffic": dram_traffic(c)}
+                   "traffic": dram_traffic(c, wl_name)}
     bytes_step = sum(per_call.values())
     out = {"workload": wl_name, "us_per_step": round(us_step, 3), "alg_bytes": bytes_step,
            "gbs": round(bytes_step / (us_step * 1e-6) / 1e9, 1), "launches_per_step": int(launches),
@@ -618,7 +620,8 @@ def main():
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     if args.traffic_from:
-        print(json.dumps(write_traffic(args.traffic_from, call=args.traffic_call, skip=args.traffic_skip)))
+        print(json.dumps(write_traffic(args.traffic_from, call=args.traffic_call, skip=args.traffic_skip,
+                                       workload=args.workload)))
         return
 
     if args.impl == "reference":
@@ -741,7 +744,7 @@ def main():
     roofline = {"bound": "hbm", "kernel": f"gemm ({gemm_kernel(M, N, K)[0]})",
                 "timing": f"CUDA events around {args.steps} back-to-back calls over {R} operand copies",
                 "achieved": round(gbs_rank, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": round(gbs_rank / peaks["hbm_gbs"], 4), "traffic": dram_traffic("gemm"),
+                "frac": round(gbs_rank / peaks["hbm_gbs"], 4), "traffic": dram_traffic("gemm", args.workload),
                 "peak_source": f"{peaks['source']} (copy bandwidth)"}
     # the same calls with MQ_GEMM_WEIGHTS_READY (a layer's weights at inference: the next
     # call's W is requested before it waits for the current one)

@@ -41,11 +41,18 @@ def test_traffic_ingestion(tmp_path):
     csv_path = tmp_path / "traffic.csv"
     csv_path.write_text("".join(lines))
     out = tmp_path / "traffic.json"
-    e = bench.write_traffic(str(csv_path), skip=1, out_path=str(out))
+    e = bench.write_traffic(str(csv_path), skip=1, out_path=str(out), workload="qwen3_32b")
     want = sum(sum(c) for c in calls[1:]) / 2
     assert e["calls"] == 2 and abs(e["bytes_per_call"] - want) <= 1
     d = json.loads(out.read_text())
     assert d["quantize_weight_delta"]["source_hash"] == bench.source_hash()
+    assert d["quantize_weight_delta"]["workload"] == "qwen3_32b"
+
+
+def test_traffic_belongs_to_its_workload():
+    # a capture taken on one workload is never reported for another
+    assert bench.dram_traffic("gemm", "llama3_8b_mlp_prefill") is None
+    assert bench.dram_traffic("gemm", "no such workload") is None
 
 
 def test_clock_summary():
