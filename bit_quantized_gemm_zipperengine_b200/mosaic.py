@@ -360,17 +360,20 @@ class Layer:
         mq_topk_blocks(self.delta, self.budget, self.rank, self.sel, stream)
         mq_pack_residual_weight(W, self.base, self.sel, self.budget, self.packed, stream)
 
-    def act_buffers(self, M: int, flags: int = 0):
-        key = (M, flags)
+    def act_buffers(self, M: int, flags: int = 0, slot: int = 0):
+        """Quantized X, Y and the GEMM workspace for M tokens (cached per M, flags and slot:
+        calls in flight together on different streams take different slots)."""
+        key = (M, flags, slot)
         if key not in self._act:
             self._act[key] = (alloc_act(M, self.K, self.device),
                               torch.empty((M, self.N), dtype=torch.bfloat16, device=self.device),
                               gemm_workspace(M, self.N, self.K, flags, self.device))
         return self._act[key]
 
-    def buffers(self, M: int, T: int, flags: int = 0, staging: bool = False) -> LayerBuffers:
-        """The ctypes struct mq_run_layer takes (staging buffers for host inputs)."""
-        xq, Y, ws = self.act_buffers(M, flags)
+    def buffers(self, M: int, T: int, flags: int = 0, staging: bool = False, slot: int = 0) -> LayerBuffers:
+        """The ctypes struct mq_run_layer takes (staging buffers for host inputs). Every slot
+        has its own activation and staging buffers; the layer's weights are shared."""
+        xq, Y, ws = self.act_buffers(M, flags, slot)
         b = LayerBuffers()
         b.base, b.resid_full, b.xq = mat(self.base), mat(self.resid), mat(xq)
         b.H, b.delta, b.rank, b.sel = _ptr(self.H), _ptr(self.delta), _ptr(self.rank), _ptr(self.sel)
@@ -378,7 +381,7 @@ class Layer:
         b.ws_quant, b.ws_quant_bytes = _ptr(self.qws), self.qws.numel()
         b.ws_gemm, b.ws_gemm_bytes = (_ptr(ws), ws.numel()) if ws is not None else (None, 0)
         if staging:
-            key = ("staging", M, T)
+            key = ("staging", M, T, slot)
             if key not in self._act:
                 bf = torch.bfloat16
                 self._act[key] = (torch.empty((self.N, self.K), dtype=bf, device=self.device),
