@@ -716,9 +716,9 @@ def main():
     ev1.record(stream)
     torch.cuda.synchronize()
     t_wall1 = time.time()
-    # the same steps for one more second, so the SM clock has samples under this load
-    # even when the timed region is shorter than the sampling interval
-    while time.time() - t_wall1 < 1.0:
+    # the same steps for three more seconds, so the SM clock has about 15 samples under
+    # this load even when the timed region is shorter than the sampling interval
+    while time.time() - t_wall1 < 3.0:
         run_steps(R * 50)
         torch.cuda.synchronize()
     t_wall2 = time.time()
@@ -733,7 +733,7 @@ def main():
     value = replica_gbs(per_call, world, ms_step)
     clocks = sampler.summary(t_wall0, t_wall2)
     if clocks:
-        clocks["window"] = "timed region + 1 s of the same steps"
+        clocks["window"] = "timed region + 3 s of the same steps"
     fl_exec, fl_dense = gemm_flops(M, N, K, budget)
     gbs_rank = per_call / (us * 1e-6) / 1e9
     fp4_burst = peaks["bf16_tflops"] * FP4_PER_BF16
