@@ -871,7 +871,8 @@ def main():
     if rank != 0:
         return
     line = {"metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
-            "warmup": warmup_done, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "warmup": args.warmup, "warmup_steps_run": warmup_done, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "nvfp4 (e2m1 x e2m1, e4m3 scales, fp32 accumulate)",
             "data": "synthetic",
             "config": {"workload": f"{args.workload} fused GEMM", "M": M, "N": N, "K": K, "budget_frac": 0.10,
